@@ -1,0 +1,376 @@
+"""Decode benchmark for factor-space KPA / TPA attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kpa|reference]
+                    [--workload tpa_decode|kpa_medium|kpa_long|tiny_kpa] [--layers L]
+
+A step is one decode pass of a model of L attention layers over one batch: per
+layer, kpa_decode of one query row per sequence against that layer's own factor
+cache (rotation of the query, factor-space scores, online softmax, value
+accumulation, split combine).  Each layer has its own cache, so a step streams
+L x (cache bytes) through HBM and the L2 (126 MB) holds none of it between uses.
+The whole step is one CUDA graph.  Throughput is cached tokens attended per
+second per layer, summed over ranks; each rank runs its own replica (the batch
+shards with no exchange).
+
+Printed: one JSON line (rank 0) with the metric, the roofline of the decode
+kernel against the measured HBM copy bandwidth, the float64 CPU oracle timed on
+a bounded sample (cpu_baseline), an end-to-end figure through the public API with
+host buffers (e2e), SM clocks sampled during the timed region, and the number of
+library kernel launches in the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode cached-tokens/s per layer; achieved HBM GB/s vs B200 peak (1 GPU)"
+PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
+KERNEL_SOURCES = ["factorised_kv_attention_b200/csrc/kpa_decode_fma.cu",
+                  "factorised_kv_attention_b200/csrc/kpa_internal.cuh"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kpa", "reference"], default="kpa")
+    ap.add_argument("--workload", default="tpa_decode")
+    ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def _dist():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def _kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _hbm_peak():
+    try:
+        with open(PEAKS) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _traffic(kernel_hash):
+    try:
+        with open(TRAFFIC) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("kernel_sources_sha") != kernel_hash:
+        return None
+    return t.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """SM clock and throttle reasons via NVML (read only), sampled every 50 ms."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hd = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hd)
+                u = u.decode() if isinstance(u, bytes) else u
+                if uuid in u or u.endswith(uuid):
+                    handle = hd
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml, self.handle = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report what we could not sample
+            self.error = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.05)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def _workload(name):
+    from workloads import DECODE_CONFIGS
+    return DECODE_CONFIGS[name]
+
+
+def _config_json(w, layers, lens, world):
+    cache_bytes = int(sum(lens)) * (w.shape.e_k + w.shape.e_v) * (2 if w.dtype == "bf16" else 4)
+    return {"workload": w.name, "batch": w.batch, "seq_len": int(max(lens)),
+            "mean_seq_len": float(np.mean(lens)), "layers": layers,
+            "factor_cache_bytes_per_layer": cache_bytes,
+            "l2": f"inputs larger than L2: {layers} distinct layer caches, "
+                  f"{layers * cache_bytes / 1e6:.0f} MB per step per GPU",
+            "parallelism": f"replicas x{world} (batch-sharded, no exchange)",
+            "accumulate": "fp32"}
+
+
+def _cpu_baseline(w, inp, seconds, steps=None):
+    """The float64 oracle, as it stands, on whole sequences of the workload."""
+    import oracle
+    from workloads import to_f64
+    oracle.build()
+    q, kf, vf = to_f64(inp["q"]), to_f64(inp["kf"]), to_f64(inp["vf"])
+    L, qp = inp["seq_len"].numpy(), inp["q_pos"].numpy()
+    cores = oracle.max_threads()
+    done_tokens, t_total, n_seq, times = 0, 0.0, 0, []
+    b = 0
+    while (steps is None and t_total < seconds) or (steps is not None and len(times) < steps):
+        t0 = time.perf_counter()
+        oracle.decode(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1], q_pos=qp[b:b + 1])
+        dt = time.perf_counter() - t0
+        times.append(dt)
+        t_total += dt
+        done_tokens += int(L[b])
+        n_seq += 1
+        b = (b + 1) % w.batch
+    return {"value": done_tokens / t_total, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_seq} whole sequences (all {w.shape.h} heads) of one layer of the "
+                      f"workload, float64 C oracle, OpenMP over heads, {t_total:.1f} s"}, times
+
+
+def run_reference(a):
+    rank, world, _ = _dist()
+    if rank != 0:
+        return 0
+    from workloads import decode_inputs
+    w = _workload(a.workload)
+    inp = decode_inputs(w)
+    _cpu_baseline(w, inp, 0, steps=a.warmup)
+    base, times = _cpu_baseline(w, inp, 0, steps=a.steps)
+    L = inp["seq_len"].numpy()
+    value = base["value"]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config_json(w, 1, L, 1),
+            "cpu_baseline": base,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    line["config"]["sample"] = "one whole sequence of one layer per step"
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_kpa(a):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+
+    import factorised_kv_attention_b200 as kpa
+    from workloads import decode_inputs
+
+    w = _workload(a.workload)
+    s = w.shape
+    elt = 2 if w.dtype == "bf16" else 4
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    first = decode_inputs(w.replace(seed=1000 * rank))
+    lens = first["seq_len"].numpy()
+    layer_bytes = int(lens.sum()) * (s.e_k + s.e_v) * elt
+    layers = a.layers or max(1, int(np.ceil(4 * l2 / max(layer_bytes, 1))))
+    cfg = kpa.make_config(s, w.dtype)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    # per-layer caches, filled through kpa_append_factors (slot = position)
+    kcs, vcs, qs = [], [], []
+    start = torch.zeros(w.batch, dtype=torch.int32, device=dev)
+    seq_len = first["seq_len"].to(dev)
+    q_pos = first["q_pos"].to(dev)
+    for layer in range(layers):
+        inp = first if layer == 0 else decode_inputs(w.replace(seed=1000 * rank + layer))
+        kc = torch.empty(w.batch * w.capacity * s.e_k, dtype=tdt, device=dev)
+        vc = torch.empty(w.batch * w.capacity * s.e_v, dtype=tdt, device=dev)
+        kpa.kpa_append_factors(cfg, w.batch, w.capacity, inp["kf"].to(dev), inp["vf"].to(dev),
+                               start, w.capacity, kc, vc)
+        kcs.append(kc)
+        vcs.append(vc)
+        qs.append(inp["q"].to(dev))
+        del inp
+    max_len = int(lens.max())
+    ws_bytes = kpa.kpa_decode_workspace_size(cfg, w.batch, max_len)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    outs = [torch.empty(w.batch, s.h, s.dh, dtype=torch.float32, device=dev) for _ in range(layers)]
+    sm_scale = 1.0 / float(np.sqrt(s.dh))
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(qsrc):
+        for layer in range(layers):
+            kpa.kpa_decode(cfg, w.batch, qsrc[layer], q_pos, kcs[layer], vcs[layer], w.capacity,
+                           seq_len, max_len, sm_scale, outs[layer], ws, stream=stream)
+
+    # warm up eagerly once (also sets kernel attributes), then capture the step
+    with torch.cuda.stream(stream):
+        step(qs)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(qs)
+
+    # e2e graph: pinned host q -> device, decode, device out -> pinned host
+    q_host = [q.cpu().pin_memory() for q in qs]
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    q_dev = [torch.empty_like(q) for q in qs]
+    graph_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_e2e, stream=stream):
+        for layer in range(layers):
+            q_dev[layer].copy_(q_host[layer], non_blocking=True)
+        step(q_dev)
+        for layer in range(layers):
+            out_host[layer].copy_(outs[layer], non_blocking=True)
+
+    sampler = ClockSampler(local)
+
+    def timed(g, steps, warmup):
+        for _ in range(warmup):
+            g.replay()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms / steps
+
+    with torch.cuda.stream(stream):
+        # settle clocks under load (untimed) while the sampler runs
+        sampler.start()
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            for _ in range(20):
+                graph.replay()
+            stream.synchronize()
+        ms_step = timed(graph, a.steps, a.warmup)
+        clocks = sampler.stop()
+        ms_e2e = timed(graph_e2e, a.steps, a.warmup)
+    code = kpa.kpa_read_device_error(stream)
+    if code != 0:
+        raise RuntimeError(f"device error word {code} after the timed region")
+
+    tokens_per_layer = int(lens.sum())
+    value = world * tokens_per_layer * layers / (ms_step * 1e-3)
+    e2e_value = world * tokens_per_layer * layers / (ms_e2e * 1e-3)
+    t_launch = ms_step * 1e-3 / layers            # average decode call (split + combine)
+    achieved = layer_bytes / t_launch / 1e9
+    peak, peak_kind = _hbm_peak()
+    khash = _kernel_hash()
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+            if w.dtype == "bf16" else "f32", "data": "synthetic (seeded, shapes of the pages' workloads)",
+            "config": _config_json(w, layers, lens, world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": _traffic(khash),
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
+                         "kernel": "kpa_decode (split + combine), per layer call",
+                         "algorithmic_bytes_per_launch": layer_bytes,
+                         "launch_us": t_launch * 1e6, "kernel_sources_sha": khash},
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(sum(q.numel() * q.element_size() for q in qs)),
+                    "d2h_bytes_per_step": int(sum(o.numel() * o.element_size() for o in outs)),
+                    "ms_per_step": ms_e2e, "path": "pinned host q -> kpa_decode x layers -> pinned host out, one CUDA graph"},
+            "clocks": clocks,
+            "gpu_launches": a.steps * layers * 2}
+
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        base, _ = _cpu_baseline(w, first, a.cpu_seconds)
+        line["cpu_baseline"] = base
+    del graph, graph_e2e
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    a = _args(argv)
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_kpa(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,289 @@
+// kpa_api.cu -- the extern "C" entry points of libkpa: argument checks, split
+// planning, workspace layout and launches.  Every check that the host can make
+// happens here, before anything is enqueued.
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "kpa_internal.cuh"
+
+namespace kpa {
+
+// Per-device error word (kpa_read_device_error).
+__device__ int g_device_error;
+
+namespace {
+
+thread_local int t_last_cuda = 0;
+
+kpa_status cuda_fail(cudaError_t e) {
+    t_last_cuda = (int)e;
+    return KPA_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int *g_err_ptr[kMaxDevices];
+int g_sms[kMaxDevices];
+
+kpa_status device_state(int **err, int *sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return KPA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_error);
+        if (e != cudaSuccess) return cuda_fail(e);
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_sms[dev] = n;
+        g_err_ptr[dev] = static_cast<int *>(p);
+    }
+    if (err) *err = g_err_ptr[dev];
+    if (sms) *sms = g_sms[dev];
+    return KPA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Shape checks shared by every call.  need_q: the query rank is used.
+kpa_status check_cfg(const kpa_config *c, bool need_q, bool need_model) {
+    if (!c) return KPA_ERR_INVALID_ARG;
+    if (c->h1 <= 0 || c->h2 <= 0 || c->d1 <= 0 || c->d2 <= 0) return KPA_ERR_INVALID_ARG;
+    if (c->r_k <= 0 || c->r_v <= 0 || c->r_q < 0) return KPA_ERR_INVALID_ARG;
+    if (need_q && c->r_q <= 0) return KPA_ERR_INVALID_ARG;
+    if (need_model && c->d_model <= 0) return KPA_ERR_INVALID_ARG;
+    if (c->dtype != KPA_F32 && c->dtype != KPA_BF16) return KPA_ERR_INVALID_ARG;
+    if (!(c->rope_base > 0.0) || !isfinite(c->rope_base)) return KPA_ERR_INVALID_ARG;
+    if (c->d2 % 2 != 0) return KPA_ERR_INVALID_ARG;        // RoPE pairs
+    const int64_t h = (int64_t)c->h1 * c->h2, dh = (int64_t)c->d1 * c->d2;
+    if (h > 4096 || dh > 4096) return KPA_ERR_UNSUPPORTED;
+    if (c->d2 > 2 * kMaxHalfD2) return KPA_ERR_UNSUPPORTED;
+    if (c->r_k > 64 || c->r_v > 64 || c->r_q > 64) return KPA_ERR_UNSUPPORTED;
+    return KPA_OK;
+}
+
+Dims dims_of(const kpa_config *c) {
+    Dims d;
+    d.h1 = c->h1; d.h2 = c->h2; d.d1 = c->d1; d.d2 = c->d2;
+    d.rk = c->r_k; d.rv = c->r_v;
+    d.h = c->h1 * c->h2;
+    d.dh = c->d1 * c->d2;
+    d.ek = c->r_k * (c->h1 * c->d1 + c->h2 * c->d2);
+    d.ev = c->r_v * (c->h1 * c->d1 + c->h2 * c->d2);
+    return d;
+}
+
+RopeTable rope_table(const kpa_config *c) {
+    RopeTable t;
+    for (int m = 0; m < kMaxHalfD2; ++m)
+        t.theta[m] = m < c->d2 / 2 ? pow(c->rope_base, -2.0 * (double)m / (double)c->d2) : 0.0;
+    return t;
+}
+
+size_t dtype_size(kpa_dtype t) { return t == KPA_BF16 ? 2 : 4; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+constexpr size_t kSmemLimit = 200 * 1024;
+
+kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int tps_req, int sms,
+                       DecodePlan *p) {
+    if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
+    int tile = 32;
+    while (tile > 8 && decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) tile /= 2;
+    if (decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) return KPA_ERR_UNSUPPORTED;
+    if ((d.h * d.dh + 255) / 256 > 32) return KPA_ERR_UNSUPPORTED;
+    int tps = tps_req;
+    if (tps == 0) {
+        const int target = 2 * (sms > 0 ? sms : 148);
+        const int per_seq = batch > 0 ? (target + batch - 1) / batch : 1;
+        const int64_t want = ((int64_t)max_len + per_seq - 1) / per_seq;
+        tps = (int)(((want + 63) / 64) * 64);
+        if (tps < 64) tps = 64;
+    }
+    p->tokens_per_split = tps;
+    p->tile = tile;
+    p->n_split = max_len > 0 ? (int)(((int64_t)max_len + tps - 1) / tps) : 1;
+    const size_t o_bytes = (size_t)batch * p->n_split * d.h * d.dh * sizeof(float);
+    const size_t ml_bytes = (size_t)batch * p->n_split * d.h * 2 * sizeof(float);
+    p->part_o_off = 0;
+    p->part_ml_off = align256(o_bytes);
+    p->bytes = p->part_ml_off + align256(ml_bytes);
+    return KPA_OK;
+}
+
+}  // namespace
+}  // namespace kpa
+
+using namespace kpa;
+
+extern "C" {
+
+const char *kpa_status_string(kpa_status s) {
+    switch (s) {
+        case KPA_OK: return "KPA_OK";
+        case KPA_ERR_INVALID_ARG: return "KPA_ERR_INVALID_ARG: invalid argument";
+        case KPA_ERR_UNSUPPORTED: return "KPA_ERR_UNSUPPORTED: shape or dtype not covered";
+        case KPA_ERR_WORKSPACE: return "KPA_ERR_WORKSPACE: workspace missing or too small";
+        case KPA_ERR_CUDA: return "KPA_ERR_CUDA: a CUDA call failed";
+        case KPA_ERR_TIMEOUT: return "KPA_ERR_TIMEOUT: a bounded device wait ran out";
+        case KPA_ERR_DEVICE_CHECK: return "KPA_ERR_DEVICE_CHECK: a device-side index check failed";
+    }
+    return "unknown kpa_status";
+}
+
+int kpa_last_cuda_error(void) { return t_last_cuda; }
+
+kpa_status kpa_cache_bytes_per_token(const kpa_config *cfg, size_t *k_bytes, size_t *v_bytes) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    const Dims d = dims_of(cfg);
+    if (k_bytes) *k_bytes = (size_t)d.ek * dtype_size(cfg->dtype);
+    if (v_bytes) *v_bytes = (size_t)d.ev * dtype_size(cfg->dtype);
+    return KPA_OK;
+}
+
+kpa_status kpa_append_factors(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                              const void *k_factors, const void *v_factors,
+                              const int32_t *start_pos, int32_t capacity, void *kcache,
+                              void *vcache, kpa_stream stream) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
+    if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
+    if (batch == 0 || n_tok == 0) return KPA_OK;
+    if (!k_factors || !v_factors || !start_pos || !kcache || !vcache) return KPA_ERR_INVALID_ARG;
+    if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(k_factors) || !aligned16(v_factors) ||
+        (reinterpret_cast<uintptr_t>(start_pos) & 3))
+        return KPA_ERR_INVALID_ARG;
+    if ((int64_t)n_tok / KPA_TOKEN_GROUP + 2 > INT32_MAX || batch > 65535) return KPA_ERR_UNSUPPORTED;
+    int *err = nullptr;
+    s = device_state(&err, nullptr);
+    if (s != KPA_OK) return s;
+    const Dims d = dims_of(cfg);
+    cudaError_t e = launch_append_factors(d, cfg->dtype, batch, n_tok, k_factors, v_factors,
+                                          start_pos, capacity, kcache, vcache, rope_table(cfg),
+                                          err, (cudaStream_t)stream);
+    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+}
+
+kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32_t max_len,
+                                     int32_t tokens_per_split, size_t *bytes) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (!bytes || batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
+    int sms = 0;
+    s = device_state(nullptr, &sms);
+    if (s != KPA_OK) return s;
+    DecodePlan p;
+    s = plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
+    if (s != KPA_OK) return s;
+    *bytes = batch == 0 ? 0 : p.bytes;
+    return KPA_OK;
+}
+
+kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
+                            const int32_t *q_pos, const void *kcache, const void *vcache,
+                            int32_t capacity, const int32_t *seq_len, int32_t max_len,
+                            float sm_scale, int32_t tokens_per_split, float *out,
+                            void *workspace, size_t ws_bytes, kpa_stream stream) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
+    if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0 || max_len > capacity)
+        return KPA_ERR_INVALID_ARG;
+    if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
+    if (batch == 0) return KPA_OK;
+    if (batch > 65535) return KPA_ERR_UNSUPPORTED;
+    if (!q || !kcache || !vcache || !seq_len || !out) return KPA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(seq_len) & 3) || (reinterpret_cast<uintptr_t>(q_pos) & 3))
+        return KPA_ERR_INVALID_ARG;
+    int *err = nullptr, sms = 0;
+    s = device_state(&err, &sms);
+    if (s != KPA_OK) return s;
+    const Dims d = dims_of(cfg);
+    DecodePlan p;
+    s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
+    if (s != KPA_OK) return s;
+    if (!workspace || ws_bytes < p.bytes) return KPA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return KPA_ERR_INVALID_ARG;
+    if (p.n_split > 65535 * 16) return KPA_ERR_UNSUPPORTED;
+
+    float *part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + p.part_o_off);
+    float *part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) + p.part_ml_off);
+    const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (max_len > 0)
+        e = launch_decode_fma(d, cfg->dtype, batch, q, q_pos, kcache, vcache, capacity, seq_len,
+                              max_len, qscale, p, part_o, part_ml, rope_table(cfg), err, st, sms);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml,
+                              (float)(1.0 / (double)d.rv), out, st);
+    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+}
+
+kpa_status kpa_decode(const kpa_config *cfg, int32_t batch, const void *q, const int32_t *q_pos,
+                      const void *kcache, const void *vcache, int32_t capacity,
+                      const int32_t *seq_len, int32_t max_len, float sm_scale, float *out,
+                      void *workspace, size_t ws_bytes, kpa_stream stream) {
+    return kpa_decode_split(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len,
+                            sm_scale, 0, out, workspace, ws_bytes, stream);
+}
+
+kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                                      size_t *bytes) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (!bytes || batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
+    *bytes = 0;
+    return KPA_ERR_UNSUPPORTED;
+}
+
+kpa_status kpa_prefill(const kpa_config *cfg, int32_t, int32_t, const void *, const int32_t *,
+                       const void *, const void *, int32_t, float, float *, void *, size_t,
+                       kpa_stream) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    return KPA_ERR_UNSUPPORTED;
+}
+
+kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                                     size_t *bytes) {
+    kpa_status s = check_cfg(cfg, true, true);
+    if (s != KPA_OK) return s;
+    if (!bytes || batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
+    *bytes = 0;
+    return KPA_ERR_UNSUPPORTED;
+}
+
+kpa_status kpa_append(const kpa_config *cfg, int32_t, int32_t, const void *, const void *,
+                      const int32_t *, int32_t, void *, void *, void *, void *, size_t,
+                      kpa_stream) {
+    kpa_status s = check_cfg(cfg, true, true);
+    if (s != KPA_OK) return s;
+    return KPA_ERR_UNSUPPORTED;
+}
+
+kpa_status kpa_read_device_error(kpa_stream stream, int32_t *code) {
+    if (!code) return KPA_ERR_INVALID_ARG;
+    int *err = nullptr;
+    kpa_status s = device_state(&err, nullptr);
+    if (s != KPA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    int host = 0;
+    cudaError_t e = cudaMemcpyAsync(&host, err, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(err, 0, sizeof(int), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *code = host;
+    return KPA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,283 @@
+// kpa_decode_fma.cu -- factor-space decode on the CUDA cores (any shape, fp32 or bf16).
+//
+// One CTA = one (sequence, split) and all heads.  The split's slots are walked in
+// shared-memory tiles; per tile (Proposition 2.2 with a dense query, scored
+// directly from the factors):
+//   score(i1,i2) = sum_r sum_j1 A^K_r[i1,j1] * (sum_j2 q[i1,i2,j1,j2] B~^K_r[i2,j2])
+//   online softmax per head in the log2 domain (running max m and sum l),
+//   o(i1,i2)[j1,j2] += p * sum_r A^V_r[i1,j1] B^V_r[i2,j2].
+// 1/R_K and the softmax scale are folded into the rotated query, 1/R_V into the
+// combine.  The CTA leaves an unnormalised partial (o, m, l) per head; the
+// combine pass merges the splits with a log-sum-exp ("online log-sum-exp",
+// FlashTPA decoding in the Tensor Product Attention explainer).
+//
+// This kernel is the general fallback (fp32 caches, shapes outside the
+// tensor-core kernel's cover).
+#include "kpa_internal.cuh"
+
+namespace kpa {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ int elem(int tok, int e, int E) {
+    return ((tok >> 3) * E + e) * kGroup + (tok & 7);
+}
+
+template <typename T>
+__device__ __forceinline__ void copy_tile(T *dst, const T *src, size_t elems) {
+    // elems * sizeof(T) is a multiple of 16 (8-token groups)
+    const size_t n16 = elems * sizeof(T) / 16;
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+    uint4 *o = reinterpret_cast<uint4 *>(dst);
+    for (size_t i = threadIdx.x; i < n16; i += blockDim.x) o[i] = __ldg(s + i);
+}
+
+template <typename T, int OPT>
+__global__ void __launch_bounds__(kThreads)
+decode_fma_kernel(Dims d, const T *__restrict__ q, const int32_t *__restrict__ q_pos,
+                  const T *__restrict__ kc, const T *__restrict__ vc, int cap,
+                  const int32_t *__restrict__ seq_len, int max_len, float qscale, int tps,
+                  int tile, int n_split, float *__restrict__ part_o,
+                  float *__restrict__ part_ml, RopeTable rope, int *err) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int b = blockIdx.y, split = blockIdx.x, tid = threadIdx.x;
+    const int h = d.h, dh = d.dh;
+
+    int L = seq_len[b];
+    if (L > max_len || L < 0) {
+        if (split == 0 && tid == 0) raise_error(err, kErrDeviceCheck);
+        L = L < 0 ? 0 : max_len;
+    }
+    const int t0 = split * tps;
+    if (t0 >= L) return;                          // empty split: the combine skips it
+    const int t1 = min(t0 + tps, L);
+
+    float *qr = reinterpret_cast<float *>(smem);  // [h][dh] rotated, scaled query
+    float *pr = qr + h * dh;                      // [h][tile] scores, then weights
+    float *m_run = pr + h * tile;
+    float *l_run = m_run + h;
+    float *alpha = l_run + h;
+    size_t off = (size_t)(h * dh + h * tile + 3 * h) * sizeof(float);
+    off = (off + 15) & ~(size_t)15;
+    T *kt = reinterpret_cast<T *>(smem + off);    // [tile/8][ek][8]
+    T *vt = kt + (size_t)tile * d.ek;             // [tile/8][ev][8]
+
+    // rotate the query: I_{d1} (x) R^(2)(q_pos), pairs (2m, 2m+1) of each d2 chunk
+    const T *qb = q + (size_t)b * h * dh;
+    const bool rotate = q_pos != nullptr;
+    const double qp = rotate ? (double)q_pos[b] : 0.0;
+    for (int i = tid; i < h * dh / 2; i += kThreads) {
+        const float x0 = to_f32(qb[2 * i]), x1 = to_f32(qb[2 * i + 1]);
+        float y0 = x0, y1 = x1;
+        if (rotate) {
+            const int m = ((2 * i) % d.d2) >> 1;
+            float c, s;
+            rope_cs(qp, rope.theta[m], c, s);
+            y0 = x0 * c - x1 * s;
+            y1 = x0 * s + x1 * c;
+        }
+        qr[2 * i] = y0 * qscale;
+        qr[2 * i + 1] = y1 * qscale;
+    }
+    for (int i = tid; i < h; i += kThreads) {
+        m_run[i] = -INFINITY;
+        l_run[i] = 0.f;
+    }
+    float o[OPT];
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) o[k] = 0.f;
+
+    const T *kb = kc + (size_t)b * cap * d.ek;
+    const T *vb = vc + (size_t)b * cap * d.ev;
+    const int a_k = d.rk * d.h1 * d.d1, a_v = d.rv * d.h1 * d.d1;
+
+    for (int s0 = t0; s0 < t1; s0 += tile) {
+        const int n = min(tile, t1 - s0);
+        const int groups = (n + kGroup - 1) / kGroup;
+        __syncthreads();                          // previous tile fully consumed
+        copy_tile(kt, kb + (size_t)s0 * d.ek, (size_t)groups * d.ek * kGroup);
+        copy_tile(vt, vb + (size_t)s0 * d.ev, (size_t)groups * d.ev * kGroup);
+        __syncthreads();
+
+        // scores, log2 domain (qscale carries sm_scale / R_K * log2 e)
+        for (int idx = tid; idx < h * tile; idx += kThreads) {
+            const int head = idx / tile, tok = idx % tile;
+            float sc = -INFINITY;
+            if (tok < n) {
+                const int i1 = head / d.h2, i2 = head % d.h2;
+                float acc = 0.f;
+                for (int r = 0; r < d.rk; ++r) {
+                    const int a_base = r * d.h1 * d.d1 + i1 * d.d1;
+                    const int b_base = a_k + r * d.h2 * d.d2 + i2 * d.d2;
+                    for (int j1 = 0; j1 < d.d1; ++j1) {
+                        const float *qrow = qr + head * dh + j1 * d.d2;
+                        float inner = 0.f;
+                        for (int j2 = 0; j2 < d.d2; ++j2)
+                            inner += qrow[j2] * to_f32(kt[elem(tok, b_base + j2, d.ek)]);
+                        acc += to_f32(kt[elem(tok, a_base + j1, d.ek)]) * inner;
+                    }
+                }
+                sc = acc;
+            }
+            pr[head * tile + tok] = sc;
+        }
+        __syncthreads();
+
+        // online softmax, one thread per head
+        for (int head = tid; head < h; head += kThreads) {
+            float *row = pr + head * tile;
+            const float m_old = m_run[head];
+            float mx = m_old;
+            for (int tok = 0; tok < n; ++tok) mx = fmaxf(mx, row[tok]);
+            const float al = (m_old == -INFINITY) ? 0.f : exp2f(m_old - mx);
+            float sum = 0.f;
+            for (int tok = 0; tok < n; ++tok) {
+                const float p = exp2f(row[tok] - mx);
+                row[tok] = p;
+                sum += p;
+            }
+            l_run[head] = l_run[head] * al + sum;
+            m_run[head] = mx;
+            alpha[head] = al;
+        }
+        __syncthreads();
+
+        // values: o += p * sum_r A^V_r[i1,j1] B^V_r[i2,j2]
+#pragma unroll
+        for (int k = 0; k < OPT; ++k) {
+            const int idx = tid + k * kThreads;
+            if (idx < h * dh) {
+                const int head = idx / dh, f = idx % dh;
+                const int i1 = head / d.h2, i2 = head % d.h2;
+                const int j1 = f / d.d2, j2 = f % d.d2;
+                const float *prow = pr + head * tile;
+                float acc = 0.f;
+                for (int tok = 0; tok < n; ++tok) {
+                    float v = 0.f;
+                    for (int r = 0; r < d.rv; ++r)
+                        v += to_f32(vt[elem(tok, r * d.h1 * d.d1 + i1 * d.d1 + j1, d.ev)]) *
+                             to_f32(vt[elem(tok, a_v + r * d.h2 * d.d2 + i2 * d.d2 + j2, d.ev)]);
+                    acc += prow[tok] * v;
+                }
+                o[k] = o[k] * alpha[head] + acc;
+            }
+        }
+    }
+
+    float *po = part_o + ((size_t)(b * n_split + split) * h) * dh;
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+        const int idx = tid + k * kThreads;
+        if (idx < h * dh) po[idx] = o[k];
+    }
+    __syncthreads();
+    float *pml = part_ml + ((size_t)(b * n_split + split) * h) * 2;
+    for (int head = tid; head < h; head += kThreads) {
+        pml[2 * head] = m_run[head];
+        pml[2 * head + 1] = l_run[head];
+    }
+}
+
+template <typename T, int OPT>
+cudaError_t launch_t(const Dims &d, int batch, const void *q, const int32_t *q_pos,
+                     const void *kc, const void *vc, int cap, const int32_t *seq_len,
+                     int max_len, float qscale, const DecodePlan &p, float *part_o,
+                     float *part_ml, const RopeTable &rope, int *err, cudaStream_t st,
+                     size_t smem) {
+    auto kern = decode_fma_kernel<T, OPT>;
+    cudaError_t e = ensure_dynamic_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)p.n_split, (unsigned)batch);
+    kern<<<grid, kThreads, smem, st>>>(d, (const T *)q, q_pos, (const T *)kc, (const T *)vc, cap,
+                                       seq_len, max_len, qscale, p.tokens_per_split, p.tile,
+                                       p.n_split, part_o, part_ml, rope, err);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch_opt(const Dims &d, int batch, const void *q, const int32_t *q_pos,
+                         const void *kc, const void *vc, int cap, const int32_t *seq_len,
+                         int max_len, float qscale, const DecodePlan &p, float *part_o,
+                         float *part_ml, const RopeTable &rope, int *err, cudaStream_t st,
+                         size_t smem) {
+    const int need = (d.h * d.dh + kThreads - 1) / kThreads;
+#define KPA_OPT_CASE(N)                                                                      \
+    if (need <= N)                                                                           \
+        return launch_t<T, N>(d, batch, q, q_pos, kc, vc, cap, seq_len, max_len, qscale, p, \
+                              part_o, part_ml, rope, err, st, smem);
+    KPA_OPT_CASE(1)
+    KPA_OPT_CASE(2)
+    KPA_OPT_CASE(4)
+    KPA_OPT_CASE(8)
+    KPA_OPT_CASE(16)
+    KPA_OPT_CASE(32)
+#undef KPA_OPT_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t decode_fma_smem_bytes(const Dims &d, kpa_dtype dt, int tile) {
+    size_t off = (size_t)(d.h * d.dh + d.h * tile + 3 * d.h) * sizeof(float);
+    off = (off + 15) & ~(size_t)15;
+    const size_t es = dt == KPA_BF16 ? 2 : 4;
+    return off + (size_t)tile * (d.ek + d.ev) * es;
+}
+
+cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void *q,
+                              const int32_t *q_pos, const void *kc, const void *vc, int cap,
+                              const int32_t *seq_len, int max_len, float qscale,
+                              const DecodePlan &plan, float *part_o, float *part_ml,
+                              const RopeTable &rope, int *err, cudaStream_t st, int /*sms*/) {
+    const size_t smem = decode_fma_smem_bytes(d, dt, plan.tile);
+    if (dt == KPA_BF16)
+        return dispatch_opt<__nv_bfloat16>(d, batch, q, q_pos, kc, vc, cap, seq_len, max_len,
+                                           qscale, plan, part_o, part_ml, rope, err, st, smem);
+    return dispatch_opt<float>(d, batch, q, q_pos, kc, vc, cap, seq_len, max_len, qscale, plan,
+                               part_o, part_ml, rope, err, st, smem);
+}
+
+// ---------------------------------------------------------------------------
+// Split combine: out = (1/R_V) * sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+__global__ void __launch_bounds__(128)
+decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, int tps,
+                      int n_split, const float *__restrict__ part_o,
+                      const float *__restrict__ part_ml, float out_scale,
+                      float *__restrict__ out) {
+    const int b = blockIdx.y;
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= d.h * d.dh) return;
+    const int head = idx / d.dh;
+    int L = seq_len[b];
+    L = L < 0 ? 0 : (L > max_len ? max_len : L);
+    const int ns = (L + tps - 1) / tps;
+    float *dst = out + (size_t)b * d.h * d.dh + idx;
+    if (ns == 0) {
+        *dst = 0.f;
+        return;
+    }
+    const float *ml = part_ml + ((size_t)b * n_split * d.h + head) * 2;
+    float M = -INFINITY;
+    for (int i = 0; i < ns; ++i) M = fmaxf(M, ml[(size_t)i * d.h * 2]);
+    float num = 0.f, den = 0.f;
+    const float *po = part_o + (size_t)b * n_split * d.h * d.dh + idx;
+    for (int i = 0; i < ns; ++i) {
+        const float w = exp2f(ml[(size_t)i * d.h * 2] - M);
+        num += w * po[(size_t)i * d.h * d.dh];
+        den += w * ml[(size_t)i * d.h * 2 + 1];
+    }
+    *dst = den > 0.f ? out_scale * num / den : 0.f;
+}
+
+cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_len,
+                                  int max_len, const DecodePlan &plan, const float *part_o,
+                                  const float *part_ml, float out_scale, float *out,
+                                  cudaStream_t st) {
+    dim3 grid((unsigned)((d.h * d.dh + 127) / 128), (unsigned)batch);
+    decode_combine_kernel<<<grid, 128, 0, st>>>(d, seq_len, max_len, plan.tokens_per_split,
+                                                plan.n_split, part_o, part_ml, out_scale, out);
+    return cudaGetLastError();
+}
+
+}  // namespace kpa

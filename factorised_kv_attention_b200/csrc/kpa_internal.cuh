@@ -1,0 +1,106 @@
+// kpa_internal.cuh -- types and helpers shared by libkpa's kernels and host code.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/kpa.h"
+
+namespace kpa {
+
+// Device-side error codes share the numbering of kpa_status.
+constexpr int kErrTimeout = KPA_ERR_TIMEOUT;
+constexpr int kErrDeviceCheck = KPA_ERR_DEVICE_CHECK;
+
+constexpr int kGroup = KPA_TOKEN_GROUP;   // tokens per interleaved cache group
+constexpr int kMaxHalfD2 = 128;           // RoPE table length (d2 <= 256)
+
+// Shape of one attention layer, with the derived sizes the kernels index by.
+struct Dims {
+    int h1, h2, d1, d2;
+    int rk, rv;
+    int h, dh;      // h1*h2, d1*d2
+    int ek, ev;     // elements per key / value record
+};
+
+// theta_m = base^(-2m/d2), m < d2/2, formed on the host in float64 and passed by
+// value (Definition 2.3; the pairing and sign are documented in kpa.h).
+struct RopeTable {
+    double theta[kMaxHalfD2];
+};
+
+// Records the first device-side error; later ones are dropped.
+__device__ __forceinline__ void raise_error(int *err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// Element offset of (slot s, element e) inside one sequence's plane of the
+// interleaved cache: group s/8 holds its records element-major, token-minor.
+__host__ __device__ __forceinline__ int64_t cache_offset(int64_t s, int e, int E) {
+    return ((s / kGroup) * E + e) * kGroup + (s % kGroup);
+}
+
+// cos/sin of pos * theta in float64, rounded to float.
+__device__ __forceinline__ void rope_cs(double pos, double theta, float &c, float &s) {
+    double sn, cs;
+    sincos(pos * theta, &sn, &cs);
+    c = (float)cs;
+    s = (float)sn;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (so later calls,
+// including ones made while a stream is being captured, launch directly).
+template <typename Kernel>
+inline cudaError_t ensure_dynamic_smem(Kernel kern, size_t bytes) {
+    static std::atomic<int> granted[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (bytes <= 48 * 1024 || (size_t)granted[dev].load() >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) granted[dev].store((int)bytes);
+    return e;
+}
+
+// ---- host-side launchers (one per kernel file) ------------------------------
+cudaError_t launch_append_factors(const Dims &d, kpa_dtype dt, int batch, int n_tok,
+                                  const void *kf, const void *vf, const int32_t *start_pos,
+                                  int cap, void *kc, void *vc, const RopeTable &rope, int *err,
+                                  cudaStream_t st);
+
+struct DecodePlan {
+    int tokens_per_split;
+    int n_split;         // splits per sequence (grid x)
+    int tile;            // tokens per shared-memory tile
+    size_t part_o_off, part_ml_off, bytes;
+};
+
+cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void *q,
+                              const int32_t *q_pos, const void *kc, const void *vc, int cap,
+                              const int32_t *seq_len, int max_len, float qscale,
+                              const DecodePlan &plan, float *part_o, float *part_ml,
+                              const RopeTable &rope, int *err, cudaStream_t st, int sms);
+
+cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_len,
+                                  int max_len, const DecodePlan &plan, const float *part_o,
+                                  const float *part_ml, float out_scale, float *out,
+                                  cudaStream_t st);
+
+size_t decode_fma_smem_bytes(const Dims &d, kpa_dtype dt, int tile);
+
+}  // namespace kpa

@@ -1,0 +1,190 @@
+/*
+ * kpa.h -- C ABI of libkpa: factor-space Kronecker Product Attention (KPA)
+ * and its degenerate split, Tensor Product Attention (TPA), on NVIDIA B200
+ * (sm_100a).
+ *
+ * Each cached key and value of token t is stored only as factors,
+ *     K_t = (1/R_K) sum_r A^K_r(t) (x) B^K_r(t),   A_r in R^{h1 x d1},
+ *     V_t = (1/R_V) sum_r A^V_r(t) (x) B^V_r(t),   B_r in R^{h2 x d2},
+ * with h = h1*h2 heads and d_h = d1*d2 features per head ("Kronecker Product
+ * Attention", section 2.2, eqs 2-4).  Setting h1 = h, d1 = 1, h2 = 1, d2 = d_h
+ * gives TPA (same section, final paragraph).  RoPE is the Kronecker-separable
+ * operator I_{d1} (x) R_theta^(2)(t) (Definition 2.3); by Theorem 2.4 it rotates
+ * only the B factors, so the cache holds B^K already rotated and A^K, A^V, B^V
+ * as projected (section 2.5).  Attention reads the factors directly: the cache
+ * is never expanded to full K/V in device memory.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Notation.  Head (i1, i2) is flat head i1*h2 + i2 and feature (j1, j2) is
+ *    flat feature j1*d2 + j2 (the block order of Definition 2.1).
+ *  - Factor record.  One token's key record holds E_K = R_K*(h1*d1 + h2*d2)
+ *    elements in the order [A_0 .. A_{R_K-1} | B_0 .. B_{R_K-1}], each A_r
+ *    row-major h1 x d1, each B_r row-major h2 x d2; the value record likewise
+ *    with R_V (E_V elements).
+ *  - RoPE.  Pairs (2m, 2m+1) of each length-d2 row of B, angle
+ *    phi = pos * rope_base^(-2m/d2), (x0, x1) -> (x0 cos phi - x1 sin phi,
+ *    x0 sin phi + x1 cos phi).  The angle is formed in float64.
+ *  - Cache layout (the planes `kcache`, `vcache`).  Slot s of sequence b holds
+ *    the token at position s.  Slots are grouped by KPA_TOKEN_GROUP (8): group
+ *    g = s / 8 stores its 8 records element-major, token-minor, so element e of
+ *    slot s lives at element offset
+ *        ((b * (capacity / 8) + s / 8) * E + e) * 8 + s % 8
+ *    (E = E_K or E_V).  `capacity` must be a positive multiple of 8.  A plane
+ *    is batch * capacity * E elements of the config dtype.
+ *  - Memory.  Every pointer is device memory unless stated otherwise, owned by
+ *    the caller, and 16-byte aligned.  The library never allocates or frees
+ *    device memory and never synchronises, except kpa_read_device_error.
+ *  - Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream);
+ *    all work is enqueued on it and the call returns without waiting.
+ *  - Errors.  Bad arguments return KPA_ERR_INVALID_ARG before anything is
+ *    enqueued; shapes the kernels do not cover return KPA_ERR_UNSUPPORTED; a
+ *    failed launch returns KPA_ERR_CUDA (kpa_last_cuda_error gives the CUDA
+ *    code).  Problems only the device can see (a slot outside the cache, a
+ *    length above max_len, a bounded wait that ran out) set a per-device error
+ *    word that kpa_read_device_error returns; the offending work is skipped,
+ *    never performed out of bounds.
+ */
+#ifndef KPA_H
+#define KPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KPA_TOKEN_GROUP 8
+
+typedef struct CUstream_st *kpa_stream; /* the same type as cudaStream_t */
+
+typedef enum {
+    KPA_OK = 0,
+    KPA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent size   */
+    KPA_ERR_UNSUPPORTED = 2,  /* valid request that no kernel here covers      */
+    KPA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required    */
+    KPA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed          */
+    KPA_ERR_TIMEOUT = 5,      /* device: a bounded wait ran out                */
+    KPA_ERR_DEVICE_CHECK = 6  /* device: an index or length failed its check   */
+} kpa_status;
+
+typedef enum { KPA_F32 = 0, KPA_BF16 = 1 } kpa_dtype;
+
+typedef struct {
+    int32_t h1, h2;     /* heads h = h1*h2                                      */
+    int32_t d1, d2;     /* features per head d_h = d1*d2; d2 even (RoPE pairs)  */
+    int32_t r_q;        /* query rank (kpa_append only; 0 elsewhere)            */
+    int32_t r_k, r_v;   /* key and value ranks                                  */
+    int32_t d_model;    /* hidden size (kpa_append only; 0 elsewhere)           */
+    double rope_base;   /* RoPE base, e.g. 10000                                */
+    kpa_dtype dtype;    /* element type of caches, factors, queries, x and W    */
+} kpa_config;
+
+/* Human-readable name of a status code (static storage). */
+const char *kpa_status_string(kpa_status status);
+
+/* CUDA error code (cudaError_t as int) behind the calling thread's most recent
+ * KPA_ERR_CUDA, or 0. */
+int kpa_last_cuda_error(void);
+
+/* Bytes one token adds to the key plane and to the value plane:
+ * E_K * sizeof(dtype) and E_V * sizeof(dtype), i.e. eq 10's
+ * (R_K + R_V)(h1 d1 + h2 d2) numbers split by plane ("Kronecker Product
+ * Attention", section 2.5; Appendix B, eq 11).  Either output may be NULL.
+ * Host only; enqueues nothing. */
+kpa_status kpa_cache_bytes_per_token(const kpa_config *cfg, size_t *k_bytes, size_t *v_bytes);
+
+/* Write given factor records into the cache (section 2.5; Theorem 2.4).
+ *   k_factors [batch][n_tok][E_K]  unrotated key records, config dtype
+ *   v_factors [batch][n_tok][E_V]  value records, config dtype
+ *   start_pos [batch] int32        token t of sequence b goes to slot
+ *                                  start_pos[b] + t, at that position
+ * B^K is rotated at its position; A^K, A^V, B^V are stored unchanged.  A token
+ * whose slot falls outside [0, capacity) is not written and sets
+ * KPA_ERR_DEVICE_CHECK.  n_tok == 0 or batch == 0 enqueues nothing. */
+kpa_status kpa_append_factors(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                              const void *k_factors, const void *v_factors,
+                              const int32_t *start_pos, int32_t capacity,
+                              void *kcache, void *vcache, kpa_stream stream);
+
+/* Workspace kpa_decode needs for `batch` sequences of at most `max_len` slots.
+ * tokens_per_split = 0 lets the library choose the split of each sequence;
+ * otherwise it must be a positive multiple of 64.  Host only. */
+kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32_t max_len,
+                                     int32_t tokens_per_split, size_t *bytes);
+
+/* Factor-space decode attention: one query row per sequence against slots
+ * 0 .. seq_len[b]-1 of the cache (Proposition 2.2 evaluated with a dense
+ * query, Theorem 2.4 for the positions; FlashTPA-style blocking over the cache
+ * with an online log-sum-exp, split across CTAs and merged by a combine pass).
+ *   q        [batch][h][d_h]  config dtype; rotated here by
+ *                             I_{d1} (x) R^(2)(q_pos[b]) when q_pos != NULL,
+ *                             used as given when q_pos == NULL
+ *   seq_len  [batch] int32    0 <= seq_len[b] <= max_len <= capacity; a longer
+ *                             length is clamped to max_len and sets
+ *                             KPA_ERR_DEVICE_CHECK
+ *   sm_scale softmax scale applied to q.k (usually 1/sqrt(d_h))
+ *   out      [batch][h][d_h] float32; a sequence with seq_len 0 gets zeros
+ *   workspace at least kpa_decode_workspace_size(cfg, batch, max_len, 0) bytes;
+ *            its contents need no initialisation and are scratch between calls
+ * Results are deterministic for a given (batch, max_len). */
+kpa_status kpa_decode(const kpa_config *cfg, int32_t batch, const void *q, const int32_t *q_pos,
+                      const void *kcache, const void *vcache, int32_t capacity,
+                      const int32_t *seq_len, int32_t max_len, float sm_scale, float *out,
+                      void *workspace, size_t ws_bytes, kpa_stream stream);
+
+/* kpa_decode with an explicit split of each sequence into pieces of
+ * tokens_per_split slots (a positive multiple of 64, or 0 for the library's
+ * choice).  The workspace must be sized with the same tokens_per_split. */
+kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
+                            const int32_t *q_pos, const void *kcache, const void *vcache,
+                            int32_t capacity, const int32_t *seq_len, int32_t max_len,
+                            float sm_scale, int32_t tokens_per_split, float *out,
+                            void *workspace, size_t ws_bytes, kpa_stream stream);
+
+/* Causal chunked attention in factor space (prefill).  Row t of sequence b is
+ * the query at position start_pos[b] + t and sees slots 0 .. start_pos[b] + t
+ * (its own key included), which must already be in the cache (kpa_append or
+ * kpa_append_factors).  K/V tiles are rebuilt from the factors on chip only.
+ *   q    [batch][n_tok][h][d_h]  config dtype, already rotated
+ *   out  [batch][n_tok][h][d_h]  float32
+ *   start_pos [batch] int32; a row whose last slot is outside the cache is
+ *   skipped (zeros) and sets KPA_ERR_DEVICE_CHECK.
+ *   workspace at least kpa_prefill_workspace_size bytes (may be 0). */
+kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                                      size_t *bytes);
+kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *q,
+                       const int32_t *start_pos, const void *kcache, const void *vcache,
+                       int32_t capacity, float sm_scale, float *out, void *workspace,
+                       size_t ws_bytes, kpa_stream stream);
+
+/* Append: merged factor projection, factor RoPE and cache write ("Kronecker
+ * Product Attention", eq 5 with the ranks merged; Theorem 2.4; section 2.5).
+ *   x  [batch][n_tok][d_model]  bf16 hidden states
+ *   w  [N][d_model]             bf16 merged weights, N = (R_Q+R_K+R_V)(h1 d1 + h2 d2),
+ *                               rows ordered [A^Q | B^Q | A^K | B^K | A^V | B^V],
+ *                               each part rank-major (r, then row, then column)
+ *   start_pos [batch] int32     token t of sequence b is at position and slot
+ *                               start_pos[b] + t
+ *   q_out [batch][n_tok][h][d_h] bf16 or NULL: the assembled query
+ *                               (1/R_Q) sum_r A^Q_r (x) B^Q_r rotated at its position
+ *   workspace at least kpa_append_workspace_size bytes.
+ * Requires dtype == KPA_BF16 and d_model a multiple of 64. */
+kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                                     size_t *bytes);
+kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *x,
+                      const void *w, const int32_t *start_pos, int32_t capacity,
+                      void *kcache, void *vcache, void *q_out, void *workspace,
+                      size_t ws_bytes, kpa_stream stream);
+
+/* Wait for `stream`, then return in *code the per-device error word
+ * (KPA_OK, KPA_ERR_TIMEOUT or KPA_ERR_DEVICE_CHECK) of the current device and
+ * clear it.  The only call that synchronises. */
+kpa_status kpa_read_device_error(kpa_stream stream, int32_t *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KPA_H */

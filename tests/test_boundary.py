@@ -1,0 +1,132 @@
+"""The C ABI: the library loads, exports every call that include/kpa.h declares,
+and rejects bad arguments before it touches a device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import factorised_kv_attention_b200 as kpa
+import oracle
+from workloads import APPEND_PREFILL, DECODE_CONFIGS, Shape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(kpa_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared_functions()
+    assert len(declared) >= 12
+    lib = ctypes.CDLL(kpa.LIB_PATH)
+    missing = [n for n in declared if not hasattr(lib, n)]
+    assert not missing, f"declared in include/ but not exported: {missing}"
+
+
+def test_status_strings():
+    for code in range(7):
+        s = kpa.kpa_status_string(code)
+        assert s.startswith("KPA_"), s
+    assert "unknown" in kpa.kpa_status_string(42)
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_CONFIGS))
+def test_cache_bytes_match_eq10(name):
+    w = DECODE_CONFIGS[name]
+    s = w.shape
+    cfg = kpa.make_config(s, w.dtype)
+    kb, vb = kpa.kpa_cache_bytes_per_token(cfg)
+    elt = 2 if w.dtype == "bf16" else 4
+    numbers = oracle.cache_numbers_per_token(s.h1, s.h2, s.d1, s.d2, s.r_k, s.r_v)
+    assert kb + vb == numbers * elt
+    assert kb * s.r_v == vb * s.r_k
+
+
+def test_cache_bytes_of_the_configs():
+    # per-token bytes of the five configurations, from eq (10)
+    want = {"tiny_kpa": 768, "tpa_decode": 640, "kpa_medium": 2560, "kpa_long": 1280}
+    for name, b in want.items():
+        w = DECODE_CONFIGS[name]
+        kb, vb = kpa.kpa_cache_bytes_per_token(kpa.make_config(w.shape, w.dtype))
+        assert kb + vb == b, name
+    kb, vb = kpa.kpa_cache_bytes_per_token(kpa.make_config(APPEND_PREFILL.shape, "bf16"))
+    assert kb + vb == 768
+
+
+BAD_SHAPES = [dict(h1=0), dict(d2=7), dict(r_k=0), dict(r_v=-1), dict(d1=-2)]
+
+
+@pytest.mark.parametrize("bad", BAD_SHAPES, ids=str)
+def test_bad_config_rejected(bad):
+    base = dict(h1=4, h2=8, d1=8, d2=16, r_k=2, r_v=2)
+    base.update(bad)
+    cfg = kpa.make_config(Shape(**base), "bf16")
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_cache_bytes_per_token(cfg)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def test_bad_dtype_and_base_rejected():
+    cfg = kpa.make_config(DECODE_CONFIGS["kpa_long"].shape, "bf16")
+    cfg.dtype = 7
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_cache_bytes_per_token(cfg)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+    cfg = kpa.make_config(DECODE_CONFIGS["kpa_long"].shape, "bf16")
+    cfg.rope_base = 0.0
+    with pytest.raises(kpa.KpaError):
+        kpa.kpa_cache_bytes_per_token(cfg)
+
+
+# Argument checks that run before any CUDA call: fake, aligned "device" addresses
+# are never dereferenced because every case below is rejected first.
+A = 1 << 20          # 16-byte aligned dummy address
+CFG = kpa.make_config(DECODE_CONFIGS["kpa_long"].shape, "bf16")
+
+
+def _decode(**over):
+    args = dict(cfg=CFG, batch=2, q=A, q_pos=None, kcache=A, vcache=A, capacity=64, seq_len=A,
+                max_len=64, sm_scale=0.1, out=A, workspace=A, ws_bytes=1 << 20)
+    args.update(over)
+    kpa.kpa_decode(args["cfg"], args["batch"], args["q"], args["q_pos"], args["kcache"],
+                   args["vcache"], args["capacity"], args["seq_len"], args["max_len"],
+                   args["sm_scale"], args["out"], args["workspace"], args["ws_bytes"], stream=0)
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(kcache=None), dict(vcache=None), dict(seq_len=None), dict(out=None),
+    dict(q=A + 2), dict(kcache=A + 8), dict(out=A + 4), dict(seq_len=A + 1),
+    dict(capacity=60), dict(capacity=0), dict(max_len=65), dict(max_len=-1), dict(batch=-1),
+    dict(sm_scale=float("nan")), dict(sm_scale=float("inf")),
+], ids=str)
+def test_decode_rejects_before_launch(over):
+    with pytest.raises(kpa.KpaError) as e:
+        _decode(**over)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def test_decode_empty_batch_is_a_no_op():
+    _decode(batch=0, q=None, kcache=None, vcache=None, seq_len=None, out=None, workspace=None)
+
+
+@pytest.mark.parametrize("over", [
+    dict(k_factors=None), dict(start_pos=None), dict(kcache=A + 2), dict(capacity=12),
+    dict(n_tok=-1),
+], ids=str)
+def test_append_factors_rejects_before_launch(over):
+    args = dict(batch=1, n_tok=4, k_factors=A, v_factors=A, start_pos=A, capacity=64, kcache=A,
+                vcache=A)
+    args.update(over)
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_append_factors(CFG, args["batch"], args["n_tok"], args["k_factors"],
+                               args["v_factors"], args["start_pos"], args["capacity"],
+                               args["kcache"], args["vcache"], stream=0)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
