@@ -1,6 +1,8 @@
 """Build libkpa.so in-tree with nvcc for sm_100a.
 
-    python -m factorised_kv_attention_b200.build [--force] [--verbose]
+    python factorised_kv_attention_b200/build.py [--force] [--verbose]
+
+(run it as a file: importing the package loads the library it builds)
 
 Each ``csrc/*.cu`` compiles to ``_build/*.o`` (in parallel), then one shared
 library is linked next to this file.  ``-Xptxas -v`` output (registers, spills,
