@@ -4,8 +4,8 @@ The functions here carry the C names of ``include/kpa.h`` and only marshal
 arguments: tensors become device pointers, ``stream=None`` becomes torch's
 current CUDA stream, and a non-OK status raises :class:`KpaError`.  Every step
 of the computation runs in the CUDA library; there is no CPU path.  Importing
-fails loudly when ``libkpa.so`` has not been built (``python -m
-factorised_kv_attention_b200.build``).
+fails loudly when ``libkpa.so`` has not been built (``python
+factorised_kv_attention_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, "libkpa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m factorised_kv_attention_b200.build`")
+                      "`python factorised_kv_attention_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -69,6 +69,8 @@ _SIGS = {
     "kpa_append": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp],
                    ctypes.c_int),
     "kpa_read_device_error": ([_vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "kpa_decode_noalloc": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp],
+                           ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -183,6 +185,18 @@ def kpa_append(cfg, batch, n_tok, x, w, start_pos, capacity, kcache, vcache, q_o
     _check(_lib.kpa_append(ctypes.byref(cfg), batch, n_tok, _addr(x), _addr(w), _addr(start_pos),
                            capacity, _addr(kcache), _addr(vcache), _addr(q_out), _addr(workspace),
                            ws_bytes, _stream(stream)), "kpa_append")
+
+
+KPA_DECODE_NOALLOC_MAX_BYTES = 16 << 20
+
+
+def kpa_decode_noalloc(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len, sm_scale,
+                       out, stream=None):
+    """kpa_decode without a workspace argument, for callers that cannot allocate:
+    the library's fixed device scratch array stands in for it (see kpa.h)."""
+    _check(_lib.kpa_decode_noalloc(ctypes.byref(cfg), batch, _addr(q), _addr(q_pos), _addr(kcache),
+                                   _addr(vcache), capacity, _addr(seq_len), max_len, sm_scale,
+                                   _addr(out), _stream(stream)), "kpa_decode_noalloc")
 
 
 def kpa_read_device_error(stream=None) -> int:

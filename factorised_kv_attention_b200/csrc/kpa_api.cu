@@ -118,6 +118,9 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
 }
 
 }  // namespace
+
+void record_cuda_error(cudaError_t e) { t_last_cuda = (int)e; }
+
 }  // namespace kpa
 
 using namespace kpa;

@@ -77,6 +77,9 @@ inline cudaError_t ensure_dynamic_smem(Kernel kern, size_t bytes) {
     return e;
 }
 
+// Remember a CUDA error for kpa_last_cuda_error (calling thread).
+void record_cuda_error(cudaError_t e);
+
 // ---- host-side launchers (one per kernel file) ------------------------------
 cudaError_t launch_append_factors(const Dims &d, kpa_dtype dt, int batch, int n_tok,
                                   const void *kf, const void *vf, const int32_t *start_pos,

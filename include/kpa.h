@@ -178,6 +178,29 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const
                       void *kcache, void *vcache, void *q_out, void *workspace,
                       size_t ws_bytes, kpa_stream stream);
 
+/* Upper bound, in bytes, of the scratch that kpa_decode_noalloc can use. */
+#define KPA_DECODE_NOALLOC_MAX_BYTES (16u << 20)
+
+/* kpa_decode for callers that cannot allocate device memory (code running
+ * while a stream is captured in a mode that forbids allocation, plugins whose
+ * host framework owns all device memory, serving loops that must not allocate
+ * on the decode path).  The pages have no counterpart: this is a deployment
+ * convenience, not part of the method.
+ * Same arguments and results as kpa_decode with the library's choice of split,
+ * minus the workspace: the scratch lives in a fixed array of
+ * KPA_DECODE_NOALLOC_MAX_BYTES in the library's own device memory, which every
+ * GPU that loads the library holds until the process exits.  A request whose
+ * kpa_decode_workspace_size exceeds that bound returns KPA_ERR_WORKSPACE and
+ * enqueues nothing.  The call allocates and frees nothing.  The first call on
+ * each device looks up the array's device address (with that device current),
+ * so make that first call before capturing a stream.  All calls on a device
+ * share the array; calls whose work overlaps on the GPU race on it and must be
+ * serialised by the caller. */
+kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, const void *q,
+                              const int32_t *q_pos, const void *kcache, const void *vcache,
+                              int32_t capacity, const int32_t *seq_len, int32_t max_len,
+                              float sm_scale, float *out, kpa_stream stream);
+
 /* Wait for `stream`, then return in *code the per-device error word
  * (KPA_OK, KPA_ERR_TIMEOUT or KPA_ERR_DEVICE_CHECK) of the current device and
  * clear it.  The only call that synchronises. */
