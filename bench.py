@@ -37,7 +37,9 @@ sys.path.insert(0, ROOT)
 METRIC = "decode cached-tokens/s per layer; achieved HBM GB/s vs B200 peak (1 GPU)"
 PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
-KERNEL_SOURCES = ["factorised_kv_attention_b200/csrc/kpa_decode_fma.cu",
+KERNEL_SOURCES = ["factorised_kv_attention_b200/csrc/kpa_decode_mma.cu",
+                  "factorised_kv_attention_b200/csrc/kpa_mma_decode.cuh",
+                  "factorised_kv_attention_b200/csrc/kpa_decode_fma.cu",
                   "factorised_kv_attention_b200/csrc/kpa_internal.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 
@@ -52,6 +54,10 @@ def _args(argv=None):
     ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0, help="override: fixed length (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override: batch (profiling)")
+    ap.add_argument("--settle-seconds", type=float, default=1.0,
+                    help="untimed load before timing while clocks are sampled (0 for profiling)")
     a = ap.parse_args(argv)
     a.warmup = max(a.warmup, 3)
     return a
@@ -148,9 +154,16 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def _workload(name):
+def _workload(name, a=None):
     from workloads import DECODE_CONFIGS
-    return DECODE_CONFIGS[name]
+    w = DECODE_CONFIGS[name]
+    if a is not None and a.seq_len:
+        cap = (a.seq_len + 7) // 8 * 8
+        w = w.replace(length=a.seq_len, ragged=(), capacity=cap,
+                      name=w.name + f" [length overridden to {a.seq_len}]")
+    if a is not None and a.batch:
+        w = w.replace(batch=a.batch, name=w.name + f" [batch overridden to {a.batch}]")
+    return w
 
 
 def _config_json(w, layers, lens, world):
@@ -193,7 +206,7 @@ def run_reference(a):
     if rank != 0:
         return 0
     from workloads import decode_inputs
-    w = _workload(a.workload)
+    w = _workload(a.workload, a)
     inp = decode_inputs(w)
     _cpu_baseline(w, inp, 0, steps=a.warmup)
     base, times = _cpu_baseline(w, inp, 0, steps=a.steps)
@@ -227,7 +240,7 @@ def run_kpa(a):
     import factorised_kv_attention_b200 as kpa
     from workloads import decode_inputs
 
-    w = _workload(a.workload)
+    w = _workload(a.workload, a)
     s = w.shape
     elt = 2 if w.dtype == "bf16" else 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -255,7 +268,7 @@ def run_kpa(a):
         del inp
     max_len = int(lens.max())
     ws_bytes = kpa.kpa_decode_workspace_size(cfg, w.batch, max_len)
-    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     outs = [torch.empty(w.batch, s.h, s.dh, dtype=torch.float32, device=dev) for _ in range(layers)]
     sm_scale = 1.0 / float(np.sqrt(s.dh))
     torch.cuda.synchronize()
@@ -315,7 +328,7 @@ def run_kpa(a):
     with torch.cuda.stream(stream):
         # settle clocks under load (untimed) while the sampler runs
         sampler.start()
-        t_end = time.time() + 1.0
+        t_end = time.time() + a.settle_seconds
         while time.time() < t_end:
             for _ in range(20):
                 graph.replay()

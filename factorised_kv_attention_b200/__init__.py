@@ -71,6 +71,7 @@ _SIGS = {
     "kpa_read_device_error": ([_vp, ctypes.POINTER(_i32)], ctypes.c_int),
     "kpa_decode_noalloc": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp],
                            ctypes.c_int),
+    "kpa_test_set_decode_hooks": ([_i32, _i32, ctypes.c_uint64], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -197,6 +198,11 @@ def kpa_decode_noalloc(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, 
     _check(_lib.kpa_decode_noalloc(ctypes.byref(cfg), batch, _addr(q), _addr(q_pos), _addr(kcache),
                                    _addr(vcache), capacity, _addr(seq_len), max_len, sm_scale,
                                    _addr(out), _stream(stream)), "kpa_decode_noalloc")
+
+
+def kpa_test_set_decode_hooks(skip_tile=-1, skip_split=-1, wait_limit_ns=1_000_000_000):
+    _check(_lib.kpa_test_set_decode_hooks(skip_tile, skip_split, wait_limit_ns),
+           "kpa_test_set_decode_hooks")
 
 
 def kpa_read_device_error(stream=None) -> int:

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "kpa_internal.cuh"
+#include "kpa_mma_decode.cuh"
 
 namespace kpa {
 
@@ -91,35 +92,101 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 constexpr size_t kSmemLimit = 200 * 1024;
 
+std::mutex g_hooks_mu;
+DecodeTestHooks g_hooks = {-1, -1, 1000000000ull};   // bounded waits give up after 1 s
+
+DecodeTestHooks current_hooks() {
+    std::lock_guard<std::mutex> lock(g_hooks_mu);
+    return g_hooks;
+}
+
+constexpr int kMaxClusterSplits = 16;
+
+// How many clusters of `size` CTAs of a tensor-core variant can be resident at once
+// on this device (cached per device).
+int cluster_capacity(int variant, int size) {
+    static std::atomic<int> known[kMaxDevices][8][kMaxClusterSplits + 1];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || variant < 0 ||
+        variant >= 8 || size < 1 || size > kMaxClusterSplits)
+        return 0;
+    int k = known[dev][variant][size].load();
+    if (k == 0) {
+        k = mma_decode_max_clusters(variant, size);
+        known[dev][variant][size].store(k > 0 ? k : -1);
+    }
+    return k > 0 ? k : 0;
+}
+
+// Split plan.  Auto splits aim at one wave of CTAs: ceil(sms * ctas_per_sm / batch)
+// pieces per sequence, each a multiple of 16 slots.
 kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int tps_req, int sms,
                        DecodePlan *p) {
     if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
-    int tile = 32;
-    while (tile > 8 && decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) tile /= 2;
-    if (decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) return KPA_ERR_UNSUPPORTED;
-    if ((d.h * d.dh + 255) / 256 > 32) return KPA_ERR_UNSUPPORTED;
+    p->variant = dt == KPA_BF16 ? mma_decode_variant(d) : -1;
+    int ctas_per_sm = 2;
+    if (p->variant >= 0) {
+        p->tile = mma_decode_tile(p->variant);
+        const size_t smem = mma_decode_smem(p->variant);
+        ctas_per_sm = smem > 0 ? (int)((227 * 1024) / smem) : 1;
+        if (ctas_per_sm < 1) ctas_per_sm = 1;
+    } else {
+        int tile = 32;
+        while (tile > 8 && decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) tile /= 2;
+        if (decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) return KPA_ERR_UNSUPPORTED;
+        if ((d.h * d.dh + 255) / 256 > 32) return KPA_ERR_UNSUPPORTED;
+        p->tile = tile;
+    }
+    const int target = ctas_per_sm * (sms > 0 ? sms : 148);
+    const int per_seq = batch > 0 ? (target > batch ? target / batch : 1) : 1;
+    // A sequence's splits merge inside one thread-block cluster (over DSMEM) when all
+    // the clusters are resident at once and still cover most of the SMs; a cluster of
+    // one CTA needs no merge at all.  Otherwise the splits of a sequence are merged
+    // through global memory.
+    int c = p->variant >= 0 ? (per_seq < kMaxClusterSplits ? per_seq : kMaxClusterSplits) : 0;
+    while (c > 1 && cluster_capacity(p->variant, c) < batch) --c;
+    const bool cluster_auto = c == 1 || (c > 1 && (int64_t)batch * c * 5 >= (int64_t)target * 4);
     int tps = tps_req;
     if (tps == 0) {
-        const int target = 2 * (sms > 0 ? sms : 148);
-        const int per_seq = batch > 0 ? (target + batch - 1) / batch : 1;
-        const int64_t want = ((int64_t)max_len + per_seq - 1) / per_seq;
-        tps = (int)(((want + 63) / 64) * 64);
+        const int want_split = cluster_auto ? c : per_seq;
+        const int64_t want = ((int64_t)max_len + want_split - 1) / want_split;
+        tps = (int)(((want + 15) / 16) * 16);
         if (tps < 64) tps = 64;
     }
     p->tokens_per_split = tps;
-    p->tile = tile;
     p->n_split = max_len > 0 ? (int)(((int64_t)max_len + tps - 1) / tps) : 1;
+    p->cluster = p->variant >= 0 && p->n_split <= kMaxClusterSplits &&
+                 (p->n_split == 1 || cluster_capacity(p->variant, p->n_split) >= batch);
+    // otherwise the last CTA of a sequence merges its splits when that read is small
+    p->fused = p->cluster ||
+               (p->variant >= 0 && (size_t)p->n_split * d.h * d.dh * sizeof(float) <= 256 * 1024);
     const size_t o_bytes = (size_t)batch * p->n_split * d.h * d.dh * sizeof(float);
     const size_t ml_bytes = (size_t)batch * p->n_split * d.h * 2 * sizeof(float);
     p->part_o_off = 0;
     p->part_ml_off = align256(o_bytes);
-    p->bytes = p->part_ml_off + align256(ml_bytes);
+    p->counters_off = p->part_ml_off + align256(ml_bytes);
+    p->bytes = p->counters_off + align256((size_t)batch * sizeof(int));
     return KPA_OK;
 }
 
 }  // namespace
 
 void record_cuda_error(cudaError_t e) { t_last_cuda = (int)e; }
+
+kpa_status decode_counter_region(const kpa_config *cfg, int batch, int max_len, size_t *offset,
+                                 size_t *bytes) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    int sms = 0;
+    s = device_state(nullptr, &sms);
+    if (s != KPA_OK) return s;
+    DecodePlan p;
+    s = plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, 0, sms, &p);
+    if (s != KPA_OK) return s;
+    *offset = p.counters_off;
+    *bytes = (size_t)batch * sizeof(int);
+    return KPA_OK;
+}
 
 }  // namespace kpa
 
@@ -222,13 +289,37 @@ kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
     float *part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) + p.part_ml_off);
     const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
     cudaStream_t st = (cudaStream_t)stream;
+    int *counters = reinterpret_cast<int *>(static_cast<char *>(workspace) + p.counters_off);
+    const float out_scale = (float)(1.0 / (double)d.rv);
     cudaError_t e = cudaSuccess;
-    if (max_len > 0)
+    if (max_len > 0 && p.variant >= 0) {
+        DecodeArgs args;
+        args.q = static_cast<const __nv_bfloat16 *>(q);
+        args.q_pos = q_pos;
+        args.kc = static_cast<const __nv_bfloat16 *>(kcache);
+        args.vc = static_cast<const __nv_bfloat16 *>(vcache);
+        args.cap = capacity;
+        args.seq_len = seq_len;
+        args.max_len = max_len;
+        args.qscale = qscale;
+        args.tps = p.tokens_per_split;
+        args.n_split = p.n_split;
+        args.part_o = part_o;
+        args.part_ml = part_ml;
+        args.counters = counters;
+        args.out = out;
+        args.out_scale = out_scale;
+        args.fused = p.fused;
+        args.cluster = p.cluster;
+        args.err = err;
+        e = launch_decode_mma(p.variant, args, batch, p, rope_table(cfg), current_hooks(), st);
+    } else if (max_len > 0) {
         e = launch_decode_fma(d, cfg->dtype, batch, q, q_pos, kcache, vcache, capacity, seq_len,
                               max_len, qscale, p, part_o, part_ml, rope_table(cfg), err, st, sms);
+    }
     if (e != cudaSuccess) return cuda_fail(e);
-    e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml,
-                              (float)(1.0 / (double)d.rv), out, st);
+    if (max_len > 0 && p.fused) return KPA_OK;
+    e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml, out_scale, out, st);
     return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 
@@ -272,6 +363,16 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t, int32_t, const void *, con
     kpa_status s = check_cfg(cfg, true, true);
     if (s != KPA_OK) return s;
     return KPA_ERR_UNSUPPORTED;
+}
+
+kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split,
+                                     uint64_t wait_limit_ns) {
+    if (wait_limit_ns == 0) return KPA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_hooks_mu);
+    g_hooks.skip_tile = skip_tile;
+    g_hooks.skip_split = skip_split;
+    g_hooks.wait_limit_ns = wait_limit_ns;
+    return KPA_OK;
 }
 
 kpa_status kpa_read_device_error(kpa_stream stream, int32_t *code) {

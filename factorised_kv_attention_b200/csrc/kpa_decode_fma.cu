@@ -186,7 +186,7 @@ cudaError_t launch_t(const Dims &d, int batch, const void *q, const int32_t *q_p
                      float *part_ml, const RopeTable &rope, int *err, cudaStream_t st,
                      size_t smem) {
     auto kern = decode_fma_kernel<T, OPT>;
-    cudaError_t e = ensure_dynamic_smem(kern, smem);
+    cudaError_t e = ensure_dynamic_smem<decode_fma_kernel<T, OPT>>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)p.n_split, (unsigned)batch);
     kern<<<grid, kThreads, smem, st>>>(d, (const T *)q, q_pos, (const T *)kc, (const T *)vc, cap,
@@ -240,43 +240,96 @@ cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void
 
 // ---------------------------------------------------------------------------
 // Split combine: out = (1/R_V) * sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
-__global__ void __launch_bounds__(128)
+// One block per (head, sequence): the split statistics are staged in shared
+// memory with all loads in flight, then each thread sums its features over the
+// splits with independent, unrolled loads.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineMaxSplits = 4096;
+
+__global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, int tps,
                       int n_split, const float *__restrict__ part_o,
                       const float *__restrict__ part_ml, float out_scale,
                       float *__restrict__ out) {
-    const int b = blockIdx.y;
-    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= d.h * d.dh) return;
-    const int head = idx / d.dh;
+    __shared__ float w[kCombineMaxSplits];
+    __shared__ float red[kCombineThreads / 32];
+    __shared__ float s_den;
+    const int head = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     int L = seq_len[b];
     L = L < 0 ? 0 : (L > max_len ? max_len : L);
     const int ns = (L + tps - 1) / tps;
-    float *dst = out + (size_t)b * d.h * d.dh + idx;
-    if (ns == 0) {
-        *dst = 0.f;
+    float *dst = out + ((size_t)b * d.h + head) * d.dh;
+    if (ns == 0 || ns > kCombineMaxSplits) {
+        for (int f = tid; f < d.dh; f += kCombineThreads) dst[f] = 0.f;
         return;
     }
-    const float *ml = part_ml + ((size_t)b * n_split * d.h + head) * 2;
+    const float2 *ml = reinterpret_cast<const float2 *>(part_ml) + (size_t)b * n_split * d.h + head;
     float M = -INFINITY;
-    for (int i = 0; i < ns; ++i) M = fmaxf(M, ml[(size_t)i * d.h * 2]);
-    float num = 0.f, den = 0.f;
-    const float *po = part_o + (size_t)b * n_split * d.h * d.dh + idx;
-    for (int i = 0; i < ns; ++i) {
-        const float w = exp2f(ml[(size_t)i * d.h * 2] - M);
-        num += w * po[(size_t)i * d.h * d.dh];
-        den += w * ml[(size_t)i * d.h * 2 + 1];
+    for (int i = tid; i < ns; i += kCombineThreads) {
+        const float m = ml[(size_t)i * d.h].x;
+        w[i] = m;
+        M = fmaxf(M, m);
     }
-    *dst = den > 0.f ? out_scale * num / den : 0.f;
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if ((tid & 31) == 0) red[tid >> 5] = M;
+    __syncthreads();
+    M = red[0];
+    for (int k = 1; k < kCombineThreads / 32; ++k) M = fmaxf(M, red[k]);
+    float den = 0.f;
+    for (int i = tid; i < ns; i += kCombineThreads) {
+        const float wi = exp2f(w[i] - M);
+        w[i] = wi;
+        den += wi * ml[(size_t)i * d.h].y;
+    }
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    __syncthreads();
+    if ((tid & 31) == 0) red[tid >> 5] = den;
+    __syncthreads();
+    if (tid == 0) {
+        float t = 0.f;
+        for (int k = 0; k < kCombineThreads / 32; ++k) t += red[k];
+        s_den = t;
+    }
+    __syncthreads();
+    if (d.dh > kCombineThreads) {                          // wide heads: one feature per pass
+        const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh;
+        for (int ff = tid; ff < d.dh; ff += kCombineThreads) {
+            float t = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < ns; ++i) t += w[i] * po[(size_t)i * d.h * d.dh + ff];
+            dst[ff] = s_den > 0.f ? out_scale * t / s_den : 0.f;
+        }
+        return;
+    }
+    // features x split phases: threads that share a feature take every P-th split
+    const int P = kCombineThreads / d.dh;
+    const int f = tid % d.dh, phase = tid / d.dh;
+    float num = 0.f;
+    if (phase < P) {
+        const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh + f;
+#pragma unroll 8
+        for (int i = phase; i < ns; i += P) num += w[i] * po[(size_t)i * d.h * d.dh];
+    }
+    __syncthreads();
+    float *acc = w;                                        // reuse: [P][dh] partial sums
+    if (phase < P) acc[phase * d.dh + f] = num;
+    __syncthreads();
+    for (int ff = tid; ff < d.dh; ff += kCombineThreads) {
+        float t = 0.f;
+        for (int ph = 0; ph < P; ++ph) t += acc[ph * d.dh + ff];
+        dst[ff] = s_den > 0.f ? out_scale * t / s_den : 0.f;
+    }
 }
 
 cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_len,
                                   int max_len, const DecodePlan &plan, const float *part_o,
                                   const float *part_ml, float out_scale, float *out,
                                   cudaStream_t st) {
-    dim3 grid((unsigned)((d.h * d.dh + 127) / 128), (unsigned)batch);
-    decode_combine_kernel<<<grid, 128, 0, st>>>(d, seq_len, max_len, plan.tokens_per_split,
-                                                plan.n_split, part_o, part_ml, out_scale, out);
+    if (plan.n_split > kCombineMaxSplits) return cudaErrorInvalidValue;
+    dim3 grid((unsigned)d.h, (unsigned)batch);
+    decode_combine_kernel<<<grid, kCombineThreads, 0, st>>>(d, seq_len, max_len,
+                                                            plan.tokens_per_split, plan.n_split,
+                                                            part_o, part_ml, out_scale, out);
     return cudaGetLastError();
 }
 

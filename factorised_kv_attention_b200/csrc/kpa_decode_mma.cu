@@ -23,8 +23,12 @@
 // 16-byte row (ldmatrix) or 32-bit word (two adjacent tokens).  Every wait is
 // bounded; on expiry the kernel records KPA_ERR_TIMEOUT, drains its copies and
 // returns.
+#include <cooperative_groups.h>
+
 #include "kpa_internal.cuh"
 #include "kpa_mma_decode.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace kpa {
 namespace {
@@ -110,36 +114,64 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// x ~= hi + lo with both parts bf16; returns the packed pairs for (x0, x1).
-__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-    __nv_bfloat162 H = __halves2bfloat162(h0, h1);
-    hi = *reinterpret_cast<uint32_t *>(&H);
-    lo = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-}
-
-__device__ __forceinline__ float2 lds_bf16x2(const unsigned char *p) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(p);
-    return __bfloat1622float2(v);
-}
-
 __device__ __forceinline__ uint32_t mask_pair(uint32_t v, bool keep0, bool keep1) {
     return (keep0 ? (v & 0xffffu) : 0u) | (keep1 ? (v & 0xffff0000u) : 0u);
+}
+
+// Packed FP32 pair arithmetic (sm_100 f32x2 forms).
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// bf16x2 word -> (low element, high element) as floats
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+__device__ __forceinline__ uint32_t lds_u32(const unsigned char *p) {
+    return *reinterpret_cast<const uint32_t *>(p);
+}
+
+// (x.x, x.y) -> bf16 hi + lo pairs, low half = x.x
+__device__ __forceinline__ void split2(float2 x, uint32_t &hi, uint32_t &lo) {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x.y), "f"(x.x));
+    const float2 r = fsub2(x, unpack_bf16x2(hi));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(r.y), "f"(r.x));
 }
 
 // ------------------------------------------------------------------- kernel
 template <class C>
 __global__ void __launch_bounds__((C::WARPS + 1) * 32, 1)
-decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ q_pos,
-                  const __nv_bfloat16 *__restrict__ kc, const __nv_bfloat16 *__restrict__ vc,
-                  int cap, const int32_t *__restrict__ seq_len, int max_len, float qscale,
-                  int tps, int n_split, float *__restrict__ part_o, float *__restrict__ part_ml,
-                  RopeTable rope, int *err, DecodeTestHooks hooks) {
+decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     constexpr int MA = C::MA, D1 = C::D1, D2 = C::D2, RK = C::RK, RV = C::RV, H2 = C::H2;
     constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
     constexpr int MT = MA / 16, KS = D2 / 16, NT = D2 / 8;
@@ -147,102 +179,144 @@ decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict
     constexpr int WARPS = C::WARPS, SLICES = C::SLICES, CHUNKS = C::CHUNKS, STAGES = C::STAGES;
     constexpr int TT = C::TT;
     constexpr int KBYTES = TT * EK * 2, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int RED_LD = C::RED_LD;               // floats per token row of the j1 scratch
+    constexpr int A_K = RK * MA, A_V = RV * MA;     // start of B in a key / value record
 
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *stage_base = smem;                                     // STAGES x (K | V)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);  // full, empty
-    float *qs = reinterpret_cast<float *>(bars + 2 * STAGES);             // [H][DH] query
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(qs + H * DH);
+    unsigned char *stage_base = smem;                                           // ring
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BARS);          // full, empty
+    float *qs = reinterpret_cast<float *>(smem + C::OFF_Q);                     // [H][DH]
+    float2 *cs = reinterpret_cast<float2 *>(smem + C::OFF_CS);                  // [D2/2]
+    float *scratch = reinterpret_cast<float *>(smem + C::OFF_SCR);              // per warp
+    volatile int *flags = reinterpret_cast<volatile int *>(smem + C::OFF_FLAGS);  // abort, last
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y, split = blockIdx.x;
-
-    int L = seq_len[b];
-    if (L > max_len || L < 0) {
-        if (split == 0 && tid == 0) raise_error(err, kErrDeviceCheck);
-        L = L < 0 ? 0 : max_len;
-    }
-    const int t0 = split * tps;
-    if (t0 >= L) return;                                   // empty split
-    const int t1 = min(t0 + tps, L);
-    const int n_tiles = (t1 - t0 + TT - 1) / TT;
-
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, WARPS);
         }
-        *abort_flag = 0;
+        flags[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // rotated, scaled query in fp32 (consumer threads; the producer starts right away)
+    // launched with programmatic stream serialization: wait for the previous grid in
+    // the stream before reading any input, and let the next grid be scheduled now
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    // The first tile's copy starts before the sequence length is known: slots
+    // [t0, t0 + TT) clipped to max_len are inside the cache whatever the length, and
+    // tokens past the length are masked later.
+    const int t0 = split * a.tps;
+    const int spec_n = min(TT, a.max_len - t0);
+    const bool spec = spec_n > 0 &&
+                      !(hooks.skip_tile == 0 && split == hooks.skip_split && b == 0);
+    if (tid == 0 && spec) {
+        const int groups = (spec_n + kGroup - 1) / kGroup;
+        const uint32_t kbytes = (uint32_t)groups * EK * kGroup * 2;
+        const uint32_t vbytes = (uint32_t)groups * EV * kGroup * 2;
+        const uint32_t dst = smem_u32(stage_base);
+        mbar_expect_tx(full0, kbytes + vbytes);
+        bulk_g2s(dst, a.kc + ((size_t)b * a.cap + t0) * EK, kbytes, full0);
+        bulk_g2s(dst + KBYTES, a.vc + ((size_t)b * a.cap + t0) * EV, vbytes, full0);
+    }
+
+    // every input of the prologue is requested at once (one round trip)
+    const bool rotate = a.q_pos != nullptr;
+    int L = a.seq_len[b];
+    const double qpos = rotate ? (double)a.q_pos[b] : 0.0;
+    constexpr int QPT = (H * DH / 2 + WARPS * 32 - 1) / (WARPS * 32);   // query pairs per thread
+    __nv_bfloat162 qv[QPT];
     if (warp < WARPS) {
-        const __nv_bfloat16 *qb = q + (size_t)b * H * DH;
-        const bool rotate = q_pos != nullptr;
-        const double qp = rotate ? (double)q_pos[b] : 0.0;
-        for (int i = tid; i < H * DH / 2; i += WARPS * 32) {
-            const float x0 = __bfloat162float(qb[2 * i]), x1 = __bfloat162float(qb[2 * i + 1]);
-            float y0 = x0, y1 = x1;
-            if (rotate) {
-                float c, s;
-                rope_cs(qp, rope.theta[((2 * i) % D2) >> 1], c, s);
-                y0 = x0 * c - x1 * s;
-                y1 = x0 * s + x1 * c;
-            }
-            qs[2 * i] = y0 * qscale;
-            qs[2 * i + 1] = y1 * qscale;
+        const __nv_bfloat162 *qb = reinterpret_cast<const __nv_bfloat162 *>(a.q + (size_t)b * H * DH);
+#pragma unroll
+        for (int k = 0; k < QPT; ++k) {
+            const int i = tid + k * WARPS * 32;
+            if (i < H * DH / 2) qv[k] = qb[i];
         }
     }
-    __syncthreads();
+    if (L > a.max_len || L < 0) {
+        if (split == 0 && tid == 0) raise_error(a.err, kErrDeviceCheck);
+        L = L < 0 ? 0 : a.max_len;
+    }
+    if (t0 >= L && !a.cluster) {                           // empty split (a cluster member stays)
+        if (tid == 0 && spec && !mbar_wait_bounded(full0, 0, hooks.wait_limit_ns))
+            raise_error(a.err, kErrTimeout);               // its speculative copy lands first
+        return;
+    }
+    const int t1 = max(t0, min(t0 + a.tps, L));
+    const int n_tiles = (t1 - t0 + TT - 1) / TT;
+    __syncthreads();                                        // barriers initialised
 
     const uint64_t limit = hooks.wait_limit_ns;
-    const __nv_bfloat16 *kb = kc + ((size_t)b * cap + t0) * EK;   // group-aligned (t0 % 8 == 0)
-    const __nv_bfloat16 *vb = vc + ((size_t)b * cap + t0) * EV;
+    const __nv_bfloat16 *kb = a.kc + ((size_t)b * a.cap + t0) * EK;   // group-aligned (t0 % 8 == 0)
+    const __nv_bfloat16 *vb = a.vc + ((size_t)b * a.cap + t0) * EV;
 
     // ------------------------------------------------------------ producer
     if (warp == WARPS) {
         if (lane == 0) {
-            int issued = 0;
-            bool ok = true;
-            for (int t = 0; t < n_tiles && ok; ++t) {
+            int issued = spec ? 1 : 0;
+            for (int t = spec ? 1 : 0; t < n_tiles; ++t) {
                 const int s = t % STAGES;
-                if (t >= STAGES) {
-                    if (!mbar_wait_bounded(empty0 + 8 * s, ((t / STAGES) - 1) & 1, limit)) {
-                        raise_error(err, kErrTimeout);
-                        *abort_flag = 1;
-                        ok = false;
-                        break;
-                    }
+                if (t >= STAGES && !mbar_wait_bounded(empty0 + 8 * s, ((t / STAGES) - 1) & 1, limit)) {
+                    raise_error(a.err, kErrTimeout);
+                    flags[0] = 1;
+                    break;
                 }
-                if (*abort_flag) break;
+                if (flags[0]) break;
                 const int n = min(TT, t1 - t0 - t * TT);
                 const int groups = (n + kGroup - 1) / kGroup;
                 const uint32_t kbytes = (uint32_t)groups * EK * kGroup * 2;
                 const uint32_t vbytes = (uint32_t)groups * EV * kGroup * 2;
-                if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) {
-                    issued = t + 1;          // test hook: this tile never arrives
-                    continue;
-                }
+                issued = t + 1;
+                if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) continue;
                 const uint32_t dst = smem_u32(stage_base + (size_t)s * STAGE_BYTES);
                 mbar_expect_tx(full0 + 8 * s, kbytes + vbytes);
                 bulk_g2s(dst, kb + (size_t)t * TT * EK, kbytes, full0 + 8 * s);
                 bulk_g2s(dst + KBYTES, vb + (size_t)t * TT * EV, vbytes, full0 + 8 * s);
-                issued = t + 1;
             }
-            // drain: every copy this thread issued must land before the CTA exits
+            // drain: every copy issued for this CTA must land before it exits
             for (int t = max(0, issued - STAGES); t < issued; ++t) {
                 if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) continue;
                 if (!mbar_wait_bounded(full0 + 8 * (t % STAGES), (t / STAGES) & 1, limit))
-                    raise_error(err, kErrTimeout);
+                    raise_error(a.err, kErrTimeout);
             }
         }
-        return;
+        if (!a.cluster) return;
+    } else {
+
+    // rotated, scaled query in fp32 (consumers, while the first copies are in flight):
+    // I_{d1} (x) R^(2)(q_pos) on pairs (2m, 2m+1), angles tabulated once per CTA
+    if (rotate && tid < D2 / 2) {
+        float cth, sth;
+        rope_cs(qpos, rope.theta[tid], cth, sth);
+        cs[tid] = make_float2(cth, sth);
     }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+#pragma unroll
+    for (int k = 0; k < QPT; ++k) {
+        const int i = tid + k * WARPS * 32;
+        if (i < H * DH / 2) {
+            const float2 x = __bfloat1622float2(qv[k]);
+            float2 y = x;
+            if (rotate) {
+                const float2 w = cs[i % (D2 / 2)];
+                y = make_float2(x.x * w.x - x.y * w.y, x.x * w.y + x.y * w.x);
+            }
+            qs[2 * i] = y.x * a.qscale;
+            qs[2 * i + 1] = y.y * a.qscale;
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
 
     // ------------------------------------------------------------ consumers
     const int i2 = warp % H2, slice = warp / H2;
     const int g = lane >> 2, c = lane & 3;
+    float *red = scratch + (size_t)warp * C::SCR_FLOATS;   // [16][RED_LD] j1 partials
+    float *pbuf = red + 16 * RED_LD;                         // [H1][16] weights
+    float *abuf = pbuf + H1 * 16;                            // [H1] rescale factors
 
     // query fragments (A operand, row = (i1, j1), k = j2), hi and lo parts
     uint32_t qa_hi[MT][KS][4], qa_lo[MT][KS][4];
@@ -256,55 +330,56 @@ decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict
                 const int j2 = ks * 16 + 2 * c + ((v & 2) ? 8 : 0);
                 const int i1 = row / D1, j1 = row % D1;
                 const float *src = qs + (i1 * H2 + i2) * DH + j1 * D2 + j2;
-                split_pack(src[0], src[1], qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
+                split2(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
             }
 
-    // running softmax state per owned row (rows g and g+8 of each m-tile), per lane
-    float m_run[MT][2], l_run[MT][2];
     float o[MT][NT][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        m_run[mt][0] = m_run[mt][1] = -INFINITY;
-        l_run[mt][0] = l_run[mt][1] = 0.f;
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    // softmax state: per owned row (D1 == 1: rows are heads) or per lane head (D1 > 1)
+    float m_row[MT][2], l_row[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        m_row[mt][0] = m_row[mt][1] = -INFINITY;
+        l_row[mt][0] = l_row[mt][1] = 0.f;
     }
+    constexpr int PPL = C::PPL;                 // (head, token) pairs per lane per chunk (D1 > 1)
+    const int my_i1 = lane % H1;                // the head this lane scores (D1 > 1)
+    float m_h = -INFINITY, l_h = 0.f;
 
-    constexpr int A_K = RK * MA;                 // start of B^K in a key record
-    constexpr int A_V = RV * MA;
     bool aborted = false;
-
     for (int t = 0; t < n_tiles; ++t) {
         const int s = t % STAGES;
         if (!mbar_wait_bounded(full0 + 8 * s, (t / STAGES) & 1, limit)) {
-            raise_error(err, kErrTimeout);
-            *abort_flag = 1;
+            raise_error(a.err, kErrTimeout);
+            flags[0] = 1;
             aborted = true;
             break;
         }
         const unsigned char *kt = stage_base + (size_t)s * STAGE_BYTES;
         const unsigned char *vt = kt + KBYTES;
-        const int n_valid = min(TT, t1 - t0 - t * TT);           // tokens of this tile
-        const int tok_base = slice * CHUNKS * 16;                 // this warp's first token
+        const int n_valid = min(TT, t1 - t0 - t * TT);
+        const int tok_base = slice * CHUNKS * 16;
 
-        float sc[CHUNKS][MT][2][4];                               // scores, then weights
-#pragma unroll
+#pragma unroll 1
         for (int ch = 0; ch < CHUNKS; ++ch) {
             const int tok0 = tok_base + ch * 16;
-            const int grp0 = tok0 >> 3;
+            if (tok0 >= n_valid) break;                       // rest of this warp's slice is past the tail
+            const bool tail = tok0 + 16 > n_valid;
+            const unsigned char *kg0 = kt + (size_t)(tok0 >> 3) * EK * 16;
+            // ---- scores: sc[mt][gi][v] = sum_r A^K_r * (Q_i2 B~^K_r), rows (i1,j1), tokens 2c, 2c+1
+            float2 sc[MT][2][2];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) sc[ch][mt][gi][v] = 0.f;
-            if (tok0 >= n_valid) continue;                        // whole chunk past the tail
+                for (int gi = 0; gi < 2; ++gi) sc[mt][gi][0] = sc[mt][gi][1] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < RK; ++r) {
 #pragma unroll
                 for (int gi = 0; gi < 2; ++gi) {
-                    const unsigned char *grp = kt + (size_t)(grp0 + gi) * EK * 16;
-                    // B~^K_r(token)[i2, :] as the B operand: rows j2, 8 tokens each (.trans)
+                    const unsigned char *grp = kg0 + (size_t)gi * EK * 16;
                     uint32_t bk[KS][2];
                     const int e_b = A_K + r * H2 * D2 + i2 * D2;
                     if constexpr (KS % 2 == 0) {
@@ -326,126 +401,150 @@ decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict
                             mma16816(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
                             mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
                         }
-                        // times A^K_r(token)[i1, j1] for rows g and g+8, tokens 2c and 2c+1
                         const int row0 = mt * 16 + g;
-                        const float2 a0 = lds_bf16x2(grp + (size_t)(r * MA + row0) * 16 + 4 * c);
-                        const float2 a1 = lds_bf16x2(grp + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
-                        sc[ch][mt][gi][0] += acc[0] * a0.x;
-                        sc[ch][mt][gi][1] += acc[1] * a0.y;
-                        sc[ch][mt][gi][2] += acc[2] * a1.x;
-                        sc[ch][mt][gi][3] += acc[3] * a1.y;
+                        const float2 a0 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MA + row0) * 16 + 4 * c));
+                        const float2 a1 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MA + row0 + 8) * 16 + 4 * c));
+                        sc[mt][gi][0] = ffma2(make_float2(acc[0], acc[1]), a0, sc[mt][gi][0]);
+                        sc[mt][gi][1] = ffma2(make_float2(acc[2], acc[3]), a1, sc[mt][gi][1]);
                     }
                 }
             }
-            // sum over j1: rows of one head are D1 consecutive rows
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi) {
-                    float *v = sc[ch][mt][gi];
-                    if constexpr (D1 == 16) {
-                        v[0] += v[2]; v[1] += v[3];
-                    }
-#pragma unroll
-                    for (int off = 4; off < 4 * (D1 < 8 ? D1 : 8); off <<= 1) {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], off);
-                    }
-                    if constexpr (D1 == 16) {
-                        v[2] = v[0]; v[3] = v[1];
-                    }
-                    // tokens past the tile's valid range
-                    const int tk = tok0 + gi * 8 + 2 * c;
-                    if (tk >= n_valid) { v[0] = -INFINITY; v[2] = -INFINITY; }
-                    if (tk + 1 >= n_valid) { v[1] = -INFINITY; v[3] = -INFINITY; }
-                }
-        }
-        // chunks entirely past the tail
-#pragma unroll
-        for (int ch = 0; ch < CHUNKS; ++ch)
-            if (tok_base + ch * 16 >= n_valid)
+
+            // ---- online softmax for this chunk; afterwards sc holds the weights p
+            if constexpr (D1 == 1) {
+                // rows are heads: row g of m-tile mt is head mt*16+g, row g+8 head mt*16+g+8
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int gi = 0; gi < 2; ++gi)
+                    for (int hr = 0; hr < 2; ++hr) {
+                        if (tail) {
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) sc[ch][mt][gi][v] = -INFINITY;
-
-        // online softmax over this tile (log2 domain), per owned row
+                            for (int gi = 0; gi < 2; ++gi) {
+                                const int tk = tok0 + gi * 8 + 2 * c;
+                                if (tk >= n_valid) sc[mt][gi][hr].x = -INFINITY;
+                                if (tk + 1 >= n_valid) sc[mt][gi][hr].y = -INFINITY;
+                            }
+                        }
+                        float mx = fmaxf(fmaxf(sc[mt][0][hr].x, sc[mt][0][hr].y),
+                                         fmaxf(sc[mt][1][hr].x, sc[mt][1][hr].y));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                        const float m_new = fmaxf(m_row[mt][hr], mx);   // finite: chunk has a valid token
+                        const float alpha = exp2f(m_row[mt][hr] - m_new);
+                        float sum = 0.f;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+                        for (int gi = 0; gi < 2; ++gi) {
+                            sc[mt][gi][hr].x = exp2f(sc[mt][gi][hr].x - m_new);
+                            sc[mt][gi][hr].y = exp2f(sc[mt][gi][hr].y - m_new);
+                            sum += sc[mt][gi][hr].x + sc[mt][gi][hr].y;
+                        }
+                        l_row[mt][hr] = l_row[mt][hr] * alpha + sum;
+                        m_row[mt][hr] = m_new;
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
+                        for (int nt = 0; nt < NT; ++nt) {
+                            o[mt][nt][2 * hr] *= alpha;
+                            o[mt][nt][2 * hr + 1] *= alpha;
+                        }
+                    }
+            } else {
+                // sum over j1 once per (head, token): partials through the warp's scratch
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int gi = 0; gi < 2; ++gi) {
+                        const int tk = gi * 8 + 2 * c, row = mt * 16 + g;
+                        red[tk * RED_LD + row] = sc[mt][gi][0].x;
+                        red[(tk + 1) * RED_LD + row] = sc[mt][gi][0].y;
+                        red[tk * RED_LD + row + 8] = sc[mt][gi][1].x;
+                        red[(tk + 1) * RED_LD + row + 8] = sc[mt][gi][1].y;
+                    }
+                __syncwarp();
+                float sp[PPL];
                 float mx = -INFINITY;
 #pragma unroll
-                for (int ch = 0; ch < CHUNKS; ++ch)
+                for (int k = 0; k < PPL; ++k) {
+                    const int tk = (lane + 32 * k) / H1;
+                    const float *src = red + tk * RED_LD + my_i1 * D1;
+                    float v = 0.f;
+                    if constexpr (D1 % 4 == 0) {
 #pragma unroll
-                    for (int gi = 0; gi < 2; ++gi)
-                        mx = fmaxf(mx, fmaxf(sc[ch][mt][gi][2 * hr], sc[ch][mt][gi][2 * hr + 1]));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float m_new = fmaxf(m_run[mt][hr], mx);
-                const float alpha = (m_run[mt][hr] == -INFINITY) ? 0.f : exp2f(m_run[mt][hr] - m_new);
+                        for (int j = 0; j < D1; j += 4) {
+                            const float4 f = *reinterpret_cast<const float4 *>(src + j);
+                            v += (f.x + f.y) + (f.z + f.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < D1; ++j) v += src[j];
+                    }
+                    if (tail && tok0 + tk >= n_valid) v = -INFINITY;
+                    sp[k] = v;
+                    mx = fmaxf(mx, v);
+                }
+#pragma unroll
+                for (int off = H1; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float m_new = fmaxf(m_h, mx);
+                const float alpha = exp2f(m_h - m_new);
                 float sum = 0.f;
 #pragma unroll
-                for (int ch = 0; ch < CHUNKS; ++ch)
-#pragma unroll
-                    for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            float &x = sc[ch][mt][gi][2 * hr + k];
-                            x = (m_new == -INFINITY) ? 0.f : exp2f(x - m_new);
-                            sum += x;
-                        }
-                l_run[mt][hr] = l_run[mt][hr] * alpha + sum;
-                m_run[mt][hr] = m_new;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    o[mt][nt][2 * hr] *= alpha;
-                    o[mt][nt][2 * hr + 1] *= alpha;
+                for (int k = 0; k < PPL; ++k) {
+                    const float p = exp2f(sp[k] - m_new);
+                    sum += p;
+                    pbuf[my_i1 * 16 + (lane + 32 * k) / H1] = p;
                 }
+                l_h = l_h * alpha + sum;
+                m_h = m_new;
+                if (lane < H1) abuf[lane] = alpha;
+                __syncwarp();
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int i1 = (mt * 16 + g + 8 * hr) / D1;
+                        const float al = abuf[i1];
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            o[mt][nt][2 * hr] *= al;
+                            o[mt][nt][2 * hr + 1] *= al;
+                        }
+#pragma unroll
+                        for (int gi = 0; gi < 2; ++gi)
+                            sc[mt][gi][hr] = *reinterpret_cast<const float2 *>(pbuf + i1 * 16 + gi * 8 + 2 * c);
+                    }
             }
 
-        // values
-#pragma unroll
-        for (int ch = 0; ch < CHUNKS; ++ch) {
-            const int tok0 = tok_base + ch * 16;
-            if (tok0 >= n_valid) continue;
-            const int grp0 = tok0 >> 3;
-            const bool tail = tok0 + 16 > n_valid;
-            const unsigned char *g0p = vt + (size_t)grp0 * EV * 16;
+            // ---- values: P'[(i1,j1), k] = p * A^V_r, k = (group, token), hi/lo bf16 parts
+            const unsigned char *g0p = vt + (size_t)(tok0 >> 3) * EV * 16;
             const unsigned char *g1p = g0p + (size_t)EV * 16;
 #pragma unroll
             for (int r = 0; r < RV; ++r) {
-                // A operand: P'[(i1,j1), k] = p * A^V_r, k = (group, token); hi/lo split
                 uint32_t pa_hi[MT][4], pa_lo[MT][4];
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     const int row0 = mt * 16 + g;
-                    const float2 a00 = lds_bf16x2(g0p + (size_t)(r * MA + row0) * 16 + 4 * c);
-                    const float2 a10 = lds_bf16x2(g0p + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
-                    const float2 a01 = lds_bf16x2(g1p + (size_t)(r * MA + row0) * 16 + 4 * c);
-                    const float2 a11 = lds_bf16x2(g1p + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
-                    const float *p0 = sc[ch][mt][0], *p1 = sc[ch][mt][1];
-                    // weights of masked tokens are exactly 0; keep garbage factors out
-                    const float w00 = p0[0] != 0.f ? p0[0] * a00.x : 0.f;
-                    const float w01 = p0[1] != 0.f ? p0[1] * a00.y : 0.f;
-                    const float w10 = p0[2] != 0.f ? p0[2] * a10.x : 0.f;
-                    const float w11 = p0[3] != 0.f ? p0[3] * a10.y : 0.f;
-                    const float w20 = p1[0] != 0.f ? p1[0] * a01.x : 0.f;
-                    const float w21 = p1[1] != 0.f ? p1[1] * a01.y : 0.f;
-                    const float w30 = p1[2] != 0.f ? p1[2] * a11.x : 0.f;
-                    const float w31 = p1[3] != 0.f ? p1[3] * a11.y : 0.f;
-                    split_pack(w00, w01, pa_hi[mt][0], pa_lo[mt][0]);
-                    split_pack(w10, w11, pa_hi[mt][1], pa_lo[mt][1]);
-                    split_pack(w20, w21, pa_hi[mt][2], pa_lo[mt][2]);
-                    split_pack(w30, w31, pa_hi[mt][3], pa_lo[mt][3]);
+                    const uint32_t w00 = lds_u32(g0p + (size_t)(r * MA + row0) * 16 + 4 * c);
+                    const uint32_t w10 = lds_u32(g0p + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
+                    const uint32_t w01 = lds_u32(g1p + (size_t)(r * MA + row0) * 16 + 4 * c);
+                    const uint32_t w11 = lds_u32(g1p + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
+                    float2 x0 = fmul2(sc[mt][0][0], unpack_bf16x2(w00));
+                    float2 x1 = fmul2(sc[mt][0][1], unpack_bf16x2(w10));
+                    float2 x2 = fmul2(sc[mt][1][0], unpack_bf16x2(w01));
+                    float2 x3 = fmul2(sc[mt][1][1], unpack_bf16x2(w11));
+                    if (tail) {   // keep garbage factors of masked tokens out (their weight is 0)
+                        const int tk = tok0 + 2 * c;
+                        if (tk >= n_valid) { x0.x = 0.f; x1.x = 0.f; }
+                        if (tk + 1 >= n_valid) { x0.y = 0.f; x1.y = 0.f; }
+                        if (tk + 8 >= n_valid) { x2.x = 0.f; x3.x = 0.f; }
+                        if (tk + 9 >= n_valid) { x2.y = 0.f; x3.y = 0.f; }
+                    }
+                    split2(x0, pa_hi[mt][0], pa_lo[mt][0]);
+                    split2(x1, pa_hi[mt][1], pa_lo[mt][1]);
+                    split2(x2, pa_hi[mt][2], pa_lo[mt][2]);
+                    split2(x3, pa_hi[mt][3], pa_lo[mt][3]);
                 }
                 const int e_b = A_V + r * H2 * D2 + i2 * D2;
                 const int mat = lane >> 3, mrow = lane & 7;
 #pragma unroll
                 for (int np = 0; np < NT / 2; ++np) {
-                    // B operand: B^V_r(token)[i2, j2], rows j2 (8 tokens each), no transpose
                     const unsigned char *gp = (mat & 1) ? g1p : g0p;
                     uint32_t b00, b01, b10, b11;
                     ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mrow) * 16), b00, b01,
@@ -466,28 +565,36 @@ decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict
                     }
                 }
             }
+            if constexpr (D1 > 1) __syncwarp();    // scratch is rewritten by the next chunk
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
-        if (*abort_flag) { aborted = true; break; }
+        if (flags[0]) { aborted = true; break; }
     }
 
-    // l: sum over the four lanes (c) that share a row
+    // l: complete sums per head
+    if constexpr (D1 == 1) {
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            float l = l_run[mt][hr];
-            l += __shfl_xor_sync(0xffffffffu, l, 1);
-            l += __shfl_xor_sync(0xffffffffu, l, 2);
-            l_run[mt][hr] = l;
-        }
+            for (int hr = 0; hr < 2; ++hr) {
+                float l = l_row[mt][hr];
+                l += __shfl_xor_sync(0xffffffffu, l, 1);
+                l += __shfl_xor_sync(0xffffffffu, l, 2);
+                l_row[mt][hr] = l;
+            }
+    } else {
+#pragma unroll
+        for (int off = H1; off < 32; off <<= 1) l_h += __shfl_xor_sync(0xffffffffu, l_h, off);
+    }
 
     // merge the token slices of the CTA through shared memory (reuses the ring)
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    if (aborted || *abort_flag) return;
+    const bool ok = !(aborted || flags[0]);
+    if (!ok && !a.cluster) return;
     float *mo = reinterpret_cast<float *>(smem);                   // [SLICES][H][DH]
     float *mm = mo + SLICES * H * DH;                              // [SLICES][H][2]
+    float *cp = mm + SLICES * H * 2;                               // merged: [H][DH] o, [H] m, [H] l
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -500,14 +607,23 @@ decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict
             for (int nt = 0; nt < NT; ++nt)
                 *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
                     make_float2(o[mt][nt][2 * hr], o[mt][nt][2 * hr + 1]);
-            if (c == 0 && j1 == 0) {
-                mm[((size_t)slice * H + head) * 2] = m_run[mt][hr];
-                mm[((size_t)slice * H + head) * 2 + 1] = l_run[mt][hr];
+            if constexpr (D1 == 1) {
+                if (c == 0) {
+                    mm[((size_t)slice * H + head) * 2] = m_row[mt][hr];
+                    mm[((size_t)slice * H + head) * 2 + 1] = l_row[mt][hr];
+                }
             }
         }
+    if constexpr (D1 > 1) {
+        if (lane < H1) {
+            const int head = lane * H2 + i2;
+            mm[((size_t)slice * H + head) * 2] = m_h;
+            mm[((size_t)slice * H + head) * 2 + 1] = l_h;
+        }
+    }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    float *po = part_o + ((size_t)(b * n_split + split) * H) * DH;
-    float *pml = part_ml + ((size_t)(b * n_split + split) * H) * 2;
+    float *po = a.part_o + ((size_t)(b * a.n_split + split) * H) * DH;
+    float *pml = a.part_ml + ((size_t)(b * a.n_split + split) * H) * 2;
     for (int idx = tid; idx < H * DH; idx += WARPS * 32) {
         const int head = idx / DH;
         float M = -INFINITY;
@@ -521,42 +637,183 @@ decode_mma_kernel(const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict
             acc += wgt * mo[((size_t)sl * H) * DH + idx];
             l += wgt * mm[((size_t)sl * H + head) * 2 + 1];
         }
-        po[idx] = acc;
-        if (idx % DH == 0) {
-            pml[2 * head] = M;
-            pml[2 * head + 1] = l;
+        if (a.cluster) {
+            cp[idx] = acc;
+            if (idx % DH == 0) {
+                cp[H * DH + head] = M;
+                cp[H * DH + H + head] = l;
+            }
+        } else {
+            po[idx] = acc;
+            if (idx % DH == 0) {
+                pml[2 * head] = M;
+                pml[2 * head + 1] = l;
+            }
         }
     }
+    if (!a.cluster) {
+    if (!a.fused) return;
+
+    // the last CTA of this sequence merges every split (log-sum-exp) into out[b]
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    const int n_b = (L + a.tps - 1) / a.tps;
+    if (tid == 0) {
+        __threadfence();                                   // the CTA's partial before the count
+        flags[1] = (atomicAdd(a.counters + b, 1) == n_b - 1) ? 1 : 0;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    if (!flags[1]) return;
+    __threadfence();
+    const float *pob = a.part_o + (size_t)b * a.n_split * H * DH;
+    const float *pmb = a.part_ml + (size_t)b * a.n_split * H * 2;
+    // split statistics first, all loads in flight together: w[i][head] = 2^(m_i - M), then l
+    float *wt = reinterpret_cast<float *>(smem);            // [n_b][H]
+    float *den = wt + (size_t)n_b * H;                      // [H]
+    float *lv = den + H;                                    // [n_b][H]
+    for (int k = tid; k < n_b * H; k += WARPS * 32) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pmb) + k);
+        wt[k] = ml.x;
+        lv[k] = ml.y;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    for (int head = tid; head < H; head += WARPS * 32) {
+        float M = -INFINITY;
+        for (int i = 0; i < n_b; ++i) M = fmaxf(M, wt[i * H + head]);
+        float d = 0.f;
+        for (int i = 0; i < n_b; ++i) {
+            const float w = exp2f(wt[i * H + head] - M);
+            wt[i * H + head] = w;
+            d += w * lv[i * H + head];
+        }
+        den[head] = d;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    // every output of this thread accumulates together, so each split's loads are in flight at once
+    constexpr int OPT = (H * DH + WARPS * 32 - 1) / (WARPS * 32);
+    float num[OPT];
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) num[k] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < n_b; ++i) {
+        const float *pi = pob + (size_t)i * H * DH;
+#pragma unroll
+        for (int k = 0; k < OPT; ++k) {
+            const int idx = tid + k * WARPS * 32;
+            if (idx < H * DH) num[k] += wt[i * H + idx / DH] * __ldcg(pi + idx);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+        const int idx = tid + k * WARPS * 32;
+        if (idx < H * DH) {
+            const float d = den[idx / DH];
+            a.out[(size_t)b * H * DH + idx] = d > 0.f ? a.out_scale * num[k] / d : 0.f;
+        }
+    }
+    if (tid == 0) a.counters[b] = 0;                 // ready for the next call
+    return;
+    }  // global merge
+    }  // consumers
+
+    // ---- cluster merge: the CTAs of a cluster are the splits of one sequence. Each
+    // keeps its merged partial in shared memory; after a cluster barrier every CTA
+    // combines a slice of the outputs, reading its peers' partials over DSMEM.
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();
+    if (warp < WARPS) {
+        const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+        const int per = (H * DH + C - 1) / C;
+        const int lo = rank * per, hi = min(H * DH, lo + per);
+        float *cpl = reinterpret_cast<float *>(smem) + SLICES * H * DH + SLICES * H * 2;
+        for (int idx = lo + tid; idx < hi; idx += WARPS * 32) {
+            const int head = idx / DH;
+            float M = -INFINITY;
+            for (int r = 0; r < C; ++r) M = fmaxf(M, cl.map_shared_rank(cpl, r)[H * DH + head]);
+            float num = 0.f, den = 0.f;
+            for (int r = 0; r < C; ++r) {
+                const float *rp = cl.map_shared_rank(cpl, r);
+                const float m = rp[H * DH + head];
+                const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+                num += w * rp[idx];
+                den += w * rp[H * DH + H + head];
+            }
+            a.out[(size_t)b * H * DH + idx] = den > 0.f ? a.out_scale * num / den : 0.f;
+        }
+    }
+    cl.sync();                                       // peers read this CTA's shared memory
 }
 
 template <class C>
-cudaError_t launch_cfg(int batch, const void *q, const int32_t *q_pos, const void *kc,
-                       const void *vc, int cap, const int32_t *seq_len, int max_len, float qscale,
-                       const DecodePlan &p, float *part_o, float *part_ml, const RopeTable &rope,
-                       int *err, const DecodeTestHooks &hooks, cudaStream_t st) {
-    auto kern = decode_mma_kernel<C>;
+cudaError_t launch_cfg(const DecodeArgs &args, int batch, const DecodePlan &p, const RopeTable &rope,
+                       const DecodeTestHooks &hooks, cudaStream_t st) {
     const size_t smem = C::smem_bytes();
-    cudaError_t e = ensure_dynamic_smem(kern, smem);
+    cudaError_t e = ensure_dynamic_smem<decode_mma_kernel<C>>(smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)p.n_split, (unsigned)batch);
-    kern<<<grid, (C::WARPS + 1) * 32, smem, st>>>(
-        (const __nv_bfloat16 *)q, q_pos, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc, cap,
-        seq_len, max_len, qscale, p.tokens_per_split, p.n_split, part_o, part_ml, rope, err, hooks);
-    return cudaGetLastError();
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)p.n_split, (unsigned)batch);
+    lc.blockDim = dim3((C::WARPS + 1) * 32);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = args.cluster ? (unsigned)p.n_split : 1u;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 2;
+    return cudaLaunchKernelEx(&lc, decode_mma_kernel<C>, args, rope, hooks);
+}
+
+// Can a cluster of `size` CTAs of this variant run on this device?
+template <class C>
+int cluster_ok_cfg(int size) {
+    const size_t smem = C::smem_bytes();
+    if (ensure_dynamic_smem<decode_mma_kernel<C>>(smem) != cudaSuccess) return 0;
+    if (size > 8 &&
+        cudaFuncSetAttribute(decode_mma_kernel<C>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)size, 1);
+    lc.blockDim = dim3((C::WARPS + 1) * 32);
+    lc.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)size;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<C>, &lc) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
 }  // namespace
 
-cudaError_t launch_decode_mma(int variant, int batch, const void *q, const int32_t *q_pos,
-                              const void *kc, const void *vc, int cap, const int32_t *seq_len,
-                              int max_len, float qscale, const DecodePlan &plan, float *part_o,
-                              float *part_ml, const RopeTable &rope, int *err,
-                              const DecodeTestHooks &hooks, cudaStream_t st) {
+int mma_decode_max_clusters(int variant, int size) {
     switch (variant) {
-#define KPA_MMA_CASE(IDX, CFG)                                                                     \
-    case IDX:                                                                                      \
-        return launch_cfg<CFG>(batch, q, q_pos, kc, vc, cap, seq_len, max_len, qscale, plan, part_o, \
-                               part_ml, rope, err, hooks, st);
+#define KPA_MMA_CL(IDX, CFG) \
+    case IDX:                \
+        return cluster_ok_cfg<CFG>(size);
+        KPA_MMA_VARIANTS(KPA_MMA_CL)
+#undef KPA_MMA_CL
+        default:
+            return 0;
+    }
+}
+
+cudaError_t launch_decode_mma(int variant, const DecodeArgs &args, int batch, const DecodePlan &plan,
+                              const RopeTable &rope, const DecodeTestHooks &hooks, cudaStream_t st) {
+    switch (variant) {
+#define KPA_MMA_CASE(IDX, CFG) \
+    case IDX:                  \
+        return launch_cfg<CFG>(args, batch, plan, rope, hooks, st);
         KPA_MMA_VARIANTS(KPA_MMA_CASE)
 #undef KPA_MMA_CASE
         default:

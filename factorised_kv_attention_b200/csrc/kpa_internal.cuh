@@ -62,17 +62,18 @@ __device__ __forceinline__ void rope_cs(double pos, double theta, float &c, floa
     s = (float)sn;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device (so later calls,
-// including ones made while a stream is being captured, launch directly).
-template <typename Kernel>
-inline cudaError_t ensure_dynamic_smem(Kernel kern, size_t bytes) {
+// Raise a kernel's dynamic shared-memory limit once per device and kernel (so
+// later calls, including ones made while a stream is being captured, launch
+// directly).  The kernel is a template argument: one cache per kernel.
+template <auto Kernel>
+inline cudaError_t ensure_dynamic_smem(size_t bytes) {
     static std::atomic<int> granted[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (bytes <= 48 * 1024 || (size_t)granted[dev].load() >= bytes) return cudaSuccess;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess) granted[dev].store((int)bytes);
     return e;
 }
@@ -87,11 +88,19 @@ cudaError_t launch_append_factors(const Dims &d, kpa_dtype dt, int batch, int n_
                                   cudaStream_t st);
 
 struct DecodePlan {
+    int variant;         // tensor-core kernel variant, or -1 for the CUDA-core kernel
     int tokens_per_split;
     int n_split;         // splits per sequence (grid x)
     int tile;            // tokens per shared-memory tile
-    size_t part_o_off, part_ml_off, bytes;
+    int fused;           // the decode kernel merges the splits itself (no combine launch)
+    int cluster;         // ... through a thread-block cluster per sequence (DSMEM)
+    size_t part_o_off, part_ml_off, counters_off, bytes;
 };
+
+// Byte range of the per-sequence counters inside a decode workspace (they must be
+// zero before a call and are zero again after every call that completes).
+kpa_status decode_counter_region(const kpa_config *cfg, int batch, int max_len, size_t *offset,
+                                 size_t *bytes);
 
 cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void *q,
                               const int32_t *q_pos, const void *kc, const void *vc, int cap,

@@ -14,6 +14,26 @@ struct DecodeTestHooks {
     unsigned long long wait_limit_ns;
 };
 
+// Arguments of one decode launch (device pointers into the caller's buffers).
+struct DecodeArgs {
+    const __nv_bfloat16 *q;
+    const int32_t *q_pos;
+    const __nv_bfloat16 *kc, *vc;
+    int cap;
+    const int32_t *seq_len;
+    int max_len;
+    float qscale;       // sm_scale / R_K * log2(e)
+    int tps;            // slots per split
+    int n_split;        // splits per sequence (grid x)
+    float *part_o, *part_ml;
+    int *counters;      // [batch] finished splits, zero between calls
+    float *out;
+    float out_scale;    // 1 / R_V
+    int fused;          // the last CTA of a sequence combines its splits
+    int cluster;        // the splits of a sequence form one cluster and merge over DSMEM
+    int *err;
+};
+
 // One instantiation per (split, ranks) family.
 //   MA = h1*d1 (rows of the per-i2 GEMMs), D1, D2, RK, RV, H2 = h2,
 //   SLICES  token slices per CTA (warps = H2 * SLICES),
@@ -27,14 +47,24 @@ struct MmaDecodeCfg {
     static constexpr int WARPS = H2 * SLICES;
     static constexpr int TT = 16 * CHUNKS * SLICES;             // tokens per stage
     static constexpr int STAGE_BYTES = TT * (EK + EV) * 2;
-    static constexpr size_t smem_bytes() {
-        return (size_t)STAGES * STAGE_BYTES + 16 * STAGES + (size_t)H * DH * 4 + 16;
-    }
+    // per-warp scratch for the sum over j1 (d1 > 1): [16 tokens][MA + 4] partials,
+    // [h1][16] weights, [h1] rescale factors
+    static constexpr int RED_LD = MA + 4;
+    static constexpr int PPL = D1 > 1 ? (H1 * 16) / 32 : 0;      // (head, token) pairs per lane
+    static constexpr int SCR_FLOATS = D1 > 1 ? ((16 * RED_LD + H1 * 16 + H1 + 3) / 4) * 4 : 0;
+    static constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
+    static constexpr size_t OFF_Q = OFF_BARS + 16 * STAGES;
+    static constexpr size_t OFF_CS = OFF_Q + (size_t)H * DH * 4;
+    static constexpr size_t OFF_SCR = (OFF_CS + (size_t)(D2 / 2) * 8 + 15) / 16 * 16;
+    static constexpr size_t OFF_FLAGS = OFF_SCR + (size_t)WARPS * SCR_FLOATS * 4;
+    static constexpr size_t smem_bytes() { return OFF_FLAGS + 16; }
     static_assert(MA % 16 == 0, "h1*d1 must be a multiple of 16");
     static_assert(D2 % 16 == 0, "d2 must be a multiple of 16");
     static_assert(D1 == 1 || D1 == 2 || D1 == 4 || D1 == 8 || D1 == 16, "d1 must be 1..16, a power of 2");
-    static_assert((size_t)SLICES * H * DH * 4 + (size_t)SLICES * H * 8 <= (size_t)STAGES * STAGE_BYTES,
-                  "slice merge must fit in the ring");
+    static_assert(D1 == 1 || (H1 >= 2 && 32 % H1 == 0), "h1 must divide 32 when d1 > 1");
+    static_assert((size_t)SLICES * H * DH * 4 + (size_t)SLICES * H * 8 + (size_t)H * DH * 4 + H * 8 <=
+                      (size_t)STAGES * STAGE_BYTES,
+                  "slice merge and merged partial must fit in the ring");
     static_assert(WARPS <= 31, "too many consumer warps");
     static_assert(smem_bytes() <= 227 * 1024, "shared memory");
 };
@@ -73,10 +103,19 @@ inline int mma_decode_tile(int variant) {
     return 0;
 }
 
-cudaError_t launch_decode_mma(int variant, int batch, const void *q, const int32_t *q_pos,
-                              const void *kc, const void *vc, int cap, const int32_t *seq_len,
-                              int max_len, float qscale, const DecodePlan &plan, float *part_o,
-                              float *part_ml, const RopeTable &rope, int *err,
-                              const DecodeTestHooks &hooks, cudaStream_t st);
+inline size_t mma_decode_smem(int variant) {
+#define KPA_MMA_SMEM(IDX, CFG) \
+    if (variant == IDX) return CFG::smem_bytes();
+    KPA_MMA_VARIANTS(KPA_MMA_SMEM)
+#undef KPA_MMA_SMEM
+    return 0;
+}
+
+// Number of clusters of `size` CTAs of a variant that fit on the current device at
+// once (0: a cluster that large cannot run).
+int mma_decode_max_clusters(int variant, int size);
+
+cudaError_t launch_decode_mma(int variant, const DecodeArgs &args, int batch, const DecodePlan &plan,
+                              const RopeTable &rope, const DecodeTestHooks &hooks, cudaStream_t st);
 
 }  // namespace kpa

@@ -12,8 +12,9 @@
 // name as a device address: the first call on each device looks the address up
 // with cudaGetSymbolAddress (with that device current) and caches it; later
 // calls reuse it.  All calls on a device share the array and it keeps the
-// previous call's contents, which the decode never reads before writing, so
-// nothing in it has to start at zero.  Calls whose work overlaps on the GPU
+// previous call's contents; the only part that must start at zero, the
+// per-sequence completion counters, is cleared on the stream before every call.
+// Calls whose work overlaps on the GPU
 // (other streams, other threads) race on the array and must be serialised by
 // the caller.
 #include <mutex>
@@ -65,6 +66,19 @@ extern "C" kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, c
     void *scratch = nullptr;
     s = scratch_address(&scratch);
     if (s != KPA_OK) return s;
+    // the decode's per-sequence counters must start at zero; an earlier call that
+    // stopped on a device error may have left them set
+    size_t off = 0, count_bytes = 0;
+    s = kpa::decode_counter_region(cfg, batch, max_len, &off, &count_bytes);
+    if (s != KPA_OK) return s;
+    if (batch > 0 && count_bytes > 0) {
+        cudaError_t e = cudaMemsetAsync(static_cast<char *>(scratch) + off, 0, count_bytes,
+                                        (cudaStream_t)stream);
+        if (e != cudaSuccess) {
+            kpa::record_cuda_error(e);
+            return KPA_ERR_CUDA;
+        }
+    }
     return kpa_decode_split(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len,
                             sm_scale, 0, out, scratch, (size_t)KPA_DECODE_NOALLOC_MAX_BYTES, stream);
 }

@@ -126,8 +126,10 @@ kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32
  *                             KPA_ERR_DEVICE_CHECK
  *   sm_scale softmax scale applied to q.k (usually 1/sqrt(d_h))
  *   out      [batch][h][d_h] float32; a sequence with seq_len 0 gets zeros
- *   workspace at least kpa_decode_workspace_size(cfg, batch, max_len, 0) bytes;
- *            its contents need no initialisation and are scratch between calls
+ *   workspace at least kpa_decode_workspace_size(cfg, batch, max_len, 0) bytes,
+ *            256-byte aligned, zero-filled before its first use (cudaMemsetAsync);
+ *            every call that completes without a device error leaves it ready for
+ *            the next one (after an error, zero it again)
  * Results are deterministic for a given (batch, max_len). */
 kpa_status kpa_decode(const kpa_config *cfg, int32_t batch, const void *q, const int32_t *q_pos,
                       const void *kcache, const void *vcache, int32_t capacity,
@@ -200,6 +202,14 @@ kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, const void *
                               const int32_t *q_pos, const void *kcache, const void *vcache,
                               int32_t capacity, const int32_t *seq_len, int32_t max_len,
                               float sm_scale, float *out, kpa_stream stream);
+
+/* Testing only: make the tensor-core decode's bounded waits observable.
+ * Every bounded wait on the device gives up after wait_limit_ns (default 1 s)
+ * and reports KPA_ERR_TIMEOUT; with skip_tile >= 0 the CTA of split
+ * `skip_split` of sequence 0 never issues the copy of its tile `skip_tile`, so
+ * its consumers' wait runs out.  (-1, -1, 1000000000) restores the defaults.
+ * Process-wide; not for concurrent use with real work. */
+kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split, uint64_t wait_limit_ns);
 
 /* Wait for `stream`, then return in *code the per-device error word
  * (KPA_OK, KPA_ERR_TIMEOUT or KPA_ERR_DEVICE_CHECK) of the current device and

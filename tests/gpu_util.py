@@ -58,7 +58,7 @@ def run_decode(lib, w, cfg, kc, vc, q, seq_len, q_pos, *, max_len=None, sm_scale
     max_len = int(seq_len.max().item()) if max_len is None else max_len
     sm_scale = 1.0 / float(np.sqrt(s.dh)) if sm_scale is None else sm_scale
     ws_bytes = lib.kpa_decode_workspace_size(cfg, w.batch, max_len, tokens_per_split)
-    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
     out = torch.full((w.batch, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
     lib.kpa_decode_split(cfg, w.batch, q.cuda().contiguous(),
                          None if q_pos is None else q_pos.cuda().contiguous(), kc, vc, w.capacity,
