@@ -353,16 +353,47 @@ kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32
     kpa_status s = check_cfg(cfg, true, true);
     if (s != KPA_OK) return s;
     if (!bytes || batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
-    *bytes = 0;
-    return KPA_ERR_UNSUPPORTED;
+    const int64_t eq = (int64_t)cfg->r_q * (cfg->h1 * cfg->d1 + cfg->h2 * cfg->d2);
+    *bytes = align256((size_t)eq * batch * n_tok * sizeof(float));
+    return KPA_OK;
 }
 
-kpa_status kpa_append(const kpa_config *cfg, int32_t, int32_t, const void *, const void *,
-                      const int32_t *, int32_t, void *, void *, void *, void *, size_t,
-                      kpa_stream) {
+kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *x,
+                      const void *w, const int32_t *start_pos, int32_t capacity, void *kcache,
+                      void *vcache, void *q_out, void *workspace, size_t ws_bytes,
+                      kpa_stream stream) {
     kpa_status s = check_cfg(cfg, true, true);
     if (s != KPA_OK) return s;
-    return KPA_ERR_UNSUPPORTED;
+    if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
+    if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
+    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    // TMA rows of x and W are d_model bf16 values: a multiple of 16 bytes
+    if (cfg->d_model % 8 != 0) return KPA_ERR_UNSUPPORTED;
+    // factor pairs (2m, 2m+1) of B must start on even columns of the projection
+    if ((cfg->h1 * cfg->d1) % 2 != 0 && (cfg->r_q % 2 != 0 || cfg->r_k % 2 != 0 || cfg->r_v % 2 != 0))
+        return KPA_ERR_UNSUPPORTED;
+    if (batch == 0 || n_tok == 0) return KPA_OK;
+    if ((int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
+    if (!x || !w || !start_pos || !kcache || !vcache) return KPA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(kcache) || !aligned16(vcache) ||
+        !aligned16(q_out) || (reinterpret_cast<uintptr_t>(start_pos) & 3))
+        return KPA_ERR_INVALID_ARG;
+    const Dims d = dims_of(cfg);
+    const size_t smem = append_smem_bytes(append_tile_n(cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) + d.ek + d.ev),
+                                          2, d.d2);
+    if (smem > 227 * 1024) return KPA_ERR_UNSUPPORTED;
+    size_t need = 0;
+    s = kpa_append_workspace_size(cfg, batch, n_tok, &need);
+    if (s != KPA_OK) return s;
+    if (q_out && (!workspace || ws_bytes < need)) return KPA_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255)) return KPA_ERR_INVALID_ARG;
+    int *err = nullptr;
+    s = device_state(&err, nullptr);
+    if (s != KPA_OK) return s;
+    cudaError_t e = launch_append(d, cfg->r_q, cfg->d_model, batch, n_tok, x, w, start_pos, capacity,
+                                  kcache, vcache, q_out, static_cast<float *>(workspace), rope_table(cfg),
+                                  err, current_hooks().wait_limit_ns, (cudaStream_t)stream);
+    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 
 kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split,

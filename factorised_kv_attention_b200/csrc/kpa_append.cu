@@ -1,0 +1,334 @@
+// kpa_append.cu -- the append step: merged factor projection on the tcgen05 tensor
+// cores, factor RoPE and the cache write in its epilogue, then the query assembly.
+//
+// "Kronecker Product Attention", eq 5 with the ranks merged: every output column of
+// F = X W^T is one factor element of one token, the columns ordered
+// [A^Q | B^Q | A^K | B^K | A^V | B^V] (rank-major inside each part).  The GEMM
+// epilogue applies R_theta^(2)(pos) to the B^Q and B^K pairs (Theorem 2.4: the
+// rotation of the reconstruction is the rotation of B alone), writes the key and
+// value factors to their cache slots in bf16, and keeps the query factors in fp32
+// for the assembly Q = (1/R_Q) sum_r A^Q_r (x) B~^Q_r (eq 2), done by a second kernel.
+//
+// GEMM: 128 x BN output tiles (BN <= 256, a multiple of 16), K in steps of 64.  Warp 0
+// issues TMA loads of X and W tiles (128-byte swizzle) into a STAGES-deep ring; one
+// thread of warp 1 issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into a TMEM
+// accumulator and commits each stage back to the producer; warps 2..5 read the
+// accumulator rows from TMEM (one row = one token per thread) and run the epilogue.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kpa_internal.cuh"
+#include "kpa_sm100.cuh"
+
+namespace kpa {
+
+struct AppendArgs {
+    int M, N, K;                 // tokens, projected factor columns, d_model
+    int BN, n_kblocks, stages;
+    int n_tok, cap;
+    const int32_t *start_pos;
+    int h1, h2, d1, d2, rq, rk, rv;
+    int eq, ek, ev;              // elements per query / key / value record
+    __nv_bfloat16 *kc, *vc;
+    float *qf;                   // [eq][M] query factors (B^Q rotated), or null
+    int *err;
+    unsigned long long wait_limit_ns;
+};
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BK = 64;
+constexpr int kThreads = 192;                 // producer, MMA, 4 epilogue warps
+constexpr uint32_t kTmemCols = 256;
+
+__device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap, int E, int s, int e,
+                                            float v) {
+    plane[(((int64_t)b * (cap / kGroup) + s / kGroup) * E + e) * kGroup + (s % kGroup)] =
+        __float2bfloat16_rn(v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
+                   AppendArgs a, RopeTable rope) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int S = a.stages, BN = a.BN;
+    const uint32_t a_bytes = BM * BK * 2, b_bytes = (uint32_t)BN * BK * 2;
+    unsigned char *a_st = smem;                                   // S x 16 KB
+    unsigned char *b_st = a_st + (size_t)S * a_bytes;             // S x BN*128 B
+    uint64_t *bars = reinterpret_cast<uint64_t *>(b_st + (size_t)S * b_bytes);   // full, empty, acc
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float2 *cs_all = reinterpret_cast<float2 *>(reinterpret_cast<unsigned char *>(bars) + 256);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile_n = blockIdx.x, tile_m = blockIdx.y;
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * S, accf = full0 + 16 * S;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(accf, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_desc(&tmx);
+        tma_prefetch_desc(&tmw);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t limit = a.wait_limit_ns;
+
+    if (warp == 0) {
+        // ---- producer: TMA tiles of X (rows tile_m) and W (rows tile_n), 64 K columns each
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < a.n_kblocks; ++kb) {
+                const int s = kb % S;
+                if (kb >= S && !mbar_wait(empty0 + 8 * s, ((kb / S) - 1) & 1, limit)) {
+                    raise_error(a.err, kErrTimeout);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_expect_tx(full0 + 8 * s, a_bytes + b_bytes);
+                tma_load_2d(smem_u32(a_st + (size_t)s * a_bytes), &tmx, kb * BK, tile_m * BM, full0 + 8 * s);
+                tma_load_2d(smem_u32(b_st + (size_t)s * b_bytes), &tmw, kb * BK, tile_n * BN, full0 + 8 * s);
+                issued = kb + 1;
+            }
+            // every copy issued must land before the CTA exits (normally already consumed)
+            if (*abort_flag)
+                for (int kb = max(0, issued - S); kb < issued; ++kb)
+                    if (!mbar_wait(full0 + 8 * (kb % S), (kb / S) & 1, limit)) raise_error(a.err, kErrTimeout);
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer: one thread drives the tensor cores
+        if (lane == 0) {
+            const uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+            bool ok = true;
+            for (int kb = 0; kb < a.n_kblocks; ++kb) {
+                const int s = kb % S;
+                if (!mbar_wait(full0 + 8 * s, (kb / S) & 1, limit)) {
+                    raise_error(a.err, kErrTimeout);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = umma_desc_k_sw128(smem_u32(a_st + (size_t)s * a_bytes));
+                const uint64_t bd = umma_desc_k_sw128(smem_u32(b_st + (size_t)s * b_bytes));
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)     // K = 16 per instruction: 32 B along the row
+                    umma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc, kb > 0 || k > 0);
+                umma_commit(empty0 + 8 * s);          // stage free once these MMAs finish
+            }
+            umma_commit(accf);                        // after every MMA issued (also on abort)
+        }
+    } else {
+        // ---- epilogue: thread = accumulator row = token
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int m = tile_m * BM + row;
+        const bool live = m < a.M;
+        int b = 0, s = 0;
+        bool slot_ok = false;
+        const int half = a.d2 / 2;
+        float2 *cs = cs_all + (size_t)row * half;
+        if (live) {
+            b = m / a.n_tok;
+            const int t = m - b * a.n_tok;
+            s = a.start_pos[b] + t;
+            slot_ok = s >= 0 && s < a.cap;
+            if (!slot_ok) raise_error(a.err, kErrDeviceCheck);
+            for (int j = 0; j < half; ++j) {
+                float c, sn;
+                rope_cs((double)s, rope.theta[j], c, sn);
+                cs[j] = make_float2(c, sn);
+            }
+        }
+        const bool acc_ok = mbar_wait(accf, 0, limit) && !*abort_flag;
+        if (!acc_ok) raise_error(a.err, kErrTimeout);
+        tc_fence_after();
+        const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1, va = a.rv * a.h1 * a.d1;
+        for (int ch = 0; ch < BN / 16; ++ch) {
+            float v[16];
+            tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16, v);   // warp-collective
+            if (!live || !acc_ok) continue;
+            const int n0 = tile_n * BN + ch * 16;
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                const int n = n0 + j;
+                if (n >= a.N) break;
+                float x0 = v[j], x1 = v[j + 1];
+                if (n < a.eq) {                                    // query factors
+                    if (n >= qa) {                                 // B^Q: rotate the pair
+                        const float2 w = cs[((n - qa) % a.d2) >> 1];
+                        const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
+                        x0 = y0;
+                        x1 = y1;
+                    }
+                    if (a.qf) {
+                        a.qf[(size_t)n * a.M + m] = x0;
+                        a.qf[(size_t)(n + 1) * a.M + m] = x1;
+                    }
+                } else if (n < a.eq + a.ek) {                      // key factors
+                    const int e = n - a.eq;
+                    if (e >= ka) {                                 // B^K: rotate the pair
+                        const float2 w = cs[((e - ka) % a.d2) >> 1];
+                        const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
+                        x0 = y0;
+                        x1 = y1;
+                    }
+                    if (slot_ok) {
+                        store_cache(a.kc, b, a.cap, a.ek, s, e, x0);
+                        store_cache(a.kc, b, a.cap, a.ek, s, e + 1, x1);
+                    }
+                } else {                                           // value factors, never rotated
+                    const int e = n - a.eq - a.ek;
+                    (void)va;
+                    if (slot_ok) {
+                        store_cache(a.vc, b, a.cap, a.ev, s, e, x0);
+                        store_cache(a.vc, b, a.cap, a.ev, s, e + 1, x1);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// q_out[m][(i1,i2)][(j1,j2)] = (1/R_Q) sum_r A^Q_r[i1,j1] * B~^Q_r[i2,j2]; one thread per
+// (token, head), threads of a block are consecutive tokens of one head.
+__global__ void __launch_bounds__(128)
+q_assemble_kernel(const float *__restrict__ qf, int M, int h1, int h2, int d1, int d2, int rq,
+                  __nv_bfloat16 *__restrict__ q_out) {
+    extern __shared__ float sh[];
+    const int head = blockIdx.y;
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    const int i1 = head / h2, i2 = head % h2;
+    const int h = h1 * h2, dh = d1 * d2;
+    const int qa = rq * h1 * d1;
+    float *A = sh + (size_t)threadIdx.x * rq * (d1 + d2);       // [rq][d1]
+    float *B = A + rq * d1;                                     // [rq][d2]
+    if (m >= M) return;
+    for (int r = 0; r < rq; ++r) {
+        for (int j1 = 0; j1 < d1; ++j1) A[r * d1 + j1] = qf[(size_t)(r * h1 * d1 + i1 * d1 + j1) * M + m];
+        for (int j2 = 0; j2 < d2; ++j2) B[r * d2 + j2] = qf[(size_t)(qa + r * h2 * d2 + i2 * d2 + j2) * M + m];
+    }
+    const float inv = 1.0f / (float)rq;
+    __nv_bfloat16 *dst = q_out + ((size_t)m * h + head) * dh;
+    for (int j1 = 0; j1 < d1; ++j1)
+        for (int j2 = 0; j2 < d2; j2 += 2) {
+            float s0 = 0.f, s1 = 0.f;
+            for (int r = 0; r < rq; ++r) {
+                const float av = A[r * d1 + j1];
+                s0 += av * B[r * d2 + j2];
+                s1 += av * B[r * d2 + j2 + 1];
+            }
+            *reinterpret_cast<__nv_bfloat162 *>(dst + j1 * d2 + j2) = __floats2bfloat162_rn(s0 * inv, s1 * inv);
+        }
+}
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), boxes of 64 columns x box_rows rows,
+// 128-byte swizzle; elements outside the tensor read as zero.
+bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t append_smem_bytes(int BN, int stages, int d2) {
+    return 1024 + (size_t)stages * (BM * BK * 2 + (size_t)BN * BK * 2) + 256 + (size_t)BM * (d2 / 2) * 8;
+}
+
+int append_tile_n(int N) {
+    const int tiles = (N + 255) / 256;
+    const int per = (N + tiles - 1) / tiles;
+    return ((per + 15) / 16) * 16;
+}
+
+cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_tok, const void *x,
+                          const void *w, const int32_t *start_pos, int cap, void *kc, void *vc,
+                          void *q_out, float *qf, const RopeTable &rope, int *err,
+                          unsigned long long wait_limit_ns, cudaStream_t st) {
+    AppendArgs a;
+    a.M = batch * n_tok;
+    a.eq = rq * (d.h1 * d.d1 + d.h2 * d.d2);
+    a.ek = d.ek;
+    a.ev = d.ev;
+    a.N = a.eq + a.ek + a.ev;
+    a.K = d_model;
+    a.BN = append_tile_n(a.N);
+    a.n_kblocks = (d_model + BK - 1) / BK;
+    a.stages = 4;
+    while (a.stages > 2 && append_smem_bytes(a.BN, a.stages, d.d2) > 227 * 1024) --a.stages;
+    if (append_smem_bytes(a.BN, a.stages, d.d2) > 227 * 1024) return cudaErrorInvalidValue;
+    a.n_tok = n_tok;
+    a.cap = cap;
+    a.start_pos = start_pos;
+    a.h1 = d.h1; a.h2 = d.h2; a.d1 = d.d1; a.d2 = d.d2;
+    a.rq = rq; a.rk = d.rk; a.rv = d.rv;
+    a.kc = static_cast<__nv_bfloat16 *>(kc);
+    a.vc = static_cast<__nv_bfloat16 *>(vc);
+    a.qf = q_out ? qf : nullptr;
+    a.err = err;
+    a.wait_limit_ns = wait_limit_ns;
+
+    CUtensorMap tmx, tmw;
+    if (!make_map(&tmx, x, (uint64_t)a.M, (uint64_t)d_model, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tmw, w, (uint64_t)a.N, (uint64_t)d_model, (uint32_t)a.BN)) return cudaErrorInvalidValue;
+    const size_t smem = append_smem_bytes(a.BN, a.stages, d.d2);
+    cudaError_t e = ensure_dynamic_smem<append_gemm_kernel>(smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((a.N + a.BN - 1) / a.BN), (unsigned)((a.M + BM - 1) / BM));
+    append_gemm_kernel<<<grid, kThreads, smem, st>>>(tmx, tmw, a, rope);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !q_out) return e;
+    const size_t qsm = (size_t)128 * rq * (d.d1 + d.d2) * sizeof(float);
+    e = ensure_dynamic_smem<q_assemble_kernel>(qsm);
+    if (e != cudaSuccess) return e;
+    dim3 g2((unsigned)((a.M + 127) / 128), (unsigned)d.h);
+    q_assemble_kernel<<<g2, 128, qsm, st>>>(qf, a.M, d.h1, d.h2, d.d1, d.d2, rq,
+                                            static_cast<__nv_bfloat16 *>(q_out));
+    return cudaGetLastError();
+}
+
+}  // namespace kpa
