@@ -336,16 +336,38 @@ kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int3
     kpa_status s = check_cfg(cfg, false, false);
     if (s != KPA_OK) return s;
     if (!bytes || batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
-    *bytes = 0;
-    return KPA_ERR_UNSUPPORTED;
+    *bytes = 0;                                  // K/V tiles live on chip only
+    return KPA_OK;
 }
 
-kpa_status kpa_prefill(const kpa_config *cfg, int32_t, int32_t, const void *, const int32_t *,
-                       const void *, const void *, int32_t, float, float *, void *, size_t,
-                       kpa_stream) {
+kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *q,
+                       const int32_t *start_pos, const void *kcache, const void *vcache,
+                       int32_t capacity, float sm_scale, float *out, void *workspace,
+                       size_t ws_bytes, kpa_stream stream) {
+    (void)workspace;
+    (void)ws_bytes;
     kpa_status s = check_cfg(cfg, false, false);
     if (s != KPA_OK) return s;
-    return KPA_ERR_UNSUPPORTED;
+    if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
+    if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
+    if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
+    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    const Dims d = dims_of(cfg);
+    if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
+    if (batch == 0 || n_tok == 0) return KPA_OK;
+    if (batch > 65535 || d.h > 65535 || (int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
+    if (!q || !start_pos || !kcache || !vcache || !out) return KPA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(start_pos) & 3))
+        return KPA_ERR_INVALID_ARG;
+    int *err = nullptr;
+    s = device_state(&err, nullptr);
+    if (s != KPA_OK) return s;
+    const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
+    cudaError_t e = launch_prefill(d, batch, n_tok, q, start_pos, kcache, vcache, capacity, qscale,
+                                   (float)(1.0 / (double)d.rv), out, err, current_hooks().wait_limit_ns,
+                                   (cudaStream_t)stream);
+    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 
 kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,

@@ -1,0 +1,112 @@
+"""kpa_prefill (causal attention with K/V rebuilt on chip from the factors, tcgen05)
+against the float64 oracle, and the append + prefill + decode-step chain of the
+append+prefill configuration (GPU)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_bf16_close, kpa, natural, planes, run_decode
+from workloads import APPEND_PREFILL, KPA_MEDIUM, Shape, append_inputs, decode_inputs, to_f64
+
+pytestmark = pytest.mark.gpu
+
+SHAPE = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, rope_base=10000.0)
+
+
+def _prefill(lib, cfg, batch, n_tok, q, start, kc, vc, cap, sm_scale):
+    out = torch.full((batch, n_tok, q.shape[2], q.shape[3]), float("nan"), dtype=torch.float32, device="cuda")
+    lib.kpa_prefill(cfg, batch, n_tok, q.cuda().contiguous(), start.cuda(), kc, vc, cap, sm_scale, out)
+    return out
+
+
+@pytest.mark.parametrize("starts,n_tok", [([0, 0], 256), ([0, 37], 200), ([5, 300], 130)])
+def test_prefill_against_oracle(starts, n_tok):
+    """Random factors in the cache (earlier context + the chunk), random rotated q."""
+    lib = kpa()
+    s = SHAPE
+    batch, cap = len(starts), 512
+    w = KPA_MEDIUM.replace(shape=s, batch=batch, capacity=cap, ragged=(), length=cap,
+                           factor_std=1.0 / np.sqrt(2.0), seed=41)
+    inp = decode_inputs(w)
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, batch, cap, "bf16")
+    zero = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    lib.kpa_append_factors(cfg, batch, cap, inp["kf"].cuda(), inp["vf"].cuda(), zero, cap, kc, vc)
+    rng = np.random.default_rng(7)
+    q = torch.from_numpy((rng.standard_normal((batch, n_tok, s.h, s.dh)) * 0.3).astype(np.float32)).to(torch.bfloat16)
+    start = torch.tensor(starts, dtype=torch.int32)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = _prefill(lib, cfg, batch, n_tok, q, start, kc, vc, cap, scale)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    kn = to_f64(natural(kc.cpu(), batch, cap, s.e_k))
+    vn = to_f64(natural(vc.cpu(), batch, cap, s.e_v))
+    want = oracle.prefill(s, to_f64(q), kn, vn, starts, keys_rotated=True, sm_scale=scale)
+    assert_bf16_close(out.cpu().numpy(), want, f"prefill starts={starts} n={n_tok}")
+
+
+def test_prefill_rows_match_decode():
+    """Row t of a prefill equals a decode of length start + t + 1 (both on the GPU)."""
+    lib = kpa()
+    s = SHAPE
+    batch, cap, n_tok = 2, 512, 160
+    w = KPA_MEDIUM.replace(shape=s, batch=batch, capacity=cap, ragged=(), length=cap, seed=42)
+    inp = decode_inputs(w)
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, batch, cap, "bf16")
+    zero = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    lib.kpa_append_factors(cfg, batch, cap, inp["kf"].cuda(), inp["vf"].cuda(), zero, cap, kc, vc)
+    q = (torch.randn(batch, n_tok, s.h, s.dh, generator=torch.Generator().manual_seed(3)) * 0.3).to(torch.bfloat16)
+    start = torch.tensor([0, 100], dtype=torch.int32)
+    scale = 1.0 / np.sqrt(s.dh)
+    pre = _prefill(lib, cfg, batch, n_tok, q, start, kc, vc, cap, scale).cpu().numpy()
+    for t in (0, 1, 63, 127, 128, 159):
+        L = start + t + 1
+        dec = run_decode(lib, w, cfg, kc, vc, q[:, t], L, None, max_len=int(L.max()), sm_scale=scale)
+        assert_bf16_close(pre[:, t], dec.cpu().numpy(), f"row {t}")
+
+
+def test_append_prefill_decode_chain_full_config():
+    """Configuration 5: append the 2048-token chunk (projection, RoPE, cache write),
+    causal prefill from q_out, then one decode step at position 2048; sampled rows
+    against the oracle fed with the GPU's bf16 q_out and cache."""
+    lib = kpa()
+    w = APPEND_PREFILL
+    s = w.shape
+    inp = append_inputs(w)
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, w.batch, w.capacity, "bf16")
+    start = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(lib.kpa_append_workspace_size(cfg, w.batch, w.n_tok), dtype=torch.uint8, device="cuda")
+    q_out = torch.empty(w.batch, w.n_tok, s.h, s.dh, dtype=torch.bfloat16, device="cuda")
+    lib.kpa_append(cfg, w.batch, w.n_tok, inp["x"].cuda(), inp["W"].cuda(), start, w.capacity, kc, vc, q_out, ws)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = torch.empty(w.batch, w.n_tok, s.h, s.dh, dtype=torch.float32, device="cuda")
+    lib.kpa_prefill(cfg, w.batch, w.n_tok, q_out, start, kc, vc, w.capacity, scale, out)
+    # decode step: append token 2048 of every sequence, attend over 2049 slots
+    ws1 = torch.zeros(max(lib.kpa_append_workspace_size(cfg, w.batch, 1), 256), dtype=torch.uint8, device="cuda")
+    q1 = torch.empty(w.batch, 1, s.h, s.dh, dtype=torch.bfloat16, device="cuda")
+    pos = torch.full((w.batch,), w.n_tok, dtype=torch.int32, device="cuda")
+    lib.kpa_append(cfg, w.batch, 1, inp["x_step"].cuda(), inp["W"].cuda(), pos, w.capacity, kc, vc, q1, ws1)
+    seq = torch.full((w.batch,), w.n_tok + 1, dtype=torch.int32)
+    dw = APPEND_PREFILL  # decode on the same cache
+    from workloads import DecodeWorkload
+    dwl = DecodeWorkload(name="c5 step", shape=s, batch=w.batch, capacity=w.capacity, dtype="bf16",
+                         factor_std=0, q_std=0, length=w.n_tok + 1)
+    dec = run_decode(lib, dwl, cfg, kc, vc, q1[:, 0], seq, None, sm_scale=scale)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    qo = to_f64(q_out.cpu())
+    got = out.cpu().numpy()
+    rng = np.random.default_rng(5)
+    rows = [(int(b), int(t)) for b, t in zip(rng.integers(0, w.batch, 12), rng.integers(0, w.n_tok, 12))]
+    rows += [(0, 0), (1, 127), (2, 128), (7, w.n_tok - 1)]
+    for b, t in rows:
+        want = oracle.decode(s, qo[b, t][None], kn[b][None], vn[b][None], [t + 1], keys_rotated=True,
+                             sm_scale=scale)
+        assert_bf16_close(got[b, t], want[0], f"prefill row ({b},{t})")
+    want = oracle.decode(s, to_f64(q1[:, 0].cpu()), kn, vn, seq.numpy(), keys_rotated=True, sm_scale=scale)
+    assert_bf16_close(dec.cpu().numpy(), want, "decode step at 2048")
