@@ -17,7 +17,7 @@
 // that rounding them costs no more than ~2^-16 relative.
 //
 // Data movement: one producer warp streams each split's cache groups through a
-// STAGES-deep shared-memory ring with cp.async.bulk (TMA, no multicast) and
+// STAGES-deep shared-memory ring with cp.async.bulk (plain bulk copies into this CTA) and
 // mbarrier transaction counts; consumer warps read the 8-token groups, whose
 // element-major/token-minor layout makes every fragment load a conflict-free
 // 16-byte row (ldmatrix) or 32-bit word (two adjacent tokens).  Every wait is
