@@ -213,35 +213,68 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
     }
 }
 
-// q_out[m][(i1,i2)][(j1,j2)] = (1/R_Q) sum_r A^Q_r[i1,j1] * B~^Q_r[i2,j2]; one thread per
-// (token, head), threads of a block are consecutive tokens of one head.
-__global__ void __launch_bounds__(128)
-q_assemble_kernel(const float *__restrict__ qf, int M, int h1, int h2, int d1, int d2, int rq,
-                  __nv_bfloat16 *__restrict__ q_out) {
-    extern __shared__ float sh[];
-    const int head = blockIdx.y;
+// Query assembly q = (1/R_Q) sum_r A^Q_r (x) B^Q_r for the queries of the chunk.
+// One thread per (token, i2): the R_Q rows B^Q_r[i2, :] stay in registers while the
+// thread walks the h1 heads (i1, i2), so each factor is read once per token and
+// head column.  Reads of the [column][token] factor buffer are coalesced across the
+// warp's tokens; each head row of q_out goes out in 16-byte stores.
+template <int RQ, int D1, int D2>
+__global__ void __launch_bounds__(64)
+q_assemble_kernel(const float *__restrict__ qf, int M, int h1, int h2, __nv_bfloat16 *__restrict__ q_out) {
     const int m = blockIdx.x * blockDim.x + threadIdx.x;
-    const int i1 = head / h2, i2 = head % h2;
-    const int h = h1 * h2, dh = d1 * d2;
-    const int qa = rq * h1 * d1;
-    float *A = sh + (size_t)threadIdx.x * rq * (d1 + d2);       // [rq][d1]
-    float *B = A + rq * d1;                                     // [rq][d2]
     if (m >= M) return;
-    for (int r = 0; r < rq; ++r) {
-        for (int j1 = 0; j1 < d1; ++j1) A[r * d1 + j1] = qf[(size_t)(r * h1 * d1 + i1 * d1 + j1) * M + m];
-        for (int j2 = 0; j2 < d2; ++j2) B[r * d2 + j2] = qf[(size_t)(qa + r * h2 * d2 + i2 * d2 + j2) * M + m];
-    }
-    const float inv = 1.0f / (float)rq;
-    __nv_bfloat16 *dst = q_out + ((size_t)m * h + head) * dh;
-    for (int j1 = 0; j1 < d1; ++j1)
-        for (int j2 = 0; j2 < d2; j2 += 2) {
-            float s0 = 0.f, s1 = 0.f;
-            for (int r = 0; r < rq; ++r) {
-                const float av = A[r * d1 + j1];
-                s0 += av * B[r * d2 + j2];
-                s1 += av * B[r * d2 + j2 + 1];
+    const int i2 = blockIdx.y;
+    const int qa = RQ * h1 * D1;
+    float B[RQ][D2];
+#pragma unroll
+    for (int r = 0; r < RQ; ++r)
+#pragma unroll
+        for (int j2 = 0; j2 < D2; ++j2) B[r][j2] = __ldg(qf + (size_t)(qa + (r * h2 + i2) * D2 + j2) * M + m);
+    const float inv = 1.0f / (float)RQ;
+    for (int i1 = 0; i1 < h1; ++i1) {
+        __nv_bfloat16 *dst = q_out + ((size_t)m * h1 * h2 + (size_t)i1 * h2 + i2) * (D1 * D2);
+#pragma unroll 2
+        for (int j1 = 0; j1 < D1; ++j1) {
+            float A[RQ];
+#pragma unroll
+            for (int r = 0; r < RQ; ++r) A[r] = __ldg(qf + (size_t)((r * h1 + i1) * D1 + j1) * M + m);
+#pragma unroll
+            for (int j2 = 0; j2 < D2; j2 += 8) {
+                uint4 u;
+                uint32_t *pu = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                    for (int r = 0; r < RQ; ++r) {
+                        s0 += A[r] * B[r][j2 + 2 * k];
+                        s1 += A[r] * B[r][j2 + 2 * k + 1];
+                    }
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(s0 * inv, s1 * inv);
+                    pu[k] = *reinterpret_cast<uint32_t *>(&hb);
+                }
+                *reinterpret_cast<uint4 *>(dst + j1 * D2 + j2) = u;
             }
-            *reinterpret_cast<__nv_bfloat162 *>(dst + j1 * d2 + j2) = __floats2bfloat162_rn(s0 * inv, s1 * inv);
+        }
+    }
+}
+
+// Any shape: one thread per (token, head), loops.
+__global__ void __launch_bounds__(128)
+q_assemble_any_kernel(const float *__restrict__ qf, int M, int h1, int h2, int d1, int d2, int rq,
+                      __nv_bfloat16 *__restrict__ q_out) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M) return;
+    const int head = blockIdx.y, i1 = head / h2, i2 = head % h2, qa = rq * h1 * d1;
+    const float inv = 1.0f / (float)rq;
+    __nv_bfloat16 *dst = q_out + ((size_t)m * h1 * h2 + head) * d1 * d2;
+    for (int j1 = 0; j1 < d1; ++j1)
+        for (int j2 = 0; j2 < d2; ++j2) {
+            float acc = 0.f;
+            for (int r = 0; r < rq; ++r)
+                acc += qf[(size_t)(r * h1 * d1 + i1 * d1 + j1) * M + m] *
+                       qf[(size_t)(qa + r * h2 * d2 + i2 * d2 + j2) * M + m];
+            dst[j1 * d2 + j2] = __float2bfloat16_rn(acc * inv);
         }
 }
 
@@ -322,12 +355,14 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     append_gemm_kernel<<<grid, kThreads, smem, st>>>(tmx, tmw, a, rope);
     e = cudaGetLastError();
     if (e != cudaSuccess || !q_out) return e;
-    const size_t qsm = (size_t)128 * rq * (d.d1 + d.d2) * sizeof(float);
-    e = ensure_dynamic_smem<q_assemble_kernel>(qsm);
-    if (e != cudaSuccess) return e;
-    dim3 g2((unsigned)((a.M + 127) / 128), (unsigned)d.h);
-    q_assemble_kernel<<<g2, 128, qsm, st>>>(qf, a.M, d.h1, d.h2, d.d1, d.d2, rq,
-                                            static_cast<__nv_bfloat16 *>(q_out));
+    __nv_bfloat16 *qo = static_cast<__nv_bfloat16 *>(q_out);
+    const dim3 g2((unsigned)((a.M + 63) / 64), (unsigned)d.h2);
+    if (rq == 6 && d.d1 == 8 && d.d2 == 16) {
+        q_assemble_kernel<6, 8, 16><<<g2, 64, 0, st>>>(qf, a.M, d.h1, d.h2, qo);
+    } else {
+        dim3 g3((unsigned)((a.M + 127) / 128), (unsigned)d.h);
+        q_assemble_any_kernel<<<g3, 128, 0, st>>>(qf, a.M, d.h1, d.h2, d.d1, d.d2, rq, qo);
+    }
     return cudaGetLastError();
 }
 

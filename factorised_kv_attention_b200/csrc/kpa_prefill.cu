@@ -1,22 +1,34 @@
 // kpa_prefill.cu -- causal chunked attention in factor space on the tcgen05 tensor cores.
 //
 // Row t of sequence b is the query at position start_pos[b] + t; it attends to cache
-// slots 0 .. start_pos[b] + t.  Keys and values exist only as factors in the cache
-// ("Kronecker Product Attention", eqs 3-4, B^K pre-rotated per Theorem 2.4); each
-// 128-token K and V tile of one head is rebuilt on chip,
+// slots 0 .. start_pos[b] + t ("Kronecker Product Attention", eqs 3-4, with B^K
+// pre-rotated in the cache per Theorem 2.4).  Keys and values exist only as factors:
+// each 128-token K and V tile of one head is rebuilt on chip,
 //     K[s][(j1,j2)] = sum_r A^K_r(s)[i1,j1] B~^K_r(s)[i2,j2]     (1/R_K folded into the scale)
 //     V[s][(j1,j2)] = sum_r A^V_r(s)[i1,j1] B^V_r(s)[i2,j2]      (1/R_V folded into the output)
-// straight into the 128-byte-swizzled K-major layouts that tcgen05.mma reads, and is
-// never written to device memory.  The tensor-core operands are fp16 (K, V and P
-// are rounded once to an 11-bit significand, 4x finer than bf16; the bf16 Q tile is
-// converted in place); a value outside the fp16 range is reported as
-// KPA_ERR_DEVICE_CHECK.  Then, per tile (FlashAttention-style):
-//     S = Q K^T on the tensor cores into TMEM; the softmax warps (one query row per
-//     thread) read S, apply the causal mask and the online softmax, write P in bf16
-//     back to shared memory and, when a row's running max grew, rescale that row of
-//     the TMEM output accumulator; then O += P V on the tensor cores, in TMEM.
-// Warps 0-3: softmax / output rows.  Warps 4-7: K/V reconstruction (one tile ahead,
-// double-buffered).  Warp 8: TMEM allocation, the Q tile's TMA load, MMA issue.
+// and is never written to device memory.
+//
+// One CTA takes 256 query rows of one (sequence, head) as two 128-row halves that
+// share every rebuilt K/V tile and take turns on the tensor pipe:
+//   - a producer warp streams the head's factor slices of each key tile into shared
+//     memory with TMA, two tiles ahead (and loads the Q tile once);
+//   - four rebuild warps form the K tile (token rows) and the V^T tile (feature rows)
+//     in the 128-byte-swizzled K-major layouts tcgen05.mma reads, from ldmatrix.trans
+//     fragments of the factors through stmatrix / stmatrix.trans; K runs one tile
+//     ahead of V, K is double-buffered;
+//   - one thread issues S_h = Q_h K^T (both operands in shared memory) and
+//     O_h += P_h V (P_h read from tensor memory) in the order S0 S1 | PV0 S0' PV1 S1' ...,
+//     so one half's softmax overlaps the other half's MMAs;
+//   - eight softmax warps (one query row per thread) read S_h from tensor memory,
+//     apply the causal mask on diagonal tiles and write P_h over S_h as fp16.
+// Tensor memory: S0 | S1 | O0 | O1, 128 columns each (all 512).
+//
+// Numerics: the tensor-core operands are fp16 (an 11-bit significand: the rebuilt K
+// and V are rounded once, P once, Q once after the softmax scale sm_scale/R_K*log2(e)
+// is folded into it); accumulation is fp32.  The running maximum is only moved when a
+// row's maximum grows by more than 2^8 (FlashAttention-4's conditional rescaling), so
+// P stays in [0, 256].  A value outside the fp16 range becomes inf and makes the row's
+// output non-finite; such a row is reported as KPA_ERR_DEVICE_CHECK.
 #include <cudaTypedefs.h>
 
 #include <cuda_fp16.h>
@@ -29,7 +41,6 @@ namespace kpa {
 struct PrefillArgs {
     int batch, n_tok, cap;
     const int32_t *start_pos;
-    const __nv_bfloat16 *kc, *vc;
     float *out;
     float qscale;       // sm_scale / R_K * log2(e)
     float out_scale;    // 1 / R_V
@@ -42,86 +53,231 @@ namespace {
 
 using namespace sm100;
 
-constexpr int TQ = 128, TK = 128;
-constexpr int kThreads = 288;
-constexpr uint32_t kTmemCols = 256;        // S: columns 0..127, O accumulator: 128..255
+constexpr int HQ = 128;                       // query rows per half
+constexpr int TK = 128;                       // keys per tile
+constexpr int kSoftmaxWarps = 8, kRebuildWarps = 4;
+constexpr int kRebuildWarp0 = kSoftmaxWarps;                  // warps 8..11
+constexpr int kMmaWarp = kSoftmaxWarps + kRebuildWarps;       // warp 12
+constexpr int kProducerWarp = kMmaWarp + 1;                   // warp 13
+constexpr int kThreads = (kProducerWarp + 1) * 32;            // 448
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.f;
+constexpr int kBox = 16 * 64 * 2;             // TMA box: 16 cache groups x (8 elements x 8 tokens) bf16
 
 template <int D1_, int D2_, int RK_, int RV_>
 struct PrefillCfg {
     static constexpr int D1 = D1_, D2 = D2_, RK = RK_, RV = RV_;
     static constexpr int DH = D1 * D2;
-    static constexpr int NH = DH / 64;             // 64-feature halves of a row
-    static_assert(DH == 64 || DH == 128, "head dim 64 or 128");
-    static_assert(D2 % 8 == 0, "d2 must be a multiple of 8");
-    static constexpr uint32_t Q_BYTES = TQ * DH * 2;
-    static constexpr uint32_t K_BYTES = TK * DH * 2;
-    static constexpr uint32_t V_BYTES = DH * TK * 2;
-    static constexpr uint32_t P_BYTES = TQ * TK * 2;
-    static constexpr size_t OFF_Q = 0;
-    static constexpr size_t OFF_K = OFF_Q + Q_BYTES;                 // 2 buffers
-    static constexpr size_t OFF_V = OFF_K + 2 * K_BYTES;             // 2 buffers
-    static constexpr size_t OFF_P = OFF_V + 2 * V_BYTES;
-    static constexpr size_t OFF_BAR = OFF_P + P_BYTES;
-    static constexpr size_t SMEM = 1024 + OFF_BAR + 64;
+    static_assert(D1 == 8 && D2 == 16, "the fragment mapping covers d1 = 8, d2 = 16");
+    static_assert(RK == 2 && RV == 2, "one ldmatrix.x4 covers the B rows of two ranks");
+    static constexpr uint32_t Q_HALF = HQ * DH * 2;
+    static constexpr uint32_t KV_TILE = TK * DH * 2;
+    static constexpr uint32_t K_ST = 3 * RK * kBox;          // A_r (1 box) and B_r (2 boxes) per rank
+    static constexpr uint32_t V_ST = 3 * RV * kBox;
+    static constexpr size_t OFF_Q = 0;                         // two halves
+    static constexpr size_t OFF_K = OFF_Q + 2 * Q_HALF;        // two buffers
+    static constexpr size_t OFF_V = OFF_K + 2 * KV_TILE;       // one buffer
+    static constexpr size_t OFF_KST = OFF_V + KV_TILE;         // two stages
+    static constexpr size_t OFF_VST = OFF_KST + 2 * K_ST;      // two stages
+    static constexpr size_t OFF_BAR = OFF_VST + 2 * V_ST;
+    static constexpr int NBAR = 24;
+    static constexpr size_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
 };
 
-// Byte offset of element k (0..63) of row `row` in a 128-byte-swizzled K-major block.
-__device__ __forceinline__ uint32_t sw128(int row, int k) {
-    return (uint32_t)row * 128 + ((((uint32_t)k >> 3) ^ ((uint32_t)row & 7)) << 4) + ((uint32_t)k & 7) * 2;
-}
+// mbarrier slots
+enum : int {
+    B_Q = 0,
+    B_QREADY = 1,      // +h
+    B_KST_FULL = 3,    // +stage
+    B_VST_FULL = 5,
+    B_KST_EMPTY = 7,
+    B_VST_EMPTY = 9,
+    B_K_FULL = 11,     // +buffer
+    B_K_EMPTY = 13,
+    B_V_FULL = 15,
+    B_V_EMPTY = 16,
+    B_S_FULL = 17,     // +h
+    B_P_FULL = 19,     // +h
+    B_O_FINAL = 21,    // +h
+    B_DRAIN = 23,
+};
 
-constexpr float kHalfMax = 65504.f;
-
-// Eight floats as fp16; `big` records whether any lies outside the fp16 range.
-__device__ __forceinline__ uint4 pack8(const float (&x)[8], bool &big) {
-    uint4 u;
-    uint32_t *p = reinterpret_cast<uint32_t *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        big |= fabsf(x[2 * i]) > kHalfMax || fabsf(x[2 * i + 1]) > kHalfMax;
-        __half2 h = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
-        p[i] = *reinterpret_cast<uint32_t *>(&h);
-    }
-    return u;
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-swizzled block.
+__device__ __forceinline__ uint32_t sw128_chunk(int row, int chunk) {
+    return (uint32_t)row * 128 + ((uint32_t)(chunk ^ (row & 7)) << 4);
 }
 
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+// (x, y) -> fp16x2 word, x in the low half
+__device__ __forceinline__ uint32_t pack_half2(float x, float y) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y), "f"(x));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T (A read from tensor memory), issued by one thread.
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                        bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+        "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+        "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+        "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&w)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]),
+        "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+        : "memory");
+}
+
+// Which tiles a half works on: both halves start at tile 0; half h stops at last[h].
+struct TilePlan {
+    bool act[2];
+    int last[2];
+    int n_kt;
+    __device__ bool active(int h, int t) const { return act[h] && t <= last[h]; }
+    __device__ int first_half(int t) const { return active(0, t) ? 0 : 1; }
+    __device__ int last_half(int t) const { return active(1, t) ? 1 : 0; }
+};
+
 template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_kernel(const __grid_constant__ CUtensorMap tmq, PrefillArgs a) {
-    constexpr int D1 = C::D1, D2 = C::D2, RK = C::RK, RV = C::RV, DH = C::DH, NH = C::NH;
+prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+               const __grid_constant__ CUtensorMap tmv, PrefillArgs a) {
+    constexpr int D1 = C::D1, RK = C::RK, RV = C::RV, DH = C::DH;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);    // q, s, pv
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + C::NBAR * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_qt = (a.n_tok + TQ - 1) / TQ;
-    const int qt = n_qt - 1 - (int)blockIdx.x;                // longest rows first
+    const int n_pairs = (a.n_tok + 2 * HQ - 1) / (2 * HQ);
+    const int pair = n_pairs - 1 - (int)blockIdx.x;             // longest rows first
     const int head = blockIdx.y, b = blockIdx.z;
     const int h = a.h1 * a.h2, i1 = head / a.h2, i2 = head % a.h2;
-    const int q0 = qt * TQ;
+    const int q0 = pair * 2 * HQ;
     const int start = a.start_pos[b];
-    int max_slot = start + min(q0 + TQ, a.n_tok) - 1;          // last slot any row of the tile sees
-    if (max_slot >= a.cap || start < 0) {
-        if (tid == 0) raise_error(a.err, kErrDeviceCheck);
-        max_slot = min(max_slot, a.cap - 1);
-    }
-    const int n_kt = max_slot >= 0 ? max_slot / TK + 1 : 0;
-    const uint32_t bar_q = smem_u32(bars), bar_s = bar_q + 8, bar_pv = bar_q + 16;
     const uint64_t limit = a.wait_limit_ns;
 
+    // Tiles: half hh covers rows q0 + hh*128 .. min(+127, n_tok-1), positions start + row.
+    TilePlan tp;
+    bool range_ok = start >= 0;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int r0 = q0 + hh * HQ;
+        tp.act[hh] = r0 < a.n_tok;
+        int last_slot = start + min(r0 + HQ, a.n_tok) - 1;
+        if (last_slot >= a.cap) {
+            range_ok = false;
+            last_slot = a.cap - 1;
+        }
+        tp.last[hh] = tp.act[hh] && last_slot >= 0 ? last_slot / TK : -1;
+        if (tp.last[hh] < 0) tp.act[hh] = false;
+    }
+    if (start < 0) tp.act[0] = tp.act[1] = false, tp.last[0] = tp.last[1] = -1;
+    tp.n_kt = max(tp.last[0], tp.last[1]) + 1;
+    // slots past the last row's position stay zero in the rebuilt tiles
+    const int max_slot = min(start + min(q0 + 2 * HQ, a.n_tok) - 1, a.cap - 1);
+    if (!range_ok && tid == 0) raise_error(a.err, kErrDeviceCheck);
+
     if (tid == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(bar_s, 1);
-        mbar_init(bar_pv, 1);
+        for (int i = 0; i < C::NBAR; ++i) {
+            uint32_t count = 1;
+            if ((i >= B_QREADY && i < B_QREADY + 2) || (i >= B_P_FULL && i < B_P_FULL + 2)) count = 4;
+            if ((i >= B_KST_EMPTY && i < B_KST_EMPTY + 2) || (i >= B_VST_EMPTY && i < B_VST_EMPTY + 2) ||
+                (i >= B_K_FULL && i < B_K_FULL + 2) || i == B_V_FULL)
+                count = kRebuildWarps;
+            mbar_init(bar(i), count);
+        }
+        *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
@@ -129,249 +285,345 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, PrefillArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (tid == 8 * 32) {           // the Q tile: rows q0.. of sequence b, this head's DH columns
-        mbar_expect_tx(bar_q, C::Q_BYTES);
-#pragma unroll
-        for (int hh = 0; hh < NH; ++hh)
-            tma_load_2d(smem_u32(smem + C::OFF_Q + hh * TQ * 128), &tmq, head * DH + hh * 64, b * a.n_tok + q0, bar_q);
-    }
 
-    const int ek = RK * (a.h1 * D1 + a.h2 * D2), ev = RV * (a.h1 * D1 + a.h2 * D2);
-    const __nv_bfloat16 *kcb = a.kc + (size_t)b * a.cap * ek;
-    const __nv_bfloat16 *vcb = a.vc + (size_t)b * a.cap * ev;
-
-    // ---- reconstruction of tile kt into buffer kt % 2 (warps 4..7)
-    auto rebuild = [&](int kt) {
-        const int rt = tid - 128;
-        bool big = false;
-        unsigned char *kbuf = smem + C::OFF_K + (kt & 1) * C::K_BYTES;
-        unsigned char *vbuf = smem + C::OFF_V + (kt & 1) * C::V_BYTES;
-        // K: thread = token row
-        {
-            const int slot = kt * TK + rt;
-            float A[RK][D1], B[RK][D2];
-            const bool live = slot <= max_slot;
-            if (live) {
-                const __nv_bfloat16 *base = kcb + ((size_t)(slot / kGroup) * ek) * kGroup + (slot % kGroup);
-#pragma unroll
-                for (int r = 0; r < RK; ++r) {
-#pragma unroll
-                    for (int j1 = 0; j1 < D1; ++j1)
-                        A[r][j1] = __bfloat162float(base[(size_t)(r * a.h1 * D1 + i1 * D1 + j1) * kGroup]);
-#pragma unroll
-                    for (int j2 = 0; j2 < D2; ++j2)
-                        B[r][j2] = __bfloat162float(
-                            base[(size_t)(RK * a.h1 * D1 + r * a.h2 * D2 + i2 * D2 + j2) * kGroup]);
+    // Bounded wait shared by every role: gives up when the time runs out or another
+    // thread has already given up, and records the timeout once.
+    auto wait = [&](int i, uint32_t parity) -> bool {
+        if (mbar_try_wait(bar(i), parity)) return true;
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 1;; ++it) {
+            if (mbar_try_wait(bar(i), parity)) return true;
+            if ((it & 15) == 0) {
+                if (*abort_flag) return false;
+                if (globaltimer() - t0 > limit) {
+                    *abort_flag = 1;
+                    raise_error(a.err, kErrTimeout);
+                    return false;
                 }
             }
-#pragma unroll
-            for (int j1 = 0; j1 < D1; ++j1)
-#pragma unroll
-                for (int c8 = 0; c8 < D2; c8 += 8) {
-                    float x[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        float acc = 0.f;
-                        if (live) {
-#pragma unroll
-                            for (int r = 0; r < RK; ++r) acc += A[r][j1] * B[r][c8 + u];
-                        }
-                        x[u] = acc;
-                    }
-                    const int f = j1 * D2 + c8;                          // first feature of the chunk
-                    *reinterpret_cast<uint4 *>(kbuf + (f / 64) * (TK * 128) + sw128(rt, f % 64)) = pack8(x, big);
-                }
         }
-        // V^T: thread = feature row f, tokens in 16-byte groups of 8
-        if (rt < DH) {
-            const int f = rt, j1 = f / D2, j2 = f % D2;
-#pragma unroll 4
-            for (int g = 0; g < TK / kGroup; ++g) {
-                const int slot0 = kt * TK + g * kGroup;
-                float x[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) x[u] = 0.f;
-                if (slot0 <= max_slot) {
-                    const __nv_bfloat16 *gb = vcb + (size_t)(slot0 / kGroup) * ev * kGroup;
-#pragma unroll
-                    for (int r = 0; r < RV; ++r) {
-                        const uint4 av = *reinterpret_cast<const uint4 *>(gb + (size_t)(r * a.h1 * D1 + i1 * D1 + j1) * kGroup);
-                        const uint4 bv = *reinterpret_cast<const uint4 *>(
-                            gb + (size_t)(RV * a.h1 * D1 + r * a.h2 * D2 + i2 * D2 + j2) * kGroup);
-                        const __nv_bfloat162 *ap = reinterpret_cast<const __nv_bfloat162 *>(&av);
-                        const __nv_bfloat162 *bp = reinterpret_cast<const __nv_bfloat162 *>(&bv);
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float2 af = __bfloat1622float2(ap[u]), bf = __bfloat1622float2(bp[u]);
-                            x[2 * u] += af.x * bf.x;
-                            x[2 * u + 1] += af.y * bf.y;
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (slot0 + u > max_slot) x[u] = 0.f;
-                }
-                const int tk = g * kGroup;                               // first token of the chunk
-                *reinterpret_cast<uint4 *>(vbuf + (tk / 64) * (DH * 128) + sw128(f, tk % 64)) = pack8(x, big);
-            }
-        }
-        if (big) raise_error(a.err, kErrDeviceCheck);
-        fence_async_smem();        // visible to the tensor cores
     };
 
-    if (warp >= 4 && warp < 8 && n_kt > 0) rebuild(0);
-
-    // softmax-row state (warps 0..3)
-    const int row = (warp & 3) * 32 + lane;
-    const int pos = start + q0 + row;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // the bf16 Q tile becomes fp16 in place once its copy has landed
-    if (warp < 4) {
-        if (!mbar_wait(bar_q, 0, limit)) {
-            raise_error(a.err, kErrTimeout);
-            ok = false;
-        }
-        bool big = false;
-        uint4 *qt4 = reinterpret_cast<uint4 *>(smem + C::OFF_Q);
-        for (int i = tid; i < (int)(C::Q_BYTES / 16); i += 128) {
-            uint4 u = qt4[i];
-            uint32_t *w = reinterpret_cast<uint32_t *>(&u);
-            float x[8];
+    if (warp == kProducerWarp) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0 && tp.n_kt > 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+            const int nh = (tp.act[0] ? 1 : 0) + (tp.act[1] ? 1 : 0);
+            mbar_expect_tx(bar(B_Q), (uint32_t)nh * C::Q_HALF);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[k]));
-                x[2 * k] = f.x;
-                x[2 * k + 1] = f.y;
-            }
-            qt4[i] = pack8(x, big);
-        }
-        if (big) raise_error(a.err, kErrDeviceCheck);
-        fence_async_smem();
-    }
-    if (warp < 4 || warp == 8) asm volatile("bar.sync 1, 160;" ::: "memory");
-
-    const uint32_t idesc_s = umma_idesc_f16_f32(TQ, TK), idesc_o = umma_idesc_f16_f32(TQ, DH);
-    const uint32_t srow = tmem + ((uint32_t)((warp & 3) * 32) << 16);    // this row's S columns
-    const uint32_t orow = srow + 128;                                     // this row's O columns
-    for (int kt = 0; kt < n_kt; ++kt) {
-        const int buf = kt & 1;
-        if (tid == 8 * 32) {                                           // S = Q K^T
-            tc_fence_after();
+            for (int hh = 0; hh < 2; ++hh)
+                if (tp.act[hh])
 #pragma unroll
-            for (int k = 0; k < DH / 16; ++k) {
-                const uint64_t qd = umma_desc_k_sw128(smem_u32(smem + C::OFF_Q + (k / 4) * TQ * 128)) + 2 * (k % 4);
-                const uint64_t kd = umma_desc_k_sw128(
-                                        smem_u32(smem + C::OFF_K + buf * C::K_BYTES + (k / 4) * TK * 128)) +
-                                    2 * (k % 4);
-                umma_bf16(tmem, qd, kd, idesc_s, k > 0);
-            }
-            umma_commit(bar_s);
-        }
-        if (warp >= 4 && warp < 8 && kt + 1 < n_kt) rebuild(kt + 1);
-        if (warp < 4) {
-            if (!mbar_wait(bar_s, kt & 1, limit)) {
-                raise_error(a.err, kErrTimeout);
-                ok = false;
-            }
-            tc_fence_after();
-            const int slot0 = kt * TK;
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < TK / 16; ++c) {
-                float v[16];
-                tmem_ld16(srow + c * 16, v);
+                    for (int cb = 0; cb < DH / 64; ++cb)
+                        tma_load_2d(smem_u32(smem + C::OFF_Q + hh * C::Q_HALF + cb * HQ * 128), &tmq,
+                                    head * DH + cb * 64, b * a.n_tok + q0 + hh * HQ, bar(B_Q));
+            const int grp0 = (int)((int64_t)b * a.cap / kGroup);
+            const int ea = RK * a.h1 * D1;     // first B element of a key record
+            const int va = RV * a.h1 * D1;
+            int issued[2][2] = {{-1, -1}, {-1, -1}};
+            bool ok = true;
+            for (int t = 0; t < tp.n_kt && ok; ++t) {
+                const int s = t & 1, grp = grp0 + t * (TK / kGroup);
+                // key factors of tile t
+                if (t >= 2 && !wait(B_KST_EMPTY + s, ((t >> 1) - 1) & 1)) { ok = false; break; }
+                mbar_expect_tx(bar(B_KST_FULL + s), C::K_ST);
+                unsigned char *kst = smem + C::OFF_KST + s * C::K_ST;
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (slot0 + c * 16 + j <= pos) mx = fmaxf(mx, v[j] * a.qscale);
-            }
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
-            float sum = 0.f;
-            unsigned char *pbuf = smem + C::OFF_P;
-#pragma unroll 1
-            for (int c = 0; c < TK / 16; ++c) {
-                float v[16];
-                tmem_ld16(srow + c * 16, v);
+                for (int r = 0; r < RK; ++r) {
+                    tma_load_2d(smem_u32(kst + r * kBox), &tmk, (r * a.h1 * D1 + i1 * D1) * kGroup, grp,
+                                bar(B_KST_FULL + s));
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int slot = slot0 + c * 16 + j;
-                    v[j] = (slot <= pos && m_new != -INFINITY) ? exp2f(v[j] * a.qscale - m_new) : 0.f;
-                    sum += v[j];
+                    for (int hb = 0; hb < 2; ++hb)
+                        tma_load_2d(smem_u32(kst + (RK + 2 * r + hb) * kBox), &tmk,
+                                    (ea + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, bar(B_KST_FULL + s));
                 }
+                issued[0][s] = t;
+                // value factors of tile t
+                if (t >= 2 && !wait(B_VST_EMPTY + s, ((t >> 1) - 1) & 1)) { ok = false; break; }
+                mbar_expect_tx(bar(B_VST_FULL + s), C::V_ST);
+                unsigned char *vst = smem + C::OFF_VST + s * C::V_ST;
+#pragma unroll
+                for (int r = 0; r < RV; ++r) {
+                    tma_load_2d(smem_u32(vst + r * kBox), &tmv, (r * a.h1 * D1 + i1 * D1) * kGroup, grp,
+                                bar(B_VST_FULL + s));
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb)
+                        tma_load_2d(smem_u32(vst + (RV + 2 * r + hb) * kBox), &tmv,
+                                    (va + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, bar(B_VST_FULL + s));
+                }
+                issued[1][s] = t;
+            }
+            // every copy this thread started lands before the CTA can exit
+            (void)mbar_wait(bar(B_Q), 0, limit);
+#pragma unroll
+            for (int pl = 0; pl < 2; ++pl)
+#pragma unroll
+                for (int s = 0; s < 2; ++s)
+                    if (issued[pl][s] >= 0)
+                        (void)mbar_wait(bar((pl ? B_VST_FULL : B_KST_FULL) + s), (issued[pl][s] >> 1) & 1, limit);
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------------------- MMA issue
+        if (lane == 0 && tp.n_kt > 0) {
+            const uint32_t idesc_s = umma_idesc_f16_f32(HQ, TK), idesc_o = umma_idesc_f16_f32(HQ, DH);
+            bool ok = true;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                if (ok && tp.act[hh] && !wait(B_QREADY + hh, 0)) ok = false;
+            auto issue_s = [&](int hh, int t) -> bool {
+                const int kb = t & 1;
+                if (!wait(B_K_FULL + kb, (t >> 1) & 1)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < DH / 16; ++k) {
+                    const uint64_t qd =
+                        umma_desc_k_sw128(smem_u32(smem + C::OFF_Q + hh * C::Q_HALF + (k / 4) * HQ * 128)) +
+                        2 * (k % 4);
+                    const uint64_t kd =
+                        umma_desc_k_sw128(smem_u32(smem + C::OFF_K + kb * C::KV_TILE + (k / 4) * TK * 128)) +
+                        2 * (k % 4);
+                    umma_bf16(tmem + hh * 128, qd, kd, idesc_s, k > 0);
+                }
+                umma_commit(bar(B_S_FULL + hh));
+                if (hh == tp.last_half(t)) umma_commit(bar(B_K_EMPTY + kb));
+                return true;
+            };
+            auto issue_pv = [&](int hh, int t) -> bool {
+                if (!wait(B_P_FULL + hh, t & 1)) return false;
+                if (hh == tp.first_half(t) && !wait(B_V_FULL, t & 1)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < TK / 16; ++k) {
+                    const uint64_t vd =
+                        umma_desc_k_sw128(smem_u32(smem + C::OFF_V + (k / 4) * DH * 128)) + 2 * (k % 4);
+                    umma_ts(tmem + 256 + hh * 128, tmem + hh * 128 + 8 * k, vd, idesc_o, t > 0 || k > 0);
+                }
+                if (hh == tp.last_half(t)) umma_commit(bar(B_V_EMPTY));
+                if (t == tp.last[hh]) umma_commit(bar(B_O_FINAL + hh));
+                return true;
+            };
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                if (ok && tp.active(hh, 0)) ok = issue_s(hh, 0);
+            for (int t = 0; t < tp.n_kt && ok; ++t) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    float x[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) x[u] = v[hh * 8 + u];
-                    const int tk = c * 16 + hh * 8;
-                    bool unused = false;
-                    *reinterpret_cast<uint4 *>(pbuf + (tk / 64) * (TQ * 128) + sw128(row, tk % 64)) = pack8(x, unused);
+                    if (ok && tp.active(hh, t)) ok = issue_pv(hh, t);
+                    if (ok && tp.active(hh, t + 1)) ok = issue_s(hh, t + 1);
                 }
             }
-            l_run = l_run * alpha + sum;
-            m_run = m_new;
-            // the accumulator row follows the new max before P V is added to it
-            // (tcgen05.ld/st are warp-collective: the warp rescales if any of its rows must)
-            if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // nothing issued here may still run when tensor memory is released
+            umma_commit(bar(B_DRAIN));
+            (void)mbar_wait(bar(B_DRAIN), 0, limit);
+        }
+    } else if (warp >= kRebuildWarp0) {
+        // ---------------------------------------------------------------- K / V rebuild
+        const int rw = warp - kRebuildWarp0;
+        const int tok = lane >> 2;                 // token of the 8-token group this lane holds
+        const int blk = lane >> 3, brow = lane & 7;   // ldmatrix / stmatrix row this lane addresses
+        // Rebuild one plane of tile t: K (token rows, stmatrix) or V^T (feature rows, stmatrix.trans).
+        auto rebuild = [&](int t, bool is_v) {
+            const unsigned char *st = smem + (is_v ? C::OFF_VST + (t & 1) * C::V_ST : C::OFF_KST + (t & 1) * C::K_ST);
+            const uint32_t dst = smem_u32(smem + (is_v ? C::OFF_V : C::OFF_K + (t & 1) * C::KV_TILE));
+            const bool edge = t * TK + TK - 1 > max_slot;
 #pragma unroll 1
-                for (int c = 0; c < DH / 16; ++c) {
-                    float v[16];
-                    tmem_ld16(orow + c * 16, v);
+            for (int gi = 0; gi < TK / kGroup / kRebuildWarps; ++gi) {
+                const int g = rw + gi * kRebuildWarps;      // group of the tile, 0..15
+                // A_r[tok][j1], r = 0, 1: one 16-byte row per j1 holds the group's 8 tokens
+                float av[2][8];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] *= alpha;
-                    tmem_st16(orow + c * 16, v);
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int j1 = 0; j1 < 8; ++j1)
+                        av[r][j1] = __uint_as_float(
+                            (uint32_t)(*reinterpret_cast<const uint16_t *>(st + r * kBox + g * 128 + j1 * 16 + tok * 2))
+                            << 16);
+                // B_r[tok][hb*8 + 2c .. +1] for (r, hb) = block 0..3
+                uint32_t bw[4];
+                ldsm_x4_t(smem_u32(st + (2 + blk) * kBox + g * 128 + brow * 16), bw);
+                float2 bf[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) bf[i] = unpack_bf16x2(bw[i]);
+                uint32_t w[8][2];
+#pragma unroll
+                for (int j1 = 0; j1 < 8; ++j1)
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb) {
+                        float2 acc = fmul2(make_float2(av[0][j1], av[0][j1]), bf[hb]);
+                        acc = ffma2(make_float2(av[1][j1], av[1][j1]), bf[2 + hb], acc);
+                        w[j1][hb] = pack_half2(acc.x, acc.y);
+                    }
+                if (edge && t * TK + g * kGroup + tok > max_slot) {
+#pragma unroll
+                    for (int j1 = 0; j1 < 8; ++j1) w[j1][0] = w[j1][1] = 0u;
                 }
-                tmem_st_wait();
-            }
-            fence_async_smem();
-            tc_fence_before();
-        }
-        if (warp < 4 || warp == 8) asm volatile("bar.sync 1, 160;" ::: "memory");     // P written
-        if (tid == 8 * 32) {                                           // O += P V
-            tc_fence_after();
+                // this lane addresses row brow of block blk of each x4 store: (j1 = 2i + blk/2, hb = blk%2)
 #pragma unroll
-            for (int k = 0; k < TK / 16; ++k) {
-                const uint64_t pd = umma_desc_k_sw128(smem_u32(smem + C::OFF_P + (k / 4) * TQ * 128)) + 2 * (k % 4);
-                const uint64_t vd = umma_desc_k_sw128(
-                                        smem_u32(smem + C::OFF_V + buf * C::V_BYTES + (k / 4) * DH * 128)) +
-                                    2 * (k % 4);
-                umma_bf16(tmem + 128, pd, vd, idesc_o, kt > 0 || k > 0);
+                for (int i = 0; i < 4; ++i) {
+                    const int f0 = (2 * i + (blk >> 1)) * 16 + (blk & 1) * 8;     // first feature of the block
+                    if (!is_v) {
+                        const int row = g * kGroup + brow;                          // token row
+                        const uint32_t ad = dst + (f0 >> 6) * (TK * 128) + sw128_chunk(row, (f0 & 63) >> 3);
+                        stsm_x4(ad, w[2 * i][0], w[2 * i][1], w[2 * i + 1][0], w[2 * i + 1][1]);
+                    } else {
+                        const int row = f0 + brow;                                  // feature row
+                        const uint32_t ad = dst + (g >> 3) * (DH * 128) + sw128_chunk(row, g & 7);
+                        stsm_x4_t(ad, w[2 * i][0], w[2 * i][1], w[2 * i + 1][0], w[2 * i + 1][1]);
+                    }
+                }
             }
-            umma_commit(bar_pv);
+        };
+        auto step = [&](int t, bool is_v) -> bool {
+            const int s = t & 1;
+            bool ok = wait((is_v ? B_VST_FULL : B_KST_FULL) + s, (t >> 1) & 1);
+            if (ok && !is_v && t >= 2) ok = wait(B_K_EMPTY + s, ((t >> 1) - 1) & 1);
+            if (ok && is_v && t >= 1) ok = wait(B_V_EMPTY, (t - 1) & 1);
+            if (!__all_sync(0xffffffffu, ok)) return false;
+            rebuild(t, is_v);
+            fence_async_smem();        // visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(is_v ? B_V_FULL : B_K_FULL + s));
+                mbar_arrive(bar((is_v ? B_VST_EMPTY : B_KST_EMPTY) + s));
+            }
+            return true;
+        };
+        if (tp.n_kt > 0) {
+            bool ok = step(0, false);
+            for (int t = 0; t < tp.n_kt && ok; ++t) {
+                if (t + 1 < tp.n_kt) ok = step(t + 1, false);
+                if (ok) ok = step(t, true);
+            }
         }
-        if (warp < 4 && !mbar_wait(bar_pv, kt & 1, limit)) {
-            raise_error(a.err, kErrTimeout);
-            ok = false;
+    } else {
+        // ---------------------------------------------------------------- softmax rows
+        const int hh = warp >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        if (tp.act[hh]) {
+            const int qrow = q0 + hh * HQ + row;
+            const int pos = start + qrow;
+            // Q_h: bf16 -> fp16 x qscale in place, once its copy has landed
+            bool ok = wait(B_Q, 0);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                uint4 *q4 = reinterpret_cast<uint4 *>(smem + C::OFF_Q + hh * C::Q_HALF);
+#pragma unroll 4
+                for (int i = row; i < (int)(C::Q_HALF / 16); i += HQ) {
+                    uint4 u = q4[i];
+                    uint32_t *wv = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = unpack_bf16x2(wv[k]);
+                        wv[k] = pack_half2(f.x * a.qscale, f.y * a.qscale);
+                    }
+                    q4[i] = u;
+                }
+                fence_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_QREADY + hh));
+
+            const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+            const uint32_t s_addr = tmem + lane_off + hh * 128;
+            const uint32_t o_addr = tmem + lane_off + 256 + hh * 128;
+            const int row_first = start + q0 + hh * HQ;              // smallest position in the half
+            float m_used = -INFINITY, l_run = 0.f;
+            for (int t = 0; t <= tp.last[hh] && ok; ++t) {
+                ok = __all_sync(0xffffffffu, wait(B_S_FULL + hh, t & 1));
+                if (!ok) break;
+                tc_fence_after();
+                const bool masked = t * TK + TK - 1 > row_first;
+                const int lim = pos - t * TK;                         // keys j <= lim are visible
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c = 0; c < TK / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(s_addr + c * 32, v);
+                    if (masked) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c * 32 + j > lim) v[j] = -INFINITY;
+                    }
+                    float m0 = fmax3(mx, v[0], v[1]);
+#pragma unroll
+                    for (int j = 2; j < 32; j += 2) m0 = fmax3(m0, v[j], v[j + 1]);
+                    mx = m0;
+                }
+                // conditional rescale: move the reference maximum only when it grew past 2^8
+                const bool grow = mx > m_used + kRescaleLog2;
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mx);
+                    m_used = mx;
+                    l_run *= alpha;
+                }
+                if (t > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+                    for (int c = 0; c < DH / 32; ++c) {
+                        float v[32];
+                        tmem_ld32(o_addr + c * 32, v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] *= alpha;
+                        tmem_st32(o_addr + c * 32, v);
+                    }
+                }
+                const float mref = m_used == -INFINITY ? 0.f : m_used;
+                float sum = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < TK / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(s_addr + c * 32, v);
+                    uint32_t pw[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float p0 = ex2(v[j] - mref), p1 = ex2(v[j + 1] - mref);
+                        if (masked) {
+                            if (c * 32 + j > lim) p0 = 0.f;
+                            if (c * 32 + j + 1 > lim) p1 = 0.f;
+                        }
+                        sum += p0 + p1;
+                        pw[j >> 1] = pack_half2(p0, p1);
+                    }
+                    tmem_st16u(s_addr + c * 16, pw);                  // P over the S columns already read
+                }
+                l_run += sum;
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_P_FULL + hh));
+            }
+            // epilogue: O / l, one row per thread
+            if (ok) ok = __all_sync(0xffffffffu, wait(B_O_FINAL + hh, 0));
+            if (ok) {
+                tc_fence_after();
+                const bool write = qrow < a.n_tok;
+                const float inv = l_run > 0.f ? a.out_scale / l_run : 0.f;
+                float *dst = a.out + (((size_t)b * a.n_tok + qrow) * h + head) * DH;
+                bool finite = true;
+#pragma unroll 1
+                for (int c = 0; c < DH / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(o_addr + c * 32, v);
+                    if (write) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 o = make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv);
+                            finite &= fabsf(o.x) <= 3.4e38f && fabsf(o.y) <= 3.4e38f && fabsf(o.z) <= 3.4e38f &&
+                                      fabsf(o.w) <= 3.4e38f;
+                            *reinterpret_cast<float4 *>(dst + c * 32 + j) = o;
+                        }
+                    }
+                }
+                if (!finite) raise_error(a.err, kErrDeviceCheck);
+            }
         }
-        tc_fence_before();
-        __syncthreads();           // next tile rebuilt; S, P and the accumulator free again
-        tc_fence_after();
     }
 
-    if (warp < 4) {
-        const bool write = q0 + row < a.n_tok && ok && n_kt > 0;
-        const float inv = l_run > 0.f ? a.out_scale / l_run : 0.f;
-        float *dst = a.out + (((size_t)b * a.n_tok + q0 + row) * h + head) * DH;
-#pragma unroll 1
-        for (int c = 0; c < DH / 16; ++c) {
-            float v[16];
-            tmem_ld16(orow + c * 16, v);                                // warp-collective
-            if (write)
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4 *>(dst + c * 16 + j) =
-                        make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv);
-        }
-    }
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -379,22 +631,43 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, PrefillArgs a) {
 
 using PrefillKpaH4x4D8x16R2 = PrefillCfg<8, 16, 2, 2>;
 
-bool make_q_map(CUtensorMap *map, const void *q, uint64_t rows, uint64_t cols) {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult qr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) != cudaSuccess ||
             qr != cudaDriverEntryPointSuccess)
-            return false;
+            return nullptr;
         fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     }
+    return fn;
+}
+
+// q [rows][cols] bf16: boxes of 64 columns x 128 rows, 128-byte swizzle.
+bool make_q_map(CUtensorMap *map, const void *q, uint64_t rows, uint64_t cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)TQ};
+    cuuint32_t box[2] = {64, (cuuint32_t)HQ};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A cache plane viewed as [groups][E x 8] bf16 (one row per 8-token group): boxes of
+// 8 elements x 8 tokens (64 values, 128 B) x 16 groups, no swizzle.
+bool make_factor_map(CUtensorMap *map, const void *plane, uint64_t groups, uint64_t e) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {e * kGroup, groups};
+    cuuint64_t strides[1] = {e * kGroup * 2};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(plane), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -415,8 +688,6 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     a.n_tok = n_tok;
     a.cap = cap;
     a.start_pos = start_pos;
-    a.kc = static_cast<const __nv_bfloat16 *>(kc);
-    a.vc = static_cast<const __nv_bfloat16 *>(vc);
     a.out = out;
     a.qscale = qscale;
     a.out_scale = out_scale;
@@ -424,12 +695,15 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     a.h2 = d.h2;
     a.err = err;
     a.wait_limit_ns = wait_limit_ns;
-    CUtensorMap tmq;
-    if (!make_q_map(&tmq, q, (uint64_t)batch * n_tok, (uint64_t)d.h * d.dh)) return cudaErrorInvalidValue;
+    CUtensorMap tmq, tmk, tmv;
+    const uint64_t groups = (uint64_t)batch * cap / kGroup;
+    if (!make_q_map(&tmq, q, (uint64_t)batch * n_tok, (uint64_t)d.h * d.dh) ||
+        !make_factor_map(&tmk, kc, groups, (uint64_t)d.ek) || !make_factor_map(&tmv, vc, groups, (uint64_t)d.ev))
+        return cudaErrorInvalidValue;
     cudaError_t e = ensure_dynamic_smem<prefill_kernel<C>>(C::SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((n_tok + TQ - 1) / TQ), (unsigned)d.h, (unsigned)batch);
-    prefill_kernel<C><<<grid, kThreads, C::SMEM, st>>>(tmq, a);
+    dim3 grid((unsigned)((n_tok + 2 * HQ - 1) / (2 * HQ)), (unsigned)d.h, (unsigned)batch);
+    prefill_kernel<C><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
     return cudaGetLastError();
 }
 

@@ -20,12 +20,18 @@ def _prefill(lib, cfg, batch, n_tok, q, start, kc, vc, cap, sm_scale):
     return out
 
 
-@pytest.mark.parametrize("starts,n_tok", [([0, 0], 256), ([0, 37], 200), ([5, 300], 130)])
-def test_prefill_against_oracle(starts, n_tok):
+# (starts, n_tok, score sharpening): one full 256-row pair; a ragged second half; two
+# rows in the second half; three pairs whose last has no second half; a start past a
+# key-tile boundary over several pairs; and scores sharpened 40x so that the row
+# maxima keep growing from tile to tile and the conditional rescale runs.
+@pytest.mark.parametrize("starts,n_tok,sharp", [([0, 0], 256, 1.0), ([0, 37], 200, 1.0), ([5, 300], 130, 1.0),
+                                               ([0, 3], 600, 1.0), ([130, 0], 520, 1.0), ([0, 64], 384, 40.0)])
+def test_prefill_against_oracle(starts, n_tok, sharp):
     """Random factors in the cache (earlier context + the chunk), random rotated q."""
     lib = kpa()
     s = SHAPE
-    batch, cap = len(starts), 512
+    batch = len(starts)
+    cap = max(512, (max(starts) + n_tok + 7) // 8 * 8)
     w = KPA_MEDIUM.replace(shape=s, batch=batch, capacity=cap, ragged=(), length=cap,
                            factor_std=1.0 / np.sqrt(2.0), seed=41)
     inp = decode_inputs(w)
@@ -36,14 +42,45 @@ def test_prefill_against_oracle(starts, n_tok):
     rng = np.random.default_rng(7)
     q = torch.from_numpy((rng.standard_normal((batch, n_tok, s.h, s.dh)) * 0.3).astype(np.float32)).to(torch.bfloat16)
     start = torch.tensor(starts, dtype=torch.int32)
-    scale = 1.0 / np.sqrt(s.dh)
+    scale = sharp / np.sqrt(s.dh)
     out = _prefill(lib, cfg, batch, n_tok, q, start, kc, vc, cap, scale)
     torch.cuda.synchronize()
     assert lib.kpa_read_device_error() == 0
     kn = to_f64(natural(kc.cpu(), batch, cap, s.e_k))
     vn = to_f64(natural(vc.cpu(), batch, cap, s.e_v))
     want = oracle.prefill(s, to_f64(q), kn, vn, starts, keys_rotated=True, sm_scale=scale)
-    assert_bf16_close(out.cpu().numpy(), want, f"prefill starts={starts} n={n_tok}")
+    assert_bf16_close(out.cpu().numpy(), want, f"prefill starts={starts} n={n_tok} sharp={sharp}")
+
+
+def test_prefill_rescale_when_the_maximum_jumps():
+    """Each query is its own key scaled up, so a row's largest score arrives in its
+    last (diagonal) key tile, far above the earlier tiles: the running maximum moves
+    by more than 2^8 and the accumulated output is rescaled."""
+    lib = kpa()
+    s = SHAPE
+    starts, n_tok, cap = [0, 64], 384, 512
+    batch = len(starts)
+    w = KPA_MEDIUM.replace(shape=s, batch=batch, capacity=cap, ragged=(), length=cap,
+                           factor_std=1.0 / np.sqrt(2.0), seed=43)
+    inp = decode_inputs(w)
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, batch, cap, "bf16")
+    zero = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    lib.kpa_append_factors(cfg, batch, cap, inp["kf"].cuda(), inp["vf"].cuda(), zero, cap, kc, vc)
+    kn = to_f64(natural(kc.cpu(), batch, cap, s.e_k))
+    vn = to_f64(natural(vc.cpu(), batch, cap, s.e_v))
+    q = np.empty((batch, n_tok, s.h, s.dh))
+    for b in range(batch):
+        for t in range(n_tok):
+            q[b, t] = 16.0 * oracle.reconstruct(s.h1, s.h2, s.d1, s.d2, s.r_k, kn[b, starts[b] + t])
+    q = torch.from_numpy(q.astype(np.float32)).to(torch.bfloat16)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = _prefill(lib, cfg, batch, n_tok, q, torch.tensor(starts, dtype=torch.int32), kc, vc, cap, scale)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    want = oracle.prefill(s, to_f64(q), kn, vn, starts, keys_rotated=True, sm_scale=scale)
+    # the self-score dominates: the output is close to the row's own value
+    assert_bf16_close(out.cpu().numpy(), want, "prefill, maximum jumps on the diagonal")
 
 
 def test_prefill_rows_match_decode():
