@@ -55,11 +55,11 @@ using namespace sm100;
 
 constexpr int HQ = 128;                       // query rows per half
 constexpr int TK = 128;                       // keys per tile
-constexpr int kSoftmaxWarps = 8, kRebuildWarps = 4;
-constexpr int kRebuildWarp0 = kSoftmaxWarps;                  // warps 8..11
-constexpr int kMmaWarp = kSoftmaxWarps + kRebuildWarps;       // warp 12
-constexpr int kProducerWarp = kMmaWarp + 1;                   // warp 13
-constexpr int kThreads = (kProducerWarp + 1) * 32;            // 448
+constexpr int kSoftmaxWarps = 8, kRebuildWarps = 8;
+constexpr int kRebuildWarp0 = kSoftmaxWarps;                  // warps 8..15
+constexpr int kMmaWarp = kSoftmaxWarps + kRebuildWarps;       // warp 16
+constexpr int kProducerWarp = kMmaWarp + 1;                   // warp 17
+constexpr int kThreads = (kProducerWarp + 1) * 32;            // 576
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kBox = 16 * 64 * 2;             // TMA box: 16 cache groups x (8 elements x 8 tokens) bf16
@@ -147,6 +147,26 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return r;
 }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
     return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
@@ -165,6 +185,27 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x (x <= 8) for a pair, on the FMA pipe instead of the transcendental unit:
+// Cody-Waite reduction x = n + f with n = round(x) and f in [-1/2, 1/2], a degree-4
+// polynomial for 2^f (coefficients fitted here for minimum relative error on that
+// interval; maximum relative error 2.7e-6), and 2^n added into the exponent field.
+// x is clamped at -126 so the scaled result stays representable (it is then ~1e-38).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kRound = 12582912.f;            // 1.5 * 2^23: x + kRound holds round(x) in its low bits
+    constexpr float c0 = 0x1.ffffe8p-1f, c1 = 0x1.62e0dep-1f, c2 = 0x1.ec06dap-3f, c3 = 0x1.ca13f8p-5f,
+                    c4 = 0x1.399750p-7f;
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 j = fadd2(x, make_float2(kRound, kRound));
+    const float2 f = fsub2(x, fsub2(j, make_float2(kRound, kRound)));
+    float2 p = ffma2(make_float2(c4, c4), f, make_float2(c3, c3));
+    p = ffma2(p, f, make_float2(c2, c2));
+    p = ffma2(p, f, make_float2(c1, c1));
+    p = ffma2(p, f, make_float2(c0, c0));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T (A read from tensor memory), issued by one thread.
@@ -310,6 +351,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
+            const int grp0 = (int)((int64_t)b * a.cap / kGroup);
+            const int ea = RK * a.h1 * D1;     // first B element of a key record
+            const int va = RV * a.h1 * D1;
+            int issued[2][2] = {{-1, -1}, {-1, -1}};
+            // the head's factor slices of tile t: A_r[i1] (one box) and B_r[i2] (two boxes) per rank
+            auto issue_factors = [&](int t, bool is_v) -> bool {
+                const int s = t & 1, grp = grp0 + t * (TK / kGroup);
+                if (t >= 2 && !wait((is_v ? B_VST_EMPTY : B_KST_EMPTY) + s, ((t >> 1) - 1) & 1)) return false;
+                const uint32_t full = bar((is_v ? B_VST_FULL : B_KST_FULL) + s);
+                mbar_expect_tx(full, is_v ? C::V_ST : C::K_ST);
+                unsigned char *st = smem + (is_v ? C::OFF_VST + s * C::V_ST : C::OFF_KST + s * C::K_ST);
+                const CUtensorMap *map = is_v ? &tmv : &tmk;
+                const int R = is_v ? RV : RK, b0 = is_v ? va : ea;
+                for (int r = 0; r < R; ++r) {
+                    tma_load_2d(smem_u32(st + r * kBox), map, (r * a.h1 * D1 + i1 * D1) * kGroup, grp, full);
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb)
+                        tma_load_2d(smem_u32(st + (R + 2 * r + hb) * kBox), map,
+                                    (b0 + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, full);
+                }
+                issued[is_v ? 1 : 0][s] = t;
+                return true;
+            };
+            // the first key tile's factors go out ahead of Q: its rebuild is the first step
+            bool ok = issue_factors(0, false);
             const int nh = (tp.act[0] ? 1 : 0) + (tp.act[1] ? 1 : 0);
             mbar_expect_tx(bar(B_Q), (uint32_t)nh * C::Q_HALF);
 #pragma unroll
@@ -319,41 +385,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     for (int cb = 0; cb < DH / 64; ++cb)
                         tma_load_2d(smem_u32(smem + C::OFF_Q + hh * C::Q_HALF + cb * HQ * 128), &tmq,
                                     head * DH + cb * 64, b * a.n_tok + q0 + hh * HQ, bar(B_Q));
-            const int grp0 = (int)((int64_t)b * a.cap / kGroup);
-            const int ea = RK * a.h1 * D1;     // first B element of a key record
-            const int va = RV * a.h1 * D1;
-            int issued[2][2] = {{-1, -1}, {-1, -1}};
-            bool ok = true;
-            for (int t = 0; t < tp.n_kt && ok; ++t) {
-                const int s = t & 1, grp = grp0 + t * (TK / kGroup);
-                // key factors of tile t
-                if (t >= 2 && !wait(B_KST_EMPTY + s, ((t >> 1) - 1) & 1)) { ok = false; break; }
-                mbar_expect_tx(bar(B_KST_FULL + s), C::K_ST);
-                unsigned char *kst = smem + C::OFF_KST + s * C::K_ST;
-#pragma unroll
-                for (int r = 0; r < RK; ++r) {
-                    tma_load_2d(smem_u32(kst + r * kBox), &tmk, (r * a.h1 * D1 + i1 * D1) * kGroup, grp,
-                                bar(B_KST_FULL + s));
-#pragma unroll
-                    for (int hb = 0; hb < 2; ++hb)
-                        tma_load_2d(smem_u32(kst + (RK + 2 * r + hb) * kBox), &tmk,
-                                    (ea + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, bar(B_KST_FULL + s));
-                }
-                issued[0][s] = t;
-                // value factors of tile t
-                if (t >= 2 && !wait(B_VST_EMPTY + s, ((t >> 1) - 1) & 1)) { ok = false; break; }
-                mbar_expect_tx(bar(B_VST_FULL + s), C::V_ST);
-                unsigned char *vst = smem + C::OFF_VST + s * C::V_ST;
-#pragma unroll
-                for (int r = 0; r < RV; ++r) {
-                    tma_load_2d(smem_u32(vst + r * kBox), &tmv, (r * a.h1 * D1 + i1 * D1) * kGroup, grp,
-                                bar(B_VST_FULL + s));
-#pragma unroll
-                    for (int hb = 0; hb < 2; ++hb)
-                        tma_load_2d(smem_u32(vst + (RV + 2 * r + hb) * kBox), &tmv,
-                                    (va + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, bar(B_VST_FULL + s));
-                }
-                issued[1][s] = t;
+            if (ok) ok = issue_factors(0, true);
+            for (int t = 1; t < tp.n_kt && ok; ++t) {
+                ok = issue_factors(t, false);
+                if (ok) ok = issue_factors(t, true);
             }
             // every copy this thread started lands before the CTA can exit
             (void)mbar_wait(bar(B_Q), 0, limit);
@@ -546,10 +581,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                         for (int j = 0; j < 32; ++j)
                             if (c * 32 + j > lim) v[j] = -INFINITY;
                     }
-                    float m0 = fmax3(mx, v[0], v[1]);
+                    float ma = fmax3(mx, v[0], v[1]), mb = fmax3(v[2], v[3], v[4]);
 #pragma unroll
-                    for (int j = 2; j < 32; j += 2) m0 = fmax3(m0, v[j], v[j + 1]);
-                    mx = m0;
+                    for (int j = 5; j < 29; j += 4) {
+                        ma = fmax3(ma, v[j], v[j + 1]);
+                        mb = fmax3(mb, v[j + 2], v[j + 3]);
+                    }
+                    mx = fmax3(ma, mb, fmax3(v[29], v[30], v[31]));
                 }
                 // conditional rescale: move the reference maximum only when it grew past 2^8
                 const bool grow = mx > m_used + kRescaleLog2;
@@ -570,25 +608,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     }
                 }
                 const float mref = m_used == -INFINITY ? 0.f : m_used;
-                float sum = 0.f;
+                const float2 mref2 = make_float2(mref, mref);
+                float2 suma = make_float2(0.f, 0.f), sumb = make_float2(0.f, 0.f);
 #pragma unroll 1
                 for (int c = 0; c < TK / 32; ++c) {
                     float v[32];
                     tmem_ld32(s_addr + c * 32, v);
                     uint32_t pw[16];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float p0 = ex2(v[j] - mref), p1 = ex2(v[j + 1] - mref);
+                    for (int jp = 0; jp < 16; ++jp) {
+                        const float2 x = fsub2(make_float2(v[2 * jp], v[2 * jp + 1]), mref2);
+                        // one pair in four on the FMA pipe, the rest on the transcendental unit
+                        float2 p = (jp & 3) == 3 ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
                         if (masked) {
-                            if (c * 32 + j > lim) p0 = 0.f;
-                            if (c * 32 + j + 1 > lim) p1 = 0.f;
+                            if (c * 32 + 2 * jp > lim) p.x = 0.f;
+                            if (c * 32 + 2 * jp + 1 > lim) p.y = 0.f;
                         }
-                        sum += p0 + p1;
-                        pw[j >> 1] = pack_half2(p0, p1);
+                        if (jp & 1)
+                            sumb = fadd2(sumb, p);
+                        else
+                            suma = fadd2(suma, p);
+                        pw[jp] = pack_half2(p.x, p.y);
                     }
                     tmem_st16u(s_addr + c * 16, pw);                  // P over the S columns already read
                 }
-                l_run += sum;
+                l_run += (suma.x + suma.y) + (sumb.x + sumb.y);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
