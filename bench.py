@@ -71,6 +71,33 @@ def _dist():
     return rank, world, local
 
 
+def rank_seed(rank: int, layer: int = 0) -> int:
+    """Seed of a rank's replica inputs: every rank draws its own batch."""
+    return 1000 * rank + layer
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (device times are taken as the max over ranks)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    """Work summed over ranks (each replica processes its own batch)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def _kernel_hash():
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
@@ -245,7 +272,7 @@ def run_kpa(a):
     s = w.shape
     elt = 2 if w.dtype == "bf16" else 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    first = decode_inputs(w.replace(seed=1000 * rank))
+    first = decode_inputs(w.replace(seed=rank_seed(rank)))
     lens = first["seq_len"].numpy()
     layer_bytes = int(lens.sum()) * (s.e_k + s.e_v) * elt
     layers = a.layers or max(1, int(np.ceil(4 * l2 / max(layer_bytes, 1))))
@@ -258,7 +285,7 @@ def run_kpa(a):
     seq_len = first["seq_len"].to(dev)
     q_pos = first["q_pos"].to(dev)
     for layer in range(layers):
-        inp = first if layer == 0 else decode_inputs(w.replace(seed=1000 * rank + layer))
+        inp = first if layer == 0 else decode_inputs(w.replace(seed=rank_seed(rank, layer)))
         kc = torch.empty(w.batch * w.capacity * s.e_k, dtype=tdt, device=dev)
         vc = torch.empty(w.batch * w.capacity * s.e_v, dtype=tdt, device=dev)
         kpa.kpa_append_factors(cfg, w.batch, w.capacity, inp["kf"].to(dev), inp["vf"].to(dev),
@@ -319,12 +346,7 @@ def run_kpa(a):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms / steps
+        return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
 
     with torch.cuda.stream(stream):
         # settle clocks under load (untimed) while the sampler runs
@@ -342,8 +364,9 @@ def run_kpa(a):
         raise RuntimeError(f"device error word {code} after the timed region")
 
     tokens_per_layer = int(lens.sum())
-    value = world * tokens_per_layer * layers / (ms_step * 1e-3)
-    e2e_value = world * tokens_per_layer * layers / (ms_e2e * 1e-3)
+    tokens_all = sum_over_ranks(tokens_per_layer, world, dev)       # every rank's own batch
+    value = tokens_all * layers / (ms_step * 1e-3)
+    e2e_value = tokens_all * layers / (ms_e2e * 1e-3)
     t_launch = ms_step * 1e-3 / layers            # average decode call (split + combine)
     achieved = layer_bytes / t_launch / 1e9
     peak, peak_kind = _hbm_peak()
@@ -365,7 +388,7 @@ def run_kpa(a):
                     "d2h_bytes_per_step": int(sum(o.numel() * o.element_size() for o in outs)),
                     "ms_per_step": ms_e2e, "path": "pinned host q -> kpa_decode x layers -> pinned host out, one CUDA graph"},
             "clocks": clocks,
-            "gpu_launches": a.steps * layers * 2}
+            "gpu_launches": a.steps * layers * kpa.kpa_decode_plan(cfg, w.batch, max_len)[2]}
 
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         base, _ = _cpu_baseline(w, first, a.cpu_seconds)
@@ -389,33 +412,54 @@ def _bf16_peak():
 
 
 def run_append_prefill(a):
-    """The append + prefill configuration: kpa_append of a 2048-token chunk per
-    sequence (merged projection, factor RoPE, cache write, query assembly) and the
-    causal kpa_prefill over it, each timed with CUDA events on its stream."""
+    """The append + prefill configuration, one step = the whole path of a prompt
+    chunk and the token after it:
+      1. kpa_append of a 2048-token chunk per sequence (merged projection, factor
+         RoPE, cache write, query assembly),
+      2. the causal kpa_prefill of the chunk over the cache,
+      3. the decode step: kpa_append of token 2048 of every sequence, then kpa_decode
+         of its query over the 2049 cached slots.
+    Each part is timed with CUDA events on its stream; the line's roofline is the
+    prefill kernel's (tensor bound)."""
     import torch
+    import torch.distributed as dist
     import factorised_kv_attention_b200 as kpa
     from workloads import APPEND_PREFILL, append_inputs
 
     rank, world, local = _dist()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     w = APPEND_PREFILL
     s = w.shape
-    inp = append_inputs(w.replace(seed=1000 * rank))
+    inp = append_inputs(w.replace(seed=rank_seed(rank)))
     cfg = kpa.make_config(s, "bf16")
-    x, W = inp["x"].to(dev), inp["W"].to(dev)
+    x, W, x1 = inp["x"].to(dev), inp["W"].to(dev), inp["x_step"].to(dev)
     kc = torch.zeros(w.batch * w.capacity * s.e_k, dtype=torch.bfloat16, device=dev)
     vc = torch.zeros(w.batch * w.capacity * s.e_v, dtype=torch.bfloat16, device=dev)
     start = torch.zeros(w.batch, dtype=torch.int32, device=dev)
     ws = torch.zeros(kpa.kpa_append_workspace_size(cfg, w.batch, w.n_tok), dtype=torch.uint8, device=dev)
     q = torch.empty(w.batch, w.n_tok, s.h, s.dh, dtype=torch.bfloat16, device=dev)
     out = torch.empty(w.batch, w.n_tok, s.h, s.dh, dtype=torch.float32, device=dev)
+    # decode step: token n_tok of every sequence, attending over n_tok + 1 slots
+    pos1 = torch.full((w.batch,), w.n_tok, dtype=torch.int32, device=dev)
+    len1 = torch.full((w.batch,), w.n_tok + 1, dtype=torch.int32, device=dev)
+    ws1 = torch.zeros(max(kpa.kpa_append_workspace_size(cfg, w.batch, 1), 256), dtype=torch.uint8, device=dev)
+    q1 = torch.empty(w.batch, 1, s.h, s.dh, dtype=torch.bfloat16, device=dev)
+    wsd = torch.zeros(max(kpa.kpa_decode_workspace_size(cfg, w.batch, w.n_tok + 1), 256), dtype=torch.uint8,
+                      device=dev)
+    out1 = torch.empty(w.batch, s.h, s.dh, dtype=torch.float32, device=dev)
     scale = 1.0 / float(np.sqrt(s.dh))
     stream = torch.cuda.Stream(device=dev)
     M = w.batch * w.n_tok
     proj_flop = 2.0 * M * s.n_proj * s.d_model
     pre_flop = 4.0 * s.h * s.dh * w.batch * (w.n_tok * (w.n_tok + 1) / 2)
+    dec_bytes = w.batch * (w.n_tok + 1) * (s.e_k + s.e_v) * 2
     sampler = ClockSampler(local)
+    _, _, dec_launches = kpa.kpa_decode_plan(cfg, w.batch, w.n_tok + 1)
+    launches_per_step = 2 + 1 + 2 + dec_launches     # append (GEMM + query assembly), prefill, step
 
     def append():
         kpa.kpa_append(cfg, w.batch, w.n_tok, x, W, start, w.capacity, kc, vc, q, ws, stream=stream)
@@ -423,53 +467,80 @@ def run_append_prefill(a):
     def prefill():
         kpa.kpa_prefill(cfg, w.batch, w.n_tok, q, start, kc, vc, w.capacity, scale, out, stream=stream)
 
+    def decode_step():
+        kpa.kpa_append(cfg, w.batch, 1, x1, W, pos1, w.capacity, kc, vc, q1, ws1, stream=stream)
+        kpa.kpa_decode(cfg, w.batch, q1, None, kc, vc, w.capacity, len1, w.n_tok + 1, scale, out1, wsd,
+                       stream=stream)
+
     with torch.cuda.stream(stream):
         for _ in range(a.warmup):
             append()
             prefill()
+            decode_step()
         stream.synchronize()
         sampler.start()
         t_end = time.time() + a.settle_seconds
         while time.time() < t_end:
             append()
             prefill()
+            decode_step()
             stream.synchronize()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * a.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4 * a.steps)]
         for i in range(a.steps):
-            ev[3 * i].record(stream)
+            ev[4 * i].record(stream)
             append()
-            ev[3 * i + 1].record(stream)
+            ev[4 * i + 1].record(stream)
             prefill()
-            ev[3 * i + 2].record(stream)
+            ev[4 * i + 2].record(stream)
+            decode_step()
+            ev[4 * i + 3].record(stream)
         stream.synchronize()
+        torch.cuda.synchronize()
         clocks = sampler.stop()
-        # end to end through the API: pinned x -> device, append + prefill, out -> pinned host
-        x_host = inp["x"].pin_memory()
+        # end to end through the API: pinned x -> device, the step, out and the step's out -> pinned host
+        x_host, x1_host = inp["x"].pin_memory(), inp["x_step"].pin_memory()
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        out1_host = torch.empty(out1.shape, dtype=out1.dtype).pin_memory()
+        if world > 1:
+            dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(a.steps):
             x.copy_(x_host, non_blocking=True)
+            x1.copy_(x1_host, non_blocking=True)
             append()
             prefill()
+            decode_step()
             out_host.copy_(out, non_blocking=True)
+            out1_host.copy_(out1, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
     code = kpa.kpa_read_device_error(stream)
     if code != 0:
         raise RuntimeError(f"device error word {code}")
-    t_app = float(np.mean([ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(a.steps)])) * 1e-3
-    t_pre = float(np.mean([ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(a.steps)])) * 1e-3
-    ms_e2e = e0.elapsed_time(e1) / a.steps
+
+    def part(k):
+        return float(np.mean([ev[4 * i + k].elapsed_time(ev[4 * i + k + 1]) for i in range(a.steps)])) * 1e-3
+
+    t_app, t_pre, t_dec = part(0), part(1), part(2)
+    t_step = max_over_ranks(t_app + t_pre + t_dec, world, dev)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / a.steps, world, dev)
+    tokens_all = sum_over_ranks(M + w.batch, world, dev)         # chunk tokens + the decoded token
     peak, peak_sus, kind = _bf16_peak()
+    hbm, hbm_kind = _hbm_peak()
     pre_tf, app_tf = pre_flop / t_pre / 1e12, proj_flop / t_app / 1e12
-    line = {"metric": "append + causal prefill tokens/s (2048-token chunks); TFLOP/s vs B200 bf16 peak",
-            "value": M / (t_app + t_pre), "unit": "tokens/s", "n_gpus": 1, "steps": a.steps,
-            "warmup": a.warmup, "ms_per_step": (t_app + t_pre) * 1e3, "higher_is_better": True,
+    line = {"metric": "append + causal prefill + decode step, tokens/s (2048-token chunks); "
+                      "TFLOP/s vs B200 bf16 peak",
+            "value": tokens_all / t_step, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate (prefill MMA in fp16)",
             "data": "synthetic (seeded)",
             "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_tok, "d_model": s.d_model,
-                       "l2": "projection input 67 MB and prefill output 134 MB per step exceed L2"},
+                       "l2": "projection input 67 MB and prefill output 134 MB per step exceed L2",
+                       "parallelism": f"replicas x{world} (batch-sharded, no exchange)"},
             "roofline": {"bound": "tensor", "achieved": pre_tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": pre_tf / peak, "traffic": None,
                          "peak_source": f"{kind} bf16_tflops (burst; fp16 dense rate is the same)",
@@ -477,11 +548,19 @@ def run_append_prefill(a):
                          "launch_us": t_pre * 1e6},
             "append": {"achieved_tflops": app_tf, "frac": app_tf / peak, "launch_us": t_app * 1e6,
                        "algorithmic_flop_per_launch": proj_flop},
-            "e2e": {"value": M / (ms_e2e * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(out_host.numel() * 4),
+            "decode_step": {"launch_us": t_dec * 1e6, "cache_bytes": dec_bytes,
+                            "achieved_gbs": dec_bytes / t_dec / 1e9, "hbm_peak_gbs": hbm,
+                            "note": "append of one token per sequence + decode over 2049 slots (latency bound)"},
+            "e2e": {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_host.numel() * 2 + x1_host.numel() * 2),
+                    "d2h_bytes_per_step": int(out_host.numel() * 4 + out1_host.numel() * 4),
                     "ms_per_step": ms_e2e},
-            "clocks": clocks, "gpu_launches": a.steps * 3}
-    print(json.dumps(line), flush=True)
+            "clocks": clocks, "gpu_launches": a.steps * launches_per_step}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     return 0
 
 

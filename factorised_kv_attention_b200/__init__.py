@@ -52,12 +52,14 @@ class KpaError(RuntimeError):
 _vp, _i32, _sz, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
 _cfgp = ctypes.POINTER(kpa_config)
 _szp = ctypes.POINTER(ctypes.c_size_t)
+_i32p = ctypes.POINTER(ctypes.c_int32)
 _SIGS = {
     "kpa_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kpa_last_cuda_error": ([], ctypes.c_int),
     "kpa_cache_bytes_per_token": ([_cfgp, _szp, _szp], ctypes.c_int),
     "kpa_append_factors": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
     "kpa_decode_workspace_size": ([_cfgp, _i32, _i32, _i32, _szp], ctypes.c_int),
+    "kpa_decode_plan": ([_cfgp, _i32, _i32, _i32, _i32p, _i32p, _i32p], ctypes.c_int),
     "kpa_decode": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp, _sz, _vp],
                    ctypes.c_int),
     "kpa_decode_split": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _i32, _vp, _vp,
@@ -137,6 +139,14 @@ def kpa_decode_workspace_size(cfg, batch, max_len, tokens_per_split=0) -> int:
     _check(_lib.kpa_decode_workspace_size(ctypes.byref(cfg), batch, max_len, tokens_per_split,
                                           ctypes.byref(n)), "kpa_decode_workspace_size")
     return n.value
+
+
+def kpa_decode_plan(cfg, batch, max_len, tokens_per_split=0):
+    """(splits per sequence, tokens per split, kernel launches per kpa_decode call)."""
+    n, t, l = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib.kpa_decode_plan(ctypes.byref(cfg), batch, max_len, tokens_per_split, ctypes.byref(n),
+                                ctypes.byref(t), ctypes.byref(l)), "kpa_decode_plan")
+    return n.value, t.value, l.value
 
 
 def kpa_decode(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len, sm_scale, out,

@@ -257,6 +257,24 @@ kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32
     return KPA_OK;
 }
 
+kpa_status kpa_decode_plan(const kpa_config *cfg, int32_t batch, int32_t max_len,
+                           int32_t tokens_per_split, int32_t *n_split, int32_t *tokens_per_split_out,
+                           int32_t *launches) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
+    int sms = 0;
+    s = device_state(nullptr, &sms);
+    if (s != KPA_OK) return s;
+    DecodePlan p;
+    s = plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
+    if (s != KPA_OK) return s;
+    if (n_split) *n_split = p.n_split;
+    if (tokens_per_split_out) *tokens_per_split_out = p.tokens_per_split;
+    if (launches) *launches = batch == 0 ? 0 : (max_len > 0 && !p.fused ? 2 : 1);
+    return KPA_OK;
+}
+
 kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
                             const int32_t *q_pos, const void *kcache, const void *vcache,
                             int32_t capacity, const int32_t *seq_len, int32_t max_len,

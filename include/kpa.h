@@ -114,6 +114,15 @@ kpa_status kpa_append_factors(const kpa_config *cfg, int32_t batch, int32_t n_to
 kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32_t max_len,
                                      int32_t tokens_per_split, size_t *bytes);
 
+/* How kpa_decode will split the work for these sizes (host only): the splits
+ * per sequence, the tokens in each split, and the kernel launches one call
+ * enqueues (1 when the splits of a sequence are merged inside the decode
+ * kernel, 2 when a separate combine kernel follows).  Any output pointer may be
+ * NULL.  Same argument rules as kpa_decode_workspace_size. */
+kpa_status kpa_decode_plan(const kpa_config *cfg, int32_t batch, int32_t max_len,
+                           int32_t tokens_per_split, int32_t *n_split,
+                           int32_t *tokens_per_split_out, int32_t *launches);
+
 /* Factor-space decode attention: one query row per sequence against slots
  * 0 .. seq_len[b]-1 of the cache (Proposition 2.2 evaluated with a dense
  * query, Theorem 2.4 for the positions; FlashTPA-style blocking over the cache
