@@ -50,6 +50,45 @@ __device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap
         __float2bfloat16_rn(v);
 }
 
+// One pair of projected columns (n, n+1) of token m: rotate it when it is a B^Q or B^K
+// pair (cs(j) = (cos, sin) of pair j of the token's position), then keep query
+// factors in fp32 and write key / value factors to the token's cache slot in bf16.
+template <class CS>
+__device__ __forceinline__ void emit_pair(const AppendArgs &a, int m, int b, int s, bool slot_ok, int n,
+                                          float x0, float x1, CS cs) {
+    const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1;
+    if (n < a.eq) {                                        // query factors
+        if (n >= qa) {                                     // B^Q: rotate the pair
+            const float2 w = cs(((n - qa) % a.d2) >> 1);
+            const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
+            x0 = y0;
+            x1 = y1;
+        }
+        if (a.qf) {
+            a.qf[(size_t)n * a.M + m] = x0;
+            a.qf[(size_t)(n + 1) * a.M + m] = x1;
+        }
+    } else if (n < a.eq + a.ek) {                          // key factors
+        const int e = n - a.eq;
+        if (e >= ka) {                                     // B^K: rotate the pair
+            const float2 w = cs(((e - ka) % a.d2) >> 1);
+            const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
+            x0 = y0;
+            x1 = y1;
+        }
+        if (slot_ok) {
+            store_cache(a.kc, b, a.cap, a.ek, s, e, x0);
+            store_cache(a.kc, b, a.cap, a.ek, s, e + 1, x1);
+        }
+    } else {                                               // value factors, never rotated
+        const int e = n - a.eq - a.ek;
+        if (slot_ok) {
+            store_cache(a.vc, b, a.cap, a.ev, s, e, x0);
+            store_cache(a.vc, b, a.cap, a.ev, s, e + 1, x1);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                    AppendArgs a, RopeTable rope) {
@@ -160,7 +199,6 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
         const bool acc_ok = mbar_wait(accf, 0, limit) && !*abort_flag;
         if (!acc_ok) raise_error(a.err, kErrTimeout);
         tc_fence_after();
-        const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1, va = a.rv * a.h1 * a.d1;
         for (int ch = 0; ch < BN / 16; ++ch) {
             float v[16];
             tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16, v);   // warp-collective
@@ -168,40 +206,8 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
             const int n0 = tile_n * BN + ch * 16;
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
-                const int n = n0 + j;
-                if (n >= a.N) break;
-                float x0 = v[j], x1 = v[j + 1];
-                if (n < a.eq) {                                    // query factors
-                    if (n >= qa) {                                 // B^Q: rotate the pair
-                        const float2 w = cs[((n - qa) % a.d2) >> 1];
-                        const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
-                        x0 = y0;
-                        x1 = y1;
-                    }
-                    if (a.qf) {
-                        a.qf[(size_t)n * a.M + m] = x0;
-                        a.qf[(size_t)(n + 1) * a.M + m] = x1;
-                    }
-                } else if (n < a.eq + a.ek) {                      // key factors
-                    const int e = n - a.eq;
-                    if (e >= ka) {                                 // B^K: rotate the pair
-                        const float2 w = cs[((e - ka) % a.d2) >> 1];
-                        const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
-                        x0 = y0;
-                        x1 = y1;
-                    }
-                    if (slot_ok) {
-                        store_cache(a.kc, b, a.cap, a.ek, s, e, x0);
-                        store_cache(a.kc, b, a.cap, a.ek, s, e + 1, x1);
-                    }
-                } else {                                           // value factors, never rotated
-                    const int e = n - a.eq - a.ek;
-                    (void)va;
-                    if (slot_ok) {
-                        store_cache(a.vc, b, a.cap, a.ev, s, e, x0);
-                        store_cache(a.vc, b, a.cap, a.ev, s, e + 1, x1);
-                    }
-                }
+                if (n0 + j >= a.N) break;
+                emit_pair(a, m, b, s, slot_ok, n0 + j, v[j], v[j + 1], [&](int k) { return cs[k]; });
             }
         }
     }
@@ -211,6 +217,122 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// The projection for a handful of tokens (a decode step): a matrix-vector product
+// that streams W once.  One CTA per pair of W rows (n, n+1), so a rotated pair is
+// formed in one place; its 8 warps split K, each lane holding 8 consecutive k of
+// both rows and of every token (X stays in L2), then the partial sums are reduced
+// with shuffles and through shared memory.  Thread m runs the epilogue of token m.
+constexpr int kSmallMaxM = 16, kSmallWarps = 8;
+
+__global__ void __launch_bounds__(kSmallWarps * 32)
+append_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, AppendArgs a,
+                    RopeTable rope) {
+    __shared__ float red[kSmallWarps][2][kSmallMaxM];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = 2 * blockIdx.x;
+    float acc0[kSmallMaxM], acc1[kSmallMaxM];
+#pragma unroll
+    for (int m = 0; m < kSmallMaxM; ++m) acc0[m] = acc1[m] = 0.f;
+    const int k8n = a.K / 8;
+    const uint4 *w0 = reinterpret_cast<const uint4 *>(w + (size_t)n * a.K);
+    const uint4 *w1 = reinterpret_cast<const uint4 *>(w + (size_t)(n + 1) * a.K);
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    for (int k8 = tid; k8 < k8n; k8 += kSmallWarps * 32) {
+        const uint4 ua = __ldg(w0 + k8), ub = __ldg(w1 + k8);
+        const __nv_bfloat162 *pa = reinterpret_cast<const __nv_bfloat162 *>(&ua);
+        const __nv_bfloat162 *pb = reinterpret_cast<const __nv_bfloat162 *>(&ub);
+        float fa[8], fb[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 ta = __bfloat1622float2(pa[i]), tb = __bfloat1622float2(pb[i]);
+            fa[2 * i] = ta.x;
+            fa[2 * i + 1] = ta.y;
+            fb[2 * i] = tb.x;
+            fb[2 * i + 1] = tb.y;
+        }
+#pragma unroll
+        for (int m = 0; m < kSmallMaxM; ++m) {
+            if (m >= a.M) break;
+            const uint4 ux = __ldg(xv + (size_t)m * k8n + k8);
+            const __nv_bfloat162 *px = reinterpret_cast<const __nv_bfloat162 *>(&ux);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 tx = __bfloat1622float2(px[i]);
+                acc0[m] = fmaf(fa[2 * i], tx.x, fmaf(fa[2 * i + 1], tx.y, acc0[m]));
+                acc1[m] = fmaf(fb[2 * i], tx.x, fmaf(fb[2 * i + 1], tx.y, acc1[m]));
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < kSmallMaxM; ++m) {
+        if (m >= a.M) break;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            acc0[m] += __shfl_xor_sync(0xffffffffu, acc0[m], off);
+            acc1[m] += __shfl_xor_sync(0xffffffffu, acc1[m], off);
+        }
+        if (lane == 0) {
+            red[warp][0][m] = acc0[m];
+            red[warp][1][m] = acc1[m];
+        }
+    }
+    __syncthreads();
+    if (tid >= a.M) return;
+    const int m = tid;
+    float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSmallWarps; ++i) {
+        x0 += red[i][0][m];
+        x1 += red[i][1][m];
+    }
+    const int b = m / a.n_tok, s = a.start_pos[b] + (m - b * a.n_tok);
+    const bool slot_ok = s >= 0 && s < a.cap;
+    if (!slot_ok && n == 0) raise_error(a.err, kErrDeviceCheck);
+    emit_pair(a, m, b, s, slot_ok, n, x0, x1, [&](int j) {
+        float c, sn;
+        rope_cs((double)s, rope.theta[j], c, sn);
+        return make_float2(c, sn);
+    });
+}
+
+// Query assembly for a handful of tokens: one thread per 16-byte chunk of q_out,
+// (token, head, j1, 8 features of j2).
+__global__ void __launch_bounds__(128)
+q_assemble_small_kernel(const float *__restrict__ qf, int M, int h1, int h2, int d1, int d2, int rq,
+                        __nv_bfloat16 *__restrict__ q_out) {
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    const int per_head = d1 * (d2 / 8), h = h1 * h2;
+    if (idx >= M * h * per_head) return;
+    const int m = idx / (h * per_head), rem = idx % (h * per_head);
+    const int head = rem / per_head, j1 = (rem % per_head) / (d2 / 8), j2 = (rem % (d2 / 8)) * 8;
+    const int i1 = head / h2, i2 = head % h2, qa = rq * h1 * d1;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // ranks in groups of 4 with every load of a group issued before its arithmetic
+    for (int r0 = 0; r0 < rq; r0 += 4) {
+        float av[4], bv[4][8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = r0 + k < rq ? r0 + k : rq - 1;
+            av[k] = r0 + k < rq ? __ldg(qf + (size_t)((r * h1 + i1) * d1 + j1) * M + m) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) bv[k][u] = __ldg(qf + (size_t)(qa + (r * h2 + i2) * d2 + j2 + u) * M + m);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] += av[k] * bv[k][u];
+    }
+    const float inv = 1.0f / (float)rq;
+    uint4 o;
+    uint32_t *po = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 hb = __floats2bfloat162_rn(acc[2 * k] * inv, acc[2 * k + 1] * inv);
+        po[k] = *reinterpret_cast<uint32_t *>(&hb);
+    }
+    *reinterpret_cast<uint4 *>(q_out + ((size_t)m * h + head) * d1 * d2 + j1 * d2 + j2) = o;
 }
 
 // Query assembly q = (1/R_Q) sum_r A^Q_r (x) B^Q_r for the queries of the chunk.
@@ -345,19 +467,31 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     a.err = err;
     a.wait_limit_ns = wait_limit_ns;
 
+    cudaError_t e;
+    const bool small = a.M <= kSmallMaxM;
+    if (small) {
+        // a decode step: stream W once with a matrix-vector kernel
+        append_small_kernel<<<(unsigned)(a.N / 2), kSmallWarps * 32, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w), a, rope);
+    } else {
     CUtensorMap tmx, tmw;
     if (!make_map(&tmx, x, (uint64_t)a.M, (uint64_t)d_model, BM)) return cudaErrorInvalidValue;
     if (!make_map(&tmw, w, (uint64_t)a.N, (uint64_t)d_model, (uint32_t)a.BN)) return cudaErrorInvalidValue;
     const size_t smem = append_smem_bytes(a.BN, a.stages, d.d2);
-    cudaError_t e = ensure_dynamic_smem<append_gemm_kernel>(smem);
+    e = ensure_dynamic_smem<append_gemm_kernel>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.N + a.BN - 1) / a.BN), (unsigned)((a.M + BM - 1) / BM));
     append_gemm_kernel<<<grid, kThreads, smem, st>>>(tmx, tmw, a, rope);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess || !q_out) return e;
     __nv_bfloat16 *qo = static_cast<__nv_bfloat16 *>(q_out);
     const dim3 g2((unsigned)((a.M + 63) / 64), (unsigned)d.h2);
-    if (rq == 6 && d.d1 == 8 && d.d2 == 16) {
+    if (small && d.d2 % 8 == 0) {
+        const int threads = a.M * d.h * d.d1 * (d.d2 / 8);
+        q_assemble_small_kernel<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(qf, a.M, d.h1, d.h2, d.d1,
+                                                                                  d.d2, rq, qo);
+    } else if (rq == 6 && d.d1 == 8 && d.d2 == 16) {
         q_assemble_kernel<6, 8, 16><<<g2, 64, 0, st>>>(qf, a.M, d.h1, d.h2, qo);
     } else {
         dim3 g3((unsigned)((a.M + 127) / 128), (unsigned)d.h);

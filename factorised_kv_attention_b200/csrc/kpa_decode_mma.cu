@@ -624,32 +624,54 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     float *po = a.part_o + ((size_t)(b * a.n_split + split) * H) * DH;
     float *pml = a.part_ml + ((size_t)(b * a.n_split + split) * H) * 2;
-    for (int idx = tid; idx < H * DH; idx += WARPS * 32) {
-        const int head = idx / DH;
-        float M = -INFINITY;
+    // log-sum-exp weights of the slices, once per head: 2^(m_slice - M) in place of m
+    if constexpr (SLICES > 1) {
+        for (int head = tid; head < H; head += WARPS * 32) {
+            float M = -INFINITY;
 #pragma unroll
-        for (int sl = 0; sl < SLICES; ++sl) M = fmaxf(M, mm[((size_t)sl * H + head) * 2]);
-        float acc = 0.f, l = 0.f;
+            for (int sl = 0; sl < SLICES; ++sl) M = fmaxf(M, mm[((size_t)sl * H + head) * 2]);
+            float l = 0.f;
 #pragma unroll
-        for (int sl = 0; sl < SLICES; ++sl) {
-            const float ms = mm[((size_t)sl * H + head) * 2];
-            const float wgt = ms == -INFINITY ? 0.f : exp2f(ms - M);
-            acc += wgt * mo[((size_t)sl * H) * DH + idx];
-            l += wgt * mm[((size_t)sl * H + head) * 2 + 1];
-        }
-        if (a.cluster) {
-            cp[idx] = acc;
-            if (idx % DH == 0) {
+            for (int sl = 0; sl < SLICES; ++sl) {
+                const float ms = mm[((size_t)sl * H + head) * 2];
+                const float wgt = ms == -INFINITY ? 0.f : exp2f(ms - M);
+                mm[((size_t)sl * H + head) * 2] = wgt;
+                l += wgt * mm[((size_t)sl * H + head) * 2 + 1];
+            }
+            if (a.cluster) {
                 cp[H * DH + head] = M;
                 cp[H * DH + H + head] = l;
-            }
-        } else {
-            po[idx] = acc;
-            if (idx % DH == 0) {
+            } else {
                 pml[2 * head] = M;
                 pml[2 * head + 1] = l;
             }
         }
+        asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    }
+    for (int idx = tid; idx < H * DH; idx += WARPS * 32) {
+        const int head = idx / DH;
+        float acc;
+        if constexpr (SLICES > 1) {
+            acc = 0.f;
+#pragma unroll
+            for (int sl = 0; sl < SLICES; ++sl)
+                acc += mm[((size_t)sl * H + head) * 2] * mo[((size_t)sl * H) * DH + idx];
+        } else {
+            acc = mo[idx];
+            if (idx % DH == 0) {
+                if (a.cluster) {
+                    cp[H * DH + head] = mm[head * 2];
+                    cp[H * DH + H + head] = mm[head * 2 + 1];
+                } else {
+                    pml[2 * head] = mm[head * 2];
+                    pml[2 * head + 1] = mm[head * 2 + 1];
+                }
+            }
+        }
+        if (a.cluster)
+            cp[idx] = acc;
+        else
+            po[idx] = acc;
     }
     if (!a.cluster) {
     if (!a.fused) return;
@@ -666,7 +688,18 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     __threadfence();
     const float *pob = a.part_o + (size_t)b * a.n_split * H * DH;
     const float *pmb = a.part_ml + (size_t)b * a.n_split * H * 2;
-    // split statistics first, all loads in flight together: w[i][head] = 2^(m_i - M), then l
+    // The first float4 column of every thread is requested for up to PF splits at once,
+    // before the split statistics, so the partials arrive in one round trip.
+    constexpr int PF = 16;
+    constexpr int N4 = H * DH / 4;
+    const float4 *pob4 = reinterpret_cast<const float4 *>(pob);
+    float4 pre[PF];
+    if (tid < N4) {
+#pragma unroll
+        for (int i = 0; i < PF; ++i)
+            if (i < n_b) pre[i] = __ldcg(pob4 + (size_t)i * N4 + tid);
+    }
+    // split statistics: w[i][head] = 2^(m_i - M), then the denominators
     float *wt = reinterpret_cast<float *>(smem);            // [n_b][H]
     float *den = wt + (size_t)n_b * H;                      // [H]
     float *lv = den + H;                                    // [n_b][H]
@@ -688,27 +721,35 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         den[head] = d;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    // every output of this thread accumulates together, so each split's loads are in flight at once
-    constexpr int OPT = (H * DH + WARPS * 32 - 1) / (WARPS * 32);
-    float num[OPT];
+    for (int c4 = tid; c4 < N4; c4 += WARPS * 32) {
+        const int head = (c4 * 4) / DH;
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        int i0 = 0;
+        if (c4 == tid) {                                    // the prefetched column
 #pragma unroll
-    for (int k = 0; k < OPT; ++k) num[k] = 0.f;
-#pragma unroll 2
-    for (int i = 0; i < n_b; ++i) {
-        const float *pi = pob + (size_t)i * H * DH;
-#pragma unroll
-        for (int k = 0; k < OPT; ++k) {
-            const int idx = tid + k * WARPS * 32;
-            if (idx < H * DH) num[k] += wt[i * H + idx / DH] * __ldcg(pi + idx);
+            for (int i = 0; i < PF; ++i)
+                if (i < n_b) {
+                    const float w = wt[i * H + head];
+                    num.x += w * pre[i].x;
+                    num.y += w * pre[i].y;
+                    num.z += w * pre[i].z;
+                    num.w += w * pre[i].w;
+                }
+            i0 = PF;
         }
-    }
-#pragma unroll
-    for (int k = 0; k < OPT; ++k) {
-        const int idx = tid + k * WARPS * 32;
-        if (idx < H * DH) {
-            const float d = den[idx / DH];
-            a.out[(size_t)b * H * DH + idx] = d > 0.f ? a.out_scale * num[k] / d : 0.f;
+#pragma unroll 8
+        for (int i = i0; i < n_b; ++i) {
+            const float4 v = __ldcg(pob4 + (size_t)i * N4 + c4);
+            const float w = wt[i * H + head];
+            num.x += w * v.x;
+            num.y += w * v.y;
+            num.z += w * v.z;
+            num.w += w * v.w;
         }
+        const float d = den[head];
+        const float f = d > 0.f ? a.out_scale / d : 0.f;
+        reinterpret_cast<float4 *>(a.out + (size_t)b * H * DH)[c4] = make_float4(num.x * f, num.y * f, num.z * f,
+                                                                                 num.w * f);
     }
     if (tid == 0) a.counters[b] = 0;                 // ready for the next call
     return;

@@ -102,3 +102,23 @@ def test_append_without_query_and_out_of_range_slot():
     kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
     _close_bf16(kn[0, :20], k_rot[0], "sequence 0")
     _close_bf16(kn[1, 50:64], k_rot[1, :14], "sequence 1, slots inside the cache")
+
+
+def test_append_few_tokens_against_oracle():
+    """A decode-sized append (batch 3 x 5 tokens: the matrix-vector path) against the
+    oracle, at start positions that are not multiples of the cache group."""
+    w = SMALL.replace(shape=SMALL_SHAPE, batch=3, n_tok=5, capacity=64, seed=9)
+    s = w.shape
+    inp = append_inputs(w)
+    start = torch.tensor([0, 13, 58], dtype=torch.int32)
+    lib = kpa()
+    _, kc, vc, q_out = _run_append(lib, w, inp, start)
+    q_rot, k_rot, v_rec, _ = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start.numpy())
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    for b in range(w.batch):
+        st = int(start[b])
+        _close_bf16(kn[b, st:st + w.n_tok], k_rot[b], f"key cache b={b}")
+        _close_bf16(vn[b, st:st + w.n_tok], v_rec[b], f"value cache b={b}")
+        assert np.all(kn[b, :st] == 0) and np.all(kn[b, st + w.n_tok:] == 0), "wrote outside its slots"
+    _close_bf16(to_f64(q_out.cpu()), q_rot, "assembled query")
