@@ -593,7 +593,8 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const bool ok = !(aborted || flags[0]);
     if (!ok && !a.cluster) return;
     float *mo = reinterpret_cast<float *>(smem);                   // [SLICES][H][DH]
-    float *mm = mo + SLICES * H * DH;                              // [SLICES][H][2]
+    constexpr int MO_LD = C::MO_LD;
+    float *mm = mo + SLICES * H * MO_LD;                           // [SLICES][H][2]
     float *cp = mm + SLICES * H * 2;                               // merged: [H][DH] o, [H] m, [H] l
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
@@ -602,7 +603,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             const int row = mt * 16 + g + 8 * hr;
             const int i1 = row / D1, j1 = row % D1;
             const int head = i1 * H2 + i2;
-            float *dst = mo + ((size_t)slice * H + head) * DH + j1 * D2;
+            float *dst = mo + ((size_t)slice * H + head) * MO_LD + j1 * D2;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
                 *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
@@ -655,9 +656,9 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             acc = 0.f;
 #pragma unroll
             for (int sl = 0; sl < SLICES; ++sl)
-                acc += mm[((size_t)sl * H + head) * 2] * mo[((size_t)sl * H) * DH + idx];
+                acc += mm[((size_t)sl * H + head) * 2] * mo[((size_t)sl * H + head) * MO_LD + (idx - head * DH)];
         } else {
-            acc = mo[idx];
+            acc = mo[(size_t)head * MO_LD + (idx - head * DH)];
             if (idx % DH == 0) {
                 if (a.cluster) {
                     cp[H * DH + head] = mm[head * 2];
@@ -680,12 +681,14 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     const int n_b = (L + a.tps - 1) / a.tps;
     if (tid == 0) {
-        __threadfence();                                   // the CTA's partial before the count
-        flags[1] = (atomicAdd(a.counters + b, 1) == n_b - 1) ? 1 : 0;
+        // acq_rel at gpu scope: releases the CTA's partial (ordered before this thread
+        // by the barrier above) and, for the last arrival, acquires every other CTA's
+        int old;
+        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(a.counters + b) : "memory");
+        flags[1] = (old == n_b - 1) ? 1 : 0;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     if (!flags[1]) return;
-    __threadfence();
     const float *pob = a.part_o + (size_t)b * a.n_split * H * DH;
     const float *pmb = a.part_ml + (size_t)b * a.n_split * H * 2;
     // The first float4 column of every thread is requested for up to PF splits at once,
@@ -699,10 +702,12 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         for (int i = 0; i < PF; ++i)
             if (i < n_b) pre[i] = __ldcg(pob4 + (size_t)i * N4 + tid);
     }
-    // split statistics: w[i][head] = 2^(m_i - M), then the denominators
+    // split statistics: w[i][head] = 2^(m_i - M) with one thread per (split, head),
+    // then the denominators
     float *wt = reinterpret_cast<float *>(smem);            // [n_b][H]
     float *den = wt + (size_t)n_b * H;                      // [H]
     float *lv = den + H;                                    // [n_b][H]
+    float *mx = lv + (size_t)n_b * H;                       // [H]
     for (int k = tid; k < n_b * H; k += WARPS * 32) {
         const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pmb) + k);
         wt[k] = ml.x;
@@ -712,12 +717,19 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     for (int head = tid; head < H; head += WARPS * 32) {
         float M = -INFINITY;
         for (int i = 0; i < n_b; ++i) M = fmaxf(M, wt[i * H + head]);
+        mx[head] = M;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    for (int k = tid; k < n_b * H; k += WARPS * 32) {
+        const float m = wt[k];
+        const float w = m == -INFINITY ? 0.f : exp2f(m - mx[k % H]);
+        wt[k] = w;
+        lv[k] *= w;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    for (int head = tid; head < H; head += WARPS * 32) {
         float d = 0.f;
-        for (int i = 0; i < n_b; ++i) {
-            const float w = exp2f(wt[i * H + head] - M);
-            wt[i * H + head] = w;
-            d += w * lv[i * H + head];
-        }
+        for (int i = 0; i < n_b; ++i) d += lv[i * H + head];
         den[head] = d;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
@@ -765,7 +777,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
         const int per = (H * DH + C - 1) / C;
         const int lo = rank * per, hi = min(H * DH, lo + per);
-        float *cpl = reinterpret_cast<float *>(smem) + SLICES * H * DH + SLICES * H * 2;
+        float *cpl = reinterpret_cast<float *>(smem) + SLICES * H * C::MO_LD + SLICES * H * 2;
         for (int idx = lo + tid; idx < hi; idx += WARPS * 32) {
             const int head = idx / DH;
             float M = -INFINITY;

@@ -58,11 +58,14 @@ struct MmaDecodeCfg {
     static constexpr size_t OFF_SCR = (OFF_CS + (size_t)(D2 / 2) * 8 + 15) / 16 * 16;
     static constexpr size_t OFF_FLAGS = OFF_SCR + (size_t)WARPS * SCR_FLOATS * 4;
     static constexpr size_t smem_bytes() { return OFF_FLAGS + 16; }
+    // row stride (floats) of the slice-merge buffer: 8 floats of padding put the rows
+    // of consecutive heads in different banks
+    static constexpr int MO_LD = D1 * D2 + 8;
     static_assert(MA % 16 == 0, "h1*d1 must be a multiple of 16");
     static_assert(D2 % 16 == 0, "d2 must be a multiple of 16");
     static_assert(D1 == 1 || D1 == 2 || D1 == 4 || D1 == 8 || D1 == 16, "d1 must be 1..16, a power of 2");
     static_assert(D1 == 1 || (H1 >= 2 && 32 % H1 == 0), "h1 must divide 32 when d1 > 1");
-    static_assert((size_t)SLICES * H * DH * 4 + (size_t)SLICES * H * 8 + (size_t)H * DH * 4 + H * 8 <=
+    static_assert((size_t)SLICES * H * MO_LD * 4 + (size_t)SLICES * H * 8 + (size_t)H * DH * 4 + H * 8 <=
                       (size_t)STAGES * STAGE_BYTES,
                   "slice merge and merged partial must fit in the ring");
     static_assert(WARPS <= 31, "too many consumer warps");
