@@ -51,7 +51,7 @@ def _args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kpa", "reference"], default="kpa")
     ap.add_argument("--workload", default="tpa_decode",
-                    help="tpa_decode | kpa_medium | kpa_long | tiny_kpa | append_prefill")
+                    help="tpa_decode | kpa_medium | kpa_long | tiny_kpa | flashtpa | append_prefill")
     ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

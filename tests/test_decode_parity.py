@@ -15,7 +15,7 @@ import torch
 import oracle
 from gpu_util import (assert_bf16_close, assert_close, assert_f32_close, errors, fill_cache, kpa,
                       natural, oracle_decode_from_cache, oracle_decode_unrotated, run_decode)
-from workloads import KPA_LONG, KPA_MEDIUM, TINY_KPA, TPA_DECODE, decode_inputs, to_f64
+from workloads import FLASHTPA_DECODE, KPA_LONG, KPA_MEDIUM, TINY_KPA, TPA_DECODE, decode_inputs, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -25,6 +25,7 @@ SMALL = {
     "kpa_medium": KPA_MEDIUM.replace(batch=4, capacity=1536, ragged=(1, 1536), seed=2),
     "kpa_long_base": KPA_LONG.replace(capacity=4104, length=4101, seed=3),
     "tiny_kpa_scaled": TINY_KPA.replace(factor_std=1.0 / np.sqrt(2.0), seed=4),
+    "flashtpa": FLASHTPA_DECODE.replace(batch=3, capacity=1536, length=0, ragged=(1, 1536), seed=6),
     "kpa_odd": KPA_MEDIUM.replace(shape=KPA_MEDIUM.shape.__class__(h1=3, h2=2, d1=2, d2=6, r_k=3,
                                                                    r_v=1, rope_base=10000.0),
                                   batch=2, capacity=200, ragged=(1, 200), seed=5),
@@ -209,7 +210,7 @@ def _sample_heads(w, seq_len, n=6, seed=0):
                   {bs[0] * w.shape.h, bs[-1] * w.shape.h + w.shape.h - 1})
 
 
-@pytest.mark.parametrize("w", [TPA_DECODE, KPA_MEDIUM, KPA_LONG], ids=lambda w: w.name.split(" (")[0])
+@pytest.mark.parametrize("w", [TPA_DECODE, KPA_MEDIUM, KPA_LONG, FLASHTPA_DECODE], ids=lambda w: w.name.split(" (")[0])
 def test_full_size_sampled_heads(w):
     """The full configurations in the launch configuration the benchmark uses,
     checked end to end on sampled (sequence, head) outputs."""

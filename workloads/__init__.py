@@ -135,8 +135,18 @@ APPEND_PREFILL = AppendWorkload(
     shape=Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, rope_base=10000.0),
     batch=8, n_tok=2048, capacity=2112, seed=0)
 
+# The decoding benchmark shape of the FlashTPA figures ("Tensor Product Attention Is
+# All You Need" explainer, decoding-speed benchmarks): d_model 2048, h = 32, d_h = 64,
+# R_Q = 16, R_K = R_V = 1, sequences 2^12 .. 2^19, batch 1 .. 16.  Here batch 1 at 2^19
+# tokens; the sweep uses the bench overrides.  The dense query path ignores R_Q.
+FLASHTPA_SHAPE = Shape(h1=32, h2=1, d1=1, d2=64, r_k=1, r_v=1, r_q=16, d_model=2048, rope_base=10000.0)
+FLASHTPA_DECODE = DecodeWorkload(
+    name="FlashTPA-shape decode (B=1, h=32x1, d_h=1x64, R=1+1, L=2^19, bf16)",
+    shape=FLASHTPA_SHAPE, batch=1, capacity=1 << 19, dtype="bf16", factor_std=1.0, q_std=1.0 / 8.0,
+    seed=0, length=1 << 19)
+
 DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
-                  "kpa_long": KPA_LONG}
+                  "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE}
 
 
 # --- draws ---------------------------------------------------------------------
