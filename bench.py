@@ -57,6 +57,8 @@ def _args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override: fixed length (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override: batch (profiling)")
+    ap.add_argument("--tokens-per-split", type=int, default=0,
+                    help="override the library's split of each sequence (profiling; multiple of 64)")
     ap.add_argument("--settle-seconds", type=float, default=1.0,
                     help="untimed load before timing while clocks are sampled (0 for profiling)")
     a = ap.parse_args(argv)
@@ -301,7 +303,8 @@ def run_kpa(a):
         qs[layer].copy_(inp["q"].to(dev))
         del inp
     max_len = int(lens.max())
-    ws_bytes = kpa.kpa_decode_workspace_size(cfg, w.batch, max_len)
+    tps = a.tokens_per_split
+    ws_bytes = kpa.kpa_decode_workspace_size(cfg, w.batch, max_len, tps)
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     sm_scale = 1.0 / float(np.sqrt(s.dh))
     torch.cuda.synchronize()
@@ -310,8 +313,8 @@ def run_kpa(a):
 
     def step(qsrc):
         for layer in range(layers):
-            kpa.kpa_decode(cfg, w.batch, qsrc[layer], q_pos, kcs[layer], vcs[layer], w.capacity,
-                           seq_len, max_len, sm_scale, outs[layer], ws, stream=stream)
+            kpa.kpa_decode_split(cfg, w.batch, qsrc[layer], q_pos, kcs[layer], vcs[layer], w.capacity,
+                                 seq_len, max_len, sm_scale, tps, outs[layer], ws, stream=stream)
 
     # warm up eagerly once (also sets kernel attributes), then capture the step
     with torch.cuda.stream(stream):
@@ -381,7 +384,9 @@ def run_kpa(a):
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
             if w.dtype == "bf16" else "f32", "data": "synthetic (seeded, shapes of the pages' workloads)",
-            "config": _config_json(w, layers, lens, world),
+            "config": dict(_config_json(w, layers, lens, world),
+                           splits_per_sequence=kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[0],
+                           tokens_per_split=kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[1]),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": _traffic(khash),
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
@@ -395,7 +400,7 @@ def run_kpa(a):
                     "path": "pinned host queries -> device (1 copy), kpa_decode x layers, outputs -> pinned host "
                             "(1 copy), one CUDA graph"},
             "clocks": clocks,
-            "gpu_launches": a.steps * layers * kpa.kpa_decode_plan(cfg, w.batch, max_len)[2]}
+            "gpu_launches": a.steps * layers * kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[2]}
 
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         base, _ = _cpu_baseline(w, first, a.cpu_seconds)

@@ -152,6 +152,13 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
         const int64_t want = ((int64_t)max_len + want_split - 1) / want_split;
         tps = (int)(((want + 15) / 16) * 16);
         if (tps < 64) tps = 64;
+        // whole tiles per split (no ragged last tile) when that keeps most of the splits
+        if (p->variant >= 0 && p->tile > 0) {
+            const int whole = (tps + p->tile - 1) / p->tile * p->tile;
+            const int64_t n0 = ((int64_t)max_len + tps - 1) / tps;
+            const int64_t n1 = ((int64_t)max_len + whole - 1) / whole;
+            if (n1 * 20 >= n0 * 17) tps = whole;
+        }
     }
     p->tokens_per_split = tps;
     p->n_split = max_len > 0 ? (int)(((int64_t)max_len + tps - 1) / tps) : 1;

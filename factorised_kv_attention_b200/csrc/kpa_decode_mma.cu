@@ -185,7 +185,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *stage_base = smem;                                           // ring
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BARS);          // full, empty
-    float *qs = reinterpret_cast<float *>(smem + C::OFF_Q);                     // [H][DH]
+    float *qs = reinterpret_cast<float *>(smem + C::OFF_Q);                     // [H][Q_LD]
     float2 *cs = reinterpret_cast<float2 *>(smem + C::OFF_CS);                  // [D2/2]
     float *scratch = reinterpret_cast<float *>(smem + C::OFF_SCR);              // per warp
     volatile int *flags = reinterpret_cast<volatile int *>(smem + C::OFF_FLAGS);  // abort, last
@@ -305,8 +305,9 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 const float2 w = cs[i % (D2 / 2)];
                 y = make_float2(x.x * w.x - x.y * w.y, x.x * w.y + x.y * w.x);
             }
-            qs[2 * i] = y.x * a.qscale;
-            qs[2 * i + 1] = y.y * a.qscale;
+            const int e = 2 * i, qh = e / DH;                // rows padded to Q_LD: no bank conflicts
+            *reinterpret_cast<float2 *>(qs + qh * C::Q_LD + (e - qh * DH)) =
+                make_float2(y.x * a.qscale, y.y * a.qscale);
         }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
@@ -329,7 +330,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 const int row = mt * 16 + g + ((v & 1) ? 8 : 0);
                 const int j2 = ks * 16 + 2 * c + ((v & 2) ? 8 : 0);
                 const int i1 = row / D1, j1 = row % D1;
-                const float *src = qs + (i1 * H2 + i2) * DH + j1 * D2 + j2;
+                const float *src = qs + (i1 * H2 + i2) * C::Q_LD + j1 * D2 + j2;
                 split2(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
             }
 

@@ -54,12 +54,18 @@ __host__ __device__ __forceinline__ int64_t cache_offset(int64_t s, int e, int E
     return ((s / kGroup) * E + e) * kGroup + (s % kGroup);
 }
 
-// cos/sin of pos * theta in float64, rounded to float.
+// cos/sin of the angle pos * theta.  The angle is formed and reduced to [-pi, pi]
+// in float64 (Cody-Waite reduction: 2 pi split into a double and its remainder, so
+// the reduced angle keeps float64 accuracy for any position below 2^31); the float
+// sine and cosine of the remainder follow.
 __device__ __forceinline__ void rope_cs(double pos, double theta, float &c, float &s) {
-    double sn, cs;
-    sincos(pos * theta, &sn, &cs);
-    c = (float)cs;
-    s = (float)sn;
+    constexpr double kInvTwoPi = 0.15915494309189535;       // 1 / (2 pi)
+    constexpr double kTwoPiHi = 6.283185307179586;          // 2 pi rounded to double
+    constexpr double kTwoPiLo = 2.4492935982947064e-16;     // 2 pi - kTwoPiHi
+    const double phi = pos * theta;
+    const double k = rint(phi * kInvTwoPi);
+    const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, phi));
+    sincosf((float)r, &s, &c);
 }
 
 // Raise a kernel's dynamic shared-memory limit once per device and kernel (so

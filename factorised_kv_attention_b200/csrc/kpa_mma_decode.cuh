@@ -54,7 +54,8 @@ struct MmaDecodeCfg {
     static constexpr int SCR_FLOATS = D1 > 1 ? ((16 * RED_LD + H1 * 16 + H1 + 3) / 4) * 4 : 0;
     static constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t OFF_Q = OFF_BARS + 16 * STAGES;
-    static constexpr size_t OFF_CS = OFF_Q + (size_t)H * DH * 4;
+    static constexpr int Q_LD = D1 * D2 + 8;                    // padded row of the fp32 query
+    static constexpr size_t OFF_CS = OFF_Q + (size_t)H * Q_LD * 4;
     static constexpr size_t OFF_SCR = (OFF_CS + (size_t)(D2 / 2) * 8 + 15) / 16 * 16;
     static constexpr size_t OFF_FLAGS = OFF_SCR + (size_t)WARPS * SCR_FLOATS * 4;
     static constexpr size_t smem_bytes() { return OFF_FLAGS + 16; }
