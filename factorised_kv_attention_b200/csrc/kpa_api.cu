@@ -145,10 +145,24 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
     // through global memory.
     int c = p->variant >= 0 ? (per_seq < kMaxClusterSplits ? per_seq : kMaxClusterSplits) : 0;
     while (c > 1 && cluster_capacity(p->variant, c) < batch) --c;
-    const bool cluster_auto = c == 1 || (c > 1 && (int64_t)batch * c * 5 >= (int64_t)target * 4);
+    // Several sequences may have different lengths (the host does not see them): up to
+    // 4 waves of shorter splits let the CTA scheduler balance the long ones, as long as
+    // every split still streams at least 1 MiB of cache.  That takes precedence over a
+    // one-wave cluster plan.
+    int over_split = 0;
+    if (batch > 1 && tps_req == 0) {
+        const int64_t bytes_tok = (int64_t)(d.ek + d.ev) * (dt == KPA_BF16 ? 2 : 4);
+        const int64_t tps_min = ((int64_t)1 << 20) / bytes_tok;
+        for (int k = 4; k > 1 && !over_split; --k) {
+            const int64_t cand = ((int64_t)max_len + (int64_t)k * per_seq - 1) / ((int64_t)k * per_seq);
+            if (cand >= tps_min) over_split = k * per_seq;
+        }
+    }
+    const bool cluster_auto =
+        !over_split && (c == 1 || (c > 1 && (int64_t)batch * c * 5 >= (int64_t)target * 4));
     int tps = tps_req;
     if (tps == 0) {
-        const int want_split = cluster_auto ? c : per_seq;
+        const int want_split = over_split ? over_split : cluster_auto ? c : per_seq;
         const int64_t want = ((int64_t)max_len + want_split - 1) / want_split;
         tps = (int)(((want + 15) / 16) * 16);
         if (tps < 64) tps = 64;
