@@ -30,6 +30,7 @@ struct AppendArgs {
     const int32_t *start_pos;
     int h1, h2, d1, d2, rq, rk, rv;
     int eq, ek, ev;              // elements per query / key / value record
+    int d2m1;                    // d2 - 1 when d2 is a power of two (pair index by mask), else -1
     __nv_bfloat16 *kc, *vc;
     float *qf;                   // [eq][M] query factors (B^Q rotated), or null
     int *err;
@@ -41,7 +42,7 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 192;                 // producer, MMA, 4 epilogue warps
+constexpr int kThreads = 320;                 // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
 constexpr uint32_t kTmemCols = 256;
 
 __device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap, int E, int s, int e,
@@ -50,37 +51,45 @@ __device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap
         __float2bfloat16_rn(v);
 }
 
+// Rotate the projected pair (n, n+1) when it is a B^Q or B^K pair (cs(j) = (cos, sin)
+// of pair j of the token's position); A factors and V pass unchanged.
+template <class CS>
+__device__ __forceinline__ void rotate_pair(const AppendArgs &a, int n, float &x0, float &x1, CS cs) {
+    const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1;
+    int r = -1;                                    // offset inside a B row
+    if (n < a.eq) {
+        if (n >= qa) r = n - qa;
+    } else if (n < a.eq + a.ek) {
+        if (n - a.eq >= ka) r = n - a.eq - ka;
+    }
+    const int j = r < 0 ? -1 : (a.d2m1 >= 0 ? (r & a.d2m1) : r % a.d2) >> 1;
+    if (j >= 0) {
+        const float2 w = cs(j);
+        const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
+        x0 = y0;
+        x1 = y1;
+    }
+}
+
 // One pair of projected columns (n, n+1) of token m: rotate it when it is a B^Q or B^K
 // pair (cs(j) = (cos, sin) of pair j of the token's position), then keep query
 // factors in fp32 and write key / value factors to the token's cache slot in bf16.
 template <class CS>
 __device__ __forceinline__ void emit_pair(const AppendArgs &a, int m, int b, int s, bool slot_ok, int n,
                                           float x0, float x1, CS cs) {
-    const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1;
+    rotate_pair(a, n, x0, x1, cs);
     if (n < a.eq) {                                        // query factors
-        if (n >= qa) {                                     // B^Q: rotate the pair
-            const float2 w = cs(((n - qa) % a.d2) >> 1);
-            const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
-            x0 = y0;
-            x1 = y1;
-        }
         if (a.qf) {
             a.qf[(size_t)n * a.M + m] = x0;
             a.qf[(size_t)(n + 1) * a.M + m] = x1;
         }
     } else if (n < a.eq + a.ek) {                          // key factors
         const int e = n - a.eq;
-        if (e >= ka) {                                     // B^K: rotate the pair
-            const float2 w = cs(((e - ka) % a.d2) >> 1);
-            const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
-            x0 = y0;
-            x1 = y1;
-        }
         if (slot_ok) {
             store_cache(a.kc, b, a.cap, a.ek, s, e, x0);
             store_cache(a.kc, b, a.cap, a.ek, s, e + 1, x1);
         }
-    } else {                                               // value factors, never rotated
+    } else {                                               // value factors
         const int e = n - a.eq - a.ek;
         if (slot_ok) {
             store_cache(a.vc, b, a.cap, a.ev, s, e, x0);
@@ -175,9 +184,11 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
             umma_commit(accf);                        // after every MMA issued (also on abort)
         }
     } else {
-        // ---- epilogue: thread = accumulator row = token
-        const int quarter = warp & 3;
+        // ---- epilogue: thread = accumulator row = token; warps 2..5 take the first
+        // half of the tile's 16-column chunks, warps 6..9 the rest
+        const int quarter = warp & 3, part = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
+        const int nch = BN / 16, ch_lo = part ? (nch + 1) / 2 : 0, ch_hi = part ? nch : (nch + 1) / 2;
         const int m = tile_m * BM + row;
         const bool live = m < a.M;
         int b = 0, s = 0;
@@ -189,17 +200,75 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
             const int t = m - b * a.n_tok;
             s = a.start_pos[b] + t;
             slot_ok = s >= 0 && s < a.cap;
-            if (!slot_ok) raise_error(a.err, kErrDeviceCheck);
-            for (int j = 0; j < half; ++j) {
+            if (!slot_ok && part == 0) raise_error(a.err, kErrDeviceCheck);
+            for (int j = part; j < half; j += 2) {          // the row's two threads split the angles
                 float c, sn;
                 rope_cs((double)s, rope.theta[j], c, sn);
                 cs[j] = make_float2(c, sn);
             }
         }
+        asm volatile("bar.sync 2, 256;" ::: "memory");              // every row's angles are in
         const bool acc_ok = mbar_wait(accf, 0, limit) && !*abort_flag;
         if (!acc_ok) raise_error(a.err, kErrTimeout);
         tc_fence_after();
-        for (int ch = 0; ch < BN / 16; ++ch) {
+        // Fast path: the tile's 128 rows are consecutive slots of one sequence starting on
+        // a cache group.  Rotated values go to shared memory transposed ([column][row], in
+        // the pipeline buffers, free once the accumulator is complete), then leave in
+        // 16-byte pieces: float4 runs of query-factor columns, whole 8-token cache groups.
+        const int m0 = tile_m * BM;
+        const int b0 = m0 / a.n_tok;
+        const int s0 = a.start_pos[b0] + (m0 - b0 * a.n_tok);
+        const bool fast = m0 + BM <= a.M && (m0 + BM - 1) / a.n_tok == b0 && s0 >= 0 && s0 % kGroup == 0 &&
+                          s0 + BM <= a.cap && a.M % 4 == 0 && (size_t)S * (a_bytes + b_bytes) >= (size_t)BN * BM * 4;
+        if (fast) {
+            float *st = reinterpret_cast<float *>(smem);        // [BN][BM]
+            for (int ch = ch_lo; ch < ch_hi; ++ch) {
+                float v[16];
+                tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16, v);   // warp-collective
+                const int n0 = tile_n * BN + ch * 16;
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    if (n0 + j >= a.N) break;
+                    float x0 = v[j], x1 = v[j + 1];
+                    rotate_pair(a, n0 + j, x0, x1, [&](int k) { return cs[k]; });
+                    st[(ch * 16 + j) * BM + row] = x0;
+                    st[(ch * 16 + j + 1) * BM + row] = x1;
+                }
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");          // the epilogue warps
+            const int te = threadIdx.x - 64;                         // 0..255
+            const int nb = tile_n * BN, ne = min(nb + BN, a.N);
+            if (acc_ok) {
+                // query-factor columns [nb, min(ne, eq)): 32 float4 per column
+                const int qe = min(ne, a.eq);
+                if (a.qf)
+                    for (int it = te; it < max(0, qe - nb) * (BM / 4); it += 256) {
+                        const int lc = it / (BM / 4), i4 = it % (BM / 4);
+                        const float4 x = reinterpret_cast<const float4 *>(st + (size_t)lc * BM)[i4];
+                        *reinterpret_cast<float4 *>(a.qf + (size_t)(nb + lc) * a.M + m0 + 4 * i4) = x;
+                    }
+                // key / value columns [max(nb, eq), ne): one 16-byte cache group per 8 rows
+                const int kb0 = max(nb, a.eq);
+                for (int it = te; it < max(0, ne - kb0) * (BM / kGroup); it += 256) {
+                    const int lc = kb0 - nb + it / (BM / kGroup), g = it % (BM / kGroup);
+                    const int n = nb + lc;
+                    const bool is_k = n < a.eq + a.ek;
+                    __nv_bfloat16 *plane = is_k ? a.kc : a.vc;
+                    const int E = is_k ? a.ek : a.ev, e = is_k ? n - a.eq : n - a.eq - a.ek;
+                    const float4 lo = reinterpret_cast<const float4 *>(st + (size_t)lc * BM + g * kGroup)[0];
+                    const float4 hi = reinterpret_cast<const float4 *>(st + (size_t)lc * BM + g * kGroup)[1];
+                    uint4 u;
+                    __nv_bfloat162 *pu = reinterpret_cast<__nv_bfloat162 *>(&u);
+                    pu[0] = __floats2bfloat162_rn(lo.x, lo.y);
+                    pu[1] = __floats2bfloat162_rn(lo.z, lo.w);
+                    pu[2] = __floats2bfloat162_rn(hi.x, hi.y);
+                    pu[3] = __floats2bfloat162_rn(hi.z, hi.w);
+                    *reinterpret_cast<uint4 *>(plane + (((int64_t)b0 * (a.cap / kGroup) + s0 / kGroup + g) * E + e) *
+                                                           kGroup) = u;
+                }
+            }
+        } else
+        for (int ch = ch_lo; ch < ch_hi; ++ch) {
             float v[16];
             tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16, v);   // warp-collective
             if (!live || !acc_ok) continue;
@@ -450,6 +519,7 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     a.ek = d.ek;
     a.ev = d.ev;
     a.N = a.eq + a.ek + a.ev;
+    a.d2m1 = (d.d2 & (d.d2 - 1)) == 0 ? d.d2 - 1 : -1;
     a.K = d_model;
     a.BN = append_tile_n(a.N);
     a.n_kblocks = (d_model + BK - 1) / BK;
