@@ -43,7 +43,8 @@ using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
 constexpr int kThreads = 320;                 // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
-constexpr uint32_t kTmemCols = 256;
+constexpr int kStageCols = 32;                // epilogue staging: columns per pass per column half
+constexpr uint32_t kTmemCols = 512;              // two accumulators of 256 columns
 
 __device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap, int E, int s, int e,
                                             float v) {
@@ -108,22 +109,28 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
     const uint32_t a_bytes = BM * BK * 2, b_bytes = (uint32_t)BN * BK * 2;
     unsigned char *a_st = smem;                                   // S x 16 KB
     unsigned char *b_st = a_st + (size_t)S * a_bytes;             // S x BN*128 B
-    uint64_t *bars = reinterpret_cast<uint64_t *>(b_st + (size_t)S * b_bytes);   // full, empty, acc
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float2 *cs_all = reinterpret_cast<float2 *>(reinterpret_cast<unsigned char *>(bars) + 256);
+    float *stg = reinterpret_cast<float *>(b_st + (size_t)S * b_bytes);   // [2 parts][kStageCols][BM]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(stg + 2 * kStageCols * BM);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    volatile int *flags = reinterpret_cast<volatile int *>(tmem_slot + 1);    // abort, epilogue abort
+    float2 *cs_all = reinterpret_cast<float2 *>(reinterpret_cast<unsigned char *>(bars) + 512);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile_n = blockIdx.x, tile_m = blockIdx.y;
-    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * S, accf = full0 + 16 * S;
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * S, accf0 = full0 + 16 * S;
+    const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
+    const int n_tn = (a.N + BN - 1) / BN, n_tiles = n_tn * ((a.M + BM - 1) / BM);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
-        mbar_init(accf, 1);
-        *abort_flag = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(accf0 + 8 * i, 1);
+            mbar_init(acce0 + 8 * i, 8);                          // the 8 epilogue warps
+        }
+        mbar_init(drain, 1);
+        flags[0] = flags[1] = 0;
         mbar_fence_init();
         tma_prefetch_desc(&tmx);
         tma_prefetch_desc(&tmw);
@@ -137,146 +144,186 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint64_t limit = a.wait_limit_ns;
+    // bounded wait that gives up when the time runs out or another role has given up
+    auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+        if (mbar_try_wait(b, parity)) return true;
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 1;; ++it) {
+            if (mbar_try_wait(b, parity)) return true;
+            if ((it & 15) == 0) {
+                if (flags[0]) return false;
+                if (globaltimer() - t0 > limit) {
+                    flags[0] = 1;
+                    raise_error(a.err, kErrTimeout);
+                    return false;
+                }
+            }
+        }
+    };
 
     if (warp == 0) {
-        // ---- producer: TMA tiles of X (rows tile_m) and W (rows tile_n), 64 K columns each
+        // ---- producer: TMA tiles of X and W for every k-block of every tile of this CTA;
+        // the stage ring runs on across tile boundaries
         if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < a.n_kblocks; ++kb) {
-                const int s = kb % S;
-                if (kb >= S && !mbar_wait(empty0 + 8 * s, ((kb / S) - 1) & 1, limit)) {
-                    raise_error(a.err, kErrTimeout);
-                    *abort_flag = 1;
-                    break;
+            int g = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                const int tm = tile / n_tn, tn = tile % n_tn;
+                for (int kb = 0; kb < a.n_kblocks; ++kb, ++g) {
+                    const int s = g % S;
+                    if (g >= S && !wait(empty0 + 8 * s, ((g / S) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(full0 + 8 * s, a_bytes + b_bytes);
+                    tma_load_2d(smem_u32(a_st + (size_t)s * a_bytes), &tmx, kb * BK, tm * BM, full0 + 8 * s);
+                    tma_load_2d(smem_u32(b_st + (size_t)s * b_bytes), &tmw, kb * BK, tn * BN, full0 + 8 * s);
                 }
-                if (*abort_flag) break;
-                mbar_expect_tx(full0 + 8 * s, a_bytes + b_bytes);
-                tma_load_2d(smem_u32(a_st + (size_t)s * a_bytes), &tmx, kb * BK, tile_m * BM, full0 + 8 * s);
-                tma_load_2d(smem_u32(b_st + (size_t)s * b_bytes), &tmw, kb * BK, tile_n * BN, full0 + 8 * s);
-                issued = kb + 1;
             }
-            // every copy issued must land before the CTA exits (normally already consumed)
-            if (*abort_flag)
-                for (int kb = max(0, issued - S); kb < issued; ++kb)
-                    if (!mbar_wait(full0 + 8 * (kb % S), (kb / S) & 1, limit)) raise_error(a.err, kErrTimeout);
+            // every copy issued lands before the CTA exits (normally already consumed)
+            for (int k = max(0, g - S); k < g; ++k) (void)mbar_wait(full0 + 8 * (k % S), (k / S) & 1, limit);
         }
     } else if (warp == 1) {
-        // ---- MMA issuer: one thread drives the tensor cores
+        // ---- MMA issuer: accumulator i&1 of this CTA's i-th tile, once the epilogue has
+        // drained it (tile i-2)
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+            int g = 0, i = 0;
             bool ok = true;
-            for (int kb = 0; kb < a.n_kblocks; ++kb) {
-                const int s = kb % S;
-                if (!mbar_wait(full0 + 8 * s, (kb / S) & 1, limit)) {
-                    raise_error(a.err, kErrTimeout);
-                    *abort_flag = 1;
-                    ok = false;
-                    break;
-                }
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++i) {
+                const int buf = i & 1;
+                if (i >= 2 && !wait(acce0 + 8 * buf, ((i >> 1) - 1) & 1)) break;
                 tc_fence_after();
-                const uint64_t ad = umma_desc_k_sw128(smem_u32(a_st + (size_t)s * a_bytes));
-                const uint64_t bd = umma_desc_k_sw128(smem_u32(b_st + (size_t)s * b_bytes));
+                for (int kb = 0; kb < a.n_kblocks; ++kb, ++g) {
+                    const int s = g % S;
+                    if (!wait(full0 + 8 * s, (g / S) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = umma_desc_k_sw128(smem_u32(a_st + (size_t)s * a_bytes));
+                    const uint64_t bd = umma_desc_k_sw128(smem_u32(b_st + (size_t)s * b_bytes));
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)     // K = 16 per instruction: 32 B along the row
-                    umma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc, kb > 0 || k > 0);
-                umma_commit(empty0 + 8 * s);          // stage free once these MMAs finish
+                    for (int k = 0; k < BK / 16; ++k)     // K = 16 per instruction: 32 B along the row
+                        umma_bf16(tmem + buf * 256, ad + 2 * k, bd + 2 * k, idesc, kb > 0 || k > 0);
+                    umma_commit(empty0 + 8 * s);          // stage free once these MMAs finish
+                }
+                if (ok) umma_commit(accf0 + 8 * buf);
             }
-            umma_commit(accf);                        // after every MMA issued (also on abort)
+            // nothing issued here may still run when tensor memory is released
+            umma_commit(drain);
+            (void)mbar_wait(drain, 0, limit);
         }
     } else {
         // ---- epilogue: thread = accumulator row = token; warps 2..5 take the first
-        // half of the tile's 16-column chunks, warps 6..9 the rest
+        // half of each tile's 16-column chunks, warps 6..9 the rest
         const int quarter = warp & 3, part = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
         const int nch = BN / 16, ch_lo = part ? (nch + 1) / 2 : 0, ch_hi = part ? nch : (nch + 1) / 2;
-        const int m = tile_m * BM + row;
-        const bool live = m < a.M;
-        int b = 0, s = 0;
-        bool slot_ok = false;
         const int half = a.d2 / 2;
         float2 *cs = cs_all + (size_t)row * half;
-        if (live) {
-            b = m / a.n_tok;
-            const int t = m - b * a.n_tok;
-            s = a.start_pos[b] + t;
-            slot_ok = s >= 0 && s < a.cap;
-            if (!slot_ok && part == 0) raise_error(a.err, kErrDeviceCheck);
-            for (int j = part; j < half; j += 2) {          // the row's two threads split the angles
-                float c, sn;
-                rope_cs((double)s, rope.theta[j], c, sn);
-                cs[j] = make_float2(c, sn);
-            }
-        }
-        asm volatile("bar.sync 2, 256;" ::: "memory");              // every row's angles are in
-        const bool acc_ok = mbar_wait(accf, 0, limit) && !*abort_flag;
-        if (!acc_ok) raise_error(a.err, kErrTimeout);
-        tc_fence_after();
-        // Fast path: the tile's 128 rows are consecutive slots of one sequence starting on
-        // a cache group.  Rotated values go to shared memory transposed ([column][row], in
-        // the pipeline buffers, free once the accumulator is complete), then leave in
-        // 16-byte pieces: float4 runs of query-factor columns, whole 8-token cache groups.
-        const int m0 = tile_m * BM;
-        const int b0 = m0 / a.n_tok;
-        const int s0 = a.start_pos[b0] + (m0 - b0 * a.n_tok);
-        const bool fast = m0 + BM <= a.M && (m0 + BM - 1) / a.n_tok == b0 && s0 >= 0 && s0 % kGroup == 0 &&
-                          s0 + BM <= a.cap && a.M % 4 == 0 && (size_t)S * (a_bytes + b_bytes) >= (size_t)BN * BM * 4;
-        if (fast) {
-            float *st = reinterpret_cast<float *>(smem);        // [BN][BM]
-            for (int ch = ch_lo; ch < ch_hi; ++ch) {
-                float v[16];
-                tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16, v);   // warp-collective
-                const int n0 = tile_n * BN + ch * 16;
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) {
-                    if (n0 + j >= a.N) break;
-                    float x0 = v[j], x1 = v[j + 1];
-                    rotate_pair(a, n0 + j, x0, x1, [&](int k) { return cs[k]; });
-                    st[(ch * 16 + j) * BM + row] = x0;
-                    st[(ch * 16 + j + 1) * BM + row] = x1;
+        float *mystg = stg + part * kStageCols * BM;
+        const int tp = (warp - 2) * 32 + lane - part * 128;           // 0..127 inside the part
+        int i = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+            const int tm = tile / n_tn, tn = tile % n_tn, buf = i & 1;
+            const uint32_t acc = tmem + buf * 256 + ((uint32_t)(quarter * 32) << 16);
+            asm volatile("bar.sync 2, 256;" ::: "memory");           // the previous tile is done with cs
+            const int m = tm * BM + row;
+            const bool live = m < a.M;
+            int b = 0, s = 0;
+            bool slot_ok = false;
+            if (live) {
+                b = m / a.n_tok;
+                s = a.start_pos[b] + (m - b * a.n_tok);
+                slot_ok = s >= 0 && s < a.cap;
+                if (!slot_ok && part == 0) raise_error(a.err, kErrDeviceCheck);
+                for (int j = part; j < half; j += 2) {             // the row's two threads split the angles
+                    float c, sn;
+                    rope_cs((double)s, rope.theta[j], c, sn);
+                    cs[j] = make_float2(c, sn);
                 }
             }
-            asm volatile("bar.sync 1, 256;" ::: "memory");          // the epilogue warps
-            const int te = threadIdx.x - 64;                         // 0..255
-            const int nb = tile_n * BN, ne = min(nb + BN, a.N);
-            if (acc_ok) {
-                // query-factor columns [nb, min(ne, eq)): 32 float4 per column
-                const int qe = min(ne, a.eq);
-                if (a.qf)
-                    for (int it = te; it < max(0, qe - nb) * (BM / 4); it += 256) {
-                        const int lc = it / (BM / 4), i4 = it % (BM / 4);
-                        const float4 x = reinterpret_cast<const float4 *>(st + (size_t)lc * BM)[i4];
-                        *reinterpret_cast<float4 *>(a.qf + (size_t)(nb + lc) * a.M + m0 + 4 * i4) = x;
+            // all 8 warps agree on whether the accumulator arrived before going on
+            const bool got = __all_sync(0xffffffffu, wait(accf0 + 8 * buf, (i >> 1) & 1));
+            if (!got && lane == 0) flags[1] = 1;
+            asm volatile("bar.sync 2, 256;" ::: "memory");           // angles in, verdicts in
+            if (flags[1]) break;
+            tc_fence_after();
+            // Fast path: the tile's 128 rows are consecutive slots of one sequence starting
+            // on a cache group.  Rotated values are staged transposed, 32 columns at a time,
+            // and leave as 16-byte pieces: float4 runs of query-factor columns, whole 8-token
+            // cache groups.
+            const int m0 = tm * BM;
+            const int b0 = m0 / a.n_tok;
+            const int s0 = a.start_pos[b0] + (m0 - b0 * a.n_tok);
+            const bool fast = m0 + BM <= a.M && (m0 + BM - 1) / a.n_tok == b0 && s0 >= 0 && s0 % kGroup == 0 &&
+                              s0 + BM <= a.cap && a.M % 4 == 0;
+            if (fast) {
+                for (int c0 = ch_lo; c0 < ch_hi; c0 += kStageCols / 16) {
+                    const int cn = min(kStageCols / 16, ch_hi - c0);   // 16-column chunks in this pass
+                    for (int cc = 0; cc < cn; ++cc) {
+                        float v[16];
+                        tmem_ld16(acc + (c0 + cc) * 16, v);             // warp-collective
+                        const int n0 = tn * BN + (c0 + cc) * 16;
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) {
+                            if (n0 + j >= a.N) break;
+                            float x0 = v[j], x1 = v[j + 1];
+                            rotate_pair(a, n0 + j, x0, x1, [&](int k) { return cs[k]; });
+                            mystg[(cc * 16 + j) * BM + row] = x0;
+                            mystg[(cc * 16 + j + 1) * BM + row] = x1;
+                        }
                     }
-                // key / value columns [max(nb, eq), ne): one 16-byte cache group per 8 rows
-                const int kb0 = max(nb, a.eq);
-                for (int it = te; it < max(0, ne - kb0) * (BM / kGroup); it += 256) {
-                    const int lc = kb0 - nb + it / (BM / kGroup), g = it % (BM / kGroup);
-                    const int n = nb + lc;
-                    const bool is_k = n < a.eq + a.ek;
-                    __nv_bfloat16 *plane = is_k ? a.kc : a.vc;
-                    const int E = is_k ? a.ek : a.ev, e = is_k ? n - a.eq : n - a.eq - a.ek;
-                    const float4 lo = reinterpret_cast<const float4 *>(st + (size_t)lc * BM + g * kGroup)[0];
-                    const float4 hi = reinterpret_cast<const float4 *>(st + (size_t)lc * BM + g * kGroup)[1];
-                    uint4 u;
-                    __nv_bfloat162 *pu = reinterpret_cast<__nv_bfloat162 *>(&u);
-                    pu[0] = __floats2bfloat162_rn(lo.x, lo.y);
-                    pu[1] = __floats2bfloat162_rn(lo.z, lo.w);
-                    pu[2] = __floats2bfloat162_rn(hi.x, hi.y);
-                    pu[3] = __floats2bfloat162_rn(hi.z, hi.w);
-                    *reinterpret_cast<uint4 *>(plane + (((int64_t)b0 * (a.cap / kGroup) + s0 / kGroup + g) * E + e) *
-                                                           kGroup) = u;
+                    if (c0 + cn >= ch_hi) {                             // last read of the accumulator
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acce0 + 8 * buf);
+                    }
+                    asm volatile("bar.sync %0, 128;" ::"r"(3 + part) : "memory");   // the part's chunk is staged
+                    const int nb = tn * BN + c0 * 16, ne = min(nb + cn * 16, a.N);
+                    const int qe = min(ne, a.eq);
+                    if (a.qf)
+                        for (int it = tp; it < max(0, qe - nb) * (BM / 4); it += 128) {
+                            const int lc = it / (BM / 4), i4 = it % (BM / 4);
+                            const float4 x = reinterpret_cast<const float4 *>(mystg + (size_t)lc * BM)[i4];
+                            *reinterpret_cast<float4 *>(a.qf + (size_t)(nb + lc) * a.M + m0 + 4 * i4) = x;
+                        }
+                    const int kb0 = max(nb, a.eq);
+                    for (int it = tp; it < max(0, ne - kb0) * (BM / kGroup); it += 128) {
+                        const int lc = kb0 - nb + it / (BM / kGroup), gq = it % (BM / kGroup);
+                        const int n = nb + lc;
+                        const bool is_k = n < a.eq + a.ek;
+                        __nv_bfloat16 *plane = is_k ? a.kc : a.vc;
+                        const int E = is_k ? a.ek : a.ev, e = is_k ? n - a.eq : n - a.eq - a.ek;
+                        const float4 lo = reinterpret_cast<const float4 *>(mystg + (size_t)lc * BM + gq * kGroup)[0];
+                        const float4 hi = reinterpret_cast<const float4 *>(mystg + (size_t)lc * BM + gq * kGroup)[1];
+                        uint4 u;
+                        __nv_bfloat162 *pu = reinterpret_cast<__nv_bfloat162 *>(&u);
+                        pu[0] = __floats2bfloat162_rn(lo.x, lo.y);
+                        pu[1] = __floats2bfloat162_rn(lo.z, lo.w);
+                        pu[2] = __floats2bfloat162_rn(hi.x, hi.y);
+                        pu[3] = __floats2bfloat162_rn(hi.z, hi.w);
+                        *reinterpret_cast<uint4 *>(
+                            plane + (((int64_t)b0 * (a.cap / kGroup) + s0 / kGroup + gq) * E + e) * kGroup) = u;
+                    }
+                    asm volatile("bar.sync %0, 128;" ::"r"(3 + part) : "memory");   // staging free again
                 }
-            }
-        } else
-        for (int ch = ch_lo; ch < ch_hi; ++ch) {
-            float v[16];
-            tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 16, v);   // warp-collective
-            if (!live || !acc_ok) continue;
-            const int n0 = tile_n * BN + ch * 16;
+            } else {
+                for (int ch = ch_lo; ch < ch_hi; ++ch) {
+                    float v[16];
+                    tmem_ld16(acc + ch * 16, v);                        // warp-collective
+                    if (!live) continue;
+                    const int n0 = tn * BN + ch * 16;
 #pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-                if (n0 + j >= a.N) break;
-                emit_pair(a, m, b, s, slot_ok, n0 + j, v[j], v[j + 1], [&](int k) { return cs[k]; });
+                    for (int j = 0; j < 16; j += 2) {
+                        if (n0 + j >= a.N) break;
+                        emit_pair(a, m, b, s, slot_ok, n0 + j, v[j], v[j + 1], [&](int k) { return cs[k]; });
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce0 + 8 * buf);
             }
         }
     }
@@ -500,7 +547,8 @@ bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, u
 }  // namespace
 
 size_t append_smem_bytes(int BN, int stages, int d2) {
-    return 1024 + (size_t)stages * (BM * BK * 2 + (size_t)BN * BK * 2) + 256 + (size_t)BM * (d2 / 2) * 8;
+    return 1024 + (size_t)stages * (BM * BK * 2 + (size_t)BN * BK * 2) + (size_t)2 * kStageCols * BM * 4 + 512 +
+           (size_t)BM * (d2 / 2) * 8;
 }
 
 int append_tile_n(int N) {
@@ -550,8 +598,14 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     const size_t smem = append_smem_bytes(a.BN, a.stages, d.d2);
     e = ensure_dynamic_smem<append_gemm_kernel>(smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.N + a.BN - 1) / a.BN), (unsigned)((a.M + BM - 1) / BM));
-    append_gemm_kernel<<<grid, kThreads, smem, st>>>(tmx, tmw, a, rope);
+    // persistent: one CTA per SM (or per tile when there are fewer tiles)
+    int sms = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int tiles = ((a.N + a.BN - 1) / a.BN) * ((a.M + BM - 1) / BM);
+    append_gemm_kernel<<<(unsigned)(tiles < sms ? tiles : sms), kThreads, smem, st>>>(tmx, tmw, a, rope);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess || !q_out) return e;
