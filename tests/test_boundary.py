@@ -130,3 +130,18 @@ def test_append_factors_rejects_before_launch(over):
                                args["v_factors"], args["start_pos"], args["capacity"],
                                args["kcache"], args["vcache"], stream=0)
     assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def test_package_refuses_to_load_without_the_library(tmp_path):
+    """The product path has no CPU fallback: without libkpa.so the import fails."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "factorised_kv_attention_b200"
+    pkg.mkdir()
+    src = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "factorised_kv_attention_b200",
+                       "__init__.py")
+    shutil.copy(src, pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import factorised_kv_attention_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "libkpa.so" in r.stderr
