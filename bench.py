@@ -459,7 +459,7 @@ def run_append_prefill(a):
     pos1 = torch.full((w.batch,), w.n_tok, dtype=torch.int32, device=dev)
     len1 = torch.full((w.batch,), w.n_tok + 1, dtype=torch.int32, device=dev)
     ws1 = torch.zeros(max(kpa.kpa_append_workspace_size(cfg, w.batch, 1), 256), dtype=torch.uint8, device=dev)
-    q1 = torch.empty(w.batch, 1, s.h, s.dh, dtype=torch.bfloat16, device=dev)
+    qf1 = ws1.view(torch.float32)             # the append leaves the query factors here: [E_Q][batch]
     wsd = torch.zeros(max(kpa.kpa_decode_workspace_size(cfg, w.batch, w.n_tok + 1), 256), dtype=torch.uint8,
                       device=dev)
     out1 = torch.empty(w.batch, s.h, s.dh, dtype=torch.float32, device=dev)
@@ -471,7 +471,7 @@ def run_append_prefill(a):
     dec_bytes = w.batch * (w.n_tok + 1) * (s.e_k + s.e_v) * 2
     sampler = ClockSampler(local)
     _, _, dec_launches = kpa.kpa_decode_plan(cfg, w.batch, w.n_tok + 1)
-    launches_per_step = 2 + 1 + 2 + dec_launches     # append (GEMM + query assembly), prefill, step
+    launches_per_step = 2 + 1 + 1 + dec_launches     # append (GEMM + query assembly), prefill, step
 
     def append():
         kpa.kpa_append(cfg, w.batch, w.n_tok, x, W, start, w.capacity, kc, vc, q, ws, stream=stream)
@@ -480,9 +480,11 @@ def run_append_prefill(a):
         kpa.kpa_prefill(cfg, w.batch, w.n_tok, q, start, kc, vc, w.capacity, scale, out, stream=stream)
 
     def decode_step():
-        kpa.kpa_append(cfg, w.batch, 1, x1, W, pos1, w.capacity, kc, vc, q1, ws1, stream=stream)
-        kpa.kpa_decode(cfg, w.batch, q1, None, kc, vc, w.capacity, len1, w.n_tok + 1, scale, out1, wsd,
-                       stream=stream)
+        # one-token append (matrix-vector projection, RoPE, cache write; query factors into
+        # its workspace), then decode straight from those query factors
+        kpa.kpa_append(cfg, w.batch, 1, x1, W, pos1, w.capacity, kc, vc, None, ws1, stream=stream)
+        kpa.kpa_decode_qf(cfg, w.batch, qf1, w.batch, 1, None, kc, vc, w.capacity, len1, w.n_tok + 1, scale, out1,
+                          wsd, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(a.warmup):
@@ -562,7 +564,8 @@ def run_append_prefill(a):
                        "algorithmic_flop_per_launch": proj_flop},
             "decode_step": {"launch_us": t_dec * 1e6, "cache_bytes": dec_bytes,
                             "achieved_gbs": dec_bytes / t_dec / 1e9, "hbm_peak_gbs": hbm,
-                            "note": "append of one token per sequence + decode over 2049 slots (latency bound)"},
+                            "note": "append of one token per sequence + decode over 2049 slots from its query "
+                                    "factors (latency bound)"},
             "e2e": {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(x_host.numel() * 2 + x1_host.numel() * 2),
                     "d2h_bytes_per_step": int(out_host.numel() * 4 + out1_host.numel() * 4),

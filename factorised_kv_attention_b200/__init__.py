@@ -60,6 +60,8 @@ _SIGS = {
     "kpa_append_factors": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
     "kpa_decode_workspace_size": ([_cfgp, _i32, _i32, _i32, _szp], ctypes.c_int),
     "kpa_decode_plan": ([_cfgp, _i32, _i32, _i32, _i32p, _i32p, _i32p], ctypes.c_int),
+    "kpa_decode_qf": ([_cfgp, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp, _sz, _vp],
+                      ctypes.c_int),
     "kpa_decode": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp, _sz, _vp],
                    ctypes.c_int),
     "kpa_decode_split": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _i32, _vp, _vp,
@@ -147,6 +149,14 @@ def kpa_decode_plan(cfg, batch, max_len, tokens_per_split=0):
     _check(_lib.kpa_decode_plan(ctypes.byref(cfg), batch, max_len, tokens_per_split, ctypes.byref(n),
                                 ctypes.byref(t), ctypes.byref(l)), "kpa_decode_plan")
     return n.value, t.value, l.value
+
+
+def kpa_decode_qf(cfg, batch, q_factors, qf_stride, qf_seq_stride, q_pos, kcache, vcache, capacity, seq_len,
+                  max_len, sm_scale, out, workspace, ws_bytes=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.kpa_decode_qf(ctypes.byref(cfg), batch, _addr(q_factors), qf_stride, qf_seq_stride, _addr(q_pos),
+                              _addr(kcache), _addr(vcache), capacity, _addr(seq_len), max_len, sm_scale,
+                              _addr(out), _addr(workspace), ws_bytes, _stream(stream)), "kpa_decode_qf")
 
 
 def kpa_decode(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len, sm_scale, out,

@@ -296,22 +296,30 @@ kpa_status kpa_decode_plan(const kpa_config *cfg, int32_t batch, int32_t max_len
     return KPA_OK;
 }
 
-kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
-                            const int32_t *q_pos, const void *kcache, const void *vcache,
-                            int32_t capacity, const int32_t *seq_len, int32_t max_len,
-                            float sm_scale, int32_t tokens_per_split, float *out,
-                            void *workspace, size_t ws_bytes, kpa_stream stream) {
+}  // extern "C"
+
+namespace kpa {
+namespace {
+
+// Shared body of the decode entry points: the query is either dense (q) or given as
+// factors (qf with strides; only the tensor-core variants take it).
+kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, const float *qf, int32_t qf_stride,
+                       int32_t qf_seq_stride, const int32_t *q_pos, const void *kcache, const void *vcache,
+                       int32_t capacity, const int32_t *seq_len, int32_t max_len, float sm_scale,
+                       int32_t tokens_per_split, float *out, void *workspace, size_t ws_bytes, kpa_stream stream) {
     kpa_status s = check_cfg(cfg, false, false);
     if (s != KPA_OK) return s;
     if (batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
     if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0 || max_len > capacity)
         return KPA_ERR_INVALID_ARG;
     if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
+    if (qf && (cfg->r_q <= 0 || qf_stride <= 0 || qf_seq_stride < 0)) return KPA_ERR_INVALID_ARG;
     if (batch == 0) return KPA_OK;
     if (batch > 65535) return KPA_ERR_UNSUPPORTED;
-    if (!q || !kcache || !vcache || !seq_len || !out) return KPA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(seq_len) & 3) || (reinterpret_cast<uintptr_t>(q_pos) & 3))
+    if ((!q && !qf) || !kcache || !vcache || !seq_len || !out) return KPA_ERR_INVALID_ARG;
+    if ((q && !aligned16(q)) || (qf && (reinterpret_cast<uintptr_t>(qf) & 3)) || !aligned16(kcache) ||
+        !aligned16(vcache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seq_len) & 3) ||
+        (reinterpret_cast<uintptr_t>(q_pos) & 3))
         return KPA_ERR_INVALID_ARG;
     int *err = nullptr, sms = 0;
     s = device_state(&err, &sms);
@@ -320,6 +328,7 @@ kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
     DecodePlan p;
     s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
     if (s != KPA_OK) return s;
+    if (qf && p.variant < 0) return KPA_ERR_UNSUPPORTED;        // query factors: tensor-core path only
     if (!workspace || ws_bytes < p.bytes) return KPA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return KPA_ERR_INVALID_ARG;
     if (p.n_split > 65535 * 16) return KPA_ERR_UNSUPPORTED;
@@ -351,6 +360,10 @@ kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
         args.fused = p.fused;
         args.cluster = p.cluster;
         args.err = err;
+        args.qf = qf;
+        args.qf_stride = qf_stride;
+        args.qf_seq_stride = qf_seq_stride;
+        args.rq = cfg->r_q;
         e = launch_decode_mma(p.variant, args, batch, p, rope_table(cfg), current_hooks(), st);
     } else if (max_len > 0) {
         e = launch_decode_fma(d, cfg->dtype, batch, q, q_pos, kcache, vcache, capacity, seq_len,
@@ -360,6 +373,28 @@ kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
     if (max_len > 0 && p.fused) return KPA_OK;
     e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml, out_scale, out, st);
     return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+}
+
+}  // namespace
+}  // namespace kpa
+
+extern "C" {
+
+kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
+                            const int32_t *q_pos, const void *kcache, const void *vcache,
+                            int32_t capacity, const int32_t *seq_len, int32_t max_len,
+                            float sm_scale, int32_t tokens_per_split, float *out,
+                            void *workspace, size_t ws_bytes, kpa_stream stream) {
+    return decode_impl(cfg, batch, q, nullptr, 0, 0, q_pos, kcache, vcache, capacity, seq_len, max_len, sm_scale,
+                       tokens_per_split, out, workspace, ws_bytes, stream);
+}
+
+kpa_status kpa_decode_qf(const kpa_config *cfg, int32_t batch, const float *q_factors, int32_t qf_stride,
+                         int32_t qf_seq_stride, const int32_t *q_pos, const void *kcache, const void *vcache,
+                         int32_t capacity, const int32_t *seq_len, int32_t max_len, float sm_scale, float *out,
+                         void *workspace, size_t ws_bytes, kpa_stream stream) {
+    return decode_impl(cfg, batch, nullptr, q_factors, qf_stride, qf_seq_stride, q_pos, kcache, vcache, capacity,
+                       seq_len, max_len, sm_scale, 0, out, workspace, ws_bytes, stream);
 }
 
 kpa_status kpa_decode(const kpa_config *cfg, int32_t batch, const void *q, const int32_t *q_pos,
@@ -446,7 +481,7 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const
     size_t need = 0;
     s = kpa_append_workspace_size(cfg, batch, n_tok, &need);
     if (s != KPA_OK) return s;
-    if (q_out && (!workspace || ws_bytes < need)) return KPA_ERR_WORKSPACE;
+    if ((q_out || workspace) && (!workspace || ws_bytes < need)) return KPA_ERR_WORKSPACE;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255)) return KPA_ERR_INVALID_ARG;
     int *err = nullptr;
     s = device_state(&err, nullptr);

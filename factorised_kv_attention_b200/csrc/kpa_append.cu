@@ -581,7 +581,7 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     a.rq = rq; a.rk = d.rk; a.rv = d.rv;
     a.kc = static_cast<__nv_bfloat16 *>(kc);
     a.vc = static_cast<__nv_bfloat16 *>(vc);
-    a.qf = q_out ? qf : nullptr;
+    a.qf = qf;                           // the query factors land in the workspace when there is one
     a.err = err;
     a.wait_limit_ns = wait_limit_ns;
 

@@ -229,7 +229,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const double qpos = rotate ? (double)a.q_pos[b] : 0.0;
     constexpr int QPT = (H * DH / 2 + WARPS * 32 - 1) / (WARPS * 32);   // query pairs per thread
     __nv_bfloat162 qv[QPT];
-    if (warp < WARPS) {
+    if (warp < WARPS && !a.qf) {
         const __nv_bfloat162 *qb = reinterpret_cast<const __nv_bfloat162 *>(a.q + (size_t)b * H * DH);
 #pragma unroll
         for (int k = 0; k < QPT; ++k) {
@@ -295,10 +295,43 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         cs[tid] = make_float2(cth, sth);
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    if (a.qf) {
+        // q = (1/R_Q) sum_r A^Q_r (x) B^Q_r assembled here from fp32 factors ("Kronecker
+        // Product Attention", eq 2); the pairs (2m, 2m+1) of each d2 chunk are rotated after
+        // the rank sum (the rotation is linear).  One thread per 8 features of a (head, j1) row.
+        constexpr int CH = D2 / 8;
+        const float *qfb = a.qf + (size_t)b * a.qf_seq_stride;
+        const int qa_b = a.rq * H1 * D1;                  // first B^Q element of the record
+        const float rs = a.qscale / (float)a.rq;
+        for (int it = tid; it < H * D1 * CH; it += WARPS * 32) {
+            const int head = it / (D1 * CH), rem = it % (D1 * CH), j1 = rem / CH, j2 = (rem % CH) * 8;
+            const int i1 = head / H2, i2h = head % H2;
+            float acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+            for (int r = 0; r < a.rq; ++r) {
+                const float av = __ldg(qfb + (size_t)((r * H1 + i1) * D1 + j1) * a.qf_stride);
+                const float *bq = qfb + (size_t)(qa_b + (r * H2 + i2h) * D2 + j2) * a.qf_stride;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] += av * __ldg(bq + (size_t)u * a.qf_stride);
+            }
+            float *dst = qs + head * C::Q_LD + j1 * D2 + j2;
+#pragma unroll
+            for (int u = 0; u < 8; u += 2) {
+                float y0 = acc[u], y1 = acc[u + 1];
+                if (rotate) {
+                    const float2 w = cs[(j2 + u) >> 1];
+                    y0 = acc[u] * w.x - acc[u + 1] * w.y;
+                    y1 = acc[u] * w.y + acc[u + 1] * w.x;
+                }
+                *reinterpret_cast<float2 *>(dst + u) = make_float2(y0 * rs, y1 * rs);
+            }
+        }
+    }
 #pragma unroll
     for (int k = 0; k < QPT; ++k) {
         const int i = tid + k * WARPS * 32;
-        if (i < H * DH / 2) {
+        if (i < H * DH / 2 && !a.qf) {
             const float2 x = __bfloat1622float2(qv[k]);
             float2 y = x;
             if (rotate) {

@@ -32,6 +32,10 @@ struct DecodeArgs {
     int fused;          // the last CTA of a sequence combines its splits
     int cluster;        // the splits of a sequence form one cluster and merge over DSMEM
     int *err;
+    // query factors instead of q (null: use q): element e of sequence b's record
+    // [A^Q_0..A^Q_{rq-1} | B^Q_0..B^Q_{rq-1}] at qf[e * qf_stride + b * qf_seq_stride]
+    const float *qf;
+    int qf_stride, qf_seq_stride, rq;
 };
 
 // One instantiation per (split, ranks) family.

@@ -154,6 +154,27 @@ kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
                             float sm_scale, int32_t tokens_per_split, float *out,
                             void *workspace, size_t ws_bytes, kpa_stream stream);
 
+/* kpa_decode with the query given as its factors ("Kronecker Product Attention",
+ * eq 2 for Q: q = (1/R_Q) sum_r A^Q_r (x) B^Q_r); the decode kernel assembles each
+ * sequence's query in float32 in its prologue, so no separate assembly runs.  (The
+ * FlashTPA decoding of the "Tensor Product Attention Is All You Need" explainer also
+ * takes the query in factored form; here the scores are then taken against the
+ * assembled query.)
+ *   q_factors  float32; element e (0 <= e < E_Q = R_Q (h1 d1 + h2 d2)) of sequence b's
+ *              record [A^Q_0 .. A^Q_{R_Q-1} | B^Q_0 .. B^Q_{R_Q-1}] (A_r row-major
+ *              h1 x d1, B_r row-major h2 x d2) at q_factors[e * qf_stride + b * qf_seq_stride]
+ *   q_pos      [batch] int32: B^Q is rotated at q_pos[b] here; NULL when the factors
+ *              are already rotated (the query factors kpa_append leaves are)
+ * kpa_append keeps its query factors, B^Q rotated, at the start of its workspace as
+ * float32 [E_Q][batch * n_tok]: after a one-token append pass that workspace with
+ * qf_stride = batch, qf_seq_stride = 1.  Requires r_q > 0 and a shape covered by a
+ * tensor-core decode variant (else KPA_ERR_UNSUPPORTED).  Everything else -- the
+ * library's choice of split, workspace, outputs, errors -- as kpa_decode. */
+kpa_status kpa_decode_qf(const kpa_config *cfg, int32_t batch, const float *q_factors, int32_t qf_stride,
+                         int32_t qf_seq_stride, const int32_t *q_pos, const void *kcache, const void *vcache,
+                         int32_t capacity, const int32_t *seq_len, int32_t max_len, float sm_scale, float *out,
+                         void *workspace, size_t ws_bytes, kpa_stream stream);
+
 /* Causal chunked attention in factor space (prefill).  Row t of sequence b is
  * the query at position start_pos[b] + t and sees slots 0 .. start_pos[b] + t
  * (its own key included), which must already be in the cache (kpa_append or
@@ -180,8 +201,11 @@ kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, cons
  *                               start_pos[b] + t
  *   q_out [batch][n_tok][h][d_h] bf16 or NULL: the assembled query
  *                               (1/R_Q) sum_r A^Q_r (x) B^Q_r rotated at its position
- *   workspace at least kpa_append_workspace_size bytes.
- * Requires dtype == KPA_BF16 and d_model a multiple of 64. */
+ *   workspace at least kpa_append_workspace_size bytes; required when q_out is
+ *             given, optional (NULL) otherwise.  When given, it holds on return the
+ *             query factors (B^Q rotated) as float32 [E_Q][batch * n_tok] (see
+ *             kpa_decode_qf)
+ * Requires dtype == KPA_BF16 and d_model a multiple of 8. */
 kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,
                                      size_t *bytes);
 kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *x,

@@ -15,7 +15,7 @@ import torch
 import oracle
 from gpu_util import (assert_bf16_close, assert_close, assert_f32_close, errors, fill_cache, kpa,
                       natural, oracle_decode_from_cache, oracle_decode_unrotated, run_decode)
-from workloads import FLASHTPA_DECODE, KPA_LONG, KPA_MEDIUM, TINY_KPA, TPA_DECODE, decode_inputs, to_f64
+from workloads import FLASHTPA_DECODE, KPA_LONG, KPA_MEDIUM, TINY_KPA, TPA_DECODE, Shape, decode_inputs, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -222,3 +222,67 @@ def test_full_size_sampled_heads(w):
     g = np.stack([got[b, hd] for b, hd in idx])
     o = np.stack([want[b, hd] for b, hd in idx])
     assert_bf16_close(g, o, w.name)
+
+
+def _qf_case(shape, batch, cap, seed):
+    w = KPA_MEDIUM.replace(shape=shape, batch=batch, capacity=cap, ragged=(1, cap), seed=seed)
+    inp = decode_inputs(w)
+    rng = np.random.default_rng(seed + 100)
+    qf = (rng.standard_normal((batch, shape.e_q)) / np.sqrt(shape.r_q)).astype(np.float32)
+    return w, inp, qf
+
+
+@pytest.mark.parametrize("shape", [
+    Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, rope_base=10000.0),
+    Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2, r_q=4, d_model=1024, rope_base=10000.0)],
+    ids=["kpa_h4x4", "tpa_h16"])
+def test_decode_from_query_factors(shape):
+    """kpa_decode_qf: the query as factor records (record layout), rotated in the kernel at
+    q_pos, against the oracle with the float64 assembly (1/R_Q) sum_r A^Q_r (x) B^Q_r."""
+    w, inp, qf = _qf_case(shape, 3, 1024, 51)
+    lib = kpa()
+    cfg, kc, vc = fill_cache(lib, w, inp)
+    L = inp["seq_len"]
+    max_len = int(L.max())
+    ws = torch.zeros(lib.kpa_decode_workspace_size(cfg, w.batch, max_len), dtype=torch.uint8, device="cuda")
+    out = torch.full((w.batch, shape.h, shape.dh), float("nan"), dtype=torch.float32, device="cuda")
+    scale = 1.0 / np.sqrt(shape.dh)
+    lib.kpa_decode_qf(cfg, w.batch, torch.from_numpy(qf).cuda(), 1, shape.e_q, inp["q_pos"].cuda(), kc, vc,
+                      w.capacity, L.cuda(), max_len, scale, out, ws)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    q_dense = np.stack([oracle.reconstruct(shape.h1, shape.h2, shape.d1, shape.d2, shape.r_q, qf[b].astype(np.float64))
+                        for b in range(w.batch)])
+    want = oracle_decode_unrotated(w, inp, q=torch.from_numpy(q_dense), sm_scale=scale)
+    assert_bf16_close(out.cpu().numpy(), want, f"decode from query factors {shape}")
+
+
+def test_decode_step_reads_the_appends_query_factors():
+    """A one-token kpa_append (no q_out) followed by kpa_decode_qf on the append's
+    workspace ([E_Q][batch] fp32, B^Q rotated): equal to the oracle's append + decode."""
+    from workloads import APPEND_PREFILL, append_inputs
+    w = APPEND_PREFILL.replace(batch=3, n_tok=1, capacity=512, seed=52)
+    s = w.shape
+    lib = kpa()
+    cfg = lib.make_config(s, "bf16")
+    # earlier context in the cache, then the new token at position start = 300 + b
+    ctx = KPA_MEDIUM.replace(shape=s, batch=w.batch, capacity=w.capacity, ragged=(), length=w.capacity, seed=53)
+    cinp = decode_inputs(ctx)
+    cfg2, kc, vc = fill_cache(lib, ctx, cinp)
+    inp = append_inputs(w)
+    start = torch.tensor([300, 301, 302], dtype=torch.int32)
+    ws = torch.zeros(max(lib.kpa_append_workspace_size(cfg, w.batch, 1), 256), dtype=torch.uint8, device="cuda")
+    lib.kpa_append(cfg, w.batch, 1, inp["x"].cuda(), inp["W"].cuda(), start.cuda(), w.capacity, kc, vc, None, ws)
+    L = start + 1
+    wsd = torch.zeros(lib.kpa_decode_workspace_size(cfg, w.batch, int(L.max())), dtype=torch.uint8, device="cuda")
+    out = torch.full((w.batch, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    scale = 1.0 / np.sqrt(s.dh)
+    lib.kpa_decode_qf(cfg, w.batch, ws.view(torch.float32), w.batch, 1, None, kc, vc, w.capacity, L.cuda(),
+                      int(L.max()), scale, out, wsd)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    q_rot, _, _, _ = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start.numpy())
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    want = oracle.decode(s, q_rot[:, 0], kn, vn, L.numpy(), keys_rotated=True, sm_scale=scale)
+    assert_bf16_close(out.cpu().numpy(), want, "decode step from the append's query factors")
