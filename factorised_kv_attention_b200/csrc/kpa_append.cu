@@ -452,49 +452,118 @@ q_assemble_small_kernel(const float *__restrict__ qf, int M, int h1, int h2, int
 }
 
 // Query assembly q = (1/R_Q) sum_r A^Q_r (x) B^Q_r for the queries of the chunk.
-// One thread per (token, i2): the R_Q rows B^Q_r[i2, :] stay in registers while the
-// thread walks the h1 heads (i1, i2), so each factor is read once per token and
-// head column.  Reads of the [column][token] factor buffer are coalesced across the
-// warp's tokens; each head row of q_out goes out in 16-byte stores.
-template <int RQ, int D1, int D2>
-__global__ void __launch_bounds__(64)
-q_assemble_kernel(const float *__restrict__ qf, int M, int h1, int h2, __nv_bfloat16 *__restrict__ q_out) {
-    const int m = blockIdx.x * blockDim.x + threadIdx.x;
-    if (m >= M) return;
-    const int i2 = blockIdx.y;
-    const int qa = RQ * h1 * D1;
-    float B[RQ][D2];
+// A CTA takes kQaTokens consecutive tokens.  Their factor columns are first staged in
+// shared memory as token rows [t][e]; the loads run along the token axis of the
+// [column][token] buffer, so they are coalesced.  Then each thread takes one
+// (token, head, 8-feature slice of d2), keeps B^Q_r[i2, slice] (R_Q x 8) in registers,
+// and walks j1, writing one 16-byte piece per j1.  A warp's 32 pieces at one j1 fill
+// whole 32-byte sectors of 16 head rows of q_out.
+constexpr int kQaTokens = 16;
+constexpr int kQaThreads = 256;
+constexpr int kQaBatch = 16;
+
+__host__ __device__ inline int qa_ld(int eq) { return (eq + 3) / 4 * 4 + 4; }   // shared-memory row stride (floats)
+
+template <int RQ>
+__global__ void __launch_bounds__(kQaThreads)
+q_assemble_kernel(const float *__restrict__ qf, int M, int h1, int h2, int d1, int d2,
+                  __nv_bfloat16 *__restrict__ q_out) {
+    extern __shared__ float4 qa_smem[];
+    float *s = reinterpret_cast<float *>(qa_smem);
+    const int qa = RQ * h1 * d1, eq = qa + RQ * h2 * d2, ld = qa_ld(eq);
+    const int m0 = blockIdx.x * kQaTokens;
+    const int nt = min(kQaTokens, M - m0);
+    // Staging: every load of a batch is issued before the first shared-memory store,
+    // so a thread has up to kQaBatch loads in flight instead of one.
+    if ((M & 3) == 0) {
+        // four tokens per 16-byte load (the column starts e*M + m0 are 16-byte aligned)
+        const int total = eq * (kQaTokens / 4);
+        for (int base = 0; base < total; base += kQaBatch * kQaThreads) {
+            float4 v[kQaBatch];
 #pragma unroll
-    for (int r = 0; r < RQ; ++r)
+            for (int k = 0; k < kQaBatch; ++k) {
+                const int idx = base + k * kQaThreads + threadIdx.x;
+                const int e = idx / (kQaTokens / 4), t = (idx % (kQaTokens / 4)) * 4;
+                v[k] = idx < total && t < nt
+                           ? __ldg(reinterpret_cast<const float4 *>(qf + (size_t)e * M + m0 + t))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-        for (int j2 = 0; j2 < D2; ++j2) B[r][j2] = __ldg(qf + (size_t)(qa + (r * h2 + i2) * D2 + j2) * M + m);
-    const float inv = 1.0f / (float)RQ;
-    for (int i1 = 0; i1 < h1; ++i1) {
-        __nv_bfloat16 *dst = q_out + ((size_t)m * h1 * h2 + (size_t)i1 * h2 + i2) * (D1 * D2);
-#pragma unroll 2
-        for (int j1 = 0; j1 < D1; ++j1) {
-            float A[RQ];
-#pragma unroll
-            for (int r = 0; r < RQ; ++r) A[r] = __ldg(qf + (size_t)((r * h1 + i1) * D1 + j1) * M + m);
-#pragma unroll
-            for (int j2 = 0; j2 < D2; j2 += 8) {
-                uint4 u;
-                uint32_t *pu = reinterpret_cast<uint32_t *>(&u);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                    for (int r = 0; r < RQ; ++r) {
-                        s0 += A[r] * B[r][j2 + 2 * k];
-                        s1 += A[r] * B[r][j2 + 2 * k + 1];
-                    }
-                    __nv_bfloat162 hb = __floats2bfloat162_rn(s0 * inv, s1 * inv);
-                    pu[k] = *reinterpret_cast<uint32_t *>(&hb);
+            for (int k = 0; k < kQaBatch; ++k) {
+                const int idx = base + k * kQaThreads + threadIdx.x;
+                const int e = idx / (kQaTokens / 4), t = (idx % (kQaTokens / 4)) * 4;
+                if (idx < total) {
+                    s[t * ld + e] = v[k].x;
+                    s[(t + 1) * ld + e] = v[k].y;
+                    s[(t + 2) * ld + e] = v[k].z;
+                    s[(t + 3) * ld + e] = v[k].w;
                 }
-                *reinterpret_cast<uint4 *>(dst + j1 * D2 + j2) = u;
+            }
+        }
+    } else {
+        const int total = eq * kQaTokens;
+        for (int base = 0; base < total; base += kQaBatch * kQaThreads) {
+            float v[kQaBatch];
+#pragma unroll
+            for (int k = 0; k < kQaBatch; ++k) {
+                const int idx = base + k * kQaThreads + threadIdx.x;
+                const int e = idx / kQaTokens, t = idx % kQaTokens;
+                v[k] = idx < total && t < nt ? __ldg(qf + (size_t)e * M + m0 + t) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < kQaBatch; ++k) {
+                const int idx = base + k * kQaThreads + threadIdx.x;
+                const int e = idx / kQaTokens, t = idx % kQaTokens;
+                if (idx < total) s[t * ld + e] = v[k];
             }
         }
     }
+    __syncthreads();
+    const int h = h1 * h2, c8 = d2 / 8, per_tok = h * c8;
+    const float inv = 1.0f / (float)RQ;
+    for (int task = threadIdx.x; task < nt * per_tok; task += kQaThreads) {
+        const int t = task / per_tok, p = task - t * per_tok;
+        const int head = p / c8, c = p - head * c8;
+        const int i1 = head / h2, i2 = head - i1 * h2;
+        const float *st = s + t * ld;
+        float B[RQ][8];
+#pragma unroll
+        for (int r = 0; r < RQ; ++r) {
+            const float4 *b4 = reinterpret_cast<const float4 *>(st + qa + (r * h2 + i2) * d2 + c * 8);
+            const float4 x = b4[0], y = b4[1];
+            B[r][0] = x.x; B[r][1] = x.y; B[r][2] = x.z; B[r][3] = x.w;
+            B[r][4] = y.x; B[r][5] = y.y; B[r][6] = y.z; B[r][7] = y.w;
+        }
+        __nv_bfloat16 *dst = q_out + ((size_t)(m0 + t) * h + head) * d1 * d2 + c * 8;
+        for (int j1 = 0; j1 < d1; ++j1) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int r = 0; r < RQ; ++r) {
+                const float a = st[(r * h1 + i1) * d1 + j1];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] += a * B[r][u];
+            }
+            uint4 o;
+            uint32_t *po = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 hb = __floats2bfloat162_rn(acc[2 * k] * inv, acc[2 * k + 1] * inv);
+                po[k] = *reinterpret_cast<uint32_t *>(&hb);
+            }
+            *reinterpret_cast<uint4 *>(dst + j1 * d2) = o;
+        }
+    }
+}
+
+template <int RQ>
+cudaError_t launch_q_assemble(const float *qf, int M, const Dims &d, __nv_bfloat16 *qo, cudaStream_t st) {
+    const int eq = RQ * (d.h1 * d.d1 + d.h2 * d.d2);
+    const size_t smem = (size_t)kQaTokens * qa_ld(eq) * sizeof(float);
+    const cudaError_t e = ensure_dynamic_smem<q_assemble_kernel<RQ>>(smem);
+    if (e != cudaSuccess) return e;
+    q_assemble_kernel<RQ><<<(unsigned)((M + kQaTokens - 1) / kQaTokens), kQaThreads, smem, st>>>(
+        qf, M, d.h1, d.h2, d.d1, d.d2, qo);
+    return cudaGetLastError();
 }
 
 // Any shape: one thread per (token, head), loops.
@@ -610,13 +679,24 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     e = cudaGetLastError();
     if (e != cudaSuccess || !q_out) return e;
     __nv_bfloat16 *qo = static_cast<__nv_bfloat16 *>(q_out);
-    const dim3 g2((unsigned)((a.M + 63) / 64), (unsigned)d.h2);
+    // the staged kernel reads B^Q slices as float4 from shared memory: d2 % 8 == 0 and
+    // the B^Q block starting on a 16-byte boundary (R_Q * h1 * d1 % 4 == 0)
+    const bool staged = d.d2 % 8 == 0 && (rq * d.h1 * d.d1) % 4 == 0 &&
+                        (size_t)kQaTokens * qa_ld(rq * (d.h1 * d.d1 + d.h2 * d.d2)) * 4 <= 96 * 1024;
     if (small && d.d2 % 8 == 0) {
         const int threads = a.M * d.h * d.d1 * (d.d2 / 8);
         q_assemble_small_kernel<<<(unsigned)((threads + 127) / 128), 128, 0, st>>>(qf, a.M, d.h1, d.h2, d.d1,
                                                                                   d.d2, rq, qo);
-    } else if (rq == 6 && d.d1 == 8 && d.d2 == 16) {
-        q_assemble_kernel<6, 8, 16><<<g2, 64, 0, st>>>(qf, a.M, d.h1, d.h2, qo);
+    } else if (staged && rq == 1) {
+        return launch_q_assemble<1>(qf, a.M, d, qo, st);
+    } else if (staged && rq == 2) {
+        return launch_q_assemble<2>(qf, a.M, d, qo, st);
+    } else if (staged && rq == 4) {
+        return launch_q_assemble<4>(qf, a.M, d, qo, st);
+    } else if (staged && rq == 6) {
+        return launch_q_assemble<6>(qf, a.M, d, qo, st);
+    } else if (staged && rq == 8) {
+        return launch_q_assemble<8>(qf, a.M, d, qo, st);
     } else {
         dim3 g3((unsigned)((a.M + 127) / 128), (unsigned)d.h);
         q_assemble_any_kernel<<<g3, 128, 0, st>>>(qf, a.M, d.h1, d.h2, d.d1, d.d2, rq, qo);

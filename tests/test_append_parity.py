@@ -63,6 +63,36 @@ def test_append_small_against_oracle():
     _close_bf16(to_f64(q_out.cpu()), q_rot, "assembled query")
 
 
+# Query assembly at other shapes: TPA-like (d1 = 1) with R_Q = 4, R_Q = 1 and 8 (the
+# staged kernel's other instantiations), R_Q = 3 (no instantiation: the generic
+# kernel), and a B^Q block that starts off a 16-byte boundary (R_Q*h1*d1 = 6).
+OTHER_SHAPES = {
+    "tpa_rq4": dict(h1=8, h2=1, d1=1, d2=64, r_k=2, r_v=2, r_q=4),
+    "kpa_rq1": dict(h1=2, h2=4, d1=4, d2=16, r_k=1, r_v=1, r_q=1),
+    "kpa_rq8": dict(h1=4, h2=2, d1=2, d2=32, r_k=2, r_v=1, r_q=8),
+    "kpa_rq3": dict(h1=2, h2=4, d1=4, d2=16, r_k=2, r_v=2, r_q=3),
+    "unaligned": dict(h1=3, h2=2, d1=1, d2=16, r_k=2, r_v=2, r_q=2),
+}
+
+
+@pytest.mark.parametrize("name", list(OTHER_SHAPES))
+def test_append_query_assembly_other_shapes(name):
+    s = SMALL_SHAPE.__class__(d_model=128, rope_base=10000.0, **OTHER_SHAPES[name])
+    w = SMALL.replace(shape=s, n_tok=53, capacity=128)
+    inp = append_inputs(w)
+    start = torch.tensor([8, 0], dtype=torch.int32)
+    lib = kpa()
+    _, kc, vc, q_out = _run_append(lib, w, inp, start)
+    q_rot, k_rot, v_rec, _ = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start.numpy())
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    for b in range(w.batch):
+        st = int(start[b])
+        _close_bf16(kn[b, st:st + w.n_tok], k_rot[b], f"{name} key cache b={b}")
+        _close_bf16(vn[b, st:st + w.n_tok], v_rec[b], f"{name} value cache b={b}")
+    _close_bf16(to_f64(q_out.cpu()), q_rot, f"{name} assembled query")
+
+
 def test_append_full_config_sampled_tokens():
     """Configuration 5 at full size (B=8, 2048 tokens, d_model 2048, R_Q=6): sampled
     tokens of the cache and of q_out checked one by one."""
