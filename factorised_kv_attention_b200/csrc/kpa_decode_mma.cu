@@ -291,7 +291,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     // I_{d1} (x) R^(2)(q_pos) on pairs (2m, 2m+1), angles tabulated once per CTA
     if (rotate && tid < D2 / 2) {
         float cth, sth;
-        rope_cs(qpos, rope.theta[tid], cth, sth);
+        rope_cs_fast(qpos, rope.theta[tid], cth, sth);
         cs[tid] = make_float2(cth, sth);
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
@@ -659,54 +659,48 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     float *po = a.part_o + ((size_t)(b * a.n_split + split) * H) * DH;
     float *pml = a.part_ml + ((size_t)(b * a.n_split + split) * H) * 2;
-    // log-sum-exp weights of the slices, once per head: 2^(m_slice - M) in place of m
-    if constexpr (SLICES > 1) {
-        for (int head = tid; head < H; head += WARPS * 32) {
-            float M = -INFINITY;
+    // One float4 column of the merged partial per thread.  Each thread forms the
+    // log-sum-exp weights 2^(m_slice - M) of its own head from the slice statistics,
+    // so the merge needs no further barrier.
+    constexpr int N4 = H * DH / 4;
+    static_assert(DH % 4 == 0 && (MO_LD % 4) == 0 && ((size_t)SLICES * H * (MO_LD + 2)) % 4 == 0,
+                  "float4 columns of the slice-merge buffer and of the merged partial");
+    for (int c4 = tid; c4 < N4; c4 += WARPS * 32) {
+        const int head = (c4 * 4) / DH, col = c4 * 4 - head * DH;
+        float4 acc;
+        float M, l;
+        if constexpr (SLICES > 1) {
+            M = -INFINITY;
 #pragma unroll
             for (int sl = 0; sl < SLICES; ++sl) M = fmaxf(M, mm[((size_t)sl * H + head) * 2]);
-            float l = 0.f;
+            l = 0.f;
+            acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int sl = 0; sl < SLICES; ++sl) {
-                const float ms = mm[((size_t)sl * H + head) * 2];
-                const float wgt = ms == -INFINITY ? 0.f : exp2f(ms - M);
-                mm[((size_t)sl * H + head) * 2] = wgt;
-                l += wgt * mm[((size_t)sl * H + head) * 2 + 1];
+                const float2 ms = *reinterpret_cast<const float2 *>(mm + ((size_t)sl * H + head) * 2);
+                const float w = ms.x == -INFINITY ? 0.f : exp2f(ms.x - M);
+                const float4 v = *reinterpret_cast<const float4 *>(mo + ((size_t)sl * H + head) * MO_LD + col);
+                l += w * ms.y;
+                acc.x += w * v.x;
+                acc.y += w * v.y;
+                acc.z += w * v.z;
+                acc.w += w * v.w;
             }
-            if (a.cluster) {
+        } else {
+            M = mm[head * 2];
+            l = mm[head * 2 + 1];
+            acc = *reinterpret_cast<const float4 *>(mo + (size_t)head * MO_LD + col);
+        }
+        if (a.cluster) {
+            *reinterpret_cast<float4 *>(cp + c4 * 4) = acc;
+            if (col == 0) {
                 cp[H * DH + head] = M;
                 cp[H * DH + H + head] = l;
-            } else {
-                pml[2 * head] = M;
-                pml[2 * head + 1] = l;
             }
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    }
-    for (int idx = tid; idx < H * DH; idx += WARPS * 32) {
-        const int head = idx / DH;
-        float acc;
-        if constexpr (SLICES > 1) {
-            acc = 0.f;
-#pragma unroll
-            for (int sl = 0; sl < SLICES; ++sl)
-                acc += mm[((size_t)sl * H + head) * 2] * mo[((size_t)sl * H + head) * MO_LD + (idx - head * DH)];
         } else {
-            acc = mo[(size_t)head * MO_LD + (idx - head * DH)];
-            if (idx % DH == 0) {
-                if (a.cluster) {
-                    cp[H * DH + head] = mm[head * 2];
-                    cp[H * DH + H + head] = mm[head * 2 + 1];
-                } else {
-                    pml[2 * head] = mm[head * 2];
-                    pml[2 * head + 1] = mm[head * 2 + 1];
-                }
-            }
+            reinterpret_cast<float4 *>(po)[c4] = acc;
+            if (col == 0) *reinterpret_cast<float2 *>(pml + 2 * head) = make_float2(M, l);
         }
-        if (a.cluster)
-            cp[idx] = acc;
-        else
-            po[idx] = acc;
     }
     if (!a.cluster) {
     if (!a.fused) return;
@@ -723,76 +717,50 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     if (!flags[1]) return;
-    const float *pob = a.part_o + (size_t)b * a.n_split * H * DH;
-    const float *pmb = a.part_ml + (size_t)b * a.n_split * H * 2;
-    // The first float4 column of every thread is requested for up to PF splits at once,
-    // before the split statistics, so the partials arrive in one round trip.
+    // One float4 output column per thread.  The column of up to PF splits and its
+    // head's statistics (m, l) of those splits are requested together, so the merge
+    // takes one round trip to L2; the weights 2^(m_i - M) are formed per thread.
+    const float4 *pob4 = reinterpret_cast<const float4 *>(a.part_o + (size_t)b * a.n_split * H * DH);
+    const float2 *pmb2 = reinterpret_cast<const float2 *>(a.part_ml + (size_t)b * a.n_split * H * 2);
     constexpr int PF = 16;
-    constexpr int N4 = H * DH / 4;
-    const float4 *pob4 = reinterpret_cast<const float4 *>(pob);
-    float4 pre[PF];
-    if (tid < N4) {
-#pragma unroll
-        for (int i = 0; i < PF; ++i)
-            if (i < n_b) pre[i] = __ldcg(pob4 + (size_t)i * N4 + tid);
-    }
-    // split statistics: w[i][head] = 2^(m_i - M) with one thread per (split, head),
-    // then the denominators
-    float *wt = reinterpret_cast<float *>(smem);            // [n_b][H]
-    float *den = wt + (size_t)n_b * H;                      // [H]
-    float *lv = den + H;                                    // [n_b][H]
-    float *mx = lv + (size_t)n_b * H;                       // [H]
-    for (int k = tid; k < n_b * H; k += WARPS * 32) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pmb) + k);
-        wt[k] = ml.x;
-        lv[k] = ml.y;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    for (int head = tid; head < H; head += WARPS * 32) {
-        float M = -INFINITY;
-        for (int i = 0; i < n_b; ++i) M = fmaxf(M, wt[i * H + head]);
-        mx[head] = M;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    for (int k = tid; k < n_b * H; k += WARPS * 32) {
-        const float m = wt[k];
-        const float w = m == -INFINITY ? 0.f : exp2f(m - mx[k % H]);
-        wt[k] = w;
-        lv[k] *= w;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    for (int head = tid; head < H; head += WARPS * 32) {
-        float d = 0.f;
-        for (int i = 0; i < n_b; ++i) d += lv[i * H + head];
-        den[head] = d;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     for (int c4 = tid; c4 < N4; c4 += WARPS * 32) {
         const int head = (c4 * 4) / DH;
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-        int i0 = 0;
-        if (c4 == tid) {                                    // the prefetched column
+        float4 pre[PF];
+        float2 st[PF];
 #pragma unroll
-            for (int i = 0; i < PF; ++i)
-                if (i < n_b) {
-                    const float w = wt[i * H + head];
-                    num.x += w * pre[i].x;
-                    num.y += w * pre[i].y;
-                    num.z += w * pre[i].z;
-                    num.w += w * pre[i].w;
-                }
-            i0 = PF;
-        }
-#pragma unroll 8
-        for (int i = i0; i < n_b; ++i) {
+        for (int i = 0; i < PF; ++i)
+            if (i < n_b) {
+                pre[i] = __ldcg(pob4 + (size_t)i * N4 + c4);
+                st[i] = __ldcg(pmb2 + (size_t)i * H + head);
+            }
+        float M = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < PF; ++i)
+            if (i < n_b) M = fmaxf(M, st[i].x);
+        for (int i = PF; i < n_b; ++i) M = fmaxf(M, __ldcg(pmb2 + (size_t)i * H + head).x);
+        float d = 0.f;
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < PF; ++i)
+            if (i < n_b) {
+                const float w = st[i].x == -INFINITY ? 0.f : exp2f(st[i].x - M);
+                d += w * st[i].y;
+                num.x += w * pre[i].x;
+                num.y += w * pre[i].y;
+                num.z += w * pre[i].z;
+                num.w += w * pre[i].w;
+            }
+#pragma unroll 4
+        for (int i = PF; i < n_b; ++i) {
+            const float2 sv = __ldcg(pmb2 + (size_t)i * H + head);
             const float4 v = __ldcg(pob4 + (size_t)i * N4 + c4);
-            const float w = wt[i * H + head];
+            const float w = sv.x == -INFINITY ? 0.f : exp2f(sv.x - M);
+            d += w * sv.y;
             num.x += w * v.x;
             num.y += w * v.y;
             num.z += w * v.z;
             num.w += w * v.w;
         }
-        const float d = den[head];
         const float f = d > 0.f ? a.out_scale / d : 0.f;
         reinterpret_cast<float4 *>(a.out + (size_t)b * H * DH)[c4] = make_float4(num.x * f, num.y * f, num.z * f,
                                                                                  num.w * f);

@@ -68,6 +68,19 @@ __device__ __forceinline__ void rope_cs(double pos, double theta, float &c, floa
     sincosf((float)r, &s, &c);
 }
 
+// The same angle with the hardware sine/cosine approximations on the reduced argument
+// r in [-pi, pi] (absolute error a few 1e-7 there): for the decode query, whose
+// rotation feeds a bf16-level dot product, at a fraction of the latency.
+__device__ __forceinline__ void rope_cs_fast(double pos, double theta, float &c, float &s) {
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    constexpr double kTwoPiHi = 6.283185307179586;
+    constexpr double kTwoPiLo = 2.4492935982947064e-16;
+    const double phi = pos * theta;
+    const double k = rint(phi * kInvTwoPi);
+    const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, phi));
+    __sincosf((float)r, &s, &c);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device and kernel (so
 // later calls, including ones made while a stream is being captured, launch
 // directly).  The kernel is a template argument: one cache per kernel.
