@@ -329,6 +329,8 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
     if (s != KPA_OK) return s;
     if (qf && p.variant < 0) return KPA_ERR_UNSUPPORTED;        // query factors: tensor-core path only
+    if (qf && (int64_t)cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) > mma_decode_qf_max(p.variant))
+        return KPA_ERR_UNSUPPORTED;                               // staged in the kernel's query rows
     if (!workspace || ws_bytes < p.bytes) return KPA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return KPA_ERR_INVALID_ARG;
     if (p.n_split > 65535 * 16) return KPA_ERR_UNSUPPORTED;

@@ -54,8 +54,9 @@ __device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap
 
 // Rotate the projected pair (n, n+1) when it is a B^Q or B^K pair (cs(j) = (cos, sin)
 // of pair j of the token's position); A factors and V pass unchanged.
-template <class CS>
-__device__ __forceinline__ void rotate_pair(const AppendArgs &a, int n, float &x0, float &x1, CS cs) {
+// RoPE pair index j of projected column n (an even column): the pair (n, n+1) is pair j
+// of a B^Q or B^K row, or -1 when the column is not rotated (A factors, values).
+__device__ __forceinline__ int rope_pair_of(const AppendArgs &a, int n) {
     const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1;
     int r = -1;                                    // offset inside a B row
     if (n < a.eq) {
@@ -63,7 +64,12 @@ __device__ __forceinline__ void rotate_pair(const AppendArgs &a, int n, float &x
     } else if (n < a.eq + a.ek) {
         if (n - a.eq >= ka) r = n - a.eq - ka;
     }
-    const int j = r < 0 ? -1 : (a.d2m1 >= 0 ? (r & a.d2m1) : r % a.d2) >> 1;
+    return r < 0 ? -1 : (a.d2m1 >= 0 ? (r & a.d2m1) : r % a.d2) >> 1;
+}
+
+template <class CS>
+__device__ __forceinline__ void rotate_pair(const AppendArgs &a, int n, float &x0, float &x1, CS cs) {
+    const int j = rope_pair_of(a, n);
     if (j >= 0) {
         const float2 w = cs(j);
         const float y0 = x0 * w.x - x1 * w.y, y1 = x0 * w.y + x1 * w.x;
@@ -340,17 +346,23 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
 // formed in one place; its 8 warps split K, each lane holding 8 consecutive k of
 // both rows and of every token (X stays in L2), then the partial sums are reduced
 // with shuffles and through shared memory.  Thread m runs the epilogue of token m.
-constexpr int kSmallMaxM = 16, kSmallWarps = 8;
+constexpr int kSmallMaxM = 16, kSmallWarps = 8;   // up to 16 tokens; MAXM = 8 or 16 below
 
-__global__ void __launch_bounds__(kSmallWarps * 32)
+template <int MAXM>
+__global__ void __launch_bounds__(kSmallWarps * 32, MAXM == 8 ? 3 : 2)
 append_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, AppendArgs a,
                     RopeTable rope) {
-    __shared__ float red[kSmallWarps][2][kSmallMaxM];
+    __shared__ float red[kSmallWarps][2][MAXM];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = 2 * blockIdx.x;
-    float acc0[kSmallMaxM], acc1[kSmallMaxM];
+    // the epilogue's own inputs (the token's start slot, the pair's RoPE frequency) are
+    // requested now, with the operand loads, instead of after the reduction
+    const int jn = rope_pair_of(a, n);
+    const int sp = tid < a.M ? a.start_pos[tid / a.n_tok] : 0;
+    const double th = tid < a.M && jn >= 0 ? rope.theta[jn] : 0.0;
+    float acc0[MAXM], acc1[MAXM];
 #pragma unroll
-    for (int m = 0; m < kSmallMaxM; ++m) acc0[m] = acc1[m] = 0.f;
+    for (int m = 0; m < MAXM; ++m) acc0[m] = acc1[m] = 0.f;
     const int k8n = a.K / 8;
     const uint4 *w0 = reinterpret_cast<const uint4 *>(w + (size_t)n * a.K);
     const uint4 *w1 = reinterpret_cast<const uint4 *>(w + (size_t)(n + 1) * a.K);
@@ -368,11 +380,15 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
             fb[2 * i] = tb.x;
             fb[2 * i + 1] = tb.y;
         }
+        // every token's x chunk is requested before the first is used (one round trip)
+        uint4 ux[MAXM];
 #pragma unroll
-        for (int m = 0; m < kSmallMaxM; ++m) {
+        for (int m = 0; m < MAXM; ++m)
+            ux[m] = m < a.M ? __ldg(xv + (size_t)m * k8n + k8) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
             if (m >= a.M) break;
-            const uint4 ux = __ldg(xv + (size_t)m * k8n + k8);
-            const __nv_bfloat162 *px = reinterpret_cast<const __nv_bfloat162 *>(&ux);
+            const __nv_bfloat162 *px = reinterpret_cast<const __nv_bfloat162 *>(&ux[m]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float2 tx = __bfloat1622float2(px[i]);
@@ -382,7 +398,7 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
         }
     }
 #pragma unroll
-    for (int m = 0; m < kSmallMaxM; ++m) {
+    for (int m = 0; m < MAXM; ++m) {
         if (m >= a.M) break;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -403,12 +419,12 @@ append_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
         x0 += red[i][0][m];
         x1 += red[i][1][m];
     }
-    const int b = m / a.n_tok, s = a.start_pos[b] + (m - b * a.n_tok);
+    const int b = m / a.n_tok, s = sp + (m - b * a.n_tok);
     const bool slot_ok = s >= 0 && s < a.cap;
     if (!slot_ok && n == 0) raise_error(a.err, kErrDeviceCheck);
-    emit_pair(a, m, b, s, slot_ok, n, x0, x1, [&](int j) {
+    emit_pair(a, m, b, s, slot_ok, n, x0, x1, [&](int) {     // the pair is jn
         float c, sn;
-        rope_cs((double)s, rope.theta[j], c, sn);
+        rope_cs((double)s, th, c, sn);
         return make_float2(c, sn);
     });
 }
@@ -658,8 +674,12 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     const bool small = a.M <= kSmallMaxM;
     if (small) {
         // a decode step: stream W once with a matrix-vector kernel
-        append_small_kernel<<<(unsigned)(a.N / 2), kSmallWarps * 32, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w), a, rope);
+        if (a.M <= 8)
+            append_small_kernel<8><<<(unsigned)(a.N / 2), kSmallWarps * 32, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w), a, rope);
+        else
+            append_small_kernel<16><<<(unsigned)(a.N / 2), kSmallWarps * 32, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w), a, rope);
     } else {
     CUtensorMap tmx, tmw;
     if (!make_map(&tmx, x, (uint64_t)a.M, (uint64_t)d_model, BM)) return cudaErrorInvalidValue;

@@ -237,6 +237,19 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             if (i < H * DH / 2) qv[k] = qb[i];
         }
     }
+    // query factors: the sequence's E_Q values (at most QF_PT per consumer thread) are
+    // requested here, in the same round trip as the other inputs
+    constexpr int QF_PT = C::QF_MAX / (WARPS * 32);
+    const int eq = a.qf ? a.rq * (H1 * D1 + H2 * D2) : 0;
+    float qfv[QF_PT];
+    if (warp < WARPS && a.qf) {
+        const float *qfb = a.qf + (size_t)b * a.qf_seq_stride;
+#pragma unroll
+        for (int k = 0; k < QF_PT; ++k) {
+            const int e = tid + k * WARPS * 32;
+            qfv[k] = e < eq ? __ldg(qfb + (size_t)e * a.qf_stride) : 0.f;
+        }
+    }
     if (L > a.max_len || L < 0) {
         if (split == 0 && tid == 0) raise_error(a.err, kErrDeviceCheck);
         L = L < 0 ? 0 : a.max_len;
@@ -298,33 +311,62 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     if (a.qf) {
         // q = (1/R_Q) sum_r A^Q_r (x) B^Q_r assembled here from fp32 factors ("Kronecker
         // Product Attention", eq 2); the pairs (2m, 2m+1) of each d2 chunk are rotated after
-        // the rank sum (the rotation is linear).  One thread per 8 features of a (head, j1) row.
-        constexpr int CH = D2 / 8;
-        const float *qfb = a.qf + (size_t)b * a.qf_seq_stride;
+        // the rank sum (the rotation is linear).  The factors are staged in the query's
+        // shared-memory rows (E_Q <= H * Q_LD, checked by the host), the outputs are kept in
+        // registers until every thread has read its factors, then written over them.
+        // One thread per 8 features of a (head, j1) row.
+        constexpr int CH = D2 / 8, ITEMS = H * D1 * CH;
+        constexpr int IPT = (ITEMS + WARPS * 32 - 1) / (WARPS * 32);
+        static_assert(C::QF_MAX <= H * C::Q_LD, "query factors staged in the query rows");
+#pragma unroll
+        for (int k = 0; k < QF_PT; ++k) {
+            const int e = tid + k * WARPS * 32;
+            if (e < eq) qs[e] = qfv[k];
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
         const int qa_b = a.rq * H1 * D1;                  // first B^Q element of the record
         const float rs = a.qscale / (float)a.rq;
-        for (int it = tid; it < H * D1 * CH; it += WARPS * 32) {
-            const int head = it / (D1 * CH), rem = it % (D1 * CH), j1 = rem / CH, j2 = (rem % CH) * 8;
-            const int i1 = head / H2, i2h = head % H2;
-            float acc[8];
+        float acc[IPT][8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-            for (int r = 0; r < a.rq; ++r) {
-                const float av = __ldg(qfb + (size_t)((r * H1 + i1) * D1 + j1) * a.qf_stride);
-                const float *bq = qfb + (size_t)(qa_b + (r * H2 + i2h) * D2 + j2) * a.qf_stride;
+        for (int k = 0; k < IPT; ++k) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) acc[u] += av * __ldg(bq + (size_t)u * a.qf_stride);
-            }
-            float *dst = qs + head * C::Q_LD + j1 * D2 + j2;
-#pragma unroll
-            for (int u = 0; u < 8; u += 2) {
-                float y0 = acc[u], y1 = acc[u + 1];
-                if (rotate) {
-                    const float2 w = cs[(j2 + u) >> 1];
-                    y0 = acc[u] * w.x - acc[u + 1] * w.y;
-                    y1 = acc[u] * w.y + acc[u + 1] * w.x;
+            for (int u = 0; u < 8; ++u) acc[k][u] = 0.f;
+            const int it = tid + k * WARPS * 32;
+            if (it < ITEMS) {
+                const int head = it / (D1 * CH), rem = it % (D1 * CH), j1 = rem / CH, j2 = (rem % CH) * 8;
+                const int i1 = head / H2, i2h = head % H2;
+                for (int r = 0; r < a.rq; ++r) {
+                    const float av = qs[(r * H1 + i1) * D1 + j1];
+                    const float4 *bq = reinterpret_cast<const float4 *>(qs + qa_b + (r * H2 + i2h) * D2 + j2);
+                    const float4 b0 = bq[0], b1 = bq[1];
+                    acc[k][0] += av * b0.x;
+                    acc[k][1] += av * b0.y;
+                    acc[k][2] += av * b0.z;
+                    acc[k][3] += av * b0.w;
+                    acc[k][4] += av * b1.x;
+                    acc[k][5] += av * b1.y;
+                    acc[k][6] += av * b1.z;
+                    acc[k][7] += av * b1.w;
                 }
-                *reinterpret_cast<float2 *>(dst + u) = make_float2(y0 * rs, y1 * rs);
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+#pragma unroll
+        for (int k = 0; k < IPT; ++k) {
+            const int it = tid + k * WARPS * 32;
+            if (it < ITEMS) {
+                const int head = it / (D1 * CH), rem = it % (D1 * CH), j1 = rem / CH, j2 = (rem % CH) * 8;
+                float *dst = qs + head * C::Q_LD + j1 * D2 + j2;
+#pragma unroll
+                for (int u = 0; u < 8; u += 2) {
+                    float y0 = acc[k][u], y1 = acc[k][u + 1];
+                    if (rotate) {
+                        const float2 w = cs[(j2 + u) >> 1];
+                        y0 = acc[k][u] * w.x - acc[k][u + 1] * w.y;
+                        y1 = acc[k][u] * w.y + acc[k][u + 1] * w.x;
+                    }
+                    *reinterpret_cast<float2 *>(dst + u) = make_float2(y0 * rs, y1 * rs);
+                }
             }
         }
     }

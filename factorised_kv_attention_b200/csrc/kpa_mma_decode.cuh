@@ -59,6 +59,9 @@ struct MmaDecodeCfg {
     static constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t OFF_Q = OFF_BARS + 16 * STAGES;
     static constexpr int Q_LD = D1 * D2 + 8;                    // padded row of the fp32 query
+    // most query-factor values (E_Q) a decode from query factors takes: staged in the
+    // query rows, eight per consumer thread
+    static constexpr int QF_MAX = 8 * WARPS * 32 < H * Q_LD ? 8 * WARPS * 32 : (H * Q_LD) / (WARPS * 32) * (WARPS * 32);
     static constexpr size_t OFF_CS = OFF_Q + (size_t)H * Q_LD * 4;
     static constexpr size_t OFF_SCR = (OFF_CS + (size_t)(D2 / 2) * 8 + 15) / 16 * 16;
     static constexpr size_t OFF_FLAGS = OFF_SCR + (size_t)WARPS * SCR_FLOATS * 4;
@@ -111,6 +114,15 @@ inline int mma_decode_tile(int variant) {
     if (variant == IDX) return CFG::TT;
     KPA_MMA_VARIANTS(KPA_MMA_TILE)
 #undef KPA_MMA_TILE
+    return 0;
+}
+
+// Most query-factor values (E_Q) a decode of this variant can take from query factors.
+inline int mma_decode_qf_max(int variant) {
+#define KPA_MMA_QFMAX(IDX, CFG) \
+    if (variant == IDX) return CFG::QF_MAX;
+    KPA_MMA_VARIANTS(KPA_MMA_QFMAX)
+#undef KPA_MMA_QFMAX
     return 0;
 }
 

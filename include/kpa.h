@@ -168,7 +168,9 @@ kpa_status kpa_decode_split(const kpa_config *cfg, int32_t batch, const void *q,
  * kpa_append keeps its query factors, B^Q rotated, at the start of its workspace as
  * float32 [E_Q][batch * n_tok]: after a one-token append pass that workspace with
  * qf_stride = batch, qf_seq_stride = 1.  Requires r_q > 0 and a shape covered by a
- * tensor-core decode variant (else KPA_ERR_UNSUPPORTED).  Everything else -- the
+ * tensor-core decode variant, with E_Q at most 2048 and at most h (d_h + 8) rounded down
+ * to a multiple of 256 (the kernel stages the factors in its query rows); otherwise
+ * KPA_ERR_UNSUPPORTED.  Everything else -- the
  * library's choice of split, workspace, outputs, errors -- as kpa_decode. */
 kpa_status kpa_decode_qf(const kpa_config *cfg, int32_t batch, const float *q_factors, int32_t qf_stride,
                          int32_t qf_seq_stride, const int32_t *q_pos, const void *kcache, const void *vcache,
