@@ -1,7 +1,8 @@
 """Decode benchmark for factor-space KPA / TPA attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kpa|reference]
-                    [--workload tpa_decode|kpa_medium|kpa_long|tiny_kpa] [--layers L]
+                    [--workload tpa_decode|tpa_shared|kpa_medium|kpa_long|tiny_kpa|flashtpa|append_prefill]
+                    [--layers L]
 
 A step is one decode pass of a model of L attention layers over one batch: per
 layer, kpa_decode of one query row per sequence against that layer's own factor
@@ -51,7 +52,7 @@ def _args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kpa", "reference"], default="kpa")
     ap.add_argument("--workload", default="tpa_decode",
-                    help="tpa_decode | kpa_medium | kpa_long | tiny_kpa | flashtpa | append_prefill")
+                    help="tpa_decode | tpa_shared | kpa_medium | kpa_long | tiny_kpa | flashtpa | append_prefill")
     ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -219,7 +220,11 @@ def _cpu_baseline(w, inp, seconds, steps=None):
     b = 0
     while (steps is None and t_total < seconds) or (steps is not None and len(times) < steps):
         t0 = time.perf_counter()
-        oracle.decode(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1], q_pos=qp[b:b + 1])
+        if w.shape.shared_b:     # one B for keys and values: value records are A^V only
+            oracle.decode_shared_b(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1],
+                                   q_pos=qp[b:b + 1])
+        else:
+            oracle.decode(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1], q_pos=qp[b:b + 1])
         dt = time.perf_counter() - t0
         times.append(dt)
         t_total += dt

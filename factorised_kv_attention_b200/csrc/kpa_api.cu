@@ -61,6 +61,8 @@ kpa_status check_cfg(const kpa_config *c, bool need_q, bool need_model) {
     if (c->dtype != KPA_F32 && c->dtype != KPA_BF16) return KPA_ERR_INVALID_ARG;
     if (!(c->rope_base > 0.0) || !isfinite(c->rope_base)) return KPA_ERR_INVALID_ARG;
     if (c->d2 % 2 != 0) return KPA_ERR_INVALID_ARG;        // RoPE pairs
+    if (c->shared_b != 0 && c->shared_b != 1) return KPA_ERR_INVALID_ARG;
+    if (c->shared_b && c->r_k != c->r_v) return KPA_ERR_INVALID_ARG;   // B^K_r = B^V_r
     const int64_t h = (int64_t)c->h1 * c->h2, dh = (int64_t)c->d1 * c->d2;
     if (h > 4096 || dh > 4096) return KPA_ERR_UNSUPPORTED;
     if (c->d2 > 2 * kMaxHalfD2) return KPA_ERR_UNSUPPORTED;
@@ -75,7 +77,8 @@ Dims dims_of(const kpa_config *c) {
     d.h = c->h1 * c->h2;
     d.dh = c->d1 * c->d2;
     d.ek = c->r_k * (c->h1 * c->d1 + c->h2 * c->d2);
-    d.ev = c->r_v * (c->h1 * c->d1 + c->h2 * c->d2);
+    d.shared = c->shared_b ? 1 : 0;
+    d.ev = d.shared ? c->r_v * c->h1 * c->d1 : c->r_v * (c->h1 * c->d1 + c->h2 * c->d2);
     return d;
 }
 
@@ -124,11 +127,15 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
                        DecodePlan *p) {
     if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
     p->variant = dt == KPA_BF16 ? mma_decode_variant(d) : -1;
+    if (d.shared && p->variant < 0) return KPA_ERR_UNSUPPORTED;   // shared B: tensor-core variants only
     int ctas_per_sm = 2;
     if (p->variant >= 0) {
         p->tile = mma_decode_tile(p->variant);
         const size_t smem = mma_decode_smem(p->variant);
         ctas_per_sm = smem > 0 ? (int)((227 * 1024) / smem) : 1;
+        // resident CTAs as the occupancy calculator counts them (registers included)
+        const int resident = cluster_capacity(p->variant, 1);
+        if (resident > 0 && sms > 0 && resident / sms < ctas_per_sm) ctas_per_sm = resident / sms;
         if (ctas_per_sm < 1) ctas_per_sm = 1;
     } else {
         int tile = 32;
@@ -429,7 +436,7 @@ kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, cons
     if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
     if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
     const Dims d = dims_of(cfg);
-    if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
+    if (d.shared || !prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
     if (batch == 0 || n_tok == 0) return KPA_OK;
     if (batch > 65535 || d.h > 65535 || (int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
     if (!q || !start_pos || !kcache || !vcache || !out) return KPA_ERR_INVALID_ARG;
@@ -464,7 +471,7 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const
     if (s != KPA_OK) return s;
     if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
     if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
-    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    if (cfg->dtype != KPA_BF16 || cfg->shared_b) return KPA_ERR_UNSUPPORTED;
     // TMA rows of x and W are d_model bf16 values: a multiple of 16 bytes
     if (cfg->d_model % 8 != 0) return KPA_ERR_UNSUPPORTED;
     // factor pairs (2m, 2m+1) of B must start on even columns of the projection

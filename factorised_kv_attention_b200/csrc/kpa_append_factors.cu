@@ -2,7 +2,9 @@
 //
 // "Kronecker Product Attention", section 2.5 and Theorem 2.4: the cache keeps
 // A^K, A^V and B^V as projected and B^K rotated at the token's position by
-// R_theta^(2)(pos); nothing else is rotated.
+// R_theta^(2)(pos); nothing else is rotated.  With one B shared by keys and values
+// ("Tensor Product Attention Is All You Need", section 5) B is stored unrotated and
+// the value record holds A^V only.
 //
 // One CTA owns one 8-token cache group of one plane of one sequence: it reads the
 // (up to) 8 natural-layout records of that group, rotates the B^K pairs and
@@ -60,7 +62,8 @@ append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__re
 
     const int half = d.d2 / 2;
     const int a_size = (is_k ? d.rk : d.rv) * d.h1 * d.d1;
-    if (is_k) {
+    const bool rot_k = is_k && !d.shared;         // a shared B is stored unrotated
+    if (rot_k) {
         for (int i = threadIdx.x; i < kGroup * half; i += blockDim.x) {
             const int k = i / half, m = i % half;
             float c, s;
@@ -71,7 +74,7 @@ append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__re
     }
 
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const bool rot = is_k && e >= a_size;
+        const bool rot = rot_k && e >= a_size;
         int partner = e, j2 = 0;
         if (rot) {
             j2 = (e - a_size) % d.d2;

@@ -114,6 +114,16 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// The same product with fp16 operands (the score of a shared-B cache, whose rotated
+// key factors are formed in registers and kept at fp16 precision).
+__device__ __forceinline__ void mma16816h(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t mask_pair(uint32_t v, bool keep0, bool keep1) {
     return (keep0 ? (v & 0xffffu) : 0u) | (keep1 ? (v & 0xffff0000u) : 0u);
 }
@@ -166,6 +176,31 @@ __device__ __forceinline__ void split2(float2 x, uint32_t &hi, uint32_t &lo) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x.y), "f"(x.x));
     const float2 r = fsub2(x, unpack_bf16x2(hi));
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(r.y), "f"(r.x));
+}
+
+// (x.x, x.y) -> fp16 hi + lo pairs, low half = x.x
+__device__ __forceinline__ void split2h(float2 x, uint32_t &hi, uint32_t &lo) {
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x.y), "f"(x.x));
+    float2 h;
+    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+        : "=f"(h.x), "=f"(h.y)
+        : "r"(hi));
+    const float2 r = fsub2(x, h);
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(r.y), "f"(r.x));
+}
+
+// RoPE pair (x0, x1) of a bf16x2 key factor word rotated by (cos, sin) = w, as fp16x2:
+// (x0 c - x1 s, x0 s + x1 c), low half first.
+__device__ __forceinline__ uint32_t rotate_to_h2(uint32_t v, float2 w) {
+    const float2 x = unpack_bf16x2(v);
+    const float y0 = x.x * w.x - x.y * w.y, y1 = x.x * w.y + x.y * w.x;
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y1), "f"(y0));
+    return r;
+}
+
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+    return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
 
 // ------------------------------------------------------------------- kernel
@@ -385,6 +420,18 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 make_float2(y.x * a.qscale, y.y * a.qscale);
         }
     }
+    if constexpr (C::SHARED) {
+        // theta_m and (cos, sin)(k theta_m), k < 16, for the in-kernel key rotation
+        double *th = reinterpret_cast<double *>(smem + C::OFF_THETA);
+        float2 *st = reinterpret_cast<float2 *>(smem + C::OFF_STEP);
+        for (int i = tid; i < D2 / 2; i += WARPS * 32) th[i] = rope.theta[i];
+        for (int i = tid; i < 16 * (D2 / 2); i += WARPS * 32) {
+            const int k = i / (D2 / 2), m = i % (D2 / 2);
+            float cth, sth;
+            rope_cs_fast((double)k, rope.theta[m], cth, sth);
+            st[i] = make_float2(cth, sth);
+        }
+    }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
 
     // ------------------------------------------------------------ consumers
@@ -406,8 +453,19 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 const int j2 = ks * 16 + 2 * c + ((v & 2) ? 8 : 0);
                 const int i1 = row / D1, j1 = row % D1;
                 const float *src = qs + (i1 * H2 + i2) * C::Q_LD + j1 * D2 + j2;
-                split2(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
+                if constexpr (C::SHARED)
+                    split2h(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
+                else
+                    split2(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
             }
+    // shared B: the keys' factors are stored unrotated, so each 16-token chunk rotates
+    // its B^K fragments at the tokens' slots ("Kronecker Product Attention", Def 2.3 and
+    // Thm 2.4: rotating B rotates the key).  (cos, sin)((p0 + k) theta_m) is formed as
+    // (cos, sin)(p0 theta_m) * (cos, sin)(k theta_m), the first per chunk, the second
+    // from a per-CTA table of the 16 offsets k.
+    const double *theta_s = reinterpret_cast<const double *>(smem + C::OFF_THETA);
+    const float2 *step_s = reinterpret_cast<const float2 *>(smem + C::OFF_STEP);
+    float2 *base_s = reinterpret_cast<float2 *>(smem + C::OFF_BASE) + (size_t)warp * (D2 / 2);
 
     float o[MT][NT][4];
 #pragma unroll
@@ -445,6 +503,27 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             if (tok0 >= n_valid) break;                       // rest of this warp's slice is past the tail
             const bool tail = tok0 + 16 > n_valid;
             const unsigned char *kg0 = kt + (size_t)(tok0 >> 3) * EK * 16;
+            float2 rc[2][KS][2];          // shared B: (cos, sin) of this lane's pairs, tokens g and 8 + g
+            if constexpr (C::SHARED) {
+                const int p0 = t0 + t * TT + tok0;        // slot (= position) of the chunk's first token
+                __syncwarp();                             // the previous chunk is done with base_s
+                for (int m = lane; m < D2 / 2; m += 32) {
+                    float cth, sth;
+                    rope_cs_fast((double)p0, theta_s[m], cth, sth);
+                    base_s[m] = make_float2(cth, sth);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            // fragment word hh of k-step ks holds features 16 ks + 8 hh + 2c, +1
+                            const int m = 8 * ks + 4 * hh + c;
+                            rc[gi][ks][hh] = cmul(base_s[m], step_s[(gi * 8 + g) * (D2 / 2) + m]);
+                        }
+            }
             // ---- scores: sc[mt][gi][v] = sum_r A^K_r * (Q_i2 B~^K_r), rows (i1,j1), tokens 2c, 2c+1
             float2 sc[MT][2][2];
 #pragma unroll
@@ -469,13 +548,32 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                             ldsm_x2_t(smem_u32(grp + (size_t)(e_b + ks * 16 + (lane & 15)) * 16), bk[ks][0],
                                       bk[ks][1]);
                     }
+                    if constexpr (C::SHARED) {
+#pragma unroll
+                        for (int ks = 0; ks < KS; ++ks) {
+                            bk[ks][0] = rotate_to_h2(bk[ks][0], rc[gi][ks][0]);
+                            bk[ks][1] = rotate_to_h2(bk[ks][1], rc[gi][ks][1]);
+                        }
+                    }
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
                         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int ks = 0; ks < KS; ++ks) {
-                            mma16816(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
-                            mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
+                            if constexpr (C::SHARED) {
+                                mma16816h(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
+                                mma16816h(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
+                            } else {
+                                mma16816(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
+                                mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
+                            }
+                        }
+                        if constexpr (C::SHARED) {
+                            // a valid token whose rotated factors left the fp16 range
+                            const int tk = tok0 + gi * 8 + 2 * c;
+                            if ((tk < n_valid && !(isfinite(acc[0]) && isfinite(acc[2]))) ||
+                                (tk + 1 < n_valid && !(isfinite(acc[1]) && isfinite(acc[3]))))
+                                raise_error(a.err, kErrDeviceCheck);
                         }
                         const int row0 = mt * 16 + g;
                         const float2 a0 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MA + row0) * 16 + 4 * c));
@@ -617,11 +715,14 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                     split2(x2, pa_hi[mt][2], pa_lo[mt][2]);
                     split2(x3, pa_hi[mt][3], pa_lo[mt][3]);
                 }
-                const int e_b = A_V + r * H2 * D2 + i2 * D2;
+                // B^V: the value record's B, or (shared) the key record's unrotated B
+                const int e_b = (C::SHARED ? A_K : A_V) + r * H2 * D2 + i2 * D2;
+                const unsigned char *b0p = C::SHARED ? kg0 : g0p;
+                const unsigned char *b1p = C::SHARED ? kg0 + (size_t)EK * 16 : g1p;
                 const int mat = lane >> 3, mrow = lane & 7;
 #pragma unroll
                 for (int np = 0; np < NT / 2; ++np) {
-                    const unsigned char *gp = (mat & 1) ? g1p : g0p;
+                    const unsigned char *gp = (mat & 1) ? b1p : b0p;
                     uint32_t b00, b01, b10, b11;
                     ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mrow) * 16), b00, b01,
                             b10, b11);

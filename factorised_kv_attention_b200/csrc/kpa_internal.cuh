@@ -24,6 +24,7 @@ struct Dims {
     int rk, rv;
     int h, dh;      // h1*h2, d1*d2
     int ek, ev;     // elements per key / value record
+    int shared;     // one B for keys and values: key record [A^K | B] (B unrotated), value record [A^V]
 };
 
 // theta_m = base^(-2m/d2), m < d2/2, formed on the host in float64 and passed by

@@ -41,13 +41,17 @@ struct DecodeArgs {
 // One instantiation per (split, ranks) family.
 //   MA = h1*d1 (rows of the per-i2 GEMMs), D1, D2, RK, RV, H2 = h2,
 //   SLICES  token slices per CTA (warps = H2 * SLICES),
-//   CHUNKS  16-token chunks per warp per stage, STAGES ring depth.
-template <int MA_, int D1_, int D2_, int RK_, int RV_, int H2_, int SLICES_, int CHUNKS_, int STAGES_>
+//   CHUNKS  16-token chunks per warp per stage, STAGES ring depth,
+//   SHARED  one B for keys and values: key record [A^K | B] (B unrotated, rotated in
+//           the kernel for the score), value record [A^V].
+template <int MA_, int D1_, int D2_, int RK_, int RV_, int H2_, int SLICES_, int CHUNKS_, int STAGES_,
+          bool SHARED_ = false>
 struct MmaDecodeCfg {
     static constexpr int MA = MA_, D1 = D1_, D2 = D2_, RK = RK_, RV = RV_, H2 = H2_;
     static constexpr int SLICES = SLICES_, CHUNKS = CHUNKS_, STAGES = STAGES_;
+    static constexpr bool SHARED = SHARED_;
     static constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
-    static constexpr int EK = RK * (MA + H2 * D2), EV = RV * (MA + H2 * D2);
+    static constexpr int EK = RK * (MA + H2 * D2), EV = SHARED ? RV * MA : RV * (MA + H2 * D2);
     static constexpr int WARPS = H2 * SLICES;
     static constexpr int TT = 16 * CHUNKS * SLICES;             // tokens per stage
     static constexpr int STAGE_BYTES = TT * (EK + EV) * 2;
@@ -65,7 +69,12 @@ struct MmaDecodeCfg {
     static constexpr size_t OFF_CS = OFF_Q + (size_t)H * Q_LD * 4;
     static constexpr size_t OFF_SCR = (OFF_CS + (size_t)(D2 / 2) * 8 + 15) / 16 * 16;
     static constexpr size_t OFF_FLAGS = OFF_SCR + (size_t)WARPS * SCR_FLOATS * 4;
-    static constexpr size_t smem_bytes() { return OFF_FLAGS + 16; }
+    // shared B: theta_m (fp64), (cos, sin)(k theta_m) for the 16 token offsets k of a
+    // chunk, and per warp (cos, sin)(p0 theta_m) at its chunk's first position p0
+    static constexpr size_t OFF_THETA = OFF_FLAGS + 16;
+    static constexpr size_t OFF_STEP = OFF_THETA + (SHARED ? (size_t)(D2 / 2) * 8 : 0);
+    static constexpr size_t OFF_BASE = OFF_STEP + (SHARED ? (size_t)16 * (D2 / 2) * 8 : 0);
+    static constexpr size_t smem_bytes() { return OFF_BASE + (SHARED ? (size_t)WARPS * (D2 / 2) * 8 : 0); }
     // row stride (floats) of the slice-merge buffer: 8 floats of padding put the rows
     // of consecutive heads in different banks
     static constexpr int MO_LD = D1 * D2 + 8;
@@ -82,6 +91,8 @@ struct MmaDecodeCfg {
 
 // TPA, h = 16, d_h = 64, R_K = R_V = 2 (the degenerate split h1 = h, d1 = 1, h2 = 1).
 using MmaTpaH16D64R2 = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2>;
+// TPA, h = 16, d_h = 64, R = 2 with one B shared by keys and values.
+using MmaTpaH16D64R2Shared = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2, true>;
 // TPA, h = 32, d_h = 64, R_K = R_V = 1 (the FlashTPA decoding benchmark's shape).
 using MmaTpaH32D64R1 = MmaDecodeCfg<32, 1, 64, 1, 1, 1, 8, 2, 2>;
 // KPA h = 4x8, d_h = 8x16, R_K = R_V = 4.
@@ -96,13 +107,14 @@ using MmaKpaH4x4D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2>;
     X(1, MmaKpaH4x8D8x16R4)        \
     X(2, MmaKpaH4x8D8x16R2)        \
     X(3, MmaKpaH4x4D8x16R2)        \
-    X(4, MmaTpaH32D64R1)
+    X(4, MmaTpaH32D64R1)           \
+    X(5, MmaTpaH16D64R2Shared)
 
 // Index of the variant that covers these dims, or -1.
 inline int mma_decode_variant(const Dims &d) {
 #define KPA_MMA_MATCH(IDX, CFG)                                                            \
     if (d.h1 * d.d1 == CFG::MA && d.d1 == CFG::D1 && d.d2 == CFG::D2 && d.rk == CFG::RK && \
-        d.rv == CFG::RV && d.h2 == CFG::H2)                                                \
+        d.rv == CFG::RV && d.h2 == CFG::H2 && (d.shared != 0) == CFG::SHARED)                \
         return IDX;
     KPA_MMA_VARIANTS(KPA_MMA_MATCH)
 #undef KPA_MMA_MATCH

@@ -79,6 +79,16 @@ typedef struct {
     int32_t d_model;    /* hidden size (kpa_append only; 0 elsewhere)           */
     double rope_base;   /* RoPE base, e.g. 10000                                */
     kpa_dtype dtype;    /* element type of caches, factors, queries, x and W    */
+    int32_t shared_b;   /* 0: separate B^K and B^V.  1: one B shared by keys and
+                         * values ("Tensor Product Attention Is All You Need",
+                         * section 5, "TPA KV with Shared B"; B^K_r = B^V_r, so
+                         * r_k == r_v).  The key record is then [A^K | B] with B
+                         * stored UNROTATED (values must not see the rotation);
+                         * the value record is [A^V] only (E_V = r_v h1 d1), and
+                         * kpa_decode rotates B for the score at each cached
+                         * token's position.  Taken by kpa_cache_bytes_per_token,
+                         * kpa_append_factors and the decode calls;
+                         * kpa_append and kpa_prefill return KPA_ERR_UNSUPPORTED. */
 } kpa_config;
 
 /* Human-readable name of a status code (static storage). */

@@ -237,6 +237,31 @@ def decode(shape, q, kf, vf, seq_len, *, q_pos=None, keys_rotated=False, sm_scal
     return out[:, 0]
 
 
+def decode_shared_b(shape, q, kf, va, seq_len, *, q_pos=None, sm_scale=None, heads=None) -> np.ndarray:
+    """Decode over a cache whose keys and values share their B factors ("Tensor Product
+    Attention Is All You Need", section 5, "TPA KV with Shared B": b_r^K = b_r^V, so
+    R_K = R_V = R).  Key of slot t: the rotation at position t of (1/R) sum_r A^K_r (x) B_r;
+    value of slot t: (1/R) sum_r A^V_r (x) B_r, with the same, unrotated, B_r.
+
+    kf [B][cap][R(h1 d1 + h2 d2)] holds [A^K | B] (B unrotated); va [B][cap][R h1 d1] holds
+    A^V.  The value record [A^V | B] is formed and the plain definition (``decode`` with
+    keys rotated at their slots) does the rest.
+    """
+    s = shape
+    R = s.r_k
+    assert s.r_v == R, "a shared B needs R_K == R_V"
+    kf, va = _f64(kf), _f64(va)
+    a = R * s.h1 * s.d1
+    assert va.shape == kf.shape[:2] + (a,), va.shape
+    vf = np.concatenate([va, kf[:, :, a:]], axis=2)
+    return decode(s, q, kf, vf, seq_len, q_pos=q_pos, keys_rotated=False, sm_scale=sm_scale, heads=heads)
+
+
+def cache_numbers_per_token_shared_b(h1, h2, d1, d2, r) -> int:
+    """Numbers cached per token with one B set for keys and values: A^K, A^V and B."""
+    return 2 * r * h1 * d1 + r * h2 * d2
+
+
 def prefill(shape, q, kf, vf, start_pos, *, q_pos=None, keys_rotated=False, sm_scale=None,
             heads=None) -> np.ndarray:
     """Causal rows: q [B][n][h][dh]; row t of sequence b sees slots 0..start_pos[b]+t."""

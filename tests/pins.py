@@ -345,11 +345,48 @@ def check_cache_sizes_golden():
         assert abs(mb - c["approx_mb"]) <= c["tol_mb"], f"{c['cite']}: {mb} MB"
 
 
+def check_shared_b_attention(seed=13):
+    """A shared-B cache ("Tensor Product Attention Is All You Need", section 5): the
+    factors A^K, A^V and B are drawn as separate arrays, K_t and V_t are formed with
+    numpy.kron from the SAME B_r, K_t is rotated with numpy.kron rotation matrices, and
+    torch's scaled_dot_product_attention gives the expected output."""
+    rng = np.random.default_rng(seed)
+    for s in [Shape(h1=16, h2=1, d1=1, d2=8, r_k=2, r_v=2), Shape(h1=2, h2=3, d1=2, d2=4, r_k=3, r_v=3),
+              Shape(h1=3, h2=2, d1=4, d2=2, r_k=1, r_v=1, rope_base=500000.0)]:
+        B, cap, R = 2, 7, s.r_k
+        AK = rng.standard_normal((B, cap, R, s.h1, s.d1))
+        AV = rng.standard_normal((B, cap, R, s.h1, s.d1))
+        Bf = rng.standard_normal((B, cap, R, s.h2, s.d2))
+        q = rng.standard_normal((B, s.h, s.dh))
+        q_pos = rng.integers(0, 600000, size=B)
+        L = np.array([cap, 4])
+        scale = 0.9 / math.sqrt(s.dh)
+        kf = np.concatenate([AK.reshape(B, cap, -1), Bf.reshape(B, cap, -1)], axis=2)
+        got = oracle.decode_shared_b(s, q, kf, AV.reshape(B, cap, -1), L, q_pos=q_pos, sm_scale=scale)
+        K = np.zeros((B, cap, s.h, s.dh)); V = np.zeros((B, cap, s.h, s.dh))
+        for b in range(B):
+            for t in range(cap):
+                rot = np.kron(np.eye(s.d1), _rot_matrix_d2(s.d2, s.rope_base, t))
+                K[b, t] = (sum(np.kron(AK[b, t, r], Bf[b, t, r]) for r in range(R)) / R) @ rot.T
+                V[b, t] = sum(np.kron(AV[b, t, r], Bf[b, t, r]) for r in range(R)) / R
+        Q = np.stack([q[b] @ np.kron(np.eye(s.d1), _rot_matrix_d2(s.d2, s.rope_base, q_pos[b])).T
+                      for b in range(B)])
+        mask = np.arange(cap)[None, :] < L[:, None]
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q)[:, :, None], torch.from_numpy(K).permute(0, 2, 1, 3),
+            torch.from_numpy(V).permute(0, 2, 1, 3), attn_mask=torch.from_numpy(mask)[:, None, None],
+            scale=scale)[:, :, 0].numpy()
+        _close(got, want, 1e-11, f"shared-B attention vs SDPA {s}")
+        # one B set instead of two: the unshared count minus R h2 d2
+        n = oracle.cache_numbers_per_token_shared_b(s.h1, s.h2, s.d1, s.d2, R)
+        assert n == oracle.cache_numbers_per_token(s.h1, s.h2, s.d1, s.d2, R, R) - R * s.h2 * s.d2
+
+
 ALL_CHECKS = [
     check_kron_is_numpy_kron, check_reconstruct_is_kron_sum, check_tpa_split_is_outer_product,
     check_prop22_factored_score, check_rope_golden_frequencies, check_rope_tpa_is_textbook,
     check_rope_kpa_is_identity_kron_rotation, check_thm24_rotating_b_equals_rotating_reconstruction,
     check_relative_position, check_attention_matches_sdpa, check_attention_closed_forms,
     check_prefill_rows_are_decodes, check_projection_is_matmul, check_append_scores_follow_eq9,
-    check_cache_sizes_golden,
+    check_cache_sizes_golden, check_shared_b_attention,
 ]

@@ -45,9 +45,13 @@ def test_cache_bytes_match_eq10(name):
     cfg = kpa.make_config(s, w.dtype)
     kb, vb = kpa.kpa_cache_bytes_per_token(cfg)
     elt = 2 if w.dtype == "bf16" else 4
-    numbers = oracle.cache_numbers_per_token(s.h1, s.h2, s.d1, s.d2, s.r_k, s.r_v)
+    if s.shared_b:
+        numbers = oracle.cache_numbers_per_token_shared_b(s.h1, s.h2, s.d1, s.d2, s.r_k)
+        assert vb == s.r_v * s.h1 * s.d1 * elt           # the value record is A^V only
+    else:
+        numbers = oracle.cache_numbers_per_token(s.h1, s.h2, s.d1, s.d2, s.r_k, s.r_v)
+        assert kb * s.r_v == vb * s.r_k
     assert kb + vb == numbers * elt
-    assert kb * s.r_v == vb * s.r_k
 
 
 def test_cache_bytes_of_the_configs():
@@ -59,6 +63,34 @@ def test_cache_bytes_of_the_configs():
         assert kb + vb == b, name
     kb, vb = kpa.kpa_cache_bytes_per_token(kpa.make_config(APPEND_PREFILL.shape, "bf16"))
     assert kb + vb == 768
+    # shared B: A^K, A^V (16 each per rank) and one B (64 per rank), R = 2, bf16
+    w = DECODE_CONFIGS["tpa_shared"]
+    assert kpa.kpa_cache_bytes_per_token(kpa.make_config(w.shape, w.dtype)) == (320, 64)
+
+
+def test_shared_b_needs_equal_ranks():
+    cfg = kpa.make_config(Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=1, shared_b=1), "bf16")
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_cache_bytes_per_token(cfg)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+    cfg = kpa.make_config(Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2), "bf16")
+    cfg.shared_b = 2
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_cache_bytes_per_token(cfg)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def test_shared_b_projection_and_prefill_unsupported():
+    """A shared-B cache is written from given factors and decoded; the merged projection
+    and the prefill do not take it (checked before any device call)."""
+    s = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, shared_b=1)
+    cfg = kpa.make_config(s, "bf16")
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_append(cfg, 1, 16, A, A, A, 64, A, A, None, None, stream=0)
+    assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)
+    assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
 
 
 BAD_SHAPES = [dict(h1=0), dict(d2=7), dict(r_k=0), dict(r_v=-1), dict(d1=-2)]

@@ -1,0 +1,104 @@
+"""Decode over a cache whose keys and values share their B factors ("Tensor Product
+Attention Is All You Need", section 5, "TPA KV with Shared B") against the float64
+oracle (GPU).  The key plane holds [A^K | B] with B unrotated, the value plane [A^V];
+the decode kernel rotates B at each cached token's slot for the score and reads the
+same, unrotated B for the values."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_bf16_close, fill_cache, kpa, natural, run_decode
+from workloads import TPA_SHARED_DECODE, decode_inputs, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle(w, inp, sm_scale, q=None):
+    return oracle.decode_shared_b(w.shape, to_f64(inp["q"] if q is None else q), to_f64(inp["kf"]),
+                                  to_f64(inp["vf"]), inp["seq_len"].numpy(), q_pos=inp["q_pos"].numpy(),
+                                  sm_scale=sm_scale)
+
+
+# (workload, tokens per split, score sharpening): automatic plan over ragged lengths;
+# explicit 64- and 128-token splits with ragged tails; scores sharpened 40x; and a long
+# cache with a large RoPE base (angles up to several thousand radians).
+CASES = {
+    "ragged_auto": (TPA_SHARED_DECODE.replace(batch=4, capacity=1024, length=0, ragged=(1, 1024), seed=61), 0, 1.0),
+    "split64": (TPA_SHARED_DECODE.replace(batch=3, capacity=512, length=0, ragged=(100, 512), seed=62), 64, 1.0),
+    "split128_sharp": (TPA_SHARED_DECODE.replace(batch=3, capacity=768, length=0, ragged=(200, 768), seed=63),
+                       128, 40.0),
+    "long_base5e5": (TPA_SHARED_DECODE.replace(
+        shape=dataclasses.replace(TPA_SHARED_DECODE.shape, rope_base=500000.0), batch=2, capacity=8192,
+        length=8192, seed=64), 0, 1.0),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_shared_b_decode_against_oracle(name):
+    w, tps, sharp = CASES[name]
+    inp = decode_inputs(w)
+    lib = kpa()
+    cfg, kc, vc = fill_cache(lib, w, inp)
+    scale = sharp / np.sqrt(w.shape.dh)
+    out = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"], sm_scale=scale,
+                     tokens_per_split=tps)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    assert_bf16_close(out.cpu().numpy(), _oracle(w, inp, scale), f"shared B {name}")
+
+
+def test_shared_b_cache_holds_the_factors_unrotated():
+    """kpa_append_factors with a shared B writes the records as given: B is not rotated
+    (the values read it), and the value plane holds A^V only (bit-exact)."""
+    w = TPA_SHARED_DECODE.replace(batch=2, capacity=64, length=0, ragged=(17, 64), seed=65)
+    inp = decode_inputs(w)
+    lib = kpa()
+    _, kc, vc = fill_cache(lib, w, inp)
+    s = w.shape
+    assert vc.numel() == w.batch * w.capacity * s.r_v * s.h1 * s.d1
+    kn = natural(kc.cpu(), w.batch, w.capacity, s.e_k)
+    vn = natural(vc.cpu(), w.batch, w.capacity, s.e_v)
+    assert torch.equal(kn, inp["kf"]) and torch.equal(vn, inp["vf"])
+
+
+def test_shared_b_decode_from_query_factors():
+    """kpa_decode_qf over a shared-B cache: the query assembled from factors in the kernel."""
+    w = TPA_SHARED_DECODE.replace(shape=dataclasses.replace(TPA_SHARED_DECODE.shape, r_q=6), batch=3,
+                                  capacity=1024, length=0, ragged=(1, 1024), seed=66)
+    s = w.shape
+    inp = decode_inputs(w)
+    rng = np.random.default_rng(166)
+    qf = (rng.standard_normal((w.batch, s.e_q)) / np.sqrt(s.r_q)).astype(np.float32)
+    lib = kpa()
+    cfg, kc, vc = fill_cache(lib, w, inp)
+    L = inp["seq_len"]
+    max_len = int(L.max())
+    ws = torch.zeros(lib.kpa_decode_workspace_size(cfg, w.batch, max_len), dtype=torch.uint8, device="cuda")
+    out = torch.full((w.batch, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    scale = 1.0 / np.sqrt(s.dh)
+    lib.kpa_decode_qf(cfg, w.batch, torch.from_numpy(qf).cuda(), 1, s.e_q, inp["q_pos"].cuda(), kc, vc,
+                      w.capacity, L.cuda(), max_len, scale, out, ws)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    q_dense = np.stack([oracle.reconstruct(s.h1, s.h2, s.d1, s.d2, s.r_q, qf[b].astype(np.float64))
+                        for b in range(w.batch)])
+    assert_bf16_close(out.cpu().numpy(), _oracle(w, inp, scale, q=torch.from_numpy(q_dense)),
+                      "shared B, query factors")
+
+
+def test_shared_b_fp16_overflow_is_reported():
+    """The rotated key factors enter the score product as fp16: a cached B value beyond
+    its range in a visible slot is reported as KPA_ERR_DEVICE_CHECK."""
+    w = TPA_SHARED_DECODE.replace(batch=2, capacity=256, length=200, seed=67)
+    inp = decode_inputs(w)
+    a = w.shape.r_k * w.shape.h1 * w.shape.d1
+    inp["kf"][1, 37, a + 5] = 1.0e6          # a B element of a visible slot of sequence 1
+    lib = kpa()
+    cfg, kc, vc = fill_cache(lib, w, inp)
+    lib.kpa_read_device_error()               # clear
+    run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"])
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == lib.KPA_ERR_DEVICE_CHECK

@@ -38,6 +38,7 @@ class Shape:
     r_q: int = 0
     d_model: int = 0
     rope_base: float = 10000.0
+    shared_b: int = 0          # 1: one B factor for keys and values (B^K_r = B^V_r, r_k == r_v)
 
     @property
     def h(self) -> int:
@@ -54,6 +55,10 @@ class Shape:
 
     @property
     def e_v(self) -> int:
+        """Elements in one token's value record: [A_0.. | B_0..], or [A_0..] alone when
+        the B factors are shared with the keys."""
+        if self.shared_b:
+            return self.r_v * self.h1 * self.d1
         return self.r_v * (self.h1 * self.d1 + self.h2 * self.d2)
 
     @property
@@ -145,8 +150,15 @@ FLASHTPA_DECODE = DecodeWorkload(
     shape=FLASHTPA_SHAPE, batch=1, capacity=1 << 19, dtype="bf16", factor_std=1.0, q_std=1.0 / 8.0,
     seed=0, length=1 << 19)
 
+# The TPA decode with one B shared by keys and values ("Tensor Product Attention Is All
+# You Need", section 5, "TPA KV with Shared B"): same sizes, key record [A^K | B]
+# (B unrotated), value record [A^V].
+TPA_SHARED_DECODE = dataclasses.replace(
+    TPA_DECODE, name="TPA decode, shared B (B=8, h=16x1, d_h=1x64, R=2, L=4096, bf16)",
+    shape=dataclasses.replace(TPA_DECODE.shape, shared_b=1))
+
 DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
-                  "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE}
+                  "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE, "tpa_shared": TPA_SHARED_DECODE}
 
 
 # --- draws ---------------------------------------------------------------------
