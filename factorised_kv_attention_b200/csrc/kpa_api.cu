@@ -471,7 +471,7 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const
     if (s != KPA_OK) return s;
     if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
     if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
-    if (cfg->dtype != KPA_BF16 || cfg->shared_b) return KPA_ERR_UNSUPPORTED;
+    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
     // TMA rows of x and W are d_model bf16 values: a multiple of 16 bytes
     if (cfg->d_model % 8 != 0) return KPA_ERR_UNSUPPORTED;
     // factor pairs (2m, 2m+1) of B must start on even columns of the projection

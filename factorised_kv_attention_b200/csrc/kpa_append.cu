@@ -31,6 +31,7 @@ struct AppendArgs {
     int h1, h2, d1, d2, rq, rk, rv;
     int eq, ek, ev;              // elements per query / key / value record
     int d2m1;                    // d2 - 1 when d2 is a power of two (pair index by mask), else -1
+    int shared;                  // one B for keys and values: columns [A^Q|B^Q|A^K|A^V|B], B unrotated
     __nv_bfloat16 *kc, *vc;
     float *qf;                   // [eq][M] query factors (B^Q rotated), or null
     int *err;
@@ -55,13 +56,14 @@ __device__ __forceinline__ void store_cache(__nv_bfloat16 *plane, int b, int cap
 // Rotate the projected pair (n, n+1) when it is a B^Q or B^K pair (cs(j) = (cos, sin)
 // of pair j of the token's position); A factors and V pass unchanged.
 // RoPE pair index j of projected column n (an even column): the pair (n, n+1) is pair j
-// of a B^Q or B^K row, or -1 when the column is not rotated (A factors, values).
+// of a B^Q or B^K row, or -1 when the column is not rotated (A factors, values, and a
+// B shared by keys and values, which the cache keeps unrotated).
 __device__ __forceinline__ int rope_pair_of(const AppendArgs &a, int n) {
     const int qa = a.rq * a.h1 * a.d1, ka = a.rk * a.h1 * a.d1;
     int r = -1;                                    // offset inside a B row
     if (n < a.eq) {
         if (n >= qa) r = n - qa;
-    } else if (n < a.eq + a.ek) {
+    } else if (!a.shared && n < a.eq + a.ek) {
         if (n - a.eq >= ka) r = n - a.eq - ka;
     }
     return r < 0 ? -1 : (a.d2m1 >= 0 ? (r & a.d2m1) : r % a.d2) >> 1;
@@ -78,6 +80,23 @@ __device__ __forceinline__ void rotate_pair(const AppendArgs &a, int n, float &x
     }
 }
 
+// Cache record of projected column n >= eq: true for the key record, with e its element.
+// Columns [A^K | B^K | A^V | B^V]; with a shared B, [A^K | A^V | B] and B belongs to the
+// key record after A^K.
+__device__ __forceinline__ bool key_column(const AppendArgs &a, int n, int &e) {
+    const int k = n - a.eq;
+    if (!a.shared) {
+        if (k < a.ek) { e = k; return true; }
+        e = k - a.ek;
+        return false;
+    }
+    const int ka = a.rk * a.h1 * a.d1;
+    if (k < ka) { e = k; return true; }            // A^K
+    if (k < 2 * ka) { e = k - ka; return false; }  // A^V
+    e = k - ka;                                    // B, after A^K in the key record
+    return true;
+}
+
 // One pair of projected columns (n, n+1) of token m: rotate it when it is a B^Q or B^K
 // pair (cs(j) = (cos, sin) of pair j of the token's position), then keep query
 // factors in fp32 and write key / value factors to the token's cache slot in bf16.
@@ -90,15 +109,12 @@ __device__ __forceinline__ void emit_pair(const AppendArgs &a, int m, int b, int
             a.qf[(size_t)n * a.M + m] = x0;
             a.qf[(size_t)(n + 1) * a.M + m] = x1;
         }
-    } else if (n < a.eq + a.ek) {                          // key factors
-        const int e = n - a.eq;
-        if (slot_ok) {
+    } else if (slot_ok) {                                  // key or value factors (a pair never
+        int e;                                             // straddles two records: even columns)
+        if (key_column(a, n, e)) {
             store_cache(a.kc, b, a.cap, a.ek, s, e, x0);
             store_cache(a.kc, b, a.cap, a.ek, s, e + 1, x1);
-        }
-    } else {                                               // value factors
-        const int e = n - a.eq - a.ek;
-        if (slot_ok) {
+        } else {
             store_cache(a.vc, b, a.cap, a.ev, s, e, x0);
             store_cache(a.vc, b, a.cap, a.ev, s, e + 1, x1);
         }
@@ -299,9 +315,10 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
                     for (int it = tp; it < max(0, ne - kb0) * (BM / kGroup); it += 128) {
                         const int lc = kb0 - nb + it / (BM / kGroup), gq = it % (BM / kGroup);
                         const int n = nb + lc;
-                        const bool is_k = n < a.eq + a.ek;
+                        int e;
+                        const bool is_k = key_column(a, n, e);
                         __nv_bfloat16 *plane = is_k ? a.kc : a.vc;
-                        const int E = is_k ? a.ek : a.ev, e = is_k ? n - a.eq : n - a.eq - a.ek;
+                        const int E = is_k ? a.ek : a.ev;
                         const float4 lo = reinterpret_cast<const float4 *>(mystg + (size_t)lc * BM + gq * kGroup)[0];
                         const float4 hi = reinterpret_cast<const float4 *>(mystg + (size_t)lc * BM + gq * kGroup)[1];
                         uint4 u;
@@ -651,6 +668,7 @@ cudaError_t launch_append(const Dims &d, int rq, int d_model, int batch, int n_t
     a.eq = rq * (d.h1 * d.d1 + d.h2 * d.d2);
     a.ek = d.ek;
     a.ev = d.ev;
+    a.shared = d.shared;
     a.N = a.eq + a.ek + a.ev;
     a.d2m1 = (d.d2 & (d.d2 - 1)) == 0 ? d.d2 - 1 : -1;
     a.K = d_model;

@@ -87,8 +87,9 @@ typedef struct {
                          * the value record is [A^V] only (E_V = r_v h1 d1), and
                          * kpa_decode rotates B for the score at each cached
                          * token's position.  Taken by kpa_cache_bytes_per_token,
-                         * kpa_append_factors and the decode calls;
-                         * kpa_append and kpa_prefill return KPA_ERR_UNSUPPORTED. */
+                         * kpa_append_factors, kpa_append (merged weight columns
+                         * [A^Q | B^Q | A^K | A^V | B]) and the decode calls;
+                         * kpa_prefill returns KPA_ERR_UNSUPPORTED.              */
 } kpa_config;
 
 /* Human-readable name of a status code (static storage). */

@@ -276,9 +276,16 @@ def prefill(shape, q, kf, vf, start_pos, *, q_pos=None, keys_rotated=False, sm_s
 # ------------------------------------------------------------------- append
 def split_columns(shape):
     """Column ranges of the merged projection output, in the order
-    [A^Q | B^Q | A^K | B^K | A^V | B^V] (a convention; see module docstring)."""
+    [A^Q | B^Q | A^K | B^K | A^V | B^V] (a convention; see module docstring).  With one
+    B shared by keys and values the order is [A^Q | B^Q | A^K | A^V | B] and the ranges
+    are returned as (A^Q, B^Q, A^K, B, A^V, B): the key and the value take the same B."""
     s = shape
     a, b = s.h1 * s.d1, s.h2 * s.d2
+    if getattr(s, "shared_b", 0):
+        widths = [s.r_q * a, s.r_q * b, s.r_k * a, s.r_k * a, s.r_k * b]
+        e = np.cumsum([0] + widths)
+        aq, bq, ak, av, bb = [(int(e[i]), int(e[i + 1])) for i in range(5)]
+        return [aq, bq, ak, bb, av, bb]
     widths = [s.r_q * a, s.r_q * b, s.r_k * a, s.r_k * b, s.r_v * a, s.r_v * b]
     edges = np.cumsum([0] + widths)
     return [(int(edges[i]), int(edges[i + 1])) for i in range(6)]
@@ -293,6 +300,9 @@ def append(shape, x, W, start_pos):
       k_rec_rot [B][n][E_K]    key records with B^K rotated at the token position
       v_rec     [B][n][E_V]    value records (never rotated)
       k_rec     [B][n][E_K]    unrotated key records
+
+    With a shared B (``shape.shared_b``) the key record is [A^K | B], v_rec is [A^V]
+    alone, and the cache keeps B unrotated: k_rec_rot is then k_rec.
     """
     s = shape
     x = _f64(x)
@@ -302,7 +312,11 @@ def append(shape, x, W, start_pos):
     cols = split_columns(s)
     q_rec = np.concatenate([fac[..., cols[0][0]:cols[0][1]], fac[..., cols[1][0]:cols[1][1]]], axis=-1)
     k_rec = np.concatenate([fac[..., cols[2][0]:cols[2][1]], fac[..., cols[3][0]:cols[3][1]]], axis=-1)
-    v_rec = np.concatenate([fac[..., cols[4][0]:cols[4][1]], fac[..., cols[5][0]:cols[5][1]]], axis=-1)
+    shared = bool(getattr(s, "shared_b", 0))
+    if shared:
+        v_rec = fac[..., cols[4][0]:cols[4][1]].copy()
+    else:
+        v_rec = np.concatenate([fac[..., cols[4][0]:cols[4][1]], fac[..., cols[5][0]:cols[5][1]]], axis=-1)
     q_rot = np.empty((B, n, h, dh))
     k_rot = np.empty_like(k_rec)
     start = np.asarray(start_pos, dtype=np.int64).reshape(B)
@@ -312,5 +326,6 @@ def append(shape, x, W, start_pos):
             Q = reconstruct(s.h1, s.h2, s.d1, s.d2, s.r_q, q_rec[b, t])
             for head in range(h):
                 q_rot[b, t, head] = rope_kpa(s.d1, s.d2, s.rope_base, pos, Q[head])
-            k_rot[b, t] = rotate_record(s.h1, s.h2, s.d1, s.d2, s.r_k, s.rope_base, pos, k_rec[b, t])
+            k_rot[b, t] = k_rec[b, t] if shared else \
+                rotate_record(s.h1, s.h2, s.d1, s.d2, s.r_k, s.rope_base, pos, k_rec[b, t])
     return q_rot, k_rot, v_rec, k_rec

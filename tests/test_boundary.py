@@ -80,14 +80,11 @@ def test_shared_b_needs_equal_ranks():
     assert e.value.status == kpa.KPA_ERR_INVALID_ARG
 
 
-def test_shared_b_projection_and_prefill_unsupported():
-    """A shared-B cache is written from given factors and decoded; the merged projection
-    and the prefill do not take it (checked before any device call)."""
+def test_shared_b_prefill_unsupported():
+    """A shared-B cache is written (from factors or the projection) and decoded; the
+    prefill does not take it (checked before any device call)."""
     s = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, shared_b=1)
     cfg = kpa.make_config(s, "bf16")
-    with pytest.raises(kpa.KpaError) as e:
-        kpa.kpa_append(cfg, 1, 16, A, A, A, 64, A, A, None, None, stream=0)
-    assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
     with pytest.raises(kpa.KpaError) as e:
         kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)
     assert e.value.status == kpa.KPA_ERR_UNSUPPORTED

@@ -102,3 +102,55 @@ def test_shared_b_fp16_overflow_is_reported():
     run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"])
     torch.cuda.synchronize()
     assert lib.kpa_read_device_error() == lib.KPA_ERR_DEVICE_CHECK
+
+
+def _close_bf16(got, want, what):
+    """Stored bf16 values: half a bf16 ulp plus the fp32 accumulation of the projection."""
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    bad = np.abs(got - want) > 2.0 ** -8 * np.abs(want) + 1e-5 * max(np.abs(want).max(), 1.0)
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} off, worst {np.abs(got - want).max():.3e}"
+
+
+@pytest.mark.parametrize("n_tok", [300, 5], ids=["gemm", "few_tokens"])
+def test_shared_b_append_then_decode(n_tok):
+    """kpa_append with a shared B (merged columns [A^Q | B^Q | A^K | A^V | B]): the key
+    records hold [A^K | B] unrotated, the value records A^V, q_out is rotated; a decode
+    over that cache then matches the oracle's shared-B decode of the stored records."""
+    from workloads import APPEND_PREFILL, append_inputs
+    s = dataclasses.replace(TPA_SHARED_DECODE.shape, r_q=4, d_model=256)
+    w = APPEND_PREFILL.replace(shape=s, batch=2, n_tok=n_tok, capacity=512, seed=68)
+    inp = append_inputs(w)
+    start = torch.tensor([0, 40], dtype=torch.int32)
+    lib = kpa()
+    cfg = lib.make_config(s, "bf16")
+    kc = torch.zeros(w.batch * w.capacity * s.e_k, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros(w.batch * w.capacity * s.e_v, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(lib.kpa_append_workspace_size(cfg, w.batch, n_tok), 256), dtype=torch.uint8,
+                     device="cuda")
+    q_out = torch.full((w.batch, n_tok, s.h, s.dh), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lib.kpa_append(cfg, w.batch, n_tok, inp["x"].cuda(), inp["W"].cuda(), start.cuda(), w.capacity, kc, vc,
+                   q_out, ws)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    q_rot, k_store, v_rec, _ = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start.numpy())
+    kn = natural(kc.cpu(), w.batch, w.capacity, s.e_k)
+    vn = natural(vc.cpu(), w.batch, w.capacity, s.e_v)
+    for b in range(w.batch):
+        st = int(start[b])
+        _close_bf16(to_f64(kn[b, st:st + n_tok]), k_store[b], f"key records b={b}")
+        _close_bf16(to_f64(vn[b, st:st + n_tok]), v_rec[b], f"value records b={b}")
+    _close_bf16(to_f64(q_out.cpu()), q_rot, "assembled query")
+    # decode of the newest token of each sequence over the slots the append wrote
+    L = start + n_tok
+    dw = TPA_SHARED_DECODE.replace(batch=w.batch, capacity=w.capacity)
+    q1 = q_out[:, -1].contiguous()
+    scale = 1.0 / np.sqrt(s.dh)
+    out = run_decode(lib, dw, cfg, kc, vc, q1.cpu(), L, None, sm_scale=scale)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    # q_out is already rotated at its position: the oracle rotates the keys at their slots and
+    # takes the query as given (position 0 = identity)
+    want = oracle.decode_shared_b(s, to_f64(q1.cpu()), to_f64(kn), to_f64(vn), L.numpy(),
+                                  q_pos=np.zeros(w.batch, dtype=np.int64), sm_scale=scale)
+    assert_bf16_close(out.cpu().numpy(), want, f"decode after shared-B append ({n_tok} tokens)")
