@@ -93,6 +93,8 @@ struct MmaDecodeCfg {
 using MmaTpaH16D64R2 = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2>;
 // TPA, h = 16, d_h = 64, R = 2 with one B shared by keys and values.
 using MmaTpaH16D64R2Shared = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2, true>;
+// KPA h = 4x4, d_h = 8x16, R = 2 with one B shared by keys and values.
+using MmaKpaH4x4D8x16R2Shared = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2, true>;
 // TPA, h = 32, d_h = 64, R_K = R_V = 1 (the FlashTPA decoding benchmark's shape).
 using MmaTpaH32D64R1 = MmaDecodeCfg<32, 1, 64, 1, 1, 1, 8, 2, 2>;
 // KPA h = 4x8, d_h = 8x16, R_K = R_V = 4.
@@ -108,7 +110,8 @@ using MmaKpaH4x4D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2>;
     X(2, MmaKpaH4x8D8x16R2)        \
     X(3, MmaKpaH4x4D8x16R2)        \
     X(4, MmaTpaH32D64R1)           \
-    X(5, MmaTpaH16D64R2Shared)
+    X(5, MmaTpaH16D64R2Shared)     \
+    X(6, MmaKpaH4x4D8x16R2Shared)
 
 // Index of the variant that covers these dims, or -1.
 inline int mma_decode_variant(const Dims &d) {

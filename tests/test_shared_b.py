@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from gpu_util import assert_bf16_close, fill_cache, kpa, natural, run_decode
-from workloads import TPA_SHARED_DECODE, decode_inputs, to_f64
+from workloads import TPA_SHARED_DECODE, Shape, decode_inputs, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -21,6 +21,8 @@ def _oracle(w, inp, sm_scale, q=None):
                                   to_f64(inp["vf"]), inp["seq_len"].numpy(), q_pos=inp["q_pos"].numpy(),
                                   sm_scale=sm_scale)
 
+
+KPA_SHARED = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, rope_base=10000.0, shared_b=1)
 
 # (workload, tokens per split, score sharpening): automatic plan over ragged lengths;
 # explicit 64- and 128-token splits with ragged tails; scores sharpened 40x; and a long
@@ -33,6 +35,11 @@ CASES = {
     "long_base5e5": (TPA_SHARED_DECODE.replace(
         shape=dataclasses.replace(TPA_SHARED_DECODE.shape, rope_base=500000.0), batch=2, capacity=8192,
         length=8192, seed=64), 0, 1.0),
+    # the Kronecker split h = 4x4, d_h = 8x16 with a shared B (rotation on the d2 pairs of B)
+    "kpa_ragged": (TPA_SHARED_DECODE.replace(shape=KPA_SHARED, batch=3, capacity=1024, length=0,
+                                             ragged=(1, 1024), factor_std=0.5, seed=69), 0, 1.0),
+    "kpa_split64_sharp": (TPA_SHARED_DECODE.replace(shape=KPA_SHARED, batch=2, capacity=512, length=0,
+                                                    ragged=(70, 512), factor_std=0.5, seed=70), 64, 20.0),
 }
 
 
@@ -112,13 +119,15 @@ def _close_bf16(got, want, what):
     assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} off, worst {np.abs(got - want).max():.3e}"
 
 
-@pytest.mark.parametrize("n_tok", [300, 5], ids=["gemm", "few_tokens"])
-def test_shared_b_append_then_decode(n_tok):
+@pytest.mark.parametrize("split,n_tok", [("tpa", 300), ("tpa", 5), ("kpa", 300)],
+                         ids=["tpa_gemm", "tpa_few_tokens", "kpa_gemm"])
+def test_shared_b_append_then_decode(split, n_tok):
     """kpa_append with a shared B (merged columns [A^Q | B^Q | A^K | A^V | B]): the key
     records hold [A^K | B] unrotated, the value records A^V, q_out is rotated; a decode
     over that cache then matches the oracle's shared-B decode of the stored records."""
     from workloads import APPEND_PREFILL, append_inputs
-    s = dataclasses.replace(TPA_SHARED_DECODE.shape, r_q=4, d_model=256)
+    base = TPA_SHARED_DECODE.shape if split == "tpa" else KPA_SHARED
+    s = dataclasses.replace(base, r_q=4, d_model=256)
     w = APPEND_PREFILL.replace(shape=s, batch=2, n_tok=n_tok, capacity=512, seed=68)
     inp = append_inputs(w)
     start = torch.tensor([0, 40], dtype=torch.int32)
@@ -143,7 +152,7 @@ def test_shared_b_append_then_decode(n_tok):
     _close_bf16(to_f64(q_out.cpu()), q_rot, "assembled query")
     # decode of the newest token of each sequence over the slots the append wrote
     L = start + n_tok
-    dw = TPA_SHARED_DECODE.replace(batch=w.batch, capacity=w.capacity)
+    dw = TPA_SHARED_DECODE.replace(shape=s, batch=w.batch, capacity=w.capacity)
     q1 = q_out[:, -1].contiguous()
     scale = 1.0 / np.sqrt(s.dh)
     out = run_decode(lib, dw, cfg, kc, vc, q1.cpu(), L, None, sm_scale=scale)
