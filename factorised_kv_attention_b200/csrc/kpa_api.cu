@@ -436,7 +436,7 @@ kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, cons
     if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
     if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
     const Dims d = dims_of(cfg);
-    if (d.shared || !prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
+    if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
     if (batch == 0 || n_tok == 0) return KPA_OK;
     if (batch > 65535 || d.h > 65535 || (int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
     if (!q || !start_pos || !kcache || !vcache || !out) return KPA_ERR_INVALID_ARG;
@@ -448,8 +448,8 @@ kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, cons
     if (s != KPA_OK) return s;
     const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
     cudaError_t e = launch_prefill(d, batch, n_tok, q, start_pos, kcache, vcache, capacity, qscale,
-                                   (float)(1.0 / (double)d.rv), out, err, current_hooks().wait_limit_ns,
-                                   (cudaStream_t)stream);
+                                   (float)(1.0 / (double)d.rv), out, rope_table(cfg), err,
+                                   current_hooks().wait_limit_ns, (cudaStream_t)stream);
     return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 

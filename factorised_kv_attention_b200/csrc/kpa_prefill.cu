@@ -47,6 +47,8 @@ struct PrefillArgs {
     int h1, h2;
     int *err;
     unsigned long long wait_limit_ns;
+    int shared;         // one B for keys and values: B unrotated in the key record, A^V alone in the value record
+    double theta[8];    // theta_m, m < d2/2 (shared B: the keys are rotated while K is rebuilt)
 };
 
 namespace {
@@ -363,12 +365,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 mbar_expect_tx(full, is_v ? C::V_ST : C::K_ST);
                 unsigned char *st = smem + (is_v ? C::OFF_VST + s * C::V_ST : C::OFF_KST + s * C::K_ST);
                 const CUtensorMap *map = is_v ? &tmv : &tmk;
-                const int R = is_v ? RV : RK, b0 = is_v ? va : ea;
+                // a shared B sits in the key record, after A^K, for the values too
+                const CUtensorMap *bmap = is_v && !a.shared ? &tmv : &tmk;
+                const int R = is_v ? RV : RK, b0 = is_v && !a.shared ? va : ea;
                 for (int r = 0; r < R; ++r) {
                     tma_load_2d(smem_u32(st + r * kBox), map, (r * a.h1 * D1 + i1 * D1) * kGroup, grp, full);
 #pragma unroll
                     for (int hb = 0; hb < 2; ++hb)
-                        tma_load_2d(smem_u32(st + (R + 2 * r + hb) * kBox), map,
+                        tma_load_2d(smem_u32(st + (R + 2 * r + hb) * kBox), bmap,
                                     (b0 + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, full);
                 }
                 issued[is_v ? 1 : 0][s] = t;
@@ -481,6 +485,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 float2 bf[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) bf[i] = unpack_bf16x2(bw[i]);
+                if (!is_v && a.shared) {
+                    // shared B is cached unrotated: rotate this lane's pairs m = c and 4 + c of its
+                    // token at the token's slot ("Kronecker Product Attention", Thm 2.4)
+                    const double pos = (double)(t * TK + g * kGroup + tok);
+                    float c0, s0, c1, s1;
+                    rope_cs_fast(pos, a.theta[lane & 3], c0, s0);
+                    rope_cs_fast(pos, a.theta[4 + (lane & 3)], c1, s1);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float cc = (i & 1) ? c1 : c0, ss = (i & 1) ? s1 : s0;
+                        bf[i] = make_float2(bf[i].x * cc - bf[i].y * ss, bf[i].x * ss + bf[i].y * cc);
+                    }
+                }
                 uint32_t w[8][2];
 #pragma unroll
                 for (int j1 = 0; j1 < 8; ++j1)
@@ -724,7 +741,8 @@ bool prefill_supported(const Dims &d) {
 
 cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const int32_t *start_pos,
                            const void *kc, const void *vc, int cap, float qscale, float out_scale,
-                           float *out, int *err, unsigned long long wait_limit_ns, cudaStream_t st) {
+                           float *out, const RopeTable &rope, int *err, unsigned long long wait_limit_ns,
+                           cudaStream_t st) {
     using C = PrefillKpaH4x4D8x16R2;
     if (!prefill_supported(d)) return cudaErrorInvalidValue;
     PrefillArgs a;
@@ -739,6 +757,8 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     a.h2 = d.h2;
     a.err = err;
     a.wait_limit_ns = wait_limit_ns;
+    a.shared = d.shared;
+    for (int m = 0; m < 8; ++m) a.theta[m] = m < C::D2 / 2 ? rope.theta[m] : 0.0;
     CUtensorMap tmq, tmk, tmv;
     const uint64_t groups = (uint64_t)batch * cap / kGroup;
     if (!make_q_map(&tmq, q, (uint64_t)batch * n_tok, (uint64_t)d.h * d.dh) ||

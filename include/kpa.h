@@ -88,8 +88,8 @@ typedef struct {
                          * kpa_decode rotates B for the score at each cached
                          * token's position.  Taken by kpa_cache_bytes_per_token,
                          * kpa_append_factors, kpa_append (merged weight columns
-                         * [A^Q | B^Q | A^K | A^V | B]) and the decode calls;
-                         * kpa_prefill returns KPA_ERR_UNSUPPORTED.              */
+                         * [A^Q | B^Q | A^K | A^V | B]), the decode calls and
+                         * kpa_prefill (which rotates B while rebuilding K).     */
 } kpa_config;
 
 /* Human-readable name of a status code (static storage). */

@@ -80,10 +80,10 @@ def test_shared_b_needs_equal_ranks():
     assert e.value.status == kpa.KPA_ERR_INVALID_ARG
 
 
-def test_shared_b_prefill_unsupported():
-    """A shared-B cache is written (from factors or the projection) and decoded; the
-    prefill does not take it (checked before any device call)."""
-    s = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, shared_b=1)
+def test_shared_b_prefill_shape_limit():
+    """The prefill kernel covers d1 = 8, d2 = 16, R = 2 whether B is shared or not; a
+    shared-B TPA shape is outside it (checked before any device call)."""
+    s = Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2, r_q=6, d_model=2048, shared_b=1)
     cfg = kpa.make_config(s, "bf16")
     with pytest.raises(kpa.KpaError) as e:
         kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)

@@ -163,3 +163,41 @@ def test_shared_b_append_then_decode(split, n_tok):
     want = oracle.decode_shared_b(s, to_f64(q1.cpu()), to_f64(kn), to_f64(vn), L.numpy(),
                                   q_pos=np.zeros(w.batch, dtype=np.int64), sm_scale=scale)
     assert_bf16_close(out.cpu().numpy(), want, f"decode after shared-B append ({n_tok} tokens)")
+
+
+def test_shared_b_append_then_prefill():
+    """kpa_append of a chunk into a shared-B cache (h = 4x4, d_h = 8x16), then the causal
+    prefill from q_out: the kernel rebuilds K with B rotated at each key's slot and V from
+    the same, unrotated B.  Sampled rows against the oracle on the stored records."""
+    from workloads import APPEND_PREFILL, append_inputs
+    s = dataclasses.replace(KPA_SHARED, r_q=6, d_model=256)
+    n_tok = 300
+    w = APPEND_PREFILL.replace(shape=s, batch=2, n_tok=n_tok, capacity=512, seed=71)
+    inp = append_inputs(w)
+    start = torch.tensor([0, 40], dtype=torch.int32)
+    lib = kpa()
+    cfg = lib.make_config(s, "bf16")
+    kc = torch.zeros(w.batch * w.capacity * s.e_k, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros(w.batch * w.capacity * s.e_v, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(lib.kpa_append_workspace_size(cfg, w.batch, n_tok), dtype=torch.uint8, device="cuda")
+    q_out = torch.empty(w.batch, n_tok, s.h, s.dh, dtype=torch.bfloat16, device="cuda")
+    lib.kpa_append(cfg, w.batch, n_tok, inp["x"].cuda(), inp["W"].cuda(), start.cuda(), w.capacity, kc, vc,
+                   q_out, ws)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = torch.full((w.batch, n_tok, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    lib.kpa_prefill(cfg, w.batch, n_tok, q_out, start.cuda(), kc, vc, w.capacity, scale, out)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    qo = to_f64(q_out.cpu())
+    got = out.cpu().numpy()
+    rng = np.random.default_rng(7)
+    rows = [(int(b), int(t)) for b, t in zip(rng.integers(0, w.batch, 10), rng.integers(0, n_tok, 10))]
+    rows += [(0, 0), (1, 0), (0, 127), (1, 128), (1, n_tok - 1)]
+    for b, t in rows:
+        L = int(start[b]) + t + 1
+        # q_out is rotated already (position 0 = identity); the oracle rotates the keys
+        want = oracle.decode_shared_b(s, qo[b, t][None], kn[b][None], vn[b][None], [L],
+                                      q_pos=[0], sm_scale=scale)
+        assert_bf16_close(got[b, t], want[0], f"shared-B prefill row ({b},{t})")
