@@ -183,6 +183,9 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
     }
     p->tokens_per_split = tps;
     p->n_split = max_len > 0 ? (int)(((int64_t)max_len + tps - 1) / tps) : 1;
+    // the last split runs to the end of its sequence: a remainder of at most a quarter of a
+    // split joins the split before it instead of becoming a split (and a partial) of its own
+    if (p->n_split > 1 && (int64_t)max_len - (int64_t)(p->n_split - 1) * tps <= tps / 4) --p->n_split;
     p->cluster = p->variant >= 0 && p->n_split <= kMaxClusterSplits &&
                  (p->n_split == 1 || cluster_capacity(p->variant, p->n_split) >= batch);
     // otherwise the last CTA of a sequence merges its splits when that read is small

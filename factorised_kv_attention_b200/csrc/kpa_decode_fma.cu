@@ -51,7 +51,7 @@ decode_fma_kernel(Dims d, const T *__restrict__ q, const int32_t *__restrict__ q
     }
     const int t0 = split * tps;
     if (t0 >= L) return;                          // empty split: the combine skips it
-    const int t1 = min(t0 + tps, L);
+    const int t1 = split == n_split - 1 ? L : min(t0 + tps, L);   // the last split runs to the end
 
     float *qr = reinterpret_cast<float *>(smem);  // [h][dh] rotated, scaled query
     float *pr = qr + h * dh;                      // [h][tile] scores, then weights
@@ -257,7 +257,7 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
     const int head = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     int L = seq_len[b];
     L = L < 0 ? 0 : (L > max_len ? max_len : L);
-    const int ns = (L + tps - 1) / tps;
+    const int ns = min(n_split, (L + tps - 1) / tps);
     float *dst = out + ((size_t)b * d.h + head) * d.dh;
     if (ns == 0 || ns > kCombineMaxSplits) {
         for (int f = tid; f < d.dh; f += kCombineThreads) dst[f] = 0.f;

@@ -294,7 +294,8 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             raise_error(a.err, kErrTimeout);               // its speculative copy lands first
         return;
     }
-    const int t1 = max(t0, min(t0 + a.tps, L));
+    // the last split runs to the end of the sequence (it may hold up to 5/4 of a split)
+    const int t1 = max(t0, split == a.n_split - 1 ? L : min(t0 + a.tps, L));
     const int n_tiles = (t1 - t0 + TT - 1) / TT;
     __syncthreads();                                        // barriers initialised
 
@@ -850,7 +851,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
 
     // the last CTA of this sequence merges every split (log-sum-exp) into out[b]
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    const int n_b = (L + a.tps - 1) / a.tps;
+    const int n_b = min(a.n_split, (L + a.tps - 1) / a.tps);   // splits holding tokens of b
     if (tid == 0) {
         // acq_rel at gpu scope: releases the CTA's partial (ordered before this thread
         // by the barrier above) and, for the last arrival, acquires every other CTA's

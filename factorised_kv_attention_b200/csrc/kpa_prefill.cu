@@ -47,7 +47,6 @@ struct PrefillArgs {
     int h1, h2;
     int *err;
     unsigned long long wait_limit_ns;
-    int shared;         // one B for keys and values: B unrotated in the key record, A^V alone in the value record
     double theta[8];    // theta_m, m < d2/2 (shared B: the keys are rotated while K is rebuilt)
 };
 
@@ -265,7 +264,7 @@ struct TilePlan {
     __device__ int last_half(int t) const { return active(1, t) ? 1 : 0; }
 };
 
-template <class C>
+template <class C, bool SHARED>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, PrefillArgs a) {
@@ -366,8 +365,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 unsigned char *st = smem + (is_v ? C::OFF_VST + s * C::V_ST : C::OFF_KST + s * C::K_ST);
                 const CUtensorMap *map = is_v ? &tmv : &tmk;
                 // a shared B sits in the key record, after A^K, for the values too
-                const CUtensorMap *bmap = is_v && !a.shared ? &tmv : &tmk;
-                const int R = is_v ? RV : RK, b0 = is_v && !a.shared ? va : ea;
+                const CUtensorMap *bmap = is_v && !SHARED ? &tmv : &tmk;
+                const int R = is_v ? RV : RK, b0 = is_v && !SHARED ? va : ea;
                 for (int r = 0; r < R; ++r) {
                     tma_load_2d(smem_u32(st + r * kBox), map, (r * a.h1 * D1 + i1 * D1) * kGroup, grp, full);
 #pragma unroll
@@ -485,7 +484,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 float2 bf[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) bf[i] = unpack_bf16x2(bw[i]);
-                if (!is_v && a.shared) {
+                if (SHARED && !is_v) {
                     // shared B is cached unrotated: rotate this lane's pairs m = c and 4 + c of its
                     // token at the token's slot ("Kronecker Product Attention", Thm 2.4)
                     const double pos = (double)(t * TK + g * kGroup + tok);
@@ -757,17 +756,20 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     a.h2 = d.h2;
     a.err = err;
     a.wait_limit_ns = wait_limit_ns;
-    a.shared = d.shared;
     for (int m = 0; m < 8; ++m) a.theta[m] = m < C::D2 / 2 ? rope.theta[m] : 0.0;
     CUtensorMap tmq, tmk, tmv;
     const uint64_t groups = (uint64_t)batch * cap / kGroup;
     if (!make_q_map(&tmq, q, (uint64_t)batch * n_tok, (uint64_t)d.h * d.dh) ||
         !make_factor_map(&tmk, kc, groups, (uint64_t)d.ek) || !make_factor_map(&tmv, vc, groups, (uint64_t)d.ev))
         return cudaErrorInvalidValue;
-    cudaError_t e = ensure_dynamic_smem<prefill_kernel<C>>(C::SMEM);
+    cudaError_t e = d.shared ? ensure_dynamic_smem<prefill_kernel<C, true>>(C::SMEM)
+                             : ensure_dynamic_smem<prefill_kernel<C, false>>(C::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((n_tok + 2 * HQ - 1) / (2 * HQ)), (unsigned)d.h, (unsigned)batch);
-    prefill_kernel<C><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
+    if (d.shared)
+        prefill_kernel<C, true><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
+    else
+        prefill_kernel<C, false><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
     return cudaGetLastError();
 }
 

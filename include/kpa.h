@@ -126,7 +126,9 @@ kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32
                                      int32_t tokens_per_split, size_t *bytes);
 
 /* How kpa_decode will split the work for these sizes (host only): the splits
- * per sequence, the tokens in each split, and the kernel launches one call
+ * per sequence, the tokens in each split (the last split of a sequence runs to
+ * its end: a remainder of at most a quarter of a split is not a split of its
+ * own, so the last may hold up to 5/4 of one), and the kernel launches one call
  * enqueues (1 when the splits of a sequence are merged inside the decode
  * kernel, 2 when a separate combine kernel follows).  Any output pointer may be
  * NULL.  Same argument rules as kpa_decode_workspace_size. */
