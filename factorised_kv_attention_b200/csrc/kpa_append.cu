@@ -121,6 +121,19 @@ __device__ __forceinline__ void emit_pair(const AppendArgs &a, int m, int b, int
     }
 }
 
+// Tile t of the persistent schedule -> (128-row block, first column, width).  The
+// tiles every CTA gets the same number of come first; the remaining tiles are split
+// into column halves of 128 and BN - 128 (both valid MMA widths), so that no CTA ends
+// a whole tile after the others.
+struct TileCols {
+    int tm, n0, nw;
+};
+__device__ __forceinline__ TileCols tile_cols(int t, int n_tn, int BN, int n_even, bool split) {
+    if (!split || t < n_even) return {t / n_tn, (t % n_tn) * BN, BN};
+    const int u = t - n_even, f = n_even + (u >> 1), h = u & 1;
+    return {f / n_tn, (f % n_tn) * BN + h * 128, h ? BN - 128 : 128};
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                    AppendArgs a, RopeTable rope) {
@@ -140,7 +153,10 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * S, accf0 = full0 + 16 * S;
     const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
-    const int n_tn = (a.N + BN - 1) / BN, n_tiles = n_tn * ((a.M + BM - 1) / BM);
+    const int n_tn = (a.N + BN - 1) / BN, whole = n_tn * ((a.M + BM - 1) / BM);
+    const int n_even = (whole / (int)gridDim.x) * (int)gridDim.x;
+    const bool split = BN > 128 && (BN - 128) % 16 == 0 && whole > n_even && 2 * (whole - n_even) <= (int)gridDim.x;
+    const int n_tiles = split ? n_even + 2 * (whole - n_even) : whole;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -190,7 +206,7 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
             int g = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-                const int tm = tile / n_tn, tn = tile % n_tn;
+                const TileCols tc = tile_cols(tile, n_tn, BN, n_even, split);
                 for (int kb = 0; kb < a.n_kblocks; ++kb, ++g) {
                     const int s = g % S;
                     if (g >= S && !wait(empty0 + 8 * s, ((g / S) - 1) & 1)) {
@@ -198,8 +214,8 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
                         break;
                     }
                     mbar_expect_tx(full0 + 8 * s, a_bytes + b_bytes);
-                    tma_load_2d(smem_u32(a_st + (size_t)s * a_bytes), &tmx, kb * BK, tm * BM, full0 + 8 * s);
-                    tma_load_2d(smem_u32(b_st + (size_t)s * b_bytes), &tmw, kb * BK, tn * BN, full0 + 8 * s);
+                    tma_load_2d(smem_u32(a_st + (size_t)s * a_bytes), &tmx, kb * BK, tc.tm * BM, full0 + 8 * s);
+                    tma_load_2d(smem_u32(b_st + (size_t)s * b_bytes), &tmw, kb * BK, tc.n0, full0 + 8 * s);
                 }
             }
             // every copy issued lands before the CTA exits (normally already consumed)
@@ -209,11 +225,11 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
         // ---- MMA issuer: accumulator i&1 of this CTA's i-th tile, once the epilogue has
         // drained it (tile i-2)
         if (lane == 0) {
-            const uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
             int g = 0, i = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++i) {
                 const int buf = i & 1;
+                const uint32_t idesc = umma_idesc_bf16_f32(BM, tile_cols(tile, n_tn, BN, n_even, split).nw);
                 if (i >= 2 && !wait(acce0 + 8 * buf, ((i >> 1) - 1) & 1)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < a.n_kblocks; ++kb, ++g) {
@@ -241,14 +257,15 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
         // half of each tile's 16-column chunks, warps 6..9 the rest
         const int quarter = warp & 3, part = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
-        const int nch = BN / 16, ch_lo = part ? (nch + 1) / 2 : 0, ch_hi = part ? nch : (nch + 1) / 2;
         const int half = a.d2 / 2;
         float2 *cs = cs_all + (size_t)row * half;
         float *mystg = stg + part * kStageCols * BM;
         const int tp = (warp - 2) * 32 + lane - part * 128;           // 0..127 inside the part
         int i = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
-            const int tm = tile / n_tn, tn = tile % n_tn, buf = i & 1;
+            const TileCols tc = tile_cols(tile, n_tn, BN, n_even, split);
+            const int tm = tc.tm, buf = i & 1;
+            const int nch = tc.nw / 16, ch_lo = part ? (nch + 1) / 2 : 0, ch_hi = part ? nch : (nch + 1) / 2;
             const uint32_t acc = tmem + buf * 256 + ((uint32_t)(quarter * 32) << 16);
             asm volatile("bar.sync 2, 256;" ::: "memory");           // the previous tile is done with cs
             const int m = tm * BM + row;
@@ -287,7 +304,7 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
                     for (int cc = 0; cc < cn; ++cc) {
                         float v[16];
                         tmem_ld16(acc + (c0 + cc) * 16, v);             // warp-collective
-                        const int n0 = tn * BN + (c0 + cc) * 16;
+                        const int n0 = tc.n0 + (c0 + cc) * 16;
 #pragma unroll
                         for (int j = 0; j < 16; j += 2) {
                             if (n0 + j >= a.N) break;
@@ -303,7 +320,7 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
                         if (lane == 0) mbar_arrive(acce0 + 8 * buf);
                     }
                     asm volatile("bar.sync %0, 128;" ::"r"(3 + part) : "memory");   // the part's chunk is staged
-                    const int nb = tn * BN + c0 * 16, ne = min(nb + cn * 16, a.N);
+                    const int nb = tc.n0 + c0 * 16, ne = min(nb + cn * 16, a.N);
                     const int qe = min(ne, a.eq);
                     if (a.qf)
                         for (int it = tp; it < max(0, qe - nb) * (BM / 4); it += 128) {
@@ -337,7 +354,7 @@ append_gemm_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constan
                     float v[16];
                     tmem_ld16(acc + ch * 16, v);                        // warp-collective
                     if (!live) continue;
-                    const int n0 = tn * BN + ch * 16;
+                    const int n0 = tc.n0 + ch * 16;
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {
                         if (n0 + j >= a.N) break;
