@@ -69,6 +69,8 @@ _SIGS = {
     "kpa_prefill_workspace_size": ([_cfgp, _i32, _i32, _szp], ctypes.c_int),
     "kpa_prefill": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _sz, _vp],
                     ctypes.c_int),
+    "kpa_prefill_qf": ([_cfgp, _i32, _i32, _vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp,
+                        _i32, _f32, _vp, _vp, _sz, _vp], ctypes.c_int),
     "kpa_append_workspace_size": ([_cfgp, _i32, _i32, _szp], ctypes.c_int),
     "kpa_append": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp],
                    ctypes.c_int),
@@ -181,6 +183,15 @@ def kpa_prefill_workspace_size(cfg, batch, n_tok) -> int:
     _check(_lib.kpa_prefill_workspace_size(ctypes.byref(cfg), batch, n_tok, ctypes.byref(n)),
            "kpa_prefill_workspace_size")
     return n.value
+
+
+def kpa_prefill_qf(cfg, batch, n_tok, q_factors, qf_stride, qf_seq_stride, qf_tok_stride, start_pos, kcache,
+                   vcache, capacity, sm_scale, out, workspace=None, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.kpa_prefill_qf(ctypes.byref(cfg), batch, n_tok, _addr(q_factors), qf_stride, qf_seq_stride,
+                               qf_tok_stride, _addr(start_pos), _addr(kcache), _addr(vcache), capacity, sm_scale,
+                               _addr(out), _addr(workspace), ws_bytes, _stream(stream)), "kpa_prefill_qf")
 
 
 def kpa_prefill(cfg, batch, n_tok, q, start_pos, kcache, vcache, capacity, sm_scale, out,

@@ -426,34 +426,60 @@ kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int3
     return KPA_OK;
 }
 
+// The prefill with a dense bf16 query (q) or with query factors (qf.ptr).
+static kpa_status prefill_impl(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *q,
+                               const PrefillQf &qf, const int32_t *start_pos, const void *kcache,
+                               const void *vcache, int32_t capacity, float sm_scale, float *out,
+                               kpa_stream stream) {
+    kpa_status s = check_cfg(cfg, qf.ptr != nullptr, false);
+    if (s != KPA_OK) return s;
+    if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
+    if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
+    if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
+    if (qf.ptr && (qf.stride <= 0 || qf.seq_stride < 0 || qf.tok_stride < 0)) return KPA_ERR_INVALID_ARG;
+    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    const Dims d = dims_of(cfg);
+    if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
+    if (qf.ptr && cfg->r_q > kPrefillQfMaxRq) return KPA_ERR_UNSUPPORTED;
+    if (batch == 0 || n_tok == 0) return KPA_OK;
+    if (batch > 65535 || d.h > 65535 || (int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
+    if ((!q && !qf.ptr) || !start_pos || !kcache || !vcache || !out) return KPA_ERR_INVALID_ARG;
+    if ((q && !aligned16(q)) || (qf.ptr && (reinterpret_cast<uintptr_t>(qf.ptr) & 3)) || !aligned16(kcache) ||
+        !aligned16(vcache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(start_pos) & 3))
+        return KPA_ERR_INVALID_ARG;
+    int *err = nullptr;
+    s = device_state(&err, nullptr);
+    if (s != KPA_OK) return s;
+    const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
+    cudaError_t e = launch_prefill(d, batch, n_tok, q, qf, start_pos, kcache, vcache, capacity, qscale,
+                                   (float)(1.0 / (double)d.rv), out, rope_table(cfg), err,
+                                   current_hooks().wait_limit_ns, (cudaStream_t)stream);
+    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+}
+
 kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *q,
                        const int32_t *start_pos, const void *kcache, const void *vcache,
                        int32_t capacity, float sm_scale, float *out, void *workspace,
                        size_t ws_bytes, kpa_stream stream) {
     (void)workspace;
     (void)ws_bytes;
-    kpa_status s = check_cfg(cfg, false, false);
-    if (s != KPA_OK) return s;
-    if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
-    if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
-    if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
-    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
-    const Dims d = dims_of(cfg);
-    if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
-    if (batch == 0 || n_tok == 0) return KPA_OK;
-    if (batch > 65535 || d.h > 65535 || (int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
-    if (!q || !start_pos || !kcache || !vcache || !out) return KPA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(start_pos) & 3))
-        return KPA_ERR_INVALID_ARG;
-    int *err = nullptr;
-    s = device_state(&err, nullptr);
-    if (s != KPA_OK) return s;
-    const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
-    cudaError_t e = launch_prefill(d, batch, n_tok, q, start_pos, kcache, vcache, capacity, qscale,
-                                   (float)(1.0 / (double)d.rv), out, rope_table(cfg), err,
-                                   current_hooks().wait_limit_ns, (cudaStream_t)stream);
-    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+    const PrefillQf none = {nullptr, 0, 0, 0, 0};
+    if (!q && batch > 0 && n_tok > 0 && check_cfg(cfg, false, false) == KPA_OK) return KPA_ERR_INVALID_ARG;
+    return prefill_impl(cfg, batch, n_tok, q, none, start_pos, kcache, vcache, capacity, sm_scale, out, stream);
+}
+
+kpa_status kpa_prefill_qf(const kpa_config *cfg, int32_t batch, int32_t n_tok, const float *q_factors,
+                          int64_t qf_stride, int64_t qf_seq_stride, int64_t qf_tok_stride,
+                          const int32_t *start_pos, const void *kcache, const void *vcache,
+                          int32_t capacity, float sm_scale, float *out, void *workspace, size_t ws_bytes,
+                          kpa_stream stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    if (!cfg) return KPA_ERR_INVALID_ARG;
+    if (!q_factors && batch > 0 && n_tok > 0) return KPA_ERR_INVALID_ARG;
+    const PrefillQf qf = {q_factors, qf_stride, qf_seq_stride, qf_tok_stride, cfg->r_q};
+    return prefill_impl(cfg, batch, n_tok, nullptr, qf, start_pos, kcache, vcache, capacity, sm_scale, out,
+                        stream);
 }
 
 kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,

@@ -136,10 +136,17 @@ cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_l
 size_t decode_fma_smem_bytes(const Dims &d, kpa_dtype dt, int tile);
 
 bool prefill_supported(const Dims &d);
-cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const int32_t *start_pos,
-                           const void *kc, const void *vc, int cap, float qscale, float out_scale,
-                           float *out, const RopeTable &rope, int *err, unsigned long long wait_limit_ns,
-                           cudaStream_t st);
+// Query factors for a prefill (ptr null: a dense bf16 query instead).
+struct PrefillQf {
+    const float *ptr;
+    long long stride, seq_stride, tok_stride;   // element, sequence and token strides (floats)
+    int rq;
+};
+constexpr int kPrefillQfMaxRq = 6;
+cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const PrefillQf &qf,
+                           const int32_t *start_pos, const void *kc, const void *vc, int cap, float qscale,
+                           float out_scale, float *out, const RopeTable &rope, int *err,
+                           unsigned long long wait_limit_ns, cudaStream_t st);
 
 size_t append_smem_bytes(int BN, int stages, int d2);
 int append_tile_n(int N);

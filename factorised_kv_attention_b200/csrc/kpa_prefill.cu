@@ -30,6 +30,7 @@
 // P stays in [0, 256].  A value outside the fp16 range becomes inf and makes the row's
 // output non-finite; such a row is reported as KPA_ERR_DEVICE_CHECK.
 #include <cudaTypedefs.h>
+#include <cstring>
 
 #include <cuda_fp16.h>
 
@@ -48,7 +49,15 @@ struct PrefillArgs {
     int *err;
     unsigned long long wait_limit_ns;
     double theta[8];    // theta_m, m < d2/2 (shared B: the keys are rotated while K is rebuilt)
+    // query factors instead of a dense query (null: q by TMA): element e of token t of
+    // sequence b at qf[e * qf_stride + b * qf_seq_stride + t * qf_tok_stride], B^Q rotated
+    const float *qf;
+    long long qf_stride, qf_seq_stride, qf_tok_stride;
+    int rq;
+    float qf_scale;     // qscale / R_Q
 };
+
+constexpr int kPrefillMaxRq = 6;    // query rank a prefill from query factors takes
 
 namespace {
 
@@ -264,7 +273,7 @@ struct TilePlan {
     __device__ int last_half(int t) const { return active(1, t) ? 1 : 0; }
 };
 
-template <class C, bool SHARED>
+template <class C, bool SHARED, bool QF>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv, PrefillArgs a) {
@@ -349,7 +358,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     if (warp == kProducerWarp) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0 && tp.n_kt > 0) {
-            tma_prefetch_desc(&tmq);
+            if (!QF) tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
             const int grp0 = (int)((int64_t)b * a.cap / kGroup);
@@ -380,21 +389,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             // the first key tile's factors go out ahead of Q: its rebuild is the first step
             bool ok = issue_factors(0, false);
             const int nh = (tp.act[0] ? 1 : 0) + (tp.act[1] ? 1 : 0);
-            mbar_expect_tx(bar(B_Q), (uint32_t)nh * C::Q_HALF);
+            if (!QF) {                           // query factors: the softmax warps assemble Q
+                mbar_expect_tx(bar(B_Q), (uint32_t)nh * C::Q_HALF);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                if (tp.act[hh])
+                for (int hh = 0; hh < 2; ++hh)
+                    if (tp.act[hh])
 #pragma unroll
-                    for (int cb = 0; cb < DH / 64; ++cb)
-                        tma_load_2d(smem_u32(smem + C::OFF_Q + hh * C::Q_HALF + cb * HQ * 128), &tmq,
-                                    head * DH + cb * 64, b * a.n_tok + q0 + hh * HQ, bar(B_Q));
+                        for (int cb = 0; cb < DH / 64; ++cb)
+                            tma_load_2d(smem_u32(smem + C::OFF_Q + hh * C::Q_HALF + cb * HQ * 128), &tmq,
+                                        head * DH + cb * 64, b * a.n_tok + q0 + hh * HQ, bar(B_Q));
+            }
             if (ok) ok = issue_factors(0, true);
             for (int t = 1; t < tp.n_kt && ok; ++t) {
                 ok = issue_factors(t, false);
                 if (ok) ok = issue_factors(t, true);
             }
             // every copy this thread started lands before the CTA can exit
-            (void)mbar_wait(bar(B_Q), 0, limit);
+            if (!QF) (void)mbar_wait(bar(B_Q), 0, limit);
 #pragma unroll
             for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
@@ -555,8 +566,56 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (tp.act[hh]) {
             const int qrow = q0 + hh * HQ + row;
             const int pos = start + qrow;
+            bool ok = true;
+            if constexpr (QF) {
+                // Q_h from the query factors ("Kronecker Product Attention", eq 2):
+                // q[j1 d2 + j2] = (1/R_Q) sum_r A^Q_r[i1][j1] B^Q_r[i2][j2], scaled and rounded
+                // once to fp16, written as 8-byte pieces into the 128-byte-swizzled K-major
+                // tile the MMA reads.  Four passes over quarters of d2 keep B^Q in registers.
+                const int t = q0 + hh * HQ + row;
+                const bool live = t < a.n_tok;
+                const float *src = a.qf + (long long)b * a.qf_seq_stride + (long long)t * a.qf_tok_stride;
+                const int qa = a.rq * a.h1 * D1;                    // first B^Q element of the record
+                unsigned char *qh = smem + C::OFF_Q + hh * C::Q_HALF;
+                // A^Q[r][i1][0..D1) of the row: every load in flight at once, then kept
+                float aq[kPrefillMaxRq][D1];
+#pragma unroll
+                for (int r = 0; r < kPrefillMaxRq; ++r)
+#pragma unroll
+                    for (int j1 = 0; j1 < D1; ++j1)
+                        aq[r][j1] = live && r < a.rq
+                                        ? __ldg(src + (long long)((r * a.h1 + i1) * D1 + j1) * a.qf_stride)
+                                        : 0.f;
+#pragma unroll 1
+                for (int hb = 0; hb < C::D2 / 4; ++hb) {            // four features of d2 per pass
+                    float bq[kPrefillMaxRq][4];
+#pragma unroll
+                    for (int r = 0; r < kPrefillMaxRq; ++r)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            bq[r][u] = live && r < a.rq
+                                           ? __ldg(src + (long long)(qa + (r * a.h2 + i2) * C::D2 + hb * 4 + u) *
+                                                             a.qf_stride)
+                                           : 0.f;
+#pragma unroll
+                    for (int j1 = 0; j1 < D1; ++j1) {
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int r = 0; r < kPrefillMaxRq; ++r)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) acc[u] += aq[r][j1] * bq[r][u];
+                        uint2 pk;
+                        pk.x = pack_half2(acc[0] * a.qf_scale, acc[1] * a.qf_scale);
+                        pk.y = pack_half2(acc[2] * a.qf_scale, acc[3] * a.qf_scale);
+                        const int f0 = j1 * C::D2 + hb * 4;          // first feature of the piece
+                        *reinterpret_cast<uint2 *>(qh + (f0 >> 6) * HQ * 128 + sw128_chunk(row, (f0 & 63) >> 3) +
+                                                   (f0 & 4) * 2) = pk;
+                    }
+                }
+                fence_async_smem();
+            } else {
             // Q_h: bf16 -> fp16 x qscale in place, once its copy has landed
-            bool ok = wait(B_Q, 0);
+            ok = wait(B_Q, 0);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 uint4 *q4 = reinterpret_cast<uint4 *>(smem + C::OFF_Q + hh * C::Q_HALF);
@@ -572,6 +631,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     q4[i] = u;
                 }
                 fence_async_smem();
+            }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_QREADY + hh));
@@ -738,10 +798,10 @@ bool prefill_supported(const Dims &d) {
            d.rk == PrefillKpaH4x4D8x16R2::RK && d.rv == PrefillKpaH4x4D8x16R2::RV;
 }
 
-cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const int32_t *start_pos,
-                           const void *kc, const void *vc, int cap, float qscale, float out_scale,
-                           float *out, const RopeTable &rope, int *err, unsigned long long wait_limit_ns,
-                           cudaStream_t st) {
+cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const PrefillQf &qf,
+                           const int32_t *start_pos, const void *kc, const void *vc, int cap, float qscale,
+                           float out_scale, float *out, const RopeTable &rope, int *err,
+                           unsigned long long wait_limit_ns, cudaStream_t st) {
     using C = PrefillKpaH4x4D8x16R2;
     if (!prefill_supported(d)) return cudaErrorInvalidValue;
     PrefillArgs a;
@@ -757,19 +817,34 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     a.err = err;
     a.wait_limit_ns = wait_limit_ns;
     for (int m = 0; m < 8; ++m) a.theta[m] = m < C::D2 / 2 ? rope.theta[m] : 0.0;
+    a.qf = qf.ptr;
+    a.qf_stride = qf.stride;
+    a.qf_seq_stride = qf.seq_stride;
+    a.qf_tok_stride = qf.tok_stride;
+    a.rq = qf.rq;
+    a.qf_scale = qf.rq > 0 ? qscale / (float)qf.rq : 0.f;
+    if (a.qf && (a.rq < 1 || a.rq > kPrefillMaxRq)) return cudaErrorInvalidValue;
     CUtensorMap tmq, tmk, tmv;
+    memset(&tmq, 0, sizeof(tmq));                   // unused (and never prefetched) with query factors
     const uint64_t groups = (uint64_t)batch * cap / kGroup;
-    if (!make_q_map(&tmq, q, (uint64_t)batch * n_tok, (uint64_t)d.h * d.dh) ||
+    if ((!a.qf && !make_q_map(&tmq, q, (uint64_t)batch * n_tok, (uint64_t)d.h * d.dh)) ||
         !make_factor_map(&tmk, kc, groups, (uint64_t)d.ek) || !make_factor_map(&tmv, vc, groups, (uint64_t)d.ev))
         return cudaErrorInvalidValue;
-    cudaError_t e = d.shared ? ensure_dynamic_smem<prefill_kernel<C, true>>(C::SMEM)
-                             : ensure_dynamic_smem<prefill_kernel<C, false>>(C::SMEM);
+    const bool use_qf = a.qf != nullptr;
+    cudaError_t e = d.shared ? (use_qf ? ensure_dynamic_smem<prefill_kernel<C, true, true>>(C::SMEM)
+                                       : ensure_dynamic_smem<prefill_kernel<C, true, false>>(C::SMEM))
+                             : (use_qf ? ensure_dynamic_smem<prefill_kernel<C, false, true>>(C::SMEM)
+                                       : ensure_dynamic_smem<prefill_kernel<C, false, false>>(C::SMEM));
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((n_tok + 2 * HQ - 1) / (2 * HQ)), (unsigned)d.h, (unsigned)batch);
-    if (d.shared)
-        prefill_kernel<C, true><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
+    if (d.shared && use_qf)
+        prefill_kernel<C, true, true><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
+    else if (d.shared)
+        prefill_kernel<C, true, false><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
+    else if (use_qf)
+        prefill_kernel<C, false, true><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
     else
-        prefill_kernel<C, false><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
+        prefill_kernel<C, false, false><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
     return cudaGetLastError();
 }
 

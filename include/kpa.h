@@ -206,6 +206,24 @@ kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, cons
                        int32_t capacity, float sm_scale, float *out, void *workspace,
                        size_t ws_bytes, kpa_stream stream);
 
+/* kpa_prefill with the queries given as factors ("Kronecker Product Attention", eq 2
+ * for Q): the kernel forms each query row (1/R_Q) sum_r A^Q_r (x) B^Q_r in fp32 and
+ * rounds it once to fp16 with the score scale folded in, so no dense query is written
+ * or read.  The factors must already be rotated at the rows' positions (as kpa_append
+ * leaves them in its workspace).
+ *   q_factors  float32; element e (0 <= e < E_Q = R_Q (h1 d1 + h2 d2)) of the record
+ *              [A^Q_0 .. | B^Q_0 ..] of row t of sequence b at
+ *              q_factors[e * qf_stride + b * qf_seq_stride + t * qf_tok_stride]
+ *              (the append's workspace: qf_stride = batch * n_tok, qf_seq_stride =
+ *              n_tok, qf_tok_stride = 1); 4-byte aligned.
+ * Requires 0 < r_q <= 6 (else KPA_ERR_UNSUPPORTED; r_q <= 0 is KPA_ERR_INVALID_ARG).
+ * Everything else as kpa_prefill. */
+kpa_status kpa_prefill_qf(const kpa_config *cfg, int32_t batch, int32_t n_tok, const float *q_factors,
+                          int64_t qf_stride, int64_t qf_seq_stride, int64_t qf_tok_stride,
+                          const int32_t *start_pos, const void *kcache, const void *vcache,
+                          int32_t capacity, float sm_scale, float *out, void *workspace, size_t ws_bytes,
+                          kpa_stream stream);
+
 /* Append: merged factor projection, factor RoPE and cache write ("Kronecker
  * Product Attention", eq 5 with the ranks merged; Theorem 2.4; section 2.5).
  *   x  [batch][n_tok][d_model]  bf16 hidden states

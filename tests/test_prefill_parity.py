@@ -147,3 +147,38 @@ def test_append_prefill_decode_chain_full_config():
         assert_bf16_close(got[b, t], want[0], f"prefill row ({b},{t})")
     want = oracle.decode(s, to_f64(q1[:, 0].cpu()), kn, vn, seq.numpy(), keys_rotated=True, sm_scale=scale)
     assert_bf16_close(dec.cpu().numpy(), want, "decode step at 2048")
+
+
+@pytest.mark.parametrize("n_tok,starts", [(300, [0, 40]), (2048, [0, 0])], ids=["ragged", "chunk2048"])
+def test_prefill_from_query_factors(n_tok, starts):
+    """kpa_append without q_out leaves the rotated query factors in its workspace;
+    kpa_prefill_qf assembles each query row from them in the kernel (fp32, one fp16
+    rounding).  Sampled rows against the oracle with the float64 projection's query."""
+    lib = kpa()
+    s = APPEND_PREFILL.shape if n_tok == 2048 else Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6,
+                                                          d_model=256, rope_base=10000.0)
+    w = APPEND_PREFILL.replace(shape=s, batch=len(starts), n_tok=n_tok, capacity=max(512, n_tok + 64), seed=73)
+    inp = append_inputs(w)
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, w.batch, w.capacity, "bf16")
+    start = torch.tensor(starts, dtype=torch.int32)
+    ws = torch.zeros(lib.kpa_append_workspace_size(cfg, w.batch, n_tok), dtype=torch.uint8, device="cuda")
+    lib.kpa_append(cfg, w.batch, n_tok, inp["x"].cuda(), inp["W"].cuda(), start.cuda(), w.capacity, kc, vc, None, ws)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = torch.full((w.batch, n_tok, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    lib.kpa_prefill_qf(cfg, w.batch, n_tok, ws.view(torch.float32), w.batch * n_tok, n_tok, 1, start.cuda(), kc, vc,
+                       w.capacity, scale, out)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    q_rot, _, _, _ = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start.numpy())
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    got = out.cpu().numpy()
+    rng = np.random.default_rng(9)
+    rows = [(int(b), int(t)) for b, t in zip(rng.integers(0, w.batch, 10), rng.integers(0, n_tok, 10))]
+    rows += [(0, 0), (w.batch - 1, 127), (w.batch - 1, 128), (w.batch - 1, n_tok - 1)]
+    for b, t in rows:
+        L = int(start[b]) + t + 1
+        want = oracle.decode(s, q_rot[b, t][None], kn[b][None], vn[b][None], [L], keys_rotated=True,
+                             sm_scale=scale)
+        assert_bf16_close(got[b, t], want[0], f"prefill from query factors, row ({b},{t})")
