@@ -201,3 +201,35 @@ def test_shared_b_append_then_prefill():
         want = oracle.decode_shared_b(s, qo[b, t][None], kn[b][None], vn[b][None], [L],
                                       q_pos=[0], sm_scale=scale)
         assert_bf16_close(got[b, t], want[0], f"shared-B prefill row ({b},{t})")
+
+
+def test_shared_b_prefill_from_query_factors():
+    """A shared-B cache written by kpa_append without q_out, then kpa_prefill_qf from the
+    append's workspace: K rebuilt with B rotated per key, Q assembled from the factors."""
+    from workloads import APPEND_PREFILL, append_inputs
+    s = dataclasses.replace(KPA_SHARED, r_q=6, d_model=256)
+    n_tok = 300
+    w = APPEND_PREFILL.replace(shape=s, batch=2, n_tok=n_tok, capacity=512, seed=74)
+    inp = append_inputs(w)
+    start = torch.tensor([0, 40], dtype=torch.int32)
+    lib = kpa()
+    cfg = lib.make_config(s, "bf16")
+    kc = torch.zeros(w.batch * w.capacity * s.e_k, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros(w.batch * w.capacity * s.e_v, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(lib.kpa_append_workspace_size(cfg, w.batch, n_tok), dtype=torch.uint8, device="cuda")
+    lib.kpa_append(cfg, w.batch, n_tok, inp["x"].cuda(), inp["W"].cuda(), start.cuda(), w.capacity, kc, vc, None, ws)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = torch.full((w.batch, n_tok, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    lib.kpa_prefill_qf(cfg, w.batch, n_tok, ws.view(torch.float32), w.batch * n_tok, n_tok, 1, start.cuda(), kc, vc,
+                       w.capacity, scale, out)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    q_rot, _, _, _ = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start.numpy())
+    kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+    vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+    got = out.cpu().numpy()
+    for b, t in [(0, 0), (0, 150), (1, 0), (1, 128), (1, n_tok - 1), (0, n_tok - 1)]:
+        L = int(start[b]) + t + 1
+        want = oracle.decode_shared_b(s, q_rot[b, t][None], kn[b][None], vn[b][None], [L], q_pos=[0],
+                                      sm_scale=scale)
+        assert_bf16_close(got[b, t], want[0], f"shared-B prefill from query factors, row ({b},{t})")
