@@ -78,6 +78,8 @@ _SIGS = {
     "kpa_decode_noalloc": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp],
                            ctypes.c_int),
     "kpa_test_set_decode_hooks": ([_i32, _i32, ctypes.c_uint64], ctypes.c_int),
+    "kpa_test_set_decode_engine": ([_i32], ctypes.c_int),
+    "kpa_decode_kernel_kind": ([_cfgp, _i32, _i32, _i32, _i32p], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -151,6 +153,17 @@ def kpa_decode_plan(cfg, batch, max_len, tokens_per_split=0):
     _check(_lib.kpa_decode_plan(ctypes.byref(cfg), batch, max_len, tokens_per_split, ctypes.byref(n),
                                 ctypes.byref(t), ctypes.byref(l)), "kpa_decode_plan")
     return n.value, t.value, l.value
+
+
+DECODE_KERNEL_NAMES = {0: "cuda_cores", 1: "mma_sync", 2: "tcgen05"}
+
+
+def kpa_decode_kernel_kind(cfg, batch, max_len, tokens_per_split=0):
+    """Name of the kernel a dense-query decode with these arguments runs."""
+    k = ctypes.c_int32()
+    _check(_lib.kpa_decode_kernel_kind(ctypes.byref(cfg), batch, max_len, tokens_per_split, ctypes.byref(k)),
+           "kpa_decode_kernel_kind")
+    return DECODE_KERNEL_NAMES[k.value]
 
 
 def kpa_decode_qf(cfg, batch, q_factors, qf_stride, qf_seq_stride, q_pos, kcache, vcache, capacity, seq_len,
@@ -234,6 +247,10 @@ def kpa_decode_noalloc(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, 
 def kpa_test_set_decode_hooks(skip_tile=-1, skip_split=-1, wait_limit_ns=1_000_000_000):
     _check(_lib.kpa_test_set_decode_hooks(skip_tile, skip_split, wait_limit_ns),
            "kpa_test_set_decode_hooks")
+
+
+def kpa_test_set_decode_engine(engine=0):
+    _check(_lib.kpa_test_set_decode_engine(engine), "kpa_test_set_decode_engine")
 
 
 def kpa_read_device_error(stream=None) -> int:

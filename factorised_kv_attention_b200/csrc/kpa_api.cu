@@ -98,6 +98,10 @@ constexpr size_t kSmemLimit = 200 * 1024;
 std::mutex g_hooks_mu;
 DecodeTestHooks g_hooks = {-1, -1, 1000000000ull};   // bounded waits give up after 1 s
 
+// 0: the default kernels; 1: the tcgen05 TPA decode where it applies (testing and
+// measurement: it is slower than the mma.sync kernel on the shapes measured so far).
+std::atomic<int> g_decode_engine{0};
+
 DecodeTestHooks current_hooks() {
     std::lock_guard<std::mutex> lock(g_hooks_mu);
     return g_hooks;
@@ -186,7 +190,10 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
     // the last split runs to the end of its sequence: a remainder of at most a quarter of a
     // split joins the split before it instead of becoming a split (and a partial) of its own
     if (p->n_split > 1 && (int64_t)max_len - (int64_t)(p->n_split - 1) * tps <= tps / 4) --p->n_split;
-    p->cluster = p->variant >= 0 && p->n_split <= kMaxClusterSplits &&
+    // the tcgen05 kernel, on request, for TPA at h = 16, d_h = 64, R = 2 (its splits merge
+    // through global memory)
+    p->engine = p->variant >= 0 && p->tile == 128 && tc_decode_supported(d) && g_decode_engine.load() == 1;
+    p->cluster = !p->engine && p->variant >= 0 && p->n_split <= kMaxClusterSplits &&
                  (p->n_split == 1 || cluster_capacity(p->variant, p->n_split) >= batch);
     // otherwise the last CTA of a sequence merges its splits when that read is small
     p->fused = p->cluster ||
@@ -306,6 +313,23 @@ kpa_status kpa_decode_plan(const kpa_config *cfg, int32_t batch, int32_t max_len
     return KPA_OK;
 }
 
+kpa_status kpa_decode_kernel_kind(const kpa_config *cfg, int32_t batch, int32_t max_len,
+                                  int32_t tokens_per_split, int32_t *kind) {
+    if (!kind) return KPA_ERR_INVALID_ARG;
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
+    int sms = 0;
+    s = device_state(nullptr, &sms);
+    if (s != KPA_OK) return s;
+    DecodePlan p;
+    s = plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
+    if (s != KPA_OK) return s;
+    *kind = p.variant < 0 ? KPA_DECODE_KERNEL_CUDA_CORES
+                          : (p.engine ? KPA_DECODE_KERNEL_TCGEN05 : KPA_DECODE_KERNEL_MMA_SYNC);
+    return KPA_OK;
+}
+
 }  // extern "C"
 
 namespace kpa {
@@ -376,7 +400,10 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
         args.qf_stride = qf_stride;
         args.qf_seq_stride = qf_seq_stride;
         args.rq = cfg->r_q;
-        e = launch_decode_mma(p.variant, args, batch, p, rope_table(cfg), current_hooks(), st);
+        if (p.engine && !qf)
+            e = launch_decode_tc(args, batch, p, rope_table(cfg), current_hooks(), st);
+        else
+            e = launch_decode_mma(p.variant, args, batch, p, rope_table(cfg), current_hooks(), st);
     } else if (max_len > 0) {
         e = launch_decode_fma(d, cfg->dtype, batch, q, q_pos, kcache, vcache, capacity, seq_len,
                               max_len, qscale, p, part_o, part_ml, rope_table(cfg), err, st, sms);
@@ -537,6 +564,12 @@ kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split,
     g_hooks.skip_tile = skip_tile;
     g_hooks.skip_split = skip_split;
     g_hooks.wait_limit_ns = wait_limit_ns;
+    return KPA_OK;
+}
+
+kpa_status kpa_test_set_decode_engine(int32_t engine) {
+    if (engine < 0 || engine > 1) return KPA_ERR_INVALID_ARG;
+    g_decode_engine.store(engine);
     return KPA_OK;
 }
 

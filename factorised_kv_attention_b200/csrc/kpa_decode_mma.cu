@@ -25,6 +25,7 @@
 // returns.
 #include <cooperative_groups.h>
 
+#include "kpa_decode_merge.cuh"
 #include "kpa_internal.cuh"
 #include "kpa_mma_decode.cuh"
 
@@ -290,6 +291,8 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         L = L < 0 ? 0 : a.max_len;
     }
     if (t0 >= L && !a.cluster) {                           // empty split (a cluster member stays)
+        if (a.fused && L == 0 && split == 0)                // an empty sequence gets zeros
+            for (int i = tid; i < H * DH; i += (WARPS + 1) * 32) a.out[(size_t)b * H * DH + i] = 0.f;
         if (tid == 0 && spec && !mbar_wait_bounded(full0, 0, hooks.wait_limit_ns))
             raise_error(a.err, kErrTimeout);               // its speculative copy lands first
         return;
@@ -861,54 +864,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     if (!flags[1]) return;
-    // One float4 output column per thread.  The column of up to PF splits and its
-    // head's statistics (m, l) of those splits are requested together, so the merge
-    // takes one round trip to L2; the weights 2^(m_i - M) are formed per thread.
-    const float4 *pob4 = reinterpret_cast<const float4 *>(a.part_o + (size_t)b * a.n_split * H * DH);
-    const float2 *pmb2 = reinterpret_cast<const float2 *>(a.part_ml + (size_t)b * a.n_split * H * 2);
-    constexpr int PF = 16;
-    for (int c4 = tid; c4 < N4; c4 += WARPS * 32) {
-        const int head = (c4 * 4) / DH;
-        float4 pre[PF];
-        float2 st[PF];
-#pragma unroll
-        for (int i = 0; i < PF; ++i)
-            if (i < n_b) {
-                pre[i] = __ldcg(pob4 + (size_t)i * N4 + c4);
-                st[i] = __ldcg(pmb2 + (size_t)i * H + head);
-            }
-        float M = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < PF; ++i)
-            if (i < n_b) M = fmaxf(M, st[i].x);
-        for (int i = PF; i < n_b; ++i) M = fmaxf(M, __ldcg(pmb2 + (size_t)i * H + head).x);
-        float d = 0.f;
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < PF; ++i)
-            if (i < n_b) {
-                const float w = st[i].x == -INFINITY ? 0.f : exp2f(st[i].x - M);
-                d += w * st[i].y;
-                num.x += w * pre[i].x;
-                num.y += w * pre[i].y;
-                num.z += w * pre[i].z;
-                num.w += w * pre[i].w;
-            }
-#pragma unroll 4
-        for (int i = PF; i < n_b; ++i) {
-            const float2 sv = __ldcg(pmb2 + (size_t)i * H + head);
-            const float4 v = __ldcg(pob4 + (size_t)i * N4 + c4);
-            const float w = sv.x == -INFINITY ? 0.f : exp2f(sv.x - M);
-            d += w * sv.y;
-            num.x += w * v.x;
-            num.y += w * v.y;
-            num.z += w * v.z;
-            num.w += w * v.w;
-        }
-        const float f = d > 0.f ? a.out_scale / d : 0.f;
-        reinterpret_cast<float4 *>(a.out + (size_t)b * H * DH)[c4] = make_float4(num.x * f, num.y * f, num.z * f,
-                                                                                 num.w * f);
-    }
+    merge_split_partials<H, DH>(a.part_o, a.part_ml, a.n_split, n_b, b, a.out_scale, a.out, tid, WARPS * 32);
     if (tid == 0) a.counters[b] = 0;                 // ready for the next call
     return;
     }  // global merge

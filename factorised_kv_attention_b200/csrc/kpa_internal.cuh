@@ -114,6 +114,7 @@ struct DecodePlan {
     int tile;            // tokens per shared-memory tile
     int fused;           // the decode kernel merges the splits itself (no combine launch)
     int cluster;         // ... through a thread-block cluster per sequence (DSMEM)
+    int engine;          // 1: the tcgen05 kernel (TPA h = 16, d_h = 64, R = 2), 0: mma.sync
     size_t part_o_off, part_ml_off, counters_off, bytes;
 };
 

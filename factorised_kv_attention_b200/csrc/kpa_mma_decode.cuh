@@ -153,6 +153,14 @@ inline size_t mma_decode_smem(int variant) {
 // once (0: a cluster that large cannot run).
 int mma_decode_max_clusters(int variant, int size);
 
+// The tcgen05 decode (TPA, h = 16, d_h = 64, R_K = R_V = 2, dense query, no cluster;
+// selected on request):
+// whether it covers these dims, its shared memory, and its launcher.
+bool tc_decode_supported(const Dims &d);
+size_t tc_decode_smem();
+cudaError_t launch_decode_tc(const DecodeArgs &args, int batch, const DecodePlan &plan, const RopeTable &rope,
+                             const DecodeTestHooks &hooks, cudaStream_t st);
+
 cudaError_t launch_decode_mma(int variant, const DecodeArgs &args, int batch, const DecodePlan &plan,
                               const RopeTable &rope, const DecodeTestHooks &hooks, cudaStream_t st);
 

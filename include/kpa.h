@@ -136,6 +136,18 @@ kpa_status kpa_decode_plan(const kpa_config *cfg, int32_t batch, int32_t max_len
                            int32_t tokens_per_split, int32_t *n_split,
                            int32_t *tokens_per_split_out, int32_t *launches);
 
+/* Which kernel a dense-query kpa_decode_split call with these arguments runs
+ * (kpa_decode_qf always takes the mma.sync kernel):
+ *   KPA_DECODE_KERNEL_CUDA_CORES  fp32 caches or shapes without a tensor-core variant
+ *   KPA_DECODE_KERNEL_MMA_SYNC    the bf16 tensor-core kernel on mma.sync
+ *   KPA_DECODE_KERNEL_TCGEN05     TPA h = 16, d_h = 64, R_K = R_V = 2 after
+ *                                 kpa_test_set_decode_engine(1): both products on
+ *                                 tcgen05
+ * Same argument checks as kpa_decode_plan. */
+enum { KPA_DECODE_KERNEL_CUDA_CORES = 0, KPA_DECODE_KERNEL_MMA_SYNC = 1, KPA_DECODE_KERNEL_TCGEN05 = 2 };
+kpa_status kpa_decode_kernel_kind(const kpa_config *cfg, int32_t batch, int32_t max_len,
+                                  int32_t tokens_per_split, int32_t *kind);
+
 /* Factor-space decode attention: one query row per sequence against slots
  * 0 .. seq_len[b]-1 of the cache (Proposition 2.2 evaluated with a dense
  * query, Theorem 2.4 for the positions; FlashTPA-style blocking over the cache
@@ -276,6 +288,15 @@ kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, const void *
  * its consumers' wait runs out.  (-1, -1, 1000000000) restores the defaults.
  * Process-wide; not for concurrent use with real work. */
 kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split, uint64_t wait_limit_ns);
+
+/* Testing and measurement: choose the decode kernel.  0 (the default) runs every
+ * bf16 tensor-core decode on the mma.sync kernel.  1 runs a dense-query decode of
+ * the TPA shape h = 16, d_h = 64, R_K = R_V = 2 on the tcgen05 kernel (both
+ * products on tcgen05, accumulators in tensor memory; its splits merge through
+ * global memory, never in a cluster); other shapes and kpa_decode_qf are
+ * unaffected.  Process-wide; returns
+ * KPA_ERR_INVALID_ARG for other values. */
+kpa_status kpa_test_set_decode_engine(int32_t engine);
 
 /* Wait for `stream`, then return in *code the per-device error word
  * (KPA_OK, KPA_ERR_TIMEOUT or KPA_ERR_DEVICE_CHECK) of the current device and
