@@ -73,17 +73,20 @@ def test_engine_selection():
     assert lib.kpa_decode_kernel_kind(cfg, w.batch, w.length) == "mma_sync"
 
 
-def test_tcgen05_special_lengths():
-    """L = 0 gives zeros, L = 1 gives V_0, tails at 8k + r and at tile edges."""
+@pytest.mark.parametrize("engine", [1, 0], ids=["tcgen05", "mma_sync"])
+def test_special_lengths_under_a_fused_plan(engine):
+    """L = 0 gives zeros (the kernel merges its own splits here, so no combine pass
+    writes them), L = 1 gives V_0, tails at 8k + r and at tile edges."""
     w = TPA_DECODE.replace(batch=8, capacity=1024, length=1024, seed=44)
     inp = decode_inputs(w)
     inp["seq_len"] = torch.tensor([0, 1, 7, 9, 127, 128, 129, 1024], dtype=torch.int32)
     inp["q_pos"] = inp["seq_len"].clone()
     lib = kpa()
     cfg, kc, vc = fill_cache(lib, w, inp)
-    lib.kpa_test_set_decode_engine(1)
+    lib.kpa_test_set_decode_engine(engine)
     try:
-        assert lib.kpa_decode_kernel_kind(cfg, w.batch, 1024) == "tcgen05"
+        assert lib.kpa_decode_kernel_kind(cfg, w.batch, 1024) == ("tcgen05" if engine else "mma_sync")
+        assert lib.kpa_decode_plan(cfg, w.batch, 1024)[2] == 1          # one launch: fused merge
         out = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"], max_len=1024)
         torch.cuda.synchronize()
         assert lib.kpa_read_device_error() == 0
