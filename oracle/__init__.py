@@ -14,6 +14,9 @@ definitions the way the pages state them:
   query / key / value records, RoPE on the B factors of keys (Theorem 2.4) and
   the assembled, rotated query (eq 2 followed by Definition 2.3).
 
+Third-order TPA (``decode_order3`` and its helpers) is composed from the pinned
+primitives above and pinned by ``tests/pins.py::check_order3_attention``.
+
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 except the column order of the merged projection weights
 ``[A^Q | B^Q | A^K | B^K | A^V | B^V]``, a convention the pages do not fix
@@ -260,6 +263,87 @@ def decode_shared_b(shape, q, kf, va, seq_len, *, q_pos=None, sm_scale=None, hea
 def cache_numbers_per_token_shared_b(h1, h2, d1, d2, r) -> int:
     """Numbers cached per token with one B set for keys and values: A^K, A^V and B."""
     return 2 * r * h1 * d1 + r * h2 * d2
+
+
+# ------------------------------------------------------------ third-order TPA
+# "Tensor Product Attention Is All You Need", Appendix C, as the explainer page
+# summarises it: a third-order factor component is a_r (x) vec(b_r (x) c_r) with
+# a_r in R^h, b_r in R^{d_b}, c_r in R^{d_c}, d_h = d_b d_c, and RoPE (Theorem C.1)
+# acts on the b factors only: (R_{d_b}(p) (x) I_{d_c}) vec(b (x) c) = vec(R_{d_b}(p) b (x) c).
+# Here vec(b (x) c) is the Kronecker product of the two vectors (b's index the slower
+# one, Definition 2.1), and R_{d_b} is Definition 2.3's rotation on a d_b-vector.
+# A record of one token is [a_0..a_{R-1} | b_0..b_{R-1} | c_0..c_{R-1}]; shapes carry
+# h1 = h, h2 = 1, d1 = d_b, d2 = d_c.
+
+def order3_as_kronecker(h, d_b, d_c, R, rec) -> np.ndarray:
+    """The same R components written as a Kronecker record of the split h1 = h, h2 = 1,
+    d1 = d_b, d2 = d_c: A_r = a_r b_r^T (h x d_b), B_r = c_r^T (1 x d_c), so that row h of
+    (1/R) sum_r A_r (x) B_r is (1/R) sum_r a_r[h] (b_r (x) c_r).
+    rec [..., R(h + d_b + d_c)] -> [..., R(h d_b + d_c)]."""
+    rec = _f64(rec)
+    lead = rec.shape[:-1]
+    assert rec.shape[-1] == R * (h + d_b + d_c), rec.shape
+    a = rec[..., :R * h].reshape(lead + (R, h))
+    b = rec[..., R * h:R * (h + d_b)].reshape(lead + (R, d_b))
+    c = rec[..., R * (h + d_b):].reshape(lead + (R, d_c))
+    A = a[..., :, :, None] * b[..., :, None, :]
+    return np.concatenate([A.reshape(lead + (R * h * d_b,)), c.reshape(lead + (R * d_c,))], axis=-1)
+
+
+def rotate_order3_b(h, d_b, d_c, R, base, pos, rec) -> np.ndarray:
+    """One record with every b_r rotated by R_{d_b}(pos) (pairs (2m, 2m+1), theta_m =
+    base^(-2m/d_b)); a and c unchanged.  Returns a new array."""
+    rec = _f64(rec).reshape(-1).copy()
+    for r in range(R):
+        o = R * h + r * d_b
+        rec[o:o + d_b] = rope_d2(d_b, base, pos, rec[o:o + d_b])
+    return rec
+
+
+def rope_order3_query(h, d_b, d_c, base, pos, q) -> np.ndarray:
+    """(R_{d_b}(pos) (x) I_{d_c}) applied to every head row of a dense query [h][d_b d_c]."""
+    q = _f64(q).reshape(h, d_b, d_c).copy()
+    for i in range(h):
+        for jc in range(d_c):
+            q[i, :, jc] = rope_d2(d_b, base, pos, q[i, :, jc])
+    return q.reshape(h, d_b * d_c)
+
+
+class _KronShape:
+    def __init__(self, h1, h2, d1, d2, r_k, r_v, rope_base):
+        self.h1, self.h2, self.d1, self.d2 = h1, h2, d1, d2
+        self.r_k, self.r_v, self.rope_base = r_k, r_v, rope_base
+
+
+def decode_order3(shape, q, kf, vf, seq_len, *, q_pos=None, keys_rotated=False, sm_scale=None,
+                  heads=None) -> np.ndarray:
+    """Decode over a third-order TPA cache: kf, vf [B][cap][R(h + d_b + d_c)] with
+    shape.h1 = h, shape.h2 = 1, shape.d1 = d_b, shape.d2 = d_c.  The key of slot t has its
+    b factors rotated at t (unless ``keys_rotated``: the cache already holds them so), the
+    query is rotated at q_pos by R_{d_b} (x) I_{d_c}, values are not rotated.  The records
+    are then written in Kronecker form and the plain attention definition (``decode`` with
+    the keys taken as rotated and the query as given) does the rest."""
+    s = shape
+    assert s.h2 == 1, "third-order TPA has its heads in the a factors"
+    h, db, dc = s.h1, s.d1, s.d2
+    q, kf, vf = _f64(q), _f64(kf), _f64(vf)
+    B = q.shape[0]
+    if not keys_rotated:
+        kf = kf.copy()
+        for b in range(B):
+            for t in range(int(np.asarray(seq_len).reshape(-1)[b])):
+                kf[b, t] = rotate_order3_b(h, db, dc, s.r_k, s.rope_base, t, kf[b, t])
+    if q_pos is not None:
+        qp = np.asarray(q_pos).reshape(-1)
+        q = np.stack([rope_order3_query(h, db, dc, s.rope_base, int(qp[b]), q[b]) for b in range(B)])
+    ks = _KronShape(h, 1, db, dc, s.r_k, s.r_v, s.rope_base)
+    return decode(ks, q, order3_as_kronecker(h, db, dc, s.r_k, kf), order3_as_kronecker(h, db, dc, s.r_v, vf),
+                  seq_len, q_pos=None, keys_rotated=True, sm_scale=sm_scale, heads=heads)
+
+
+def cache_numbers_per_token_order3(h, d_b, d_c, r_k, r_v) -> int:
+    """Numbers cached per token by a third-order TPA cache: (R_K + R_V)(h + d_b + d_c)."""
+    return (r_k + r_v) * (h + d_b + d_c)
 
 
 def prefill(shape, q, kf, vf, start_pos, *, q_pos=None, keys_rotated=False, sm_scale=None,

@@ -182,7 +182,7 @@ int oracle_attend(int h1, int h2, int d1, int d2, int r_k, int r_v, double rope_
     const int ek = r_k * (h1 * d1 + h2 * d2), ev = r_v * (h1 * d1 + h2 * d2);
     if (h <= 0 || dh <= 0 || r_k <= 0 || r_v <= 0 || batch < 0 || n_q < 0 || cap < 0)
         return -1;
-    if (d2 % 2 != 0) return -1;
+    if (d2 % 2 != 0 && (q_pos || !keys_rotated)) return -1;   /* RoPE pairs, when it rotates */
     const int total = heads ? n_heads : batch * h;
     int failed = 0;
 

@@ -382,11 +382,63 @@ def check_shared_b_attention(seed=13):
         assert n == oracle.cache_numbers_per_token(s.h1, s.h2, s.d1, s.d2, R, R) - R * s.h2 * s.d2
 
 
+def check_order3_attention(seed=14):
+    """Third-order TPA ("Tensor Product Attention Is All You Need", Appendix C, as the
+    explainer summarises it): a, b and c are drawn as separate arrays; K_t and V_t are
+    built with numpy.kron as (1/R) sum_r a_r (x) (b_r (x) c_r); K_t is rotated with the
+    block matrix numpy.kron(R_{d_b}(t), I_{d_c}) (RoPE on b, Theorem C.1) and the query
+    with numpy.kron(R_{d_b}(q_pos), I_{d_c}); torch's scaled_dot_product_attention gives
+    the expected output.  With d_c = 1 the cache is a second-order TPA cache with
+    B_r = c_r b_r, and the plain decode of that cache must agree."""
+    rng = np.random.default_rng(seed)
+    for (h, db, dc, R, base) in [(4, 4, 2, 2, 10000.0), (3, 2, 3, 1, 500000.0), (2, 6, 1, 3, 10000.0)]:
+        B, cap = 2, 9
+        a = rng.standard_normal((2, B, cap, R, h))
+        b = rng.standard_normal((2, B, cap, R, db))
+        c = rng.standard_normal((2, B, cap, R, dc))
+        q = rng.standard_normal((B, h, db * dc))
+        q_pos = rng.integers(0, 600000, size=B)
+        L = np.array([cap, 5])
+        scale = 1.1 / math.sqrt(db * dc)
+        s3 = Shape(h1=h, h2=1, d1=db, d2=dc, r_k=R, r_v=R, rope_base=base, order=3)
+        kf = np.concatenate([a[0].reshape(B, cap, -1), b[0].reshape(B, cap, -1), c[0].reshape(B, cap, -1)], axis=2)
+        vf = np.concatenate([a[1].reshape(B, cap, -1), b[1].reshape(B, cap, -1), c[1].reshape(B, cap, -1)], axis=2)
+        got = oracle.decode_order3(s3, q, kf, vf, L, q_pos=q_pos, sm_scale=scale)
+        K = np.zeros((B, cap, h, db * dc)); V = np.zeros((B, cap, h, db * dc))
+        for bb in range(B):
+            for t in range(cap):
+                rot = np.kron(_rot_matrix_d2(db, base, t), np.eye(dc))
+                K[bb, t] = (sum(np.kron(a[0, bb, t, r][:, None], np.kron(b[0, bb, t, r], c[0, bb, t, r])[None, :])
+                                for r in range(R)) / R) @ rot.T
+                V[bb, t] = sum(np.kron(a[1, bb, t, r][:, None], np.kron(b[1, bb, t, r], c[1, bb, t, r])[None, :])
+                               for r in range(R)) / R
+        Q = np.stack([q[bb] @ np.kron(_rot_matrix_d2(db, base, q_pos[bb]), np.eye(dc)).T for bb in range(B)])
+        mask = np.arange(cap)[None, :] < L[:, None]
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q)[:, :, None], torch.from_numpy(K).permute(0, 2, 1, 3),
+            torch.from_numpy(V).permute(0, 2, 1, 3), attn_mask=torch.from_numpy(mask)[:, None, None],
+            scale=scale)[:, :, 0].numpy()
+        _close(got, want, 1e-11, f"third-order attention vs SDPA {(h, db, dc, R)}")
+        # the rotated cache (b rotated at each slot) read with keys_rotated gives the same
+        kr = np.stack([np.stack([oracle.rotate_order3_b(h, db, dc, R, base, t, kf[bb, t]) for t in range(cap)])
+                       for bb in range(B)])
+        _close(oracle.decode_order3(s3, q, kr, vf, L, q_pos=q_pos, sm_scale=scale, keys_rotated=True), want,
+               1e-11, "third-order, keys stored rotated")
+        if dc == 1:
+            s2 = Shape(h1=h, h2=1, d1=1, d2=db, r_k=R, r_v=R, rope_base=base)
+            k2 = np.concatenate([a[0].reshape(B, cap, -1), (b[0] * c[0]).reshape(B, cap, -1)], axis=2)
+            v2 = np.concatenate([a[1].reshape(B, cap, -1), (b[1] * c[1]).reshape(B, cap, -1)], axis=2)
+            _close(got, oracle.decode(s2, q, k2, v2, L, q_pos=q_pos, sm_scale=scale), 1e-11,
+                   "third-order with d_c = 1 is second-order TPA with B = c b")
+        # cache size: R (h + d_b + d_c) numbers per key or value record
+        assert oracle.cache_numbers_per_token_order3(h, db, dc, R, R) == kf.shape[2] + vf.shape[2]
+
+
 ALL_CHECKS = [
     check_kron_is_numpy_kron, check_reconstruct_is_kron_sum, check_tpa_split_is_outer_product,
     check_prop22_factored_score, check_rope_golden_frequencies, check_rope_tpa_is_textbook,
     check_rope_kpa_is_identity_kron_rotation, check_thm24_rotating_b_equals_rotating_reconstruction,
     check_relative_position, check_attention_matches_sdpa, check_attention_closed_forms,
     check_prefill_rows_are_decodes, check_projection_is_matmul, check_append_scores_follow_eq9,
-    check_cache_sizes_golden, check_shared_b_attention,
+    check_cache_sizes_golden, check_shared_b_attention, check_order3_attention,
 ]

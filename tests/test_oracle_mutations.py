@@ -65,3 +65,43 @@ def test_planted_causal_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "prefill", _prefill_without_self)
     with pytest.raises(AssertionError):
         pins.check_prefill_rows_are_decodes()
+
+
+def _order3_transposed_a_b(h, d_b, d_c, R, rec):
+    """A planted mistake: A_r laid out as b_r a_r^T (d_b x h) instead of a_r b_r^T."""
+    rec = oracle._f64(rec)
+    lead = rec.shape[:-1]
+    a = rec[..., :R * h].reshape(lead + (R, h))
+    b = rec[..., R * h:R * (h + d_b)].reshape(lead + (R, d_b))
+    c = rec[..., R * (h + d_b):].reshape(lead + (R, d_c))
+    A = b[..., :, :, None] * a[..., :, None, :]
+    return oracle.np.concatenate([A.reshape(lead + (R * h * d_b,)), c.reshape(lead + (R * d_c,))], axis=-1)
+
+
+_rotate_b = oracle.rotate_order3_b
+_rope_q3 = oracle.rope_order3_query
+
+
+def _order3_key_rotated_one_slot_late(h, d_b, d_c, R, base, pos, rec):
+    return _rotate_b(h, d_b, d_c, R, base, pos + 1, rec)
+
+
+def _order3_query_rotated_on_c(h, d_b, d_c, base, pos, q):
+    """A planted mistake: the query's rotation acts on the c index instead of b."""
+    q = oracle._f64(q).reshape(h, d_b, d_c).copy()
+    if d_c % 2:
+        return _rope_q3(h, d_b, d_c, base, pos + 1, q.reshape(h, -1))
+    for i in range(h):
+        for jb in range(d_b):
+            q[i, jb, :] = oracle.rope_d2(d_c, base, pos, q[i, jb, :])
+    return q.reshape(h, d_b * d_c)
+
+
+@pytest.mark.parametrize("attr,bad", [("order3_as_kronecker", _order3_transposed_a_b),
+                                      ("rotate_order3_b", _order3_key_rotated_one_slot_late),
+                                      ("rope_order3_query", _order3_query_rotated_on_c)],
+                         ids=["a and b transposed", "key rotated one slot late", "query rotated on c"])
+def test_planted_order3_mistake_is_caught(monkeypatch, attr, bad):
+    monkeypatch.setattr(oracle, attr, bad)
+    with pytest.raises((AssertionError, ValueError)):
+        pins.check_order3_attention()

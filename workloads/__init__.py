@@ -39,6 +39,7 @@ class Shape:
     d_model: int = 0
     rope_base: float = 10000.0
     shared_b: int = 0          # 1: one B factor for keys and values (B^K_r = B^V_r, r_k == r_v)
+    order: int = 2             # 3: third-order TPA, key a (x) b (x) c with h2 = 1, d1 = d_b, d2 = d_c
 
     @property
     def h(self) -> int:
@@ -50,13 +51,18 @@ class Shape:
 
     @property
     def e_k(self) -> int:
-        """Elements in one token's key record [A_0..A_{R-1} | B_0..B_{R-1}]."""
+        """Elements in one token's key record [A_0..A_{R-1} | B_0..B_{R-1}], or for a
+        third-order shape [a_0..a_{R-1} | b_0..b_{R-1} | c_0..c_{R-1}]."""
+        if self.order == 3:
+            return self.r_k * (self.h1 + self.d1 + self.d2)
         return self.r_k * (self.h1 * self.d1 + self.h2 * self.d2)
 
     @property
     def e_v(self) -> int:
         """Elements in one token's value record: [A_0.. | B_0..], or [A_0..] alone when
         the B factors are shared with the keys."""
+        if self.order == 3:
+            return self.r_v * (self.h1 + self.d1 + self.d2)
         if self.shared_b:
             return self.r_v * self.h1 * self.d1
         return self.r_v * (self.h1 * self.d1 + self.h2 * self.d2)
@@ -157,8 +163,21 @@ TPA_SHARED_DECODE = dataclasses.replace(
     TPA_DECODE, name="TPA decode, shared B (B=8, h=16x1, d_h=1x64, R=2, L=4096, bf16)",
     shape=dataclasses.replace(TPA_DECODE.shape, shared_b=1))
 
+# Third-order TPA ("Tensor Product Attention Is All You Need", Appendix C, as the
+# explainer summarises it): the key of head h is (1/R) sum_r a_r[h] (b_r (x) c_r), b in
+# R^{d_b}, c in R^{d_c}, d_h = d_b d_c = 64, so the sizes match the TPA decode above.
+# The pages give no shape for it; this one keeps h, d_h, R, B and L of the TPA decode
+# and splits d_h as 8 x 8.  Factors ~ N(0, 2^(1/3)) make a key entry's variance
+# sigma^6 / R = 1.
+TPA3_DECODE = DecodeWorkload(
+    name="third-order TPA decode (B=8, h=16, d_h=8x8, R=2+2, L=4096, bf16)",
+    shape=Shape(h1=16, h2=1, d1=8, d2=8, r_k=2, r_v=2, rope_base=10000.0, order=3),
+    batch=8, capacity=4096, dtype="bf16", factor_std=float(2.0 ** (1.0 / 6.0)), q_std=1.0 / 8.0,
+    seed=0, length=4096)
+
 DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
-                  "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE, "tpa_shared": TPA_SHARED_DECODE}
+                  "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE, "tpa_shared": TPA_SHARED_DECODE,
+                  "tpa_order3": TPA3_DECODE}
 
 
 # --- draws ---------------------------------------------------------------------
