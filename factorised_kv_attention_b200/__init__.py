@@ -37,7 +37,7 @@ class kpa_config(ctypes.Structure):
     _fields_ = [("h1", ctypes.c_int32), ("h2", ctypes.c_int32), ("d1", ctypes.c_int32),
                 ("d2", ctypes.c_int32), ("r_q", ctypes.c_int32), ("r_k", ctypes.c_int32),
                 ("r_v", ctypes.c_int32), ("d_model", ctypes.c_int32), ("rope_base", ctypes.c_double),
-                ("dtype", ctypes.c_int), ("shared_b", ctypes.c_int32)]
+                ("dtype", ctypes.c_int), ("shared_b", ctypes.c_int32), ("order", ctypes.c_int32)]
 
 
 class KpaError(RuntimeError):
@@ -89,11 +89,12 @@ for _name, (_args, _res) in _SIGS.items():
 
 def make_config(shape, dtype: str = "bf16") -> kpa_config:
     """kpa_config from any object with h1, h2, d1, d2, r_k, r_v (and optionally
-    r_q, d_model, rope_base, shared_b)."""
+    r_q, d_model, rope_base, shared_b, order)."""
     return kpa_config(int(shape.h1), int(shape.h2), int(shape.d1), int(shape.d2),
                       int(getattr(shape, "r_q", 0)), int(shape.r_k), int(shape.r_v),
                       int(getattr(shape, "d_model", 0)), float(getattr(shape, "rope_base", 10000.0)),
-                      KPA_BF16 if dtype == "bf16" else KPA_F32, int(getattr(shape, "shared_b", 0)))
+                      KPA_BF16 if dtype == "bf16" else KPA_F32, int(getattr(shape, "shared_b", 0)),
+                      int(getattr(shape, "order", 2)))
 
 
 def _addr(x):

@@ -60,7 +60,14 @@ kpa_status check_cfg(const kpa_config *c, bool need_q, bool need_model) {
     if (need_model && c->d_model <= 0) return KPA_ERR_INVALID_ARG;
     if (c->dtype != KPA_F32 && c->dtype != KPA_BF16) return KPA_ERR_INVALID_ARG;
     if (!(c->rope_base > 0.0) || !isfinite(c->rope_base)) return KPA_ERR_INVALID_ARG;
-    if (c->d2 % 2 != 0) return KPA_ERR_INVALID_ARG;        // RoPE pairs
+    if (c->order != 0 && c->order != 2 && c->order != 3) return KPA_ERR_INVALID_ARG;
+    if (c->order == 3) {
+        // third-order TPA: heads in a, RoPE pairs on b (d1 = d_b), no shared B
+        if (c->h2 != 1 || c->d1 % 2 != 0 || c->shared_b != 0) return KPA_ERR_INVALID_ARG;
+        if (c->d1 > 2 * kMaxHalfD2) return KPA_ERR_UNSUPPORTED;
+    } else if (c->d2 % 2 != 0) {
+        return KPA_ERR_INVALID_ARG;                           // RoPE pairs
+    }
     if (c->shared_b != 0 && c->shared_b != 1) return KPA_ERR_INVALID_ARG;
     if (c->shared_b && c->r_k != c->r_v) return KPA_ERR_INVALID_ARG;   // B^K_r = B^V_r
     const int64_t h = (int64_t)c->h1 * c->h2, dh = (int64_t)c->d1 * c->d2;
@@ -79,13 +86,19 @@ Dims dims_of(const kpa_config *c) {
     d.ek = c->r_k * (c->h1 * c->d1 + c->h2 * c->d2);
     d.shared = c->shared_b ? 1 : 0;
     d.ev = d.shared ? c->r_v * c->h1 * c->d1 : c->r_v * (c->h1 * c->d1 + c->h2 * c->d2);
+    d.order = c->order == 3 ? 3 : 2;
+    if (d.order == 3) {                                       // record [a | b | c]
+        d.ek = c->r_k * (c->h1 + c->d1 + c->d2);
+        d.ev = c->r_v * (c->h1 + c->d1 + c->d2);
+    }
     return d;
 }
 
 RopeTable rope_table(const kpa_config *c) {
     RopeTable t;
+    const int n = c->order == 3 ? c->d1 : c->d2;              // the rotated factor's length
     for (int m = 0; m < kMaxHalfD2; ++m)
-        t.theta[m] = m < c->d2 / 2 ? pow(c->rope_base, -2.0 * (double)m / (double)c->d2) : 0.0;
+        t.theta[m] = m < n / 2 ? pow(c->rope_base, -2.0 * (double)m / (double)n) : 0.0;
     return t;
 }
 
@@ -130,7 +143,7 @@ int cluster_capacity(int variant, int size) {
 kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int tps_req, int sms,
                        DecodePlan *p) {
     if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
-    p->variant = dt == KPA_BF16 ? mma_decode_variant(d) : -1;
+    p->variant = dt == KPA_BF16 && d.order != 3 ? mma_decode_variant(d) : -1;
     if (d.shared && p->variant < 0) return KPA_ERR_UNSUPPORTED;   // shared B: tensor-core variants only
     int ctas_per_sm = 2;
     if (p->variant >= 0) {
@@ -141,6 +154,9 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
         const int resident = cluster_capacity(p->variant, 1);
         if (resident > 0 && sms > 0 && resident / sms < ctas_per_sm) ctas_per_sm = resident / sms;
         if (ctas_per_sm < 1) ctas_per_sm = 1;
+    } else if (d.order == 3) {
+        if (!order3_decode_supported(d, dt)) return KPA_ERR_UNSUPPORTED;
+        p->tile = kOrder3Tile;
     } else {
         int tile = 32;
         while (tile > 8 && decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) tile /= 2;
@@ -363,6 +379,7 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
     if (s != KPA_OK) return s;
     if (qf && p.variant < 0) return KPA_ERR_UNSUPPORTED;        // query factors: tensor-core path only
+                                                                  // (never a third-order cache)
     if (qf && (int64_t)cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) > mma_decode_qf_max(p.variant))
         return KPA_ERR_UNSUPPORTED;                               // staged in the kernel's query rows
     if (!workspace || ws_bytes < p.bytes) return KPA_ERR_WORKSPACE;
@@ -404,6 +421,9 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
             e = launch_decode_tc(args, batch, p, rope_table(cfg), current_hooks(), st);
         else
             e = launch_decode_mma(p.variant, args, batch, p, rope_table(cfg), current_hooks(), st);
+    } else if (max_len > 0 && d.order == 3) {
+        e = launch_decode_order3(d, cfg->dtype, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len,
+                                 qscale, p, part_o, part_ml, rope_table(cfg), err, st);
     } else if (max_len > 0) {
         e = launch_decode_fma(d, cfg->dtype, batch, q, q_pos, kcache, vcache, capacity, seq_len,
                               max_len, qscale, p, part_o, part_ml, rope_table(cfg), err, st, sms);
@@ -464,7 +484,7 @@ static kpa_status prefill_impl(const kpa_config *cfg, int32_t batch, int32_t n_t
     if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
     if (!isfinite(sm_scale)) return KPA_ERR_INVALID_ARG;
     if (qf.ptr && (qf.stride <= 0 || qf.seq_stride < 0 || qf.tok_stride < 0)) return KPA_ERR_INVALID_ARG;
-    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    if (cfg->dtype != KPA_BF16 || cfg->order == 3) return KPA_ERR_UNSUPPORTED;
     const Dims d = dims_of(cfg);
     if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
     if (qf.ptr && cfg->r_q > kPrefillQfMaxRq) return KPA_ERR_UNSUPPORTED;
@@ -513,6 +533,7 @@ kpa_status kpa_append_workspace_size(const kpa_config *cfg, int32_t batch, int32
                                      size_t *bytes) {
     kpa_status s = check_cfg(cfg, true, true);
     if (s != KPA_OK) return s;
+    if (cfg->order == 3) return KPA_ERR_UNSUPPORTED;             // the merged projection: Kronecker form
     if (!bytes || batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
     const int64_t eq = (int64_t)cfg->r_q * (cfg->h1 * cfg->d1 + cfg->h2 * cfg->d2);
     *bytes = align256((size_t)eq * batch * n_tok * sizeof(float));
@@ -527,7 +548,7 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const
     if (s != KPA_OK) return s;
     if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
     if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
-    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    if (cfg->dtype != KPA_BF16 || cfg->order == 3) return KPA_ERR_UNSUPPORTED;
     // TMA rows of x and W are d_model bf16 values: a multiple of 16 bytes
     if (cfg->d_model % 8 != 0) return KPA_ERR_UNSUPPORTED;
     // factor pairs (2m, 2m+1) of B must start on even columns of the projection

@@ -4,7 +4,8 @@
 // A^K, A^V and B^V as projected and B^K rotated at the token's position by
 // R_theta^(2)(pos); nothing else is rotated.  With one B shared by keys and values
 // ("Tensor Product Attention Is All You Need", section 5) B is stored unrotated and
-// the value record holds A^V only.
+// the value record holds A^V only.  A third-order TPA record [a | b | c] has its b
+// factors rotated instead (R_{d_b}(pos) (x) I_{d_c}, the same paper's Appendix C).
 //
 // One CTA owns one 8-token cache group of one plane of one sequence: it reads the
 // (up to) 8 natural-layout records of that group, rotates the B^K pairs and
@@ -60,8 +61,13 @@ append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__re
     const T *src = (is_k ? kf : vf) + ((size_t)b * n_tok) * E;
     T *dst = (is_k ? kc : vc) + ((size_t)b * cap) * E + (size_t)g * E * kGroup;
 
-    const int half = d.d2 / 2;
-    const int a_size = (is_k ? d.rk : d.rv) * d.h1 * d.d1;
+    // the rotated factor: B^K (length d2, after the A factors), or for a third-order
+    // record [a | b | c] the b factors (length d1, after the a factors)
+    const int R = is_k ? d.rk : d.rv;
+    const int period = d.order == 3 ? d.d1 : d.d2;
+    const int half = period / 2;
+    const int a_size = d.order == 3 ? R * d.h1 : R * d.h1 * d.d1;
+    const int rot_end = d.order == 3 ? a_size + R * d.d1 : E;
     const bool rot_k = is_k && !d.shared;         // a shared B is stored unrotated
     if (rot_k) {
         for (int i = threadIdx.x; i < kGroup * half; i += blockDim.x) {
@@ -74,10 +80,10 @@ append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__re
     }
 
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const bool rot = rot_k && e >= a_size;
+        const bool rot = rot_k && e >= a_size && e < rot_end;
         int partner = e, j2 = 0;
         if (rot) {
-            j2 = (e - a_size) % d.d2;
+            j2 = (e - a_size) % period;
             partner = (j2 & 1) ? e - 1 : e + 1;
         }
         T vals[kGroup];

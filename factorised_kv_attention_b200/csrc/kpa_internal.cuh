@@ -25,10 +25,12 @@ struct Dims {
     int h, dh;      // h1*h2, d1*d2
     int ek, ev;     // elements per key / value record
     int shared;     // one B for keys and values: key record [A^K | B] (B unrotated), value record [A^V]
+    int order;      // 2: Kronecker form; 3: third-order TPA, record [a | b | c] (h2 = 1, d1 = d_b, d2 = d_c)
 };
 
-// theta_m = base^(-2m/d2), m < d2/2, formed on the host in float64 and passed by
-// value (Definition 2.3; the pairing and sign are documented in kpa.h).
+// theta_m = base^(-2m/n), m < n/2, formed on the host in float64 and passed by
+// value (Definition 2.3; the pairing and sign are documented in kpa.h).  n is d2,
+// or d_b = d1 for a third-order cache (RoPE on the b factors).
 struct RopeTable {
     double theta[kMaxHalfD2];
 };
@@ -135,6 +137,15 @@ cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_l
                                   cudaStream_t st);
 
 size_t decode_fma_smem_bytes(const Dims &d, kpa_dtype dt, int tile);
+
+// Third-order TPA decode (CUDA cores): whether it covers these dims, and its launcher
+// (unnormalised split partials for launch_decode_combine).
+constexpr int kOrder3Tile = 32;
+bool order3_decode_supported(const Dims &d, kpa_dtype dt);
+cudaError_t launch_decode_order3(const Dims &d, kpa_dtype dt, int batch, const void *q, const int32_t *q_pos,
+                                 const void *kc, const void *vc, int cap, const int32_t *seq_len, int max_len,
+                                 float qscale, const DecodePlan &p, float *part_o, float *part_ml,
+                                 const RopeTable &rope, int *err, cudaStream_t st);
 
 bool prefill_supported(const Dims &d);
 // Query factors for a prefill (ptr null: a dense bf16 query instead).

@@ -90,6 +90,22 @@ typedef struct {
                          * kpa_append_factors, kpa_append (merged weight columns
                          * [A^Q | B^Q | A^K | A^V | B]), the decode calls and
                          * kpa_prefill (which rotates B while rebuilding K).     */
+    int32_t order;      /* 0 or 2: the Kronecker form above.  3: third-order TPA
+                         * ("Tensor Product Attention Is All You Need", Appendix C):
+                         * the key of head h is (1/R_K) sum_r a_r[h] (b_r (x) c_r)
+                         * with a_r in R^h1, b_r in R^d1, c_r in R^d2 (d_h = d1 d2,
+                         * b's index the slower one); h2 must be 1, d1 even, and
+                         * shared_b 0.  A record is [a_0..a_{R-1} | b_0..b_{R-1} |
+                         * c_0..c_{R-1}] (E = R (h1 + d1 + d2)); RoPE acts on the b
+                         * factors only, R_{d1}(pos) (x) I_{d2} with theta_m =
+                         * base^(-2m/d1), so kpa_append_factors rotates the keys' b
+                         * and kpa_decode rotates the query by the same block
+                         * matrix.  Taken by kpa_cache_bytes_per_token,
+                         * kpa_append_factors, kpa_decode_workspace_size,
+                         * kpa_decode_plan, kpa_decode_kernel_kind, kpa_decode,
+                         * kpa_decode_split and kpa_decode_noalloc (d1, d2 <= 16,
+                         * h1 <= 32); the projection, the prefill and the
+                         * query-factor decode return KPA_ERR_UNSUPPORTED.       */
 } kpa_config;
 
 /* Human-readable name of a status code (static storage). */

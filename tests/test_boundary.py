@@ -1,6 +1,7 @@
 """The C ABI: the library loads, exports every call that include/kpa.h declares,
 and rejects bad arguments before it touches a device (CPU only)."""
 import ctypes
+import dataclasses
 import os
 import re
 
@@ -45,7 +46,10 @@ def test_cache_bytes_match_eq10(name):
     cfg = kpa.make_config(s, w.dtype)
     kb, vb = kpa.kpa_cache_bytes_per_token(cfg)
     elt = 2 if w.dtype == "bf16" else 4
-    if s.shared_b:
+    if s.order == 3:
+        numbers = oracle.cache_numbers_per_token_order3(s.h1, s.d1, s.d2, s.r_k, s.r_v)
+        assert kb * s.r_v == vb * s.r_k
+    elif s.shared_b:
         numbers = oracle.cache_numbers_per_token_shared_b(s.h1, s.h2, s.d1, s.d2, s.r_k)
         assert vb == s.r_v * s.h1 * s.d1 * elt           # the value record is A^V only
     else:
@@ -88,6 +92,28 @@ def test_shared_b_prefill_shape_limit():
     with pytest.raises(kpa.KpaError) as e:
         kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)
     assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
+
+
+def test_third_order_entry_points():
+    """A third-order cache ([a | b | c] records, RoPE on b) is taken by the cache write
+    and the decode; the projection and the prefill refuse it before any device call,
+    and its own shape rules hold (h2 = 1, d1 even, no shared B)."""
+    s = DECODE_CONFIGS["tpa_order3"].shape
+    cfg = kpa.make_config(s, "bf16")
+    assert kpa.kpa_cache_bytes_per_token(cfg) == (2 * s.r_k * (s.h1 + s.d1 + s.d2),) * 2
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)
+    assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
+    cfg_q = kpa.make_config(dataclasses.replace(s, r_q=4, d_model=256), "bf16")
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_append_workspace_size(cfg_q, 1, 16)
+    assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
+    # d2 (= d_c) may be odd; d1 (= d_b, the rotated factor) may not
+    assert kpa.kpa_cache_bytes_per_token(kpa.make_config(dataclasses.replace(s, d2=3), "bf16"))[0] > 0
+    for bad in (dict(d1=7), dict(h2=2), dict(shared_b=1), dict(order=4)):
+        with pytest.raises(kpa.KpaError) as e:
+            kpa.kpa_cache_bytes_per_token(kpa.make_config(dataclasses.replace(s, **bad), "bf16"))
+        assert e.value.status == kpa.KPA_ERR_INVALID_ARG, bad
 
 
 BAD_SHAPES = [dict(h1=0), dict(d2=7), dict(r_k=0), dict(r_v=-1), dict(d1=-2)]
