@@ -41,7 +41,8 @@ TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = ["factorised_kv_attention_b200/csrc/kpa_decode_mma.cu",
                   "factorised_kv_attention_b200/csrc/kpa_mma_decode.cuh",
                   "factorised_kv_attention_b200/csrc/kpa_decode_fma.cu",
-                  "factorised_kv_attention_b200/csrc/kpa_internal.cuh"]
+                  "factorised_kv_attention_b200/csrc/kpa_internal.cuh",
+                  "factorised_kv_attention_b200/csrc/kpa_decode_merge.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -52,7 +53,8 @@ def _args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kpa", "reference"], default="kpa")
     ap.add_argument("--workload", default="tpa_decode",
-                    help="tpa_decode | tpa_shared | kpa_medium | kpa_long | tiny_kpa | flashtpa | append_prefill")
+                    help="tpa_decode | tpa_shared | tpa_order3 | kpa_medium | kpa_long | tiny_kpa | flashtpa | "
+                         "append_prefill")
     ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -117,13 +119,15 @@ def _hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _traffic(kernel_hash):
+def _traffic(kernel_hash, workload):
+    """DRAM bytes per launch from the committed ncu record, when it was taken on this
+    workload and on the current decode sources (else None)."""
     try:
         with open(TRAFFIC) as f:
             t = json.load(f)
     except Exception:
         return None
-    if t.get("kernel_sources_sha") != kernel_hash:
+    if t.get("kernel_sources_sha") != kernel_hash or t.get("workload") != workload:
         return None
     return t.get("dram_bytes_per_launch")
 
@@ -220,7 +224,9 @@ def _cpu_baseline(w, inp, seconds, steps=None):
     b = 0
     while (steps is None and t_total < seconds) or (steps is not None and len(times) < steps):
         t0 = time.perf_counter()
-        if w.shape.shared_b:     # one B for keys and values: value records are A^V only
+        if w.shape.order == 3:   # third-order records [a | b | c], RoPE on b
+            oracle.decode_order3(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1], q_pos=qp[b:b + 1])
+        elif w.shape.shared_b:   # one B for keys and values: value records are A^V only
             oracle.decode_shared_b(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1],
                                    q_pos=qp[b:b + 1])
         else:
@@ -384,6 +390,24 @@ def run_kpa(a):
     achieved = layer_bytes / t_launch / 1e9
     peak, peak_kind = _hbm_peak()
     khash = _kernel_hash()
+    traffic_workload = a.workload if not (a.seq_len or a.batch or a.tokens_per_split) else None
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": _traffic(khash, traffic_workload),
+                "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
+                "kernel": "kpa_decode (split + combine), per layer call",
+                "algorithmic_bytes_per_launch": layer_bytes,
+                "launch_us": t_launch * 1e6, "kernel_sources_sha": khash}
+    if s.order == 3:
+        # a third-order record is too small for HBM to bound the decode: its FP32
+        # multiply-adds do (see _order3_flops_per_token)
+        flops = tokens_per_layer * _order3_flops_per_token(s)
+        roofline = {"bound": "alu", "achieved": flops / t_launch / 1e12, "peak": FP32_PEAK_TFLOPS,
+                    "unit": "TFLOP/s", "frac": flops / t_launch / 1e12 / FP32_PEAK_TFLOPS, "traffic": None,
+                    "peak_source": "148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz (nominal unit counts and "
+                                   "max SM clock)",
+                    "kernel": "kpa_decode on a third-order cache (split + combine), per layer call",
+                    "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": layer_bytes,
+                    "hbm_frac": achieved / peak, "launch_us": t_launch * 1e6}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
@@ -392,12 +416,7 @@ def run_kpa(a):
             "config": dict(_config_json(w, layers, lens, world),
                            splits_per_sequence=kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[0],
                            tokens_per_split=kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[1]),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": _traffic(khash),
-                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
-                         "kernel": "kpa_decode (split + combine), per layer call",
-                         "algorithmic_bytes_per_launch": layer_bytes,
-                         "launch_us": t_launch * 1e6, "kernel_sources_sha": khash},
+            "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
                     "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
@@ -417,6 +436,20 @@ def run_kpa(a):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+# FP32 CUDA-core peak: 148 SMs x 128 lanes x 2 flops per FMA x 1.965 GHz.
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def _order3_flops_per_token(s):
+    """Multiply-adds a third-order decode needs per cached token, x 2: the score's
+    bilinear form per head and key rank, h R_K (d_b d_c + d_b) + h R_K; the products
+    b^V (x) c^V once per value rank, R_V d_b d_c; the value update per head and value
+    rank, h R_V d_b d_c (plus h R_V for p a^V)."""
+    h, db, dc = s.h1, s.d1, s.d2
+    fma = h * s.r_k * (db * dc + db + 1) + s.r_v * db * dc + h * s.r_v * (db * dc + 1)
+    return 2 * fma
 
 
 def _bf16_peak():

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kpa_internal.cuh"
@@ -157,6 +158,9 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
     } else if (d.order == 3) {
         if (!order3_decode_supported(d, dt)) return KPA_ERR_UNSUPPORTED;
         p->tile = kOrder3Tile;
+        // latency-bound CUDA-core kernel: fill every CTA slot the occupancy query allows
+        // (up to 4 per SM; more splits only add partials to merge)
+        ctas_per_sm = std::min(4, order3_ctas_per_sm(d, dt));
     } else {
         int tile = 32;
         while (tile > 8 && decode_fma_smem_bytes(d, dt, tile) > kSmemLimit) tile /= 2;

@@ -142,6 +142,7 @@ size_t decode_fma_smem_bytes(const Dims &d, kpa_dtype dt, int tile);
 // (unnormalised split partials for launch_decode_combine).
 constexpr int kOrder3Tile = 32;
 bool order3_decode_supported(const Dims &d, kpa_dtype dt);
+int order3_ctas_per_sm(const Dims &d, kpa_dtype dt);
 cudaError_t launch_decode_order3(const Dims &d, kpa_dtype dt, int batch, const void *q, const int32_t *q_pos,
                                  const void *kc, const void *vc, int cap, const int32_t *seq_len, int max_len,
                                  float qscale, const DecodePlan &p, float *part_o, float *part_ml,
