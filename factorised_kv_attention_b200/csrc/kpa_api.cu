@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <mutex>
 
+#include "kpa_decode_factored.cuh"
 #include "kpa_internal.cuh"
 #include "kpa_mma_decode.cuh"
 
@@ -112,8 +113,9 @@ constexpr size_t kSmemLimit = 200 * 1024;
 std::mutex g_hooks_mu;
 DecodeTestHooks g_hooks = {-1, -1, 1000000000ull};   // bounded waits give up after 1 s
 
-// 0: the default kernels; 1: the tcgen05 TPA decode where it applies (testing and
-// measurement: it is slower than the mma.sync kernel on the shapes measured so far).
+// 0: the default kernels; 1: the tcgen05 TPA decode where it applies; 2: the factored
+// score for decodes from query factors on TPA shapes (testing and measurement: both are
+// slower than the defaults on the shapes measured so far).
 std::atomic<int> g_decode_engine{0};
 
 DecodeTestHooks current_hooks() {
@@ -382,9 +384,12 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     DecodePlan p;
     s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
     if (s != KPA_OK) return s;
-    if (qf && p.variant < 0) return KPA_ERR_UNSUPPORTED;        // query factors: tensor-core path only
-                                                                  // (never a third-order cache)
-    if (qf && (int64_t)cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) > mma_decode_qf_max(p.variant))
+    // query factors: the factored score on request (TPA shapes), else the tensor-core
+    // kernel, which assembles the query (never a third-order cache)
+    const bool factored = qf && g_decode_engine.load() == 2 && cfg->dtype == KPA_BF16 &&
+                          factored_decode_supported(d, cfg->r_q);
+    if (qf && !factored && p.variant < 0) return KPA_ERR_UNSUPPORTED;
+    if (qf && !factored && (int64_t)cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) > mma_decode_qf_max(p.variant))
         return KPA_ERR_UNSUPPORTED;                               // staged in the kernel's query rows
     if (!workspace || ws_bytes < p.bytes) return KPA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return KPA_ERR_INVALID_ARG;
@@ -397,6 +402,14 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     int *counters = reinterpret_cast<int *>(static_cast<char *>(workspace) + p.counters_off);
     const float out_scale = (float)(1.0 / (double)d.rv);
     cudaError_t e = cudaSuccess;
+    if (max_len > 0 && factored) {
+        const float fscale = (float)((double)sm_scale / ((double)cfg->r_q * d.rk) * 1.4426950408889634);
+        e = launch_decode_factored(d, cfg->r_q, batch, qf, qf_stride, qf_seq_stride, q_pos, kcache, vcache, capacity,
+                                   seq_len, max_len, fscale, p, part_o, part_ml, rope_table(cfg), err, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml, out_scale, out, st);
+        return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+    }
     if (max_len > 0 && p.variant >= 0) {
         DecodeArgs args;
         args.q = static_cast<const __nv_bfloat16 *>(q);
@@ -593,7 +606,7 @@ kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split,
 }
 
 kpa_status kpa_test_set_decode_engine(int32_t engine) {
-    if (engine < 0 || engine > 1) return KPA_ERR_INVALID_ARG;
+    if (engine < 0 || engine > 2) return KPA_ERR_INVALID_ARG;
     g_decode_engine.store(engine);
     return KPA_OK;
 }

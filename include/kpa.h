@@ -153,7 +153,8 @@ kpa_status kpa_decode_plan(const kpa_config *cfg, int32_t batch, int32_t max_len
                            int32_t *tokens_per_split_out, int32_t *launches);
 
 /* Which kernel a dense-query kpa_decode_split call with these arguments runs
- * (kpa_decode_qf always takes the mma.sync kernel):
+ * (kpa_decode_qf takes the mma.sync kernel, or the factored score after
+ * kpa_test_set_decode_engine(2)):
  *   KPA_DECODE_KERNEL_CUDA_CORES  fp32 caches or shapes without a tensor-core variant
  *   KPA_DECODE_KERNEL_MMA_SYNC    the bf16 tensor-core kernel on mma.sync
  *   KPA_DECODE_KERNEL_TCGEN05     TPA h = 16, d_h = 64, R_K = R_V = 2 after
@@ -310,8 +311,11 @@ kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split, uint
  * the TPA shape h = 16, d_h = 64, R_K = R_V = 2 on the tcgen05 kernel (both
  * products on tcgen05, accumulators in tensor memory; its splits merge through
  * global memory, never in a cluster); other shapes and kpa_decode_qf are
- * unaffected.  Process-wide; returns
- * KPA_ERR_INVALID_ARG for other values. */
+ * unaffected.  2 runs kpa_decode_qf on TPA shapes (h2 = 1, d1 = 1, d_h = 64, h <= 32,
+ * R_Q R_K <= 32, R_K and R_V <= 4, bf16) with the factored score of Proposition 2.2
+ * (the FlashTPA form: head-shared dots B^Q_r . B^K_r' per token, then a rank mix per
+ * head) on CUDA cores, its splits merged by the combine pass; other calls are
+ * unaffected.  Process-wide; returns KPA_ERR_INVALID_ARG for other values. */
 kpa_status kpa_test_set_decode_engine(int32_t engine);
 
 /* Wait for `stream`, then return in *code the per-device error word
