@@ -143,13 +143,19 @@ int cluster_capacity(int variant, int size) {
 
 // Split plan.  Auto splits aim at one wave of CTAs: ceil(sms * ctas_per_sm / batch)
 // pieces per sequence, each a multiple of 16 slots.
+// factored_rq > 0: the plan of the factored-score decode from query factors of that rank
 kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int tps_req, int sms,
-                       DecodePlan *p) {
+                       DecodePlan *p, int factored_rq = 0) {
     if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
-    p->variant = dt == KPA_BF16 && d.order != 3 ? mma_decode_variant(d) : -1;
+    p->variant = dt == KPA_BF16 && d.order != 3 && factored_rq == 0 ? mma_decode_variant(d) : -1;
     if (d.shared && p->variant < 0) return KPA_ERR_UNSUPPORTED;   // shared B: tensor-core variants only
     int ctas_per_sm = 2;
-    if (p->variant >= 0) {
+    if (factored_rq > 0) {
+        if (!factored_decode_supported(d, factored_rq)) return KPA_ERR_UNSUPPORTED;
+        p->tile = 32;
+        // latency-bound CUDA-core kernel: every CTA slot the occupancy query allows (up to 4)
+        ctas_per_sm = std::min(4, factored_ctas_per_sm(d, factored_rq));
+    } else if (p->variant >= 0) {
         p->tile = mma_decode_tile(p->variant);
         const size_t smem = mma_decode_smem(p->variant);
         ctas_per_sm = smem > 0 ? (int)((227 * 1024) / smem) : 1;
@@ -313,7 +319,14 @@ kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32
     DecodePlan p;
     s = plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
     if (s != KPA_OK) return s;
-    *bytes = batch == 0 ? 0 : p.bytes;
+    size_t need = p.bytes;
+    // with the factored-score engine selected, room for its plan too
+    if (g_decode_engine.load() == 2 && cfg->dtype == KPA_BF16 && factored_decode_supported(dims_of(cfg), cfg->r_q)) {
+        DecodePlan pf;
+        if (plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, tokens_per_split, sms, &pf, cfg->r_q) == KPA_OK)
+            need = std::max(need, pf.bytes);
+    }
+    *bytes = batch == 0 ? 0 : need;
     return KPA_OK;
 }
 
@@ -403,11 +416,17 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     const float out_scale = (float)(1.0 / (double)d.rv);
     cudaError_t e = cudaSuccess;
     if (max_len > 0 && factored) {
+        DecodePlan pf;
+        s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &pf, cfg->r_q);
+        if (s != KPA_OK) return s;
+        if (ws_bytes < pf.bytes) return KPA_ERR_WORKSPACE;
+        float *fo = reinterpret_cast<float *>(static_cast<char *>(workspace) + pf.part_o_off);
+        float *fml = reinterpret_cast<float *>(static_cast<char *>(workspace) + pf.part_ml_off);
         const float fscale = (float)((double)sm_scale / ((double)cfg->r_q * d.rk) * 1.4426950408889634);
         e = launch_decode_factored(d, cfg->r_q, batch, qf, qf_stride, qf_seq_stride, q_pos, kcache, vcache, capacity,
-                                   seq_len, max_len, fscale, p, part_o, part_ml, rope_table(cfg), err, st);
+                                   seq_len, max_len, fscale, pf, fo, fml, rope_table(cfg), err, st);
         if (e != cudaSuccess) return cuda_fail(e);
-        e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml, out_scale, out, st);
+        e = launch_decode_combine(d, batch, seq_len, max_len, pf, fo, fml, out_scale, out, st);
         return e == cudaSuccess ? KPA_OK : cuda_fail(e);
     }
     if (max_len > 0 && p.variant >= 0) {

@@ -74,7 +74,7 @@ struct FqLayout {
 };
 
 template <int DH, int NP_>
-__global__ void __launch_bounds__(kFqThreads) decode_factored_kernel(FactoredArgs a, RopeTable rope) {
+__global__ void __launch_bounds__(kFqThreads, 2) decode_factored_kernel(FactoredArgs a, RopeTable rope) {
     constexpr int JPL = DH / 32;                                  // features per lane
     const int H = a.h, RQ = a.rq, RK = a.rk, RV = a.rv, NP = NP_ ? NP_ : RQ * RK;
     const int EK = RK * (H + DH), EV = RV * (H + DH);
@@ -295,6 +295,22 @@ bool factored_decode_supported(const Dims &d, int rq) {
     return d.order == 2 && !d.shared && d.h2 == 1 && d.d1 == 1 && d.dh == 64 && d.h <= 8 * kFqMaxHpw && rq > 0 &&
            rq * d.rk <= kFqMaxPairs && d.rk <= kFqMaxR && d.rv <= kFqMaxR &&
            FqLayout(d.h, d.dh, rq, d.rk, d.rv).bytes <= 200 * 1024;
+}
+
+int factored_ctas_per_sm(const Dims &d, int rq) {
+    const size_t smem = FqLayout(d.h, d.dh, rq, d.rk, d.rv).bytes;
+    return with_factored_kernel(rq, d.rk, [&](auto kernel) -> int {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+            cudaGetLastError();
+            return 1;
+        }
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kFqThreads, smem) != cudaSuccess) {
+            cudaGetLastError();
+            return 1;
+        }
+        return n > 0 ? n : 1;
+    });
 }
 
 cudaError_t launch_decode_factored(const Dims &d, int rq, int batch, const float *qf, long long qf_stride,

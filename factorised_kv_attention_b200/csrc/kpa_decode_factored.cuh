@@ -9,6 +9,9 @@ namespace kpa {
 // h <= 32, R_Q R_K <= 32, R_K and R_V <= 4) with query rank rq.
 bool factored_decode_supported(const Dims &d, int rq);
 
+// CTAs of the kernel that one SM holds at once (occupancy query).
+int factored_ctas_per_sm(const Dims &d, int rq);
+
 // Unnormalised split partials (o, m, l) for launch_decode_combine.  qscale is
 // sm_scale / (R_Q R_K) * log2(e).
 cudaError_t launch_decode_factored(const Dims &d, int rq, int batch, const float *qf, long long qf_stride,

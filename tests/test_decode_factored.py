@@ -34,11 +34,12 @@ def _case(shape, batch, cap, seed, ragged=True):
 def _decode_qf(lib, w, cfg, kc, vc, inp, qf_dev, qf_stride, qf_seq_stride, engine, scale):
     L = inp["seq_len"]
     max_len = int(L.max())
-    ws = torch.zeros(max(lib.kpa_decode_workspace_size(cfg, w.batch, max_len), 256), dtype=torch.uint8,
-                     device="cuda")
     out = torch.full((w.batch, w.shape.h, w.shape.dh), float("nan"), dtype=torch.float32, device="cuda")
     lib.kpa_test_set_decode_engine(engine)
     try:
+        # sized with the engine selected: the factored score plans its own splits
+        ws = torch.zeros(max(lib.kpa_decode_workspace_size(cfg, w.batch, max_len), 256), dtype=torch.uint8,
+                         device="cuda")
         lib.kpa_decode_qf(cfg, w.batch, qf_dev, qf_stride, qf_seq_stride, inp["q_pos"].cuda(), kc, vc, w.capacity,
                           L.cuda(), max_len, scale, out, ws)
         torch.cuda.synchronize()
