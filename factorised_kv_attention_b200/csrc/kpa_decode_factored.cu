@@ -20,9 +20,12 @@
 // split combine merges the splits.
 #include "kpa_decode_factored.cuh"
 #include "kpa_internal.cuh"
+#include "kpa_sm100.cuh"
 
 namespace kpa {
 namespace {
+
+using sm100::cp_async16;
 
 constexpr int kFqThreads = 256;
 constexpr int kFqTile = 32;           // tokens per tile (4 groups)
@@ -43,10 +46,6 @@ struct FactoredArgs {
     float *part_o, *part_ml;
     int *err;
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 
 // element e of token t in a tile of 8-token groups at byte stride g; a bf16 widened by a shift
 __device__ __forceinline__ float tile_elem(const unsigned char *tile, int g, int t, int e) {

@@ -20,9 +20,12 @@
 // lane = output feature for the value accumulation.  Each CTA leaves an
 // unnormalised partial (o, m, l) per head; the split combine merges them.
 #include "kpa_internal.cuh"
+#include "kpa_sm100.cuh"
 
 namespace kpa {
 namespace {
+
+using sm100::cp_async16;
 
 constexpr int kO3Threads = 256;
 constexpr int kO3Tile = kOrder3Tile;  // tokens per tile (4 groups)
@@ -42,10 +45,6 @@ struct Order3Args {
     float *part_o, *part_ml;
     int *err;
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 
 // Shared memory: the query [h][d_h], the weights p a^V [h][R_V][32], the value outer
 // products b^V (x) c^V of a tile [R_V][8][d_h][4] (4 tokens per float4), the rotation
