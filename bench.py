@@ -336,9 +336,9 @@ def run_kpa(a):
         step(qs)
 
     # e2e graph: every layer's query comes from pinned host memory and every output goes
-    # back to it, each step.  The copies overlap the decodes on a side stream: layer 0's
-    # query first, the other layers' while layer 0 runs; each group of layers' outputs
-    # while the next group runs.
+    # back to it, each step.  The copies overlap the decodes on a side stream: the first
+    # two layers' queries first, the others' while those run; each group of layers'
+    # outputs while the next group runs, the last layers' one by one.
     q_host = q_all.cpu().pin_memory()
     out_host = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
     q_dev_all = torch.empty_like(q_all)
@@ -349,22 +349,25 @@ def run_kpa(a):
         kpa.kpa_decode_split(cfg, w.batch, q_dev_all[layer], q_pos, kcs[layer], vcs[layer], w.capacity,
                              seq_len, max_len, sm_scale, tps, outs[layer], ws, stream=stream)
 
+    head = min(2, layers)                         # layers whose queries go first
     graph_e2e = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_e2e, stream=stream):
-        q_dev_all[0].copy_(q_host[0], non_blocking=True)
+        q_dev_all[:head].copy_(q_host[:head], non_blocking=True)
         side.wait_stream(stream)
-        if layers > 1:
+        if layers > head:
             with torch.cuda.stream(side):
-                q_dev_all[1:].copy_(q_host[1:], non_blocking=True)
+                q_dev_all[head:].copy_(q_host[head:], non_blocking=True)
+        lo = 0
         for layer in range(layers):
-            if layer == 1:
+            if layer == head:
                 stream.wait_stream(side)          # the other layers' queries are in
             decode_layer(layer)
-            if (layer + 1) % group == 0 or layer == layers - 1:
-                lo = (layer // group) * group
+            # outputs in groups of `group` layers; the last two layers one by one
+            if (layer + 1) % group == 0 or layer >= layers - 3:
                 side.wait_stream(stream)
                 with torch.cuda.stream(side):
                     out_host[lo:layer + 1].copy_(out_all[lo:layer + 1], non_blocking=True)
+                lo = layer + 1
         stream.wait_stream(side)
 
     sampler = ClockSampler(local)
@@ -442,8 +445,9 @@ def run_kpa(a):
                     "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
                     "ms_per_step": ms_e2e,
                     "path": "pinned host queries -> device, kpa_decode x layers, outputs -> pinned host, every "
-                            "step, one CUDA graph; the copies overlap the decodes on a second stream (layer 0's "
-                            "query first, then the rest; outputs in groups of 4 layers)"},
+                            "step, one CUDA graph; the copies overlap the decodes on a second stream (the first "
+                            "two layers' queries first, then the rest; outputs in groups of 4 layers, the last "
+                            "ones singly)"},
             "clocks": clocks,
             "gpu_launches": a.steps * layers * kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[2]}
 
