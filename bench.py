@@ -420,9 +420,13 @@ def run_kpa(a):
                 "kernel": "kpa_decode (split + combine), per layer call",
                 "algorithmic_bytes_per_launch": layer_bytes,
                 "launch_us": t_launch * 1e6, "kernel_sources_sha": khash}
+    kind = kpa.kpa_decode_kernel_kind(cfg, w.batch, max_len, tps)
+    roofline["decode_kernel"] = kind
     if s.order == 3:
-        # a third-order record is too small for HBM to bound the decode: its FP32
-        # multiply-adds do (see _order3_flops_per_token)
+        roofline["algorithmic_flops_per_launch"] = tokens_per_layer * _order3_flops_per_token(s)
+    if s.order == 3 and kind == "cuda_cores":
+        # on the CUDA-core kernel a third-order record is too small for HBM to bound the
+        # decode: its FP32 multiply-adds do (see _order3_flops_per_token)
         flops = tokens_per_layer * _order3_flops_per_token(s)
         roofline = {"bound": "alu", "achieved": flops / t_launch / 1e12, "peak": FP32_PEAK_TFLOPS,
                     "unit": "TFLOP/s", "frac": flops / t_launch / 1e12 / FP32_PEAK_TFLOPS, "traffic": None,

@@ -147,7 +147,7 @@ int cluster_capacity(int variant, int size) {
 kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int tps_req, int sms,
                        DecodePlan *p, int factored_rq = 0) {
     if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
-    p->variant = dt == KPA_BF16 && d.order != 3 && factored_rq == 0 ? mma_decode_variant(d) : -1;
+    p->variant = dt == KPA_BF16 && factored_rq == 0 ? mma_decode_variant(d) : -1;
     if (d.shared && p->variant < 0) return KPA_ERR_UNSUPPORTED;   // shared B: tensor-core variants only
     int ctas_per_sm = 2;
     if (factored_rq > 0) {
@@ -401,7 +401,7 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     // kernel, which assembles the query (never a third-order cache)
     const bool factored = qf && g_decode_engine.load() == 2 && cfg->dtype == KPA_BF16 &&
                           factored_decode_supported(d, cfg->r_q);
-    if (qf && !factored && p.variant < 0) return KPA_ERR_UNSUPPORTED;
+    if (qf && (d.order == 3 || (!factored && p.variant < 0))) return KPA_ERR_UNSUPPORTED;
     if (qf && !factored && (int64_t)cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) > mma_decode_qf_max(p.variant))
         return KPA_ERR_UNSUPPORTED;                               // staged in the kernel's query rows
     if (!workspace || ws_bytes < p.bytes) return KPA_ERR_WORKSPACE;

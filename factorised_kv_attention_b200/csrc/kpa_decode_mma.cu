@@ -200,6 +200,18 @@ __device__ __forceinline__ uint32_t rotate_to_h2(uint32_t v, float2 w) {
     return r;
 }
 
+// (lo, hi) floats -> fp16x2 word, lo in the low half
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// bf16 element of one token in a group row (2-byte load), widened by a shift
+__device__ __forceinline__ float lds_bf16f(const unsigned char *p) {
+    return __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short *>(p) << 16);
+}
+
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
     return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
@@ -217,6 +229,14 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     constexpr int KBYTES = TT * EK * 2, STAGE_BYTES = C::STAGE_BYTES;
     constexpr int RED_LD = C::RED_LD;               // floats per token row of the j1 scratch
     constexpr int A_K = RK * MA, A_V = RV * MA;     // start of B in a key / value record
+    // third order: query pair i = (head, m, jc) -> its first feature (head, 2m, jc); the
+    // records' b and c factors start at A_K (A_V) and A_K + RK DB (A_V + RV DB)
+    auto o3_pair_feature = [](int i) {
+        constexpr int PH = (C::DB / 2) * C::DC;       // pairs per head
+        const int h = i / PH, rem = i % PH;
+        return h * DH + (rem / C::DC) * 2 * C::DC + rem % C::DC;
+    };
+    constexpr int C_K = A_K + RK * C::DB, C_V = A_V + RV * C::DB;
 
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *stage_base = smem;                                           // ring
@@ -270,7 +290,15 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
 #pragma unroll
         for (int k = 0; k < QPT; ++k) {
             const int i = tid + k * WARPS * 32;
-            if (i < H * DH / 2) qv[k] = qb[i];
+            if (i < H * DH / 2) {
+                if constexpr (C::ORDER3) {
+                    // third order: the RoPE pair of (head, m, c index) is features (2m DC + jc, + DC)
+                    const int e0 = o3_pair_feature(i);
+                    qv[k] = __halves2bfloat162(a.q[(size_t)b * H * DH + e0], a.q[(size_t)b * H * DH + e0 + C::DC]);
+                } else {
+                    qv[k] = qb[i];
+                }
+            }
         }
     }
     // query factors: the sequence's E_Q values (at most QF_PT per consumer thread) are
@@ -415,13 +443,24 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         if (i < H * DH / 2 && !a.qf) {
             const float2 x = __bfloat1622float2(qv[k]);
             float2 y = x;
-            if (rotate) {
-                const float2 w = cs[i % (D2 / 2)];
-                y = make_float2(x.x * w.x - x.y * w.y, x.x * w.y + x.y * w.x);
+            if constexpr (C::ORDER3) {
+                // R_{d_b}(q_pos) (x) I_{d_c}: pair m of the b index, for every c index
+                if (rotate) {
+                    const float2 w = cs[(i % ((C::DB / 2) * C::DC)) / C::DC];
+                    y = make_float2(x.x * w.x - x.y * w.y, x.x * w.y + x.y * w.x);
+                }
+                const int e = o3_pair_feature(i), qh = e / DH;
+                qs[qh * C::Q_LD + (e - qh * DH)] = y.x * a.qscale;
+                qs[qh * C::Q_LD + (e - qh * DH) + C::DC] = y.y * a.qscale;
+            } else {
+                if (rotate) {
+                    const float2 w = cs[i % (D2 / 2)];
+                    y = make_float2(x.x * w.x - x.y * w.y, x.x * w.y + x.y * w.x);
+                }
+                const int e = 2 * i, qh = e / DH;            // rows padded to Q_LD: no bank conflicts
+                *reinterpret_cast<float2 *>(qs + qh * C::Q_LD + (e - qh * DH)) =
+                    make_float2(y.x * a.qscale, y.y * a.qscale);
             }
-            const int e = 2 * i, qh = e / DH;                // rows padded to Q_LD: no bank conflicts
-            *reinterpret_cast<float2 *>(qs + qh * C::Q_LD + (e - qh * DH)) =
-                make_float2(y.x * a.qscale, y.y * a.qscale);
         }
     }
     if constexpr (C::SHARED) {
@@ -457,7 +496,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 const int j2 = ks * 16 + 2 * c + ((v & 2) ? 8 : 0);
                 const int i1 = row / D1, j1 = row % D1;
                 const float *src = qs + (i1 * H2 + i2) * C::Q_LD + j1 * D2 + j2;
-                if constexpr (C::SHARED)
+                if constexpr (C::SHARED || C::ORDER3)
                     split2h(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
                 else
                     split2(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
@@ -541,7 +580,20 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                     const unsigned char *grp = kg0 + (size_t)gi * EK * 16;
                     uint32_t bk[KS][2];
                     const int e_b = A_K + r * H2 * D2 + i2 * D2;
-                    if constexpr (KS % 2 == 0) {
+                    if constexpr (C::ORDER3) {
+                        // the key's features b (x) c of token g, as the B fragment: word 0 of
+                        // k-step ks holds features (2ks, 2c), (2ks, 2c+1), word 1 (2ks+1, 2c), (2ks+1, 2c+1)
+                        const unsigned char *tg = grp + 2 * g;
+                        const float c0 = lds_bf16f(tg + (size_t)(C_K + r * C::DC + 2 * c) * 16);
+                        const float c1 = lds_bf16f(tg + (size_t)(C_K + r * C::DC + 2 * c + 1) * 16);
+#pragma unroll
+                        for (int ks = 0; ks < KS; ++ks) {
+                            const float b0 = lds_bf16f(tg + (size_t)(A_K + r * C::DB + 2 * ks) * 16);
+                            const float b1 = lds_bf16f(tg + (size_t)(A_K + r * C::DB + 2 * ks + 1) * 16);
+                            bk[ks][0] = pack_h2(b0 * c0, b0 * c1);
+                            bk[ks][1] = pack_h2(b1 * c0, b1 * c1);
+                        }
+                    } else if constexpr (KS % 2 == 0) {
 #pragma unroll
                         for (int kp = 0; kp < KS / 2; ++kp)
                             ldsm_x4_t(smem_u32(grp + (size_t)(e_b + kp * 32 + lane) * 16), bk[2 * kp][0],
@@ -564,7 +616,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int ks = 0; ks < KS; ++ks) {
-                            if constexpr (C::SHARED) {
+                            if constexpr (C::SHARED || C::ORDER3) {
                                 mma16816h(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
                                 mma16816h(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
                             } else {
@@ -572,8 +624,8 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                                 mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
                             }
                         }
-                        if constexpr (C::SHARED) {
-                            // a valid token whose rotated factors left the fp16 range
+                        if constexpr (C::SHARED || C::ORDER3) {
+                            // a valid token whose fp16 key factors left the fp16 range
                             const int tk = tok0 + gi * 8 + 2 * c;
                             if ((tk < n_valid && !(isfinite(acc[0]) && isfinite(acc[2]))) ||
                                 (tk + 1 < n_valid && !(isfinite(acc[1]) && isfinite(acc[3]))))
@@ -714,22 +766,48 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         if (tk + 8 >= n_valid) { x2.x = 0.f; x3.x = 0.f; }
                         if (tk + 9 >= n_valid) { x2.y = 0.f; x3.y = 0.f; }
                     }
-                    split2(x0, pa_hi[mt][0], pa_lo[mt][0]);
-                    split2(x1, pa_hi[mt][1], pa_lo[mt][1]);
-                    split2(x2, pa_hi[mt][2], pa_lo[mt][2]);
-                    split2(x3, pa_hi[mt][3], pa_lo[mt][3]);
+                    if constexpr (C::ORDER3) {       // fp16 operands: the values' b (x) c are fp16
+                        split2h(x0, pa_hi[mt][0], pa_lo[mt][0]);
+                        split2h(x1, pa_hi[mt][1], pa_lo[mt][1]);
+                        split2h(x2, pa_hi[mt][2], pa_lo[mt][2]);
+                        split2h(x3, pa_hi[mt][3], pa_lo[mt][3]);
+                    } else {
+                        split2(x0, pa_hi[mt][0], pa_lo[mt][0]);
+                        split2(x1, pa_hi[mt][1], pa_lo[mt][1]);
+                        split2(x2, pa_hi[mt][2], pa_lo[mt][2]);
+                        split2(x3, pa_hi[mt][3], pa_lo[mt][3]);
+                    }
                 }
                 // B^V: the value record's B, or (shared) the key record's unrotated B
                 const int e_b = (C::SHARED ? A_K : A_V) + r * H2 * D2 + i2 * D2;
                 const unsigned char *b0p = C::SHARED ? kg0 : g0p;
                 const unsigned char *b1p = C::SHARED ? kg0 + (size_t)EK * 16 : g1p;
                 const int mat = lane >> 3, mrow = lane & 7;
+                // third order: c^V of feature g for this lane's tokens (2c, 2c+1 of both groups)
+                float2 cv0 = make_float2(0.f, 0.f), cv1 = cv0;
+                if constexpr (C::ORDER3) {
+                    cv0 = unpack_bf16x2(lds_u32(g0p + (size_t)(C_V + r * C::DC + g) * 16 + 4 * c));
+                    cv1 = unpack_bf16x2(lds_u32(g1p + (size_t)(C_V + r * C::DC + g) * 16 + 4 * c));
+                }
 #pragma unroll
                 for (int np = 0; np < NT / 2; ++np) {
                     const unsigned char *gp = (mat & 1) ? b1p : b0p;
                     uint32_t b00, b01, b10, b11;
-                    ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mrow) * 16), b00, b01,
-                            b10, b11);
+                    if constexpr (C::ORDER3) {
+                        // features 16 np + g (b index 2np) and 16 np + 8 + g (b index 2np + 1), c index g
+                        const int eb = A_V + r * C::DB + 2 * np;
+                        const float2 p00 = fmul2(unpack_bf16x2(lds_u32(g0p + (size_t)eb * 16 + 4 * c)), cv0);
+                        const float2 p01 = fmul2(unpack_bf16x2(lds_u32(g1p + (size_t)eb * 16 + 4 * c)), cv1);
+                        const float2 p10 = fmul2(unpack_bf16x2(lds_u32(g0p + (size_t)(eb + 1) * 16 + 4 * c)), cv0);
+                        const float2 p11 = fmul2(unpack_bf16x2(lds_u32(g1p + (size_t)(eb + 1) * 16 + 4 * c)), cv1);
+                        b00 = pack_h2(p00.x, p00.y);
+                        b01 = pack_h2(p01.x, p01.y);
+                        b10 = pack_h2(p10.x, p10.y);
+                        b11 = pack_h2(p11.x, p11.y);
+                    } else {
+                        ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mrow) * 16), b00, b01,
+                                b10, b11);
+                    }
                     if (tail) {
                         const int tk = tok0 + 2 * c;
                         b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
@@ -739,6 +817,13 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                     }
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
+                        if constexpr (C::ORDER3) {
+                            mma16816h(o[mt][2 * np], pa_hi[mt], b00, b01);
+                            mma16816h(o[mt][2 * np], pa_lo[mt], b00, b01);
+                            mma16816h(o[mt][2 * np + 1], pa_hi[mt], b10, b11);
+                            mma16816h(o[mt][2 * np + 1], pa_lo[mt], b10, b11);
+                            continue;
+                        }
                         mma16816(o[mt][2 * np], pa_hi[mt], b00, b01);
                         mma16816(o[mt][2 * np], pa_lo[mt], b00, b01);
                         mma16816(o[mt][2 * np + 1], pa_hi[mt], b10, b11);
@@ -751,6 +836,18 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
         if (flags[0]) { aborted = true; break; }
+    }
+
+    if constexpr (C::ORDER3) {
+        // the values' fp16 features b (x) c: an overflow makes the partial non-finite
+        bool fin = true;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) fin = fin && isfinite(o[mt][nt][v]);
+        if (!fin) raise_error(a.err, kErrDeviceCheck);
     }
 
     // l: complete sums per head

@@ -44,14 +44,20 @@ struct DecodeArgs {
 //   CHUNKS  16-token chunks per warp per stage, STAGES ring depth,
 //   SHARED  one B for keys and values: key record [A^K | B] (B unrotated, rotated in
 //           the kernel for the score), value record [A^V].
+//   DB      > 0: a third-order TPA cache (h = MA heads, d1 = 1, d2 = d_h = DB * DC):
+//           records [a | b | c] with b in R^DB, c in R^DC, and the keys' features
+//           b (x) c formed in registers as fp16 for both products.
 template <int MA_, int D1_, int D2_, int RK_, int RV_, int H2_, int SLICES_, int CHUNKS_, int STAGES_,
-          bool SHARED_ = false>
+          bool SHARED_ = false, int DB_ = 0>
 struct MmaDecodeCfg {
     static constexpr int MA = MA_, D1 = D1_, D2 = D2_, RK = RK_, RV = RV_, H2 = H2_;
     static constexpr int SLICES = SLICES_, CHUNKS = CHUNKS_, STAGES = STAGES_;
     static constexpr bool SHARED = SHARED_;
+    static constexpr bool ORDER3 = DB_ > 0;
+    static constexpr int DB = ORDER3 ? DB_ : 1, DC = ORDER3 ? D2_ / DB : D2_;
     static constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
-    static constexpr int EK = RK * (MA + H2 * D2), EV = SHARED ? RV * MA : RV * (MA + H2 * D2);
+    static constexpr int EK = ORDER3 ? RK * (MA + DB + DC) : RK * (MA + H2 * D2);
+    static constexpr int EV = ORDER3 ? RV * (MA + DB + DC) : SHARED ? RV * MA : RV * (MA + H2 * D2);
     static constexpr int WARPS = H2 * SLICES;
     static constexpr int TT = 16 * CHUNKS * SLICES;             // tokens per stage
     static constexpr int STAGE_BYTES = TT * (EK + EV) * 2;
@@ -87,6 +93,8 @@ struct MmaDecodeCfg {
                   "slice merge and merged partial must fit in the ring");
     static_assert(WARPS <= 31, "too many consumer warps");
     static_assert(smem_bytes() <= 227 * 1024, "shared memory");
+    static_assert(!ORDER3 || (D1 == 1 && H2 == 1 && !SHARED && DB == 8 && DC == 8),
+                  "third-order mode: TPA split, d_b = d_c = 8 (one c pair per fragment lane)");
 };
 
 // TPA, h = 16, d_h = 64, R_K = R_V = 2 (the degenerate split h1 = h, d1 = 1, h2 = 1).
@@ -103,6 +111,8 @@ using MmaKpaH4x8D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 8, 1, 2, 2>;
 using MmaKpaH4x8D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 8, 1, 4, 2>;
 // KPA h = 4x4, d_h = 8x16, R_K = R_V = 2.
 using MmaKpaH4x4D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2>;
+// Third-order TPA, h = 16, d_h = 8 x 8, R_K = R_V = 2.
+using MmaTpa3H16D8x8R2 = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2, false, 8>;
 
 #define KPA_MMA_VARIANTS(X)        \
     X(0, MmaTpaH16D64R2)           \
@@ -111,13 +121,16 @@ using MmaKpaH4x4D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2>;
     X(3, MmaKpaH4x4D8x16R2)        \
     X(4, MmaTpaH32D64R1)           \
     X(5, MmaTpaH16D64R2Shared)     \
-    X(6, MmaKpaH4x4D8x16R2Shared)
+    X(6, MmaKpaH4x4D8x16R2Shared)  \
+    X(7, MmaTpa3H16D8x8R2)
 
 // Index of the variant that covers these dims, or -1.
 inline int mma_decode_variant(const Dims &d) {
-#define KPA_MMA_MATCH(IDX, CFG)                                                            \
-    if (d.h1 * d.d1 == CFG::MA && d.d1 == CFG::D1 && d.d2 == CFG::D2 && d.rk == CFG::RK && \
-        d.rv == CFG::RV && d.h2 == CFG::H2 && (d.shared != 0) == CFG::SHARED)                \
+#define KPA_MMA_MATCH(IDX, CFG)                                                                    \
+    if (d.rk == CFG::RK && d.rv == CFG::RV &&                                                      \
+        (CFG::ORDER3 ? (d.order == 3 && d.h1 == CFG::MA && d.h2 == 1 && d.d1 == CFG::DB && d.d2 == CFG::DC) \
+                     : (d.order != 3 && d.h1 * d.d1 == CFG::MA && d.d1 == CFG::D1 && d.d2 == CFG::D2 &&  \
+                        d.h2 == CFG::H2 && (d.shared != 0) == CFG::SHARED)))                       \
         return IDX;
     KPA_MMA_VARIANTS(KPA_MMA_MATCH)
 #undef KPA_MMA_MATCH

@@ -96,7 +96,7 @@ def test_order3_special_lengths_and_splits():
     inp["q_pos"] = inp["seq_len"].clone()
     lib = kpa()
     cfg, kc, vc = fill_cache(lib, w, inp)
-    assert lib.kpa_decode_kernel_kind(cfg, w.batch, 1024) == "cuda_cores"
+    assert lib.kpa_decode_kernel_kind(cfg, w.batch, 1024) == "mma_sync"   # the d_b = d_c = 8 variant
     outs = []
     for tps in (0, 64, 256, 1024):
         out = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"], max_len=1024,
