@@ -56,6 +56,8 @@ def _args(argv=None):
                     help="tpa_decode | tpa_shared | tpa_order3 | kpa_medium | kpa_long | tiny_kpa | flashtpa | "
                          "append_prefill")
     ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
+    ap.add_argument("--decode-engine", type=int, default=0, choices=(0, 1),
+                    help="1: the opt-in tcgen05 decode for the TPA shape h=16, d_h=64, R=2 (measurement)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override: fixed length (profiling)")
@@ -291,6 +293,7 @@ def run_kpa(a):
     layers = a.layers or max(1, int(np.ceil(4 * l2 / max(layer_bytes, 1))))
     cfg = kpa.make_config(s, w.dtype)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    kpa.kpa_test_set_decode_engine(a.decode_engine)
 
     # per-layer caches, filled through kpa_append_factors (slot = position)
     kcs, vcs = [], []
@@ -413,7 +416,7 @@ def run_kpa(a):
     achieved = layer_bytes / t_launch / 1e9
     peak, peak_kind = _hbm_peak()
     khash = _kernel_hash()
-    traffic_workload = a.workload if not (a.seq_len or a.batch or a.tokens_per_split) else None
+    traffic_workload = a.workload if not (a.seq_len or a.batch or a.tokens_per_split or a.decode_engine) else None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": _traffic(khash, traffic_workload),
                 "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
