@@ -9,9 +9,11 @@
 //   score   = sum_r a^K_r[h] sum_jb b~_r[jb] sum_jc Qs[h, jb d_c + jc] c_r[jc]
 //   values  O[h, (jb, jc)] += sum_r (p[h] a^V_r[h]) b^V_r[jb] c^V_r[jc]
 // where Qs is the query rotated by R_{d_b}(q_pos) (x) I_{d_c} and scaled by
-// sm_scale / R_K * log2(e).  The products are far too small for the tensor cores
-// (a d_b x d_c bilinear form per head and a rank-R_V outer-product update), so the
-// kernel is bound by FP32 issue, not by HBM: a record is R (h + d_b + d_c) numbers.
+// sm_scale / R_K * log2(e).  This kernel computes them as written, on the CUDA cores
+// (a d_b x d_c bilinear form per head and a rank-R_V outer-product update), for the
+// shapes and element types the tensor-core decode does not take: d_b = d_c = 8 in bf16
+// runs there instead, with the features b (x) c formed in registers.  Here the FP32
+// work, not HBM, bounds the decode: a record is only R (h + d_b + d_c) numbers.
 //
 // One CTA per (split, sequence), 8 warps.  A tile of 32 tokens (4 cache groups)
 // is copied with cp.async into shared memory at a padded group stride, double
