@@ -133,3 +133,33 @@ def test_order3_full_size_sampled_heads():
     g = got.reshape(w.batch * s.h, -1)[flat]
     wv = want.reshape(w.batch * s.h, -1)[flat]
     assert_close(w.dtype, g, wv, "full size, sampled heads")
+
+
+@pytest.mark.parametrize("mode", ["peaked_q", "peaked_scale", "zero_q", "prerotated"])
+def test_order3_softmax_edges(mode):
+    """Logit gaps far above 10 (q x 64, exact in bf16; or sm_scale x 64), a zero query (the
+    mean of the values) and a query used as given (q_pos = NULL), on the tensor-core variant
+    and on the CUDA-core kernel (another shape).  Stage parity: the oracle reads the cache the
+    GPU wrote, so a x64 scale does not also amplify the rounding at the cache write."""
+    lib = kpa()
+    for w in (SMALL["h16_8x8"], SMALL["h12_4x3_r3"]):
+        inp = decode_inputs(w)
+        sm_scale = 1.0 / np.sqrt(w.shape.dh)
+        if mode == "peaked_q":
+            inp["q"] = inp["q"] * 64
+        elif mode == "peaked_scale":
+            sm_scale *= 64
+        elif mode == "zero_q":
+            inp["q"] = torch.zeros_like(inp["q"])
+        q_pos = None if mode == "prerotated" else inp["q_pos"]
+        cfg, kc, vc = fill_cache(lib, w, inp)
+        out = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], q_pos, sm_scale=float(sm_scale))
+        torch.cuda.synchronize()
+        assert lib.kpa_read_device_error() == 0
+        s = w.shape
+        kn = to_f64(natural(kc.cpu(), w.batch, w.capacity, s.e_k))
+        vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
+        want = oracle.decode_order3(s, to_f64(inp["q"]), kn, vn, inp["seq_len"].numpy(),
+                                    q_pos=None if q_pos is None else q_pos.numpy(), keys_rotated=True,
+                                    sm_scale=sm_scale)
+        assert_close(w.dtype, out.cpu().numpy(), want, f"{mode} {w.shape}")
