@@ -56,8 +56,11 @@ def _args(argv=None):
                     help="tpa_decode | tpa_shared | tpa_order3 | kpa_medium | kpa_long | tiny_kpa | flashtpa | "
                          "append_prefill")
     ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
-    ap.add_argument("--decode-engine", type=int, default=0, choices=(0, 1),
-                    help="1: the opt-in tcgen05 decode for the TPA shape h=16, d_h=64, R=2 (measurement)")
+    ap.add_argument("--decode-engine", type=int, default=0, choices=(0, 1, 2),
+                    help="1: the opt-in tcgen05 decode for the TPA shape h=16, d_h=64, R=2; 2: the factored "
+                         "score on CUDA cores (with --query-factors) (measurement)")
+    ap.add_argument("--query-factors", action="store_true",
+                    help="decode from the query's factors (kpa_decode_qf) instead of a dense query")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override: fixed length (profiling)")
@@ -68,6 +71,12 @@ def _args(argv=None):
                     help="untimed load before timing while clocks are sampled (0 for profiling)")
     a = ap.parse_args(argv)
     a.warmup = max(a.warmup, 3)
+    if a.decode_engine == 1 and a.query_factors:
+        ap.error("--decode-engine 1 (tcgen05) takes dense queries only")
+    if a.decode_engine == 2 and not a.query_factors:
+        ap.error("--decode-engine 2 (the factored score) needs --query-factors")
+    if a.query_factors and a.tokens_per_split:
+        ap.error("--query-factors takes the library's split (no --tokens-per-split)")
     return a
 
 
@@ -214,12 +223,16 @@ def _config_json(w, layers, lens, world):
             "accumulate": "fp32"}
 
 
-def _cpu_baseline(w, inp, seconds, steps=None):
-    """The float64 oracle, as it stands, on whole sequences of the workload."""
+def _cpu_baseline(w, inp, seconds, steps=None, q_factors=None):
+    """The float64 oracle, as it stands, on whole sequences of the workload.  With
+    q_factors ([B][E_Q]) the query is assembled from them first (eq 2 for Q)."""
     import oracle
     from workloads import to_f64
     oracle.build()
     q, kf, vf = to_f64(inp["q"]), to_f64(inp["kf"]), to_f64(inp["vf"])
+    if q_factors is not None:
+        s = w.shape
+        q = np.stack([oracle.reconstruct(s.h1, s.h2, s.d1, s.d2, s.r_q, f) for f in to_f64(q_factors)])
     L, qp = inp["seq_len"].numpy(), inp["q_pos"].numpy()
     cores = oracle.max_threads()
     done_tokens, t_total, n_seq, times = 0, 0.0, 0, []
@@ -281,10 +294,13 @@ def run_kpa(a):
                                 device_id=dev)
 
     import factorised_kv_attention_b200 as kpa
-    from workloads import decode_inputs
+    from workloads import decode_inputs, query_factor_inputs
 
     w = _workload(a.workload, a)
     s = w.shape
+    qf_mode = a.query_factors            # the query as its factors, through kpa_decode_qf
+    if qf_mode and s.r_q <= 0:
+        raise SystemExit(f"--query-factors: the {a.workload} shape has no query factors (r_q = 0)")
     elt = 2 if w.dtype == "bf16" else 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     first = decode_inputs(w.replace(seed=rank_seed(rank)))
@@ -299,7 +315,8 @@ def run_kpa(a):
     kcs, vcs = [], []
     # every layer's query and output are views of one buffer each, so a step's inputs
     # and results move between host and device in one copy each way
-    q_all = torch.empty(layers, w.batch, s.h, s.dh, dtype=tdt, device=dev)
+    q_all = (torch.empty(layers, w.batch, s.e_q, dtype=torch.float32, device=dev) if qf_mode
+             else torch.empty(layers, w.batch, s.h, s.dh, dtype=tdt, device=dev))
     out_all = torch.empty(layers, w.batch, s.h, s.dh, dtype=torch.float32, device=dev)
     qs = [q_all[layer] for layer in range(layers)]
     outs = [out_all[layer] for layer in range(layers)]
@@ -314,7 +331,7 @@ def run_kpa(a):
                                start, w.capacity, kc, vc)
         kcs.append(kc)
         vcs.append(vc)
-        qs[layer].copy_(inp["q"].to(dev))
+        qs[layer].copy_((query_factor_inputs(w, rank_seed(rank, layer)) if qf_mode else inp["q"]).to(dev))
         del inp
     max_len = int(lens.max())
     tps = a.tokens_per_split
@@ -325,10 +342,17 @@ def run_kpa(a):
 
     stream = torch.cuda.Stream(device=dev)
 
+    def decode(q_layer, layer):
+        if qf_mode:   # factor records [batch][E_Q]: element stride 1, sequence stride E_Q
+            kpa.kpa_decode_qf(cfg, w.batch, q_layer, 1, s.e_q, q_pos, kcs[layer], vcs[layer], w.capacity,
+                              seq_len, max_len, sm_scale, outs[layer], ws, stream=stream)
+        else:
+            kpa.kpa_decode_split(cfg, w.batch, q_layer, q_pos, kcs[layer], vcs[layer], w.capacity,
+                                 seq_len, max_len, sm_scale, tps, outs[layer], ws, stream=stream)
+
     def step(qsrc):
         for layer in range(layers):
-            kpa.kpa_decode_split(cfg, w.batch, qsrc[layer], q_pos, kcs[layer], vcs[layer], w.capacity,
-                                 seq_len, max_len, sm_scale, tps, outs[layer], ws, stream=stream)
+            decode(qsrc[layer], layer)
 
     # warm up eagerly once (also sets kernel attributes), then capture the step
     with torch.cuda.stream(stream):
@@ -349,8 +373,7 @@ def run_kpa(a):
     group = 4
 
     def decode_layer(layer):
-        kpa.kpa_decode_split(cfg, w.batch, q_dev_all[layer], q_pos, kcs[layer], vcs[layer], w.capacity,
-                             seq_len, max_len, sm_scale, tps, outs[layer], ws, stream=stream)
+        decode(q_dev_all[layer], layer)
 
     head = min(2, layers)                         # layers whose queries go first
     graph_e2e = torch.cuda.CUDAGraph()
@@ -416,7 +439,8 @@ def run_kpa(a):
     achieved = layer_bytes / t_launch / 1e9
     peak, peak_kind = _hbm_peak()
     khash = _kernel_hash()
-    traffic_workload = a.workload if not (a.seq_len or a.batch or a.tokens_per_split or a.decode_engine) else None
+    traffic_workload = (a.workload if not (a.seq_len or a.batch or a.tokens_per_split or a.decode_engine
+                                           or qf_mode) else None)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": _traffic(khash, traffic_workload),
                 "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
@@ -424,6 +448,12 @@ def run_kpa(a):
                 "algorithmic_bytes_per_launch": layer_bytes,
                 "launch_us": t_launch * 1e6, "kernel_sources_sha": khash}
     kind = kpa.kpa_decode_kernel_kind(cfg, w.batch, max_len, tps)
+    plan = kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)
+    if qf_mode:
+        roofline["kernel"] = "kpa_decode_qf (query factors; split + combine), per layer call"
+        if a.decode_engine == 2:
+            # the factored score plans its own splits and always ends with the combine kernel
+            kind, plan = "factored_score_cuda_cores", (None, None, 2 if max_len > 0 else 1)
     roofline["decode_kernel"] = kind
     if s.order == 3:
         roofline["algorithmic_flops_per_launch"] = tokens_per_layer * _order3_flops_per_token(s)
@@ -444,22 +474,25 @@ def run_kpa(a):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
             if w.dtype == "bf16" else "f32", "data": "synthetic (seeded, shapes of the pages' workloads)",
             "config": dict(_config_json(w, layers, lens, world),
-                           splits_per_sequence=kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[0],
-                           tokens_per_split=kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[1]),
+                           splits_per_sequence=plan[0], tokens_per_split=plan[1],
+                           query="factors [batch][E_Q] float32 (kpa_decode_qf)" if qf_mode
+                           else "dense [batch][h][d_h]"),
             "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
                     "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
                     "ms_per_step": ms_e2e,
-                    "path": "pinned host queries -> device, kpa_decode x layers, outputs -> pinned host, every "
+                    "path": f"pinned host queries -> device, {'kpa_decode_qf' if qf_mode else 'kpa_decode'} x "
+                            "layers, outputs -> pinned host, every "
                             "step, one CUDA graph; the copies overlap the decodes on a second stream (the first "
                             "two layers' queries first, then the rest; outputs in groups of 4 layers, the last "
                             "ones singly)"},
             "clocks": clocks,
-            "gpu_launches": a.steps * layers * kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)[2]}
+            "gpu_launches": a.steps * layers * plan[2]}
 
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        base, _ = _cpu_baseline(w, first, a.cpu_seconds)
+        base, _ = _cpu_baseline(w, first, a.cpu_seconds,
+                                q_factors=query_factor_inputs(w, rank_seed(rank, 0)) if qf_mode else None)
         line["cpu_baseline"] = base
     del graph, graph_e2e
     if world > 1:

@@ -204,7 +204,10 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
         const int want_split = over_split ? over_split : cluster_auto ? c : per_seq;
         const int64_t want = ((int64_t)max_len + want_split - 1) / want_split;
         tps = (int)(((want + 15) / 16) * 16);
-        if (tps < 64) tps = 64;
+        // the generic CUDA-core kernel walks its split tile by tile through latency
+        // chains, so a short sequence goes faster over more SMs: splits down to 16 slots
+        const int tps_floor = p->variant < 0 && d.order != 3 && factored_rq == 0 ? 16 : 64;
+        if (tps < tps_floor) tps = tps_floor;
         // whole tiles per split (no ragged last tile) when that keeps most of the splits
         if (p->variant >= 0 && p->tile > 0) {
             const int whole = (tps + p->tile - 1) / p->tile * p->tile;

@@ -101,6 +101,33 @@ def test_special_lengths():
     assert_bf16_close(got[1:], want[1:], "ragged tails")
 
 
+def test_cuda_core_kernel_short_splits():
+    """The CUDA-core kernel's own plan splits short sequences down to 16 slots (the fp32
+    configuration: 256 slots over 16 CTAs).  Tails around a split's end and the last
+    split's absorbed remainder (up to a quarter of a split) against the oracle in fp32,
+    and against a user split of 64 slots."""
+    w = TINY_KPA.replace(batch=10, seed=8)
+    inp = decode_inputs(w)
+    inp["seq_len"] = torch.tensor([0, 1, 15, 16, 17, 20, 21, 33, 100, 256], dtype=torch.int32)
+    inp["q_pos"] = inp["seq_len"].clone()
+    lib = kpa()
+    cfg, kc, vc = fill_cache(lib, w, inp)
+    assert lib.kpa_decode_kernel_kind(cfg, w.batch, 256) == "cuda_cores"
+    n_split, tps, _ = lib.kpa_decode_plan(cfg, 1, 256)
+    assert (n_split, tps) == (16, 16)
+    outs = []
+    for split in (0, 64):
+        out = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"], max_len=256,
+                         tokens_per_split=split)
+        torch.cuda.synchronize()
+        assert lib.kpa_read_device_error() == 0
+        outs.append(out.cpu().numpy())
+    assert np.all(outs[0][0] == 0.0)
+    want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"])
+    assert_f32_close(outs[0][1:], want[1:], "16-slot splits")
+    assert_f32_close(outs[1][1:], want[1:], "64-slot splits")
+
+
 def test_zero_query_gives_the_mean():
     w = SMALL["tpa"]
     inp = decode_inputs(w)

@@ -226,6 +226,19 @@ def decode_inputs(w: DecodeWorkload) -> dict:
     }
 
 
+def query_factor_inputs(w: DecodeWorkload, seed: int) -> torch.Tensor:
+    """Seeded query factor records [B][E_Q], float32 ([A^Q_0..A^Q_{R_Q-1} | B^Q_0..],
+    unrotated), each element ~ N(0, sigma^2) with sigma^2 = q_std sqrt(R_Q): the
+    assembled query (1/R_Q) sum_r A^Q_r (x) B^Q_r then has the dense query's spread
+    q_std per element."""
+    s = w.shape
+    if s.r_q <= 0:
+        raise ValueError("the shape has no query factors (r_q = 0)")
+    rng = np.random.default_rng([seed, 7])
+    sigma = np.float32(np.sqrt(w.q_std * np.sqrt(s.r_q)))
+    return torch.from_numpy(rng.standard_normal((w.batch, s.e_q), dtype=np.float32) * sigma)
+
+
 def append_inputs(w: AppendWorkload) -> dict:
     """x [B][n][d_model] and W [N][d_model] (bf16), the decode-step x [B][1][d_model]
     and int32 ``start_pos`` [B]."""
