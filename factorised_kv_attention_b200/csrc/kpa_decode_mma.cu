@@ -87,6 +87,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// hint a global range (16-byte aligned, a multiple of 16 bytes) into L2.  No data is
+// bound to the issuing thread, and L2 stays coherent with later writes to the range.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                         uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -232,9 +238,10 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     // third order: query pair i = (head, m, jc) -> its first feature (head, 2m, jc); the
     // records' b and c factors start at A_K (A_V) and A_K + RK DB (A_V + RV DB)
     auto o3_pair_feature = [](int i) {
-        constexpr int PH = (C::DB / 2) * C::DC;       // pairs per head
+        constexpr int DCN = C::ORDER3 ? C::DC : 1;     // (1 keeps other shapes' unused copy defined)
+        constexpr int PH = C::ORDER3 ? (C::DB / 2) * C::DC : 1;   // pairs per head
         const int h = i / PH, rem = i % PH;
-        return h * DH + (rem / C::DC) * 2 * C::DC + rem % C::DC;
+        return h * DH + (rem / DCN) * 2 * DCN + rem % DCN;
     };
     constexpr int C_K = A_K + RK * C::DB, C_V = A_V + RV * C::DB;
 
@@ -256,6 +263,21 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         }
         flags[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // Ahead of the dependency on the previous grid: hint this CTA's first ring of tiles
+    // into L2.  A prefetch binds no data and L2 stays coherent with anything the
+    // previous grid still writes, so it reads no input early; the cache streams in
+    // while the previous call finishes (its split merge).  Only kernel parameters are
+    // used here.  Slots [p0, p1) clipped to max_len, rounded up to whole 8-slot groups,
+    // stay inside the cache (capacity >= max_len, a multiple of 8).
+    if (tid == 0) {
+        const int p0 = split * a.tps;
+        const int p1 = min(p0 + STAGES * TT, a.max_len);
+        if (p1 > p0) {
+            const uint32_t groups = (uint32_t)((p1 - p0 + kGroup - 1) / kGroup);
+            bulk_prefetch_l2(a.kc + ((size_t)b * a.cap + p0) * EK, groups * EK * kGroup * 2);
+            bulk_prefetch_l2(a.vc + ((size_t)b * a.cap + p0) * EV, groups * EV * kGroup * 2);
+        }
     }
     // launched with programmatic stream serialization: wait for the previous grid in
     // the stream before reading any input, and let the next grid be scheduled now
@@ -973,16 +995,16 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();
     if (warp < WARPS) {
-        const int C = (int)cl.num_blocks(), rank = (int)cl.block_rank();
-        const int per = (H * DH + C - 1) / C;
+        const int n_cl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+        const int per = (H * DH + n_cl - 1) / n_cl;
         const int lo = rank * per, hi = min(H * DH, lo + per);
         float *cpl = reinterpret_cast<float *>(smem) + SLICES * H * C::MO_LD + SLICES * H * 2;
         for (int idx = lo + tid; idx < hi; idx += WARPS * 32) {
             const int head = idx / DH;
             float M = -INFINITY;
-            for (int r = 0; r < C; ++r) M = fmaxf(M, cl.map_shared_rank(cpl, r)[H * DH + head]);
+            for (int r = 0; r < n_cl; ++r) M = fmaxf(M, cl.map_shared_rank(cpl, r)[H * DH + head]);
             float num = 0.f, den = 0.f;
-            for (int r = 0; r < C; ++r) {
+            for (int r = 0; r < n_cl; ++r) {
                 const float *rp = cl.map_shared_rank(cpl, r);
                 const float m = rp[H * DH + head];
                 const float w = m == -INFINITY ? 0.f : exp2f(m - M);
