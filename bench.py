@@ -52,10 +52,11 @@ def _args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kpa", "reference"], default="kpa")
-    ap.add_argument("--workload", default="tpa_decode",
+    ap.add_argument("--workload", default="kpa_long",
                     help="tpa_decode | tpa_shared | tpa_order3 | kpa_medium | kpa_long | tiny_kpa | flashtpa | "
                          "append_prefill")
-    ap.add_argument("--layers", type=int, default=0, help="0 = enough layers to exceed 4 x L2")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="0 = enough layer caches to exceed 4 x L2 (at least 2)")
     ap.add_argument("--decode-engine", type=int, default=0, choices=(0, 1, 2),
                     help="1: the opt-in tcgen05 decode for the TPA shape h=16, d_h=64, R=2; 2: the factored "
                          "score on CUDA cores (with --query-factors) (measurement)")
@@ -67,6 +68,9 @@ def _args(argv=None):
     ap.add_argument("--batch", type=int, default=0, help="override: batch (profiling)")
     ap.add_argument("--tokens-per-split", type=int, default=0,
                     help="override the library's split of each sequence (profiling; multiple of 64)")
+    ap.add_argument("--sweep", choices=["flashtpa"], default=None,
+                    help="flashtpa: the FlashTPA decoding shape over sequence lengths 2^12..2^19 and batch "
+                         "1, 2, 4, 8, 16 (one JSON line per point, then none of the other lines)")
     ap.add_argument("--settle-seconds", type=float, default=1.0,
                     help="untimed load before timing while clocks are sampled (0 for profiling)")
     a = ap.parse_args(argv)
@@ -131,16 +135,17 @@ def _hbm_peak():
 
 
 def _traffic(kernel_hash, workload):
-    """DRAM bytes per launch from the committed ncu record, when it was taken on this
+    """DRAM bytes per launch from the committed ncu records, when one was taken on this
     workload and on the current decode sources (else None)."""
     try:
         with open(TRAFFIC) as f:
             t = json.load(f)
     except Exception:
         return None
-    if t.get("kernel_sources_sha") != kernel_hash or t.get("workload") != workload:
-        return None
-    return t.get("dram_bytes_per_launch")
+    for r in t.get("records", []):
+        if r.get("kernel_sources_sha") == kernel_hash and r.get("workload") == workload:
+            return r.get("dram_bytes_per_launch")
+    return None
 
 
 class ClockSampler:
@@ -223,38 +228,77 @@ def _config_json(w, layers, lens, world):
             "accumulate": "fp32"}
 
 
-def _cpu_baseline(w, inp, seconds, steps=None, q_factors=None):
-    """The float64 oracle, as it stands, on whole sequences of the workload.  With
-    q_factors ([B][E_Q]) the query is assembled from them first (eq 2 for Q)."""
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def _cpu_baseline(w, inp, seconds, steps=None, q_factors=None, call_seconds=2.5, single_thread=True):
+    """The float64 oracle, as it stands, on the workload's sequences.  A call decodes one
+    sequence's query over its first n slots: the whole sequence when that fits in about
+    call_seconds, else a prefix of it sized from a first short call (the work per slot
+    is the same).  Calls run over the sequences in turn until `seconds` have passed (or
+    `steps` calls); then, unless single_thread is False, the same for a share of the time
+    on one core.  With q_factors ([B][E_Q]) the query is assembled from them first (eq 2
+    for Q).  Returns the line's cpu_baseline object and the per-call times (all cores)."""
     import oracle
     from workloads import to_f64
     oracle.build()
-    q, kf, vf = to_f64(inp["q"]), to_f64(inp["kf"]), to_f64(inp["vf"])
-    if q_factors is not None:
-        s = w.shape
-        q = np.stack([oracle.reconstruct(s.h1, s.h2, s.d1, s.d2, s.r_q, f) for f in to_f64(q_factors)])
+    s = w.shape
     L, qp = inp["seq_len"].numpy(), inp["q_pos"].numpy()
-    cores = oracle.max_threads()
-    done_tokens, t_total, n_seq, times = 0, 0.0, 0, []
-    b = 0
-    while (steps is None and t_total < seconds) or (steps is not None and len(times) < steps):
+    if q_factors is not None:
+        qf64 = to_f64(q_factors)
+        q_of = lambda b: oracle.reconstruct(s.h1, s.h2, s.d1, s.d2, s.r_q, qf64[b])[None]   # noqa: E731
+    else:
+        q_of = lambda b: to_f64(inp["q"][b:b + 1])                                        # noqa: E731
+    fn = oracle.decode_order3 if s.order == 3 else oracle.decode_shared_b if s.shared_b else oracle.decode
+
+    def call(b, n):
+        q = q_of(b)
+        kf, vf = to_f64(inp["kf"][b:b + 1, :n]), to_f64(inp["vf"][b:b + 1, :n])
         t0 = time.perf_counter()
-        if w.shape.order == 3:   # third-order records [a | b | c], RoPE on b
-            oracle.decode_order3(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1], q_pos=qp[b:b + 1])
-        elif w.shape.shared_b:   # one B for keys and values: value records are A^V only
-            oracle.decode_shared_b(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1],
-                                   q_pos=qp[b:b + 1])
-        else:
-            oracle.decode(w.shape, q[b:b + 1], kf[b:b + 1], vf[b:b + 1], L[b:b + 1], q_pos=qp[b:b + 1])
-        dt = time.perf_counter() - t0
-        times.append(dt)
-        t_total += dt
-        done_tokens += int(L[b])
-        n_seq += 1
-        b = (b + 1) % w.batch
-    return {"value": done_tokens / t_total, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n_seq} whole sequences (all {w.shape.h} heads) of one layer of the "
-                      f"workload, float64 C oracle, OpenMP over heads, {t_total:.1f} s"}, times
+        fn(s, q, kf, vf, np.array([n], dtype=np.int32), q_pos=qp[b:b + 1])
+        return time.perf_counter() - t0
+
+    def leg(budget, n_calls):
+        n_probe = int(min(L.max(), 512))
+        rate = n_probe / max(call(int(np.argmax(L)), n_probe), 1e-6)          # slots per second
+        n_max = max(64, int(rate * call_seconds))
+        done, t_total, times, n_seq, n_prefix, b = 0, 0.0, [], 0, 0, 0
+        while (n_calls is None and t_total < budget) or (n_calls is not None and len(times) < n_calls):
+            n = int(min(L[b], n_max))
+            if n > 0:
+                dt = call(b, n)
+                times.append(dt)
+                t_total += dt
+                done += n
+                n_seq += 1
+                n_prefix += n < L[b]
+            b = (b + 1) % w.batch
+        return done / t_total, t_total, times, n_seq, n_prefix, n_max
+
+    cores = oracle.max_threads()
+    value, t_all, times, n_seq, n_prefix, n_max = leg(seconds, steps)
+    what = (f"{n_seq} calls of one layer's decode (all {s.h} heads) over the workload's sequences in turn, "
+            + (f"{n_prefix} of them over a prefix of at most {n_max} slots, " if n_prefix else "whole sequences, ")
+            + f"float64 C oracle, OpenMP over heads, {t_all:.1f} s")
+    base = {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what,
+            "cpu_model": _cpu_model(), "cpus_in_affinity": len(os.sched_getaffinity(0))}
+    if single_thread:
+        oracle.set_threads(1)
+        try:
+            v1, t1, _, n1, p1, m1 = leg(max(seconds / 2, 1.0), None if steps is None else max(1, steps // 4))
+        finally:
+            oracle.set_threads(cores)
+        base["single_thread"] = {"value": v1, "unit": "tokens/s", "cores": 1,
+                                 "sample": f"{n1} calls, {p1} over a prefix of at most {m1} slots, {t1:.1f} s"}
+    return base, times
 
 
 def run_reference(a):
@@ -264,19 +308,21 @@ def run_reference(a):
     from workloads import decode_inputs
     w = _workload(a.workload, a)
     inp = decode_inputs(w)
-    _cpu_baseline(w, inp, 0, steps=a.warmup)
-    base, times = _cpu_baseline(w, inp, 0, steps=a.steps)
+    # each step one bounded call, sized so warm-up and steps take about two minutes
+    per_call = min(2.5, 120.0 / max(a.steps + a.warmup, 1))
+    _cpu_baseline(w, inp, 0, steps=a.warmup, call_seconds=per_call, single_thread=False)
+    base, times = _cpu_baseline(w, inp, 0, steps=a.steps, call_seconds=per_call, single_thread=False)
     L = inp["seq_len"].numpy()
     value = base["value"]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
+            "ms_per_step": 1e3 * float(np.sum(times)) / max(len(times), 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config_json(w, 1, L, 1),
             "cpu_baseline": base,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
-    line["config"]["sample"] = "one whole sequence of one layer per step"
+    line["config"]["sample"] = "one decode call of one layer per step (a whole sequence, or a prefix of it)"
     print(json.dumps(line), flush=True)
     return 0
 
@@ -306,7 +352,7 @@ def run_kpa(a):
     first = decode_inputs(w.replace(seed=rank_seed(rank)))
     lens = first["seq_len"].numpy()
     layer_bytes = int(lens.sum()) * (s.e_k + s.e_v) * elt
-    layers = a.layers or max(1, int(np.ceil(4 * l2 / max(layer_bytes, 1))))
+    layers = a.layers or max(2, int(np.ceil(4 * l2 / max(layer_bytes, 1))))
     cfg = kpa.make_config(s, w.dtype)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     kpa.kpa_test_set_decode_engine(a.decode_engine)
@@ -405,16 +451,19 @@ def run_kpa(a):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record(stream)
+        for i in range(steps):
             g.replay()
-        e1.record(stream)
-        e1.synchronize()
+            ev[i + 1].record(stream)
+        ev[-1].synchronize()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+        per = np.array([ev[i].elapsed_time(ev[i + 1]) for i in range(steps)])
+        dist_ms = {"median": float(np.median(per)), "p10": float(np.percentile(per, 10)),
+                   "p90": float(np.percentile(per, 90)), "min": float(per.min()), "max": float(per.max())}
+        return max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev) / steps, dist_ms
 
     with torch.cuda.stream(stream):
         # settle clocks under load (untimed) while the sampler runs
@@ -424,9 +473,9 @@ def run_kpa(a):
             for _ in range(20):
                 graph.replay()
             stream.synchronize()
-        ms_step = timed(graph, a.steps, a.warmup)
+        ms_step, step_dist = timed(graph, a.steps, a.warmup)
         clocks = sampler.stop()
-        ms_e2e = timed(graph_e2e, a.steps, a.warmup)
+        ms_e2e, e2e_dist = timed(graph_e2e, a.steps, a.warmup)
     code = kpa.kpa_read_device_error(stream)
     if code != 0:
         raise RuntimeError(f"device error word {code} after the timed region")
@@ -446,7 +495,8 @@ def run_kpa(a):
                 "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json copy test)",
                 "kernel": "kpa_decode (split + combine), per layer call",
                 "algorithmic_bytes_per_launch": layer_bytes,
-                "launch_us": t_launch * 1e6, "kernel_sources_sha": khash}
+                "launch_us": t_launch * 1e6, "kernel_sources_sha": khash,
+                "launch_us_per_step_percentiles": {k: v * 1e3 / layers for k, v in step_dist.items()}}
     kind = kpa.kpa_decode_kernel_kind(cfg, w.batch, max_len, tps)
     plan = kpa.kpa_decode_plan(cfg, w.batch, max_len, tps)
     if qf_mode:
@@ -481,12 +531,13 @@ def run_kpa(a):
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
                     "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
-                    "ms_per_step": ms_e2e,
+                    "ms_per_step": ms_e2e, "ms_per_step_percentiles": e2e_dist,
                     "path": f"pinned host queries -> device, {'kpa_decode_qf' if qf_mode else 'kpa_decode'} x "
                             "layers, outputs -> pinned host, every "
                             "step, one CUDA graph; the copies overlap the decodes on a second stream (the first "
                             "two layers' queries first, then the rest; outputs in groups of 4 layers, the last "
                             "ones singly)"},
+            "ms_per_step_percentiles": step_dist,
             "clocks": clocks,
             "gpu_launches": a.steps * layers * plan[2]}
 
@@ -682,10 +733,92 @@ def run_append_prefill(a):
     return 0
 
 
+def run_sweep(a):
+    """The FlashTPA decoding benchmark grid ("Tensor Product Attention Is All You Need"
+    explainer, decoding-speed figures: sequence 2^12 .. 2^19, batch 1 .. 16) on the
+    pages' TPA shape (h = 32, d_h = 64, R_K = R_V = 1).  Per point: caches filled through
+    kpa_append_factors from device-drawn factors, enough layer copies to exceed 4 x L2
+    (at least 2), the decodes of one step in a CUDA graph, timed with CUDA events over
+    a.steps replays after a.warmup.  One JSON line per point (rank 0, 1 GPU)."""
+    import torch
+    import factorised_kv_attention_b200 as kpa
+    from workloads import FLASHTPA_DECODE, device_decode_factors
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = _hbm_peak()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    s = FLASHTPA_DECODE.shape
+    cfg = kpa.make_config(s, "bf16")
+    stream = torch.cuda.Stream(device=dev)
+    for log_len in range(12, 20):
+        for batch in (1, 2, 4, 8, 16):
+            L = 1 << log_len
+            w = FLASHTPA_DECODE.replace(batch=batch, capacity=L, length=L, name=f"FlashTPA shape B={batch} L={L}")
+            layer_bytes = batch * L * (s.e_k + s.e_v) * 2
+            layers = max(2, int(np.ceil(4 * l2 / layer_bytes)))
+            start = torch.zeros(batch, dtype=torch.int32, device=dev)
+            seq_len = torch.full((batch,), L, dtype=torch.int32, device=dev)
+            q_pos = seq_len.clone()
+            kcs, vcs, qs = [], [], []
+            for layer in range(layers):
+                kf, vf, q = device_decode_factors(w, dev, 1000 * log_len + 10 * batch + layer)
+                kc = torch.empty(batch * L * s.e_k, dtype=torch.bfloat16, device=dev)
+                vc = torch.empty(batch * L * s.e_v, dtype=torch.bfloat16, device=dev)
+                kpa.kpa_append_factors(cfg, batch, L, kf, vf, start, L, kc, vc)
+                kcs.append(kc)
+                vcs.append(vc)
+                qs.append(q)
+                del kf, vf
+            outs = [torch.empty(batch, s.h, s.dh, dtype=torch.float32, device=dev) for _ in range(layers)]
+            ws = torch.zeros(max(kpa.kpa_decode_workspace_size(cfg, batch, L), 256), dtype=torch.uint8, device=dev)
+            scale = 1.0 / float(np.sqrt(s.dh))
+
+            def step():
+                for i in range(layers):
+                    kpa.kpa_decode(cfg, batch, qs[i], q_pos, kcs[i], vcs[i], L, seq_len, L, scale, outs[i], ws,
+                                   stream=stream)
+
+            with torch.cuda.stream(stream):
+                step()
+            stream.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+            for _ in range(a.warmup):
+                graph.replay()
+            stream.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps + 1)]
+            ev[0].record(stream)
+            for i in range(a.steps):
+                graph.replay()
+                ev[i + 1].record(stream)
+            ev[-1].synchronize()
+            per = np.array([ev[i].elapsed_time(ev[i + 1]) for i in range(a.steps)]) / layers * 1e3   # us per call
+            code = kpa.kpa_read_device_error(stream)
+            if code != 0:
+                raise RuntimeError(f"device error word {code}")
+            us = float(np.median(per))
+            n_split, tps, launches = kpa.kpa_decode_plan(cfg, batch, L)
+            print(json.dumps({"sweep": "flashtpa", "batch": batch, "seq_len": L, "layers": layers,
+                              "us_per_call_median": us, "us_p10": float(np.percentile(per, 10)),
+                              "us_p90": float(np.percentile(per, 90)),
+                              "cached_tokens_per_s": batch * L / (us * 1e-6),
+                              "achieved_gbs": layer_bytes / (us * 1e-6) / 1e9, "peak_gbs": peak,
+                              "frac": layer_bytes / (us * 1e-6) / 1e9 / peak, "peak_source": peak_kind,
+                              "splits_per_sequence": n_split, "tokens_per_split": tps, "launches": launches}),
+                  flush=True)
+            del graph, kcs, vcs, qs, outs, ws
+            torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     a = _args(argv)
     if a.impl == "reference":
         return run_reference(a)
+    if a.sweep:
+        return run_sweep(a)
     if a.workload == "append_prefill":
         return run_append_prefill(a)
     return run_kpa(a)

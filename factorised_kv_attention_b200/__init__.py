@@ -80,6 +80,7 @@ _SIGS = {
     "kpa_test_set_decode_hooks": ([_i32, _i32, ctypes.c_uint64], ctypes.c_int),
     "kpa_test_set_decode_engine": ([_i32], ctypes.c_int),
     "kpa_decode_kernel_kind": ([_cfgp, _i32, _i32, _i32, _i32p], ctypes.c_int),
+    "kpa_test_exp2_poly": ([_vp, _vp, ctypes.c_int64, _vp], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -252,6 +253,14 @@ def kpa_test_set_decode_hooks(skip_tile=-1, skip_split=-1, wait_limit_ns=1_000_0
 
 def kpa_test_set_decode_engine(engine=0):
     _check(_lib.kpa_test_set_decode_engine(engine), "kpa_test_set_decode_engine")
+
+
+def kpa_test_exp2_poly(x, y, stream=None):
+    """y = 2^x (float32 device tensors of the same size) through the prefill's
+    polynomial exponential (testing)."""
+    if x.numel() != y.numel():
+        raise ValueError("x and y differ in size")
+    _check(_lib.kpa_test_exp2_poly(_addr(x), _addr(y), x.numel(), _stream(stream)), "kpa_test_exp2_poly")
 
 
 def kpa_read_device_error(stream=None) -> int:

@@ -110,28 +110,28 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 constexpr size_t kSmemLimit = 200 * 1024;
 
-std::mutex g_hooks_mu;
-DecodeTestHooks g_hooks = {-1, -1, 1000000000ull};   // bounded waits give up after 1 s
+// Test and measurement switches, scoped to the host thread that sets them (a caller
+// that flips them changes only its own later calls, never another thread's).
+// The bounded waits give up after 1 s unless a test shortens them.
+thread_local DecodeTestHooks t_hooks = {-1, -1, 1000000000ull};
 
 // 0: the default kernels; 1: the tcgen05 TPA decode where it applies; 2: the factored
 // score for decodes from query factors on TPA shapes (testing and measurement: both are
 // slower than the defaults on the shapes measured so far).
-std::atomic<int> g_decode_engine{0};
+thread_local int t_decode_engine = 0;
 
-DecodeTestHooks current_hooks() {
-    std::lock_guard<std::mutex> lock(g_hooks_mu);
-    return g_hooks;
-}
+DecodeTestHooks current_hooks() { return t_hooks; }
 
 constexpr int kMaxClusterSplits = 16;
 
 // How many clusters of `size` CTAs of a tensor-core variant can be resident at once
 // on this device (cached per device).
 int cluster_capacity(int variant, int size) {
-    static std::atomic<int> known[kMaxDevices][8][kMaxClusterSplits + 1];
+    constexpr int kMaxVariants = 16;
+    static std::atomic<int> known[kMaxDevices][kMaxVariants][kMaxClusterSplits + 1];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || variant < 0 ||
-        variant >= 8 || size < 1 || size > kMaxClusterSplits)
+        variant >= kMaxVariants || size < 1 || size > kMaxClusterSplits)
         return 0;
     int k = known[dev][variant][size].load();
     if (k == 0) {
@@ -223,10 +223,15 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
     if (p->n_split > 1 && (int64_t)max_len - (int64_t)(p->n_split - 1) * tps <= tps / 4) --p->n_split;
     // the tcgen05 kernel, on request, for TPA at h = 16, d_h = 64, R = 2 (its splits merge
     // through global memory)
-    p->engine = p->variant >= 0 && p->tile == 128 && tc_decode_supported(d) && g_decode_engine.load() == 1;
+    p->engine = p->variant >= 0 && p->tile == 128 && tc_decode_supported(d) && t_decode_engine == 1;
     p->cluster = !p->engine && p->variant >= 0 && p->n_split <= kMaxClusterSplits &&
                  (p->n_split == 1 || cluster_capacity(p->variant, p->n_split) >= batch);
     // otherwise the last CTA of a sequence merges its splits when that read is small
+    // In a grid of one wave the first tile's latency is on every CTA's critical path, so
+    // the kernel requests it before reading the length (a split past a sequence's end then
+    // copies one tile for nothing).  In several waves the later CTAs' latency overlaps the
+    // running ones, and the copies of empty splits would only add DRAM traffic.
+    p->spec = (int64_t)batch * p->n_split <= (int64_t)target;
     p->fused = p->cluster ||
                (p->variant >= 0 && (size_t)p->n_split * d.h * d.dh * sizeof(float) <= 256 * 1024);
     const size_t o_bytes = (size_t)batch * p->n_split * d.h * d.dh * sizeof(float);
@@ -242,8 +247,8 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
 
 void record_cuda_error(cudaError_t e) { t_last_cuda = (int)e; }
 
-kpa_status decode_counter_region(const kpa_config *cfg, int batch, int max_len, size_t *offset,
-                                 size_t *bytes) {
+kpa_status decode_dense_plan(const kpa_config *cfg, int batch, int max_len, size_t *total, size_t *offset,
+                             size_t *bytes) {
     kpa_status s = check_cfg(cfg, false, false);
     if (s != KPA_OK) return s;
     int sms = 0;
@@ -252,6 +257,7 @@ kpa_status decode_counter_region(const kpa_config *cfg, int batch, int max_len, 
     DecodePlan p;
     s = plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, 0, sms, &p);
     if (s != KPA_OK) return s;
+    *total = batch == 0 ? 0 : p.bytes;
     *offset = p.counters_off;
     *bytes = (size_t)batch * sizeof(int);
     return KPA_OK;
@@ -324,7 +330,7 @@ kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32
     if (s != KPA_OK) return s;
     size_t need = p.bytes;
     // with the factored-score engine selected, room for its plan too
-    if (g_decode_engine.load() == 2 && cfg->dtype == KPA_BF16 && factored_decode_supported(dims_of(cfg), cfg->r_q)) {
+    if (t_decode_engine == 2 && cfg->dtype == KPA_BF16 && factored_decode_supported(dims_of(cfg), cfg->r_q)) {
         DecodePlan pf;
         if (plan_decode(dims_of(cfg), cfg->dtype, batch, max_len, tokens_per_split, sms, &pf, cfg->r_q) == KPA_OK)
             need = std::max(need, pf.bytes);
@@ -402,7 +408,7 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     if (s != KPA_OK) return s;
     // query factors: the factored score on request (TPA shapes), else the tensor-core
     // kernel, which assembles the query (never a third-order cache)
-    const bool factored = qf && g_decode_engine.load() == 2 && cfg->dtype == KPA_BF16 &&
+    const bool factored = qf && t_decode_engine == 2 && cfg->dtype == KPA_BF16 &&
                           factored_decode_supported(d, cfg->r_q);
     if (qf && (d.order == 3 || (!factored && p.variant < 0))) return KPA_ERR_UNSUPPORTED;
     if (qf && !factored && (int64_t)cfg->r_q * (d.h1 * d.d1 + d.h2 * d.d2) > mma_decode_qf_max(p.variant))
@@ -451,6 +457,7 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
         args.out_scale = out_scale;
         args.fused = p.fused;
         args.cluster = p.cluster;
+        args.spec = p.spec;
         args.err = err;
         args.qf = qf;
         args.qf_stride = qf_stride;
@@ -620,16 +627,15 @@ kpa_status kpa_append(const kpa_config *cfg, int32_t batch, int32_t n_tok, const
 kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split,
                                      uint64_t wait_limit_ns) {
     if (wait_limit_ns == 0) return KPA_ERR_INVALID_ARG;
-    std::lock_guard<std::mutex> lock(g_hooks_mu);
-    g_hooks.skip_tile = skip_tile;
-    g_hooks.skip_split = skip_split;
-    g_hooks.wait_limit_ns = wait_limit_ns;
+    t_hooks.skip_tile = skip_tile;
+    t_hooks.skip_split = skip_split;
+    t_hooks.wait_limit_ns = wait_limit_ns;
     return KPA_OK;
 }
 
 kpa_status kpa_test_set_decode_engine(int32_t engine) {
     if (engine < 0 || engine > 2) return KPA_ERR_INVALID_ARG;
-    g_decode_engine.store(engine);
+    t_decode_engine = engine;
     return KPA_OK;
 }
 

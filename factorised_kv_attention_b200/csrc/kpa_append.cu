@@ -11,9 +11,10 @@
 //
 // GEMM: 128 x BN output tiles (BN <= 256, a multiple of 16), K in steps of 64.  Warp 0
 // issues TMA loads of X and W tiles (128-byte swizzle) into a STAGES-deep ring; one
-// thread of warp 1 issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into a TMEM
-// accumulator and commits each stage back to the producer; warps 2..5 read the
-// accumulator rows from TMEM (one row = one token per thread) and run the epilogue.
+// thread of warp 1 issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into one of two
+// TMEM accumulators and commits each stage back to the producer; warps 2..9 read the
+// accumulator rows from TMEM (one row = one token per thread; two warps per TMEM lane
+// quarter, each taking half of a tile's 32-column passes) and run the epilogue.
 #include <cudaTypedefs.h>
 
 #include <mutex>

@@ -26,66 +26,29 @@
 #include <cooperative_groups.h>
 
 #include "kpa_decode_merge.cuh"
+#include "kpa_f32x2.cuh"
 #include "kpa_internal.cuh"
 #include "kpa_mma_decode.cuh"
+#include "kpa_sm100.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace kpa {
 namespace {
 
+using f32x2::fadd2;
+using f32x2::ffma2;
+using f32x2::fmul2;
+using f32x2::fsub2;
+using f32x2::unpack_bf16x2;
+
 // ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Wait for phase `parity` of an mbarrier, for at most limit_ns nanoseconds.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 15) == 0 && globaltimer() - t0 > limit_ns) return false;
-    }
-}
-
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
+using sm100::bulk_g2s;
+using sm100::mbar_arrive;
+using sm100::mbar_expect_tx;
+using sm100::mbar_init;
+using sm100::mbar_wait;
+using sm100::smem_u32;
 
 // hint a global range (16-byte aligned, a multiple of 16 bytes) into L2.  No data is
 // bound to the issuing thread, and L2 stays coherent with later writes to the range.
@@ -107,6 +70,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x1_t(uint32_t addr, uint32_t &r0) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x1.trans.shared.b16 {%0}, [%1];" : "=r"(r0) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
 __device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t &r0, uint32_t &r1) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
                  : "=r"(r0), "=r"(r1)
@@ -119,6 +90,14 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         "{%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// m16n8k8 (k = d2 = 8): A rows g, g + 8 at k 2c, 2c + 1; B k 2c, 2c + 1 at n g
+__device__ __forceinline__ void mma16808(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(b0));
 }
 
 // The same product with fp16 operands (the score of a shared-B cache, whose rotated
@@ -135,44 +114,9 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t v, bool keep0, bool keep1
     return (keep0 ? (v & 0xffffu) : 0u) | (keep1 ? (v & 0xffff0000u) : 0u);
 }
 
-// Packed FP32 pair arithmetic (sm_100 f32x2 forms).
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-    float2 r;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rc, ra, rb;\n\t"
-        "mov.b64 {%0, %1}, rc;\n\t}"
-        : "=f"(r.x), "=f"(r.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return r;
-}
 
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    float2 r;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
-        "mov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(r.x), "=f"(r.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return r;
-}
 
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-    float2 r;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "sub.rn.f32x2 rc, ra, rb;\n\t"
-        "mov.b64 {%0, %1}, rc;\n\t}"
-        : "=f"(r.x), "=f"(r.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return r;
-}
 
-// bf16x2 word -> (low element, high element) as floats
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
-    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
-}
 
 __device__ __forceinline__ uint32_t lds_u32(const unsigned char *p) {
     return *reinterpret_cast<const uint32_t *>(p);
@@ -213,6 +157,30 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     return r;
 }
 
+// A-factor fragments of the d1 = 8 decode for MT m-tiles: words (row half 0, 1) of each
+// m-tile, two m-tiles per ldmatrix.x4 (4 x d1 rows of 16 bytes apart), an odd last one
+// by ldmatrix.x2 (its lanes 0..15 give the row addresses).  abase: this lane's row.
+template <int MT, int D1>
+__device__ __forceinline__ void a_frags(uint32_t abase, uint32_t (&w)[MT][2]) {
+#pragma unroll
+    for (int mp = 0; mp < MT / 2; ++mp)
+        ldsm_x4(abase + mp * 4 * D1 * 16, w[2 * mp][0], w[2 * mp][1], w[2 * mp + 1][0], w[2 * mp + 1][1]);
+    if constexpr (MT % 2 == 1) ldsm_x2(abase + (MT / 2) * 4 * D1 * 16, w[MT - 1][0], w[MT - 1][1]);
+}
+
+// bf16x2 word -> fp16x2 word (exact for values in fp16's normal range)
+__device__ __forceinline__ uint32_t bf16x2_to_h2(uint32_t v) {
+    const float2 x = unpack_bf16x2(v);
+    return pack_h2(x.x, x.y);
+}
+
+// 2^x on the special-function unit (ex2.approx: relative error about 2^-22; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // bf16 element of one token in a group row (2-byte load), widened by a shift
 __device__ __forceinline__ float lds_bf16f(const unsigned char *p) {
     return __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short *>(p) << 16);
@@ -224,7 +192,7 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
 
 // ------------------------------------------------------------------- kernel
 template <class C>
-__global__ void __launch_bounds__((C::WARPS + 1) * 32, 1)
+__global__ void __launch_bounds__(C::THREADS, 1)
 decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     constexpr int MA = C::MA, D1 = C::D1, D2 = C::D2, RK = C::RK, RV = C::RV, H2 = C::H2;
     constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
@@ -261,7 +229,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, WARPS);
         }
-        flags[0] = 0;
+        for (int i = 0; i < 16; ++i) flags[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // Ahead of the dependency on the previous grid: hint this CTA's first ring of tiles
@@ -269,8 +237,10 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     // previous grid still writes, so it reads no input early; the cache streams in
     // while the previous call finishes (its split merge).  Only kernel parameters are
     // used here.  Slots [p0, p1) clipped to max_len, rounded up to whole 8-slot groups,
-    // stay inside the cache (capacity >= max_len, a multiple of 8).
-    if (tid == 0) {
+    // stay inside the cache (capacity >= max_len, a multiple of 8).  Only in a grid of
+    // one wave (a.spec): with several waves a split past its sequence's end would read
+    // its slots for nothing.
+    if (tid == 0 && a.spec) {
         const int p0 = split * a.tps;
         const int p1 = min(p0 + STAGES * TT, a.max_len);
         if (p1 > p0) {
@@ -284,12 +254,12 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    // The first tile's copy starts before the sequence length is known: slots
-    // [t0, t0 + TT) clipped to max_len are inside the cache whatever the length, and
-    // tokens past the length are masked later.
+    // In a grid of one wave the first tile's copy starts before the sequence length is
+    // known: slots [t0, t0 + TT) clipped to max_len are inside the cache whatever the
+    // length, and tokens past the length are masked later.
     const int t0 = split * a.tps;
     const int spec_n = min(TT, a.max_len - t0);
-    const bool spec = spec_n > 0 &&
+    const bool spec = a.spec && spec_n > 0 &&
                       !(hooks.skip_tile == 0 && split == hooks.skip_split && b == 0);
     if (tid == 0 && spec) {
         const int groups = (spec_n + kGroup - 1) / kGroup;
@@ -342,8 +312,8 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     }
     if (t0 >= L && !a.cluster) {                           // empty split (a cluster member stays)
         if (a.fused && L == 0 && split == 0)                // an empty sequence gets zeros
-            for (int i = tid; i < H * DH; i += (WARPS + 1) * 32) a.out[(size_t)b * H * DH + i] = 0.f;
-        if (tid == 0 && spec && !mbar_wait_bounded(full0, 0, hooks.wait_limit_ns))
+            for (int i = tid; i < H * DH; i += C::THREADS) a.out[(size_t)b * H * DH + i] = 0.f;
+        if (tid == 0 && spec && !mbar_wait(full0, 0, hooks.wait_limit_ns))
             raise_error(a.err, kErrTimeout);               // its speculative copy lands first
         return;
     }
@@ -356,35 +326,50 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const __nv_bfloat16 *kb = a.kc + ((size_t)b * a.cap + t0) * EK;   // group-aligned (t0 % 8 == 0)
     const __nv_bfloat16 *vb = a.vc + ((size_t)b * a.cap + t0) * EV;
 
+    // tile t of this split into stage t % STAGES (the test hook may withhold one)
+    auto issue_tile = [&](int t) {
+        const int s = t % STAGES;
+        const int n = min(TT, t1 - t0 - t * TT);
+        const int groups = (n + kGroup - 1) / kGroup;
+        const uint32_t kbytes = (uint32_t)groups * EK * kGroup * 2;
+        const uint32_t vbytes = (uint32_t)groups * EV * kGroup * 2;
+        if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) return;
+        const uint32_t dst = smem_u32(stage_base + (size_t)s * STAGE_BYTES);
+        mbar_expect_tx(full0 + 8 * s, kbytes + vbytes);
+        bulk_g2s(dst, kb + (size_t)t * TT * EK, kbytes, full0 + 8 * s);
+        bulk_g2s(dst + KBYTES, vb + (size_t)t * TT * EV, vbytes, full0 + 8 * s);
+    };
+    // every copy issued for this CTA (tiles below `issued`) lands before it exits
+    auto drain = [&](int issued) {
+        for (int t = max(0, issued - STAGES); t < issued; ++t) {
+            if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) continue;
+            if (!mbar_wait(full0 + 8 * (t % STAGES), (t / STAGES) & 1, limit)) raise_error(a.err, kErrTimeout);
+        }
+    };
+    if constexpr (!C::PRODUCER_WARP) {
+        if (tid == 0) {                                    // the rest of the first ring
+            const int first = min(STAGES, n_tiles);
+            for (int t = spec ? 1 : 0; t < first; ++t) issue_tile(t);
+            flags[2] = max(first, spec ? 1 : 0);
+        }
+    }
+
     // ------------------------------------------------------------ producer
-    if (warp == WARPS) {
+    if (C::PRODUCER_WARP && warp == WARPS) {
         if (lane == 0) {
             int issued = spec ? 1 : 0;
             for (int t = spec ? 1 : 0; t < n_tiles; ++t) {
                 const int s = t % STAGES;
-                if (t >= STAGES && !mbar_wait_bounded(empty0 + 8 * s, ((t / STAGES) - 1) & 1, limit)) {
+                if (t >= STAGES && !mbar_wait(empty0 + 8 * s, ((t / STAGES) - 1) & 1, limit)) {
                     raise_error(a.err, kErrTimeout);
                     flags[0] = 1;
                     break;
                 }
                 if (flags[0]) break;
-                const int n = min(TT, t1 - t0 - t * TT);
-                const int groups = (n + kGroup - 1) / kGroup;
-                const uint32_t kbytes = (uint32_t)groups * EK * kGroup * 2;
-                const uint32_t vbytes = (uint32_t)groups * EV * kGroup * 2;
                 issued = t + 1;
-                if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) continue;
-                const uint32_t dst = smem_u32(stage_base + (size_t)s * STAGE_BYTES);
-                mbar_expect_tx(full0 + 8 * s, kbytes + vbytes);
-                bulk_g2s(dst, kb + (size_t)t * TT * EK, kbytes, full0 + 8 * s);
-                bulk_g2s(dst + KBYTES, vb + (size_t)t * TT * EV, vbytes, full0 + 8 * s);
+                issue_tile(t);
             }
-            // drain: every copy issued for this CTA must land before it exits
-            for (int t = max(0, issued - STAGES); t < issued; ++t) {
-                if (hooks.skip_tile == t && split == hooks.skip_split && b == 0) continue;
-                if (!mbar_wait_bounded(full0 + 8 * (t % STAGES), (t / STAGES) & 1, limit))
-                    raise_error(a.err, kErrTimeout);
-            }
+            drain(issued);
         }
         if (!a.cluster) return;
     } else {
@@ -502,6 +487,295 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     // ------------------------------------------------------------ consumers
     const int i2 = warp % H2, slice = warp / H2;
     const int g = lane >> 2, c = lane & 3;
+    float *mo = reinterpret_cast<float *>(smem);                   // [SLICES][H][DH] (after the loop)
+    constexpr int MO_LD = C::MO_LD;
+    float *mm = mo + SLICES * H * MO_LD;                           // [SLICES][H][2]
+    float *cp = mm + SLICES * H * 2;                               // merged: [H][DH] o, [H] m, [H] l
+    bool aborted = false;
+    if constexpr (C::KPA8) {
+    // d1 = 8.  Row g of m-tile mt stands for the query row (i1, j1) = (2 mt + (g >> 2),
+    // 2 (g & 3)) and row g + 8 for (i1, j1 + 1): a lane's two rows belong to one head, so
+    // after the A^K product both add into one score, the sum over j1 is two shuffle
+    // levels (lanes g & 3), and every lane then holds the full scores, the weights p
+    // and the softmax state of its head for its four tokens (2c, 2c + 1 of each
+    // 8-token group).  The A-factor fragments are loaded with ldmatrix from the
+    // permuted rows.  The value product P' B^V runs once in fp16: P' = p A^V is
+    // rounded once to fp16 (relative 2^-11), B^V (bf16) converts to fp16 exactly in
+    // fp16's normal range; a value outside fp16's range makes the partial non-finite,
+    // which is reported as a device check.
+    // d2 = 8: the score is one m16n8k8 per m-tile (A words 0, 1 of each fragment) and the
+    // value product has one 8-column n-tile
+    constexpr bool K8 = D2 == 8;
+    constexpr int KQ = K8 ? 1 : KS, VQ = K8 ? 2 : 4;
+    const int hi1 = g >> 2, jp = 2 * (g & 3);
+    uint32_t qa_hi[MT][KQ][4], qa_lo[MT][KQ][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int ks = 0; ks < KQ; ++ks)
+#pragma unroll
+            for (int v = 0; v < VQ; ++v) {
+                const int i1 = 2 * mt + hi1, j1 = jp + (v & 1);
+                const int j2 = ks * 16 + 2 * c + ((v & 2) ? 8 : 0);
+                const float *src = qs + (i1 * H2 + i2) * C::Q_LD + j1 * D2 + j2;
+                split2(make_float2(src[0], src[1]), qa_hi[mt][ks][v], qa_lo[mt][ks][v]);
+            }
+    // ldmatrix row address (bytes inside a group) of this lane for the A factors: matrix
+    // mj = (m-tile 2 mp + (mj >> 1), row half mj & 1) of m-tile pair mp, matrix row mrow
+    const int mj = lane >> 3, mrow = lane & 7;
+    const uint32_t a_off =
+        (uint32_t)(((2 * (mj >> 1) + (mrow >> 2)) * D1 + 2 * (mrow & 3) + (mj & 1)) * 16);
+    float o[MT][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    float m_k[MT], l_k[MT];              // running max and this lane's share of the sum, head 2 mt + hi1
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        m_k[mt] = -INFINITY;
+        l_k[mt] = 0.f;
+    }
+
+    for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % STAGES;
+        if (!mbar_wait(full0 + 8 * s, (t / STAGES) & 1, limit)) {
+            raise_error(a.err, kErrTimeout);
+            flags[0] = 1;
+            aborted = true;
+            break;
+        }
+        const unsigned char *kt = stage_base + (size_t)s * STAGE_BYTES;
+        const unsigned char *vt = kt + KBYTES;
+        const int n_valid = min(TT, t1 - t0 - t * TT);
+        const int tok_base = slice * CHUNKS * 16;
+
+#pragma unroll 1
+        for (int ch = 0; ch < CHUNKS; ++ch) {
+            const int tok0 = tok_base + ch * 16;
+            if (tok0 >= n_valid) break;
+            const bool tail = tok0 + 16 > n_valid;
+            const unsigned char *kg0 = kt + (size_t)(tok0 >> 3) * EK * 16;
+            // ---- scores of head 2 mt + hi1, tokens (gi, 2c) and (gi, 2c + 1)
+            float2 sc[MT][2];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) sc[mt][0] = sc[mt][1] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < RK; ++r) {
+#pragma unroll
+                for (int gi = 0; gi < 2; ++gi) {
+                    const unsigned char *grp = kg0 + (size_t)gi * EK * 16;
+                    uint32_t bk[KQ][2];
+                    const int e_b = A_K + r * H2 * D2 + i2 * D2;
+                    if constexpr (K8) {
+                        ldsm_x1_t(smem_u32(grp + (size_t)(e_b + (lane & 7)) * 16), bk[0][0]);
+                    } else if constexpr (KS % 2 == 0) {
+#pragma unroll
+                        for (int kp = 0; kp < KS / 2; ++kp)
+                            ldsm_x4_t(smem_u32(grp + (size_t)(e_b + kp * 32 + lane) * 16), bk[2 * kp][0],
+                                      bk[2 * kp][1], bk[2 * kp + 1][0], bk[2 * kp + 1][1]);
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < KS; ++ks)
+                            ldsm_x2_t(smem_u32(grp + (size_t)(e_b + ks * 16 + (lane & 15)) * 16), bk[ks][0],
+                                      bk[ks][1]);
+                    }
+                    uint32_t ak[MT][2];
+                    a_frags<MT, D1>(smem_u32(grp + (size_t)r * MA * 16) + a_off, ak);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                        if constexpr (K8) {
+                            mma16808(acc, qa_hi[mt][0][0], qa_hi[mt][0][1], bk[0][0]);
+                            mma16808(acc, qa_lo[mt][0][0], qa_lo[mt][0][1], bk[0][0]);
+                        } else {
+#pragma unroll
+                            for (int ks = 0; ks < KS; ++ks) {
+                                mma16816(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
+                                mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
+                            }
+                        }
+                        sc[mt][gi] = ffma2(make_float2(acc[0], acc[1]), unpack_bf16x2(ak[mt][0]), sc[mt][gi]);
+                        sc[mt][gi] = ffma2(make_float2(acc[2], acc[3]), unpack_bf16x2(ak[mt][1]), sc[mt][gi]);
+                    }
+                }
+            }
+            // ---- the sum over j1: lanes that differ in g & 3
+#pragma unroll
+            for (int off = 4; off <= 8; off <<= 1)
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int gi = 0; gi < 2; ++gi) {
+                        sc[mt][gi].x += __shfl_xor_sync(0xffffffffu, sc[mt][gi].x, off);
+                        sc[mt][gi].y += __shfl_xor_sync(0xffffffffu, sc[mt][gi].y, off);
+                    }
+            if (tail) {
+#pragma unroll
+                for (int gi = 0; gi < 2; ++gi) {
+                    const int tk = tok0 + gi * 8 + 2 * c;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        if (tk >= n_valid) sc[mt][gi].x = -INFINITY;
+                        if (tk + 1 >= n_valid) sc[mt][gi].y = -INFINITY;
+                    }
+                }
+            }
+            // ---- online softmax of this lane's head over the chunk's 16 tokens
+            bool grow = false;
+            float alpha[MT];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                float mx = fmaxf(fmaxf(sc[mt][0].x, sc[mt][0].y), fmaxf(sc[mt][1].x, sc[mt][1].y));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                alpha[mt] = 1.f;
+                if (mx > m_k[mt]) {                     // finite: the chunk has a valid token
+                    alpha[mt] = ex2_approx(m_k[mt] - mx);
+                    m_k[mt] = mx;
+                    grow = true;
+                }
+                const float m_new = m_k[mt];
+#pragma unroll
+                for (int gi = 0; gi < 2; ++gi) {
+                    sc[mt][gi].x = ex2_approx(sc[mt][gi].x - m_new);
+                    sc[mt][gi].y = ex2_approx(sc[mt][gi].y - m_new);
+                }
+                l_k[mt] = l_k[mt] * alpha[mt] + ((sc[mt][0].x + sc[mt][0].y) + (sc[mt][1].x + sc[mt][1].y));
+            }
+            if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) o[mt][nt][v] *= alpha[mt];
+            }
+            // ---- values: P'[(i1, j1), token] = p * A^V_r in fp16 (A operand: rows g, g + 8,
+            // tokens 2c, 2c + 1 of group 0 then of group 1)
+            const unsigned char *g0p = vt + (size_t)(tok0 >> 3) * EV * 16;
+            const unsigned char *g1p = g0p + (size_t)EV * 16;
+#pragma unroll
+            for (int r = 0; r < RV; ++r) {
+                uint32_t av[2][MT][2];
+#pragma unroll
+                for (int gi = 0; gi < 2; ++gi) {
+                    a_frags<MT, D1>(smem_u32((gi ? g1p : g0p) + (size_t)r * MA * 16) + a_off, av[gi]);
+                }
+                uint32_t pa[MT][4];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+                        for (int hr = 0; hr < 2; ++hr) {
+                            float2 x = fmul2(sc[mt][gi], unpack_bf16x2(av[gi][mt][hr]));
+                            if (tail) {   // garbage factors of masked tokens stay out (their weight is 0)
+                                const int tk = tok0 + gi * 8 + 2 * c;
+                                if (tk >= n_valid) x.x = 0.f;
+                                if (tk + 1 >= n_valid) x.y = 0.f;
+                            }
+                            pa[mt][2 * gi + hr] = pack_h2(x.x, x.y);
+                        }
+                }
+                const int e_b = A_V + r * H2 * D2 + i2 * D2;
+                const int mat = lane >> 3, mr = lane & 7;
+                if constexpr (K8) {
+                    // one n-tile: matrices (group 0, group 1) of the 8 features, lanes 0..15
+                    uint32_t b00, b01;
+                    ldsm_x2(smem_u32(((mat & 1) ? g1p : g0p) + (size_t)(e_b + mr) * 16), b00, b01);
+                    b00 = bf16x2_to_h2(b00);
+                    b01 = bf16x2_to_h2(b01);
+                    if (tail) {
+                        const int tk = tok0 + 2 * c;
+                        b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
+                        b01 = mask_pair(b01, tk + 8 < n_valid, tk + 9 < n_valid);
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) mma16816h(o[mt][0], pa[mt], b00, b01);
+                }
+#pragma unroll
+                for (int np = 0; np < NT / 2; ++np) {
+                    const unsigned char *gp = (mat & 1) ? g1p : g0p;
+                    uint32_t b00, b01, b10, b11;
+                    ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mr) * 16), b00, b01, b10,
+                            b11);
+                    b00 = bf16x2_to_h2(b00);
+                    b01 = bf16x2_to_h2(b01);
+                    b10 = bf16x2_to_h2(b10);
+                    b11 = bf16x2_to_h2(b11);
+                    if (tail) {
+                        const int tk = tok0 + 2 * c;
+                        b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
+                        b10 = mask_pair(b10, tk < n_valid, tk + 1 < n_valid);
+                        b01 = mask_pair(b01, tk + 8 < n_valid, tk + 9 < n_valid);
+                        b11 = mask_pair(b11, tk + 8 < n_valid, tk + 9 < n_valid);
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        mma16816h(o[mt][2 * np], pa[mt], b00, b01);
+                        mma16816h(o[mt][2 * np + 1], pa[mt], b10, b11);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) {
+            // the warp is done with stage s: the last of the WARPS releases issues tile
+            // t + STAGES into it (acq_rel: every warp's reads of the stage come first)
+            uint32_t old;
+            asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                         : "=r"(old)
+                         : "r"(smem_u32((const void *)(flags + 4 + s)))
+                         : "memory");
+            if ((old + 1) % WARPS == 0 && t + STAGES < n_tiles && !flags[0]) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                issue_tile(t + STAGES);
+                flags[2] = t + STAGES + 1;
+            }
+        }
+        if (flags[0]) { aborted = true; break; }
+    }
+
+    {   // fp16 operands of the value product: an out-of-range value makes the partial non-finite
+        bool fin = true;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) fin = fin && isfinite(o[mt][nt][v]);
+        if (!fin) raise_error(a.err, kErrDeviceCheck);
+    }
+    // the sum of each head over the lanes of its tokens (c); lanes g & 3 hold copies
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        l_k[mt] += __shfl_xor_sync(0xffffffffu, l_k[mt], 1);
+        l_k[mt] += __shfl_xor_sync(0xffffffffu, l_k[mt], 2);
+    }
+
+    // merge the token slices of the CTA through shared memory (reuses the ring)
+    asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
+    if (tid == 0) drain(flags[2]);               // copies still in flight after an abort
+    const bool ok = !(aborted || flags[0]);
+    if (!ok && !a.cluster) return;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int head = (2 * mt + hi1) * H2 + i2;
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            float *dst = mo + ((size_t)slice * H + head) * MO_LD + (jp + hr) * D2;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                *reinterpret_cast<float2 *>(dst + nt * 8 + 2 * c) =
+                    make_float2(o[mt][nt][2 * hr], o[mt][nt][2 * hr + 1]);
+        }
+        if ((lane & 15) == 0) {
+            mm[((size_t)slice * H + head) * 2] = m_k[mt];
+            mm[((size_t)slice * H + head) * 2 + 1] = l_k[mt];
+        }
+    }
+    } else {
     float *red = scratch + (size_t)warp * C::SCR_FLOATS;   // [16][RED_LD] j1 partials
     float *pbuf = red + 16 * RED_LD;                         // [H1][16] weights
     float *abuf = pbuf + H1 * 16;                            // [H1] rescale factors
@@ -548,10 +822,9 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const int my_i1 = lane % H1;                // the head this lane scores (D1 > 1)
     float m_h = -INFINITY, l_h = 0.f;
 
-    bool aborted = false;
     for (int t = 0; t < n_tiles; ++t) {
         const int s = t % STAGES;
-        if (!mbar_wait_bounded(full0 + 8 * s, (t / STAGES) & 1, limit)) {
+        if (!mbar_wait(full0 + 8 * s, (t / STAGES) & 1, limit)) {
             raise_error(a.err, kErrTimeout);
             flags[0] = 1;
             aborted = true;
@@ -892,10 +1165,6 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     const bool ok = !(aborted || flags[0]);
     if (!ok && !a.cluster) return;
-    float *mo = reinterpret_cast<float *>(smem);                   // [SLICES][H][DH]
-    constexpr int MO_LD = C::MO_LD;
-    float *mm = mo + SLICES * H * MO_LD;                           // [SLICES][H][2]
-    float *cp = mm + SLICES * H * 2;                               // merged: [H][DH] o, [H] m, [H] l
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -922,6 +1191,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             mm[((size_t)slice * H + head) * 2 + 1] = l_h;
         }
     }
+    }  // KPA8
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     float *po = a.part_o + ((size_t)(b * a.n_split + split) * H) * DH;
     float *pml = a.part_ml + ((size_t)(b * a.n_split + split) * H) * 2;
@@ -1025,7 +1295,7 @@ cudaError_t launch_cfg(const DecodeArgs &args, int batch, const DecodePlan &p, c
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3((unsigned)p.n_split, (unsigned)batch);
-    lc.blockDim = dim3((C::WARPS + 1) * 32);
+    lc.blockDim = dim3(C::THREADS);
     lc.dynamicSmemBytes = smem;
     lc.stream = st;
     cudaLaunchAttribute attr[2];
@@ -1051,7 +1321,7 @@ int cluster_ok_cfg(int size) {
         return 0;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3((unsigned)size, 1);
-    lc.blockDim = dim3((C::WARPS + 1) * 32);
+    lc.blockDim = dim3(C::THREADS);
     lc.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -117,13 +117,16 @@ struct DecodePlan {
     int fused;           // the decode kernel merges the splits itself (no combine launch)
     int cluster;         // ... through a thread-block cluster per sequence (DSMEM)
     int engine;          // 1: the tcgen05 kernel (TPA h = 16, d_h = 64, R = 2), 0: mma.sync
+    int spec;            // every CTA is resident at once (one wave): the decode copies its first
+                         // tiles before it has read the sequence length
     size_t part_o_off, part_ml_off, counters_off, bytes;
 };
 
-// Byte range of the per-sequence counters inside a decode workspace (they must be
-// zero before a call and are zero again after every call that completes).
-kpa_status decode_counter_region(const kpa_config *cfg, int batch, int max_len, size_t *offset,
-                                 size_t *bytes);
+// Workspace of a decode with a dense query and the automatic split: its size (total)
+// and the byte range of its per-sequence counters (they must be zero before a call and
+// are zero again after every call that completes).
+kpa_status decode_dense_plan(const kpa_config *cfg, int batch, int max_len, size_t *total, size_t *offset,
+                             size_t *bytes);
 
 cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void *q,
                               const int32_t *q_pos, const void *kc, const void *vc, int cap,

@@ -31,6 +31,8 @@ struct DecodeArgs {
     float out_scale;    // 1 / R_V
     int fused;          // the last CTA of a sequence combines its splits
     int cluster;        // the splits of a sequence form one cluster and merge over DSMEM
+    int spec;           // the grid is one wave: hint and copy the first tiles before the
+                        // sequence length is read (else only slots below the length)
     int *err;
     // query factors instead of q (null: use q): element e of sequence b's record
     // [A^Q_0..A^Q_{rq-1} | B^Q_0..B^Q_{rq-1}] at qf[e * qf_stride + b * qf_seq_stride]
@@ -58,14 +60,24 @@ struct MmaDecodeCfg {
     static constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
     static constexpr int EK = ORDER3 ? RK * (MA + DB + DC) : RK * (MA + H2 * D2);
     static constexpr int EV = ORDER3 ? RV * (MA + DB + DC) : SHARED ? RV * MA : RV * (MA + H2 * D2);
+    // d1 = 8 (no shared B, second order): the rows of each 16-row query tile pair up
+    // two j1 of one head per lane, so the sum over j1 and the softmax stay in registers,
+    // and the value product runs once in fp16 (P' = p A^V and B^V rounded to fp16)
+    static constexpr bool KPA8 = D1 == 8 && !SHARED && !ORDER3;
     static constexpr int WARPS = H2 * SLICES;
+    // A warp of its own streams the tiles, or (KPA8) the last consumer warp to release a
+    // stage issues its next tile: sixteen consumer warps then keep 128 registers each
+    // (a seventeenth warp would put five warps, at most 96 registers each, on one SM
+    // sub-partition).
+    static constexpr bool PRODUCER_WARP = !KPA8;
+    static constexpr int THREADS = (WARPS + (PRODUCER_WARP ? 1 : 0)) * 32;
     static constexpr int TT = 16 * CHUNKS * SLICES;             // tokens per stage
     static constexpr int STAGE_BYTES = TT * (EK + EV) * 2;
     // per-warp scratch for the sum over j1 (d1 > 1): [16 tokens][MA + 4] partials,
     // [h1][16] weights, [h1] rescale factors
     static constexpr int RED_LD = MA + 4;
     static constexpr int PPL = D1 > 1 ? (H1 * 16) / 32 : 0;      // (head, token) pairs per lane
-    static constexpr int SCR_FLOATS = D1 > 1 ? ((16 * RED_LD + H1 * 16 + H1 + 3) / 4) * 4 : 0;
+    static constexpr int SCR_FLOATS = D1 > 1 && !KPA8 ? ((16 * RED_LD + H1 * 16 + H1 + 3) / 4) * 4 : 0;
     static constexpr size_t OFF_BARS = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t OFF_Q = OFF_BARS + 16 * STAGES;
     static constexpr int Q_LD = D1 * D2 + 8;                    // padded row of the fp32 query
@@ -77,7 +89,8 @@ struct MmaDecodeCfg {
     static constexpr size_t OFF_FLAGS = OFF_SCR + (size_t)WARPS * SCR_FLOATS * 4;
     // shared B: theta_m (fp64), (cos, sin)(k theta_m) for the 16 token offsets k of a
     // chunk, and per warp (cos, sin)(p0 theta_m) at its chunk's first position p0
-    static constexpr size_t OFF_THETA = OFF_FLAGS + 16;
+    // flags: [0] abort, [1] last CTA, [2] tiles issued, [4 + s] releases of stage s
+    static constexpr size_t OFF_THETA = OFF_FLAGS + 64;
     static constexpr size_t OFF_STEP = OFF_THETA + (SHARED ? (size_t)(D2 / 2) * 8 : 0);
     static constexpr size_t OFF_BASE = OFF_STEP + (SHARED ? (size_t)16 * (D2 / 2) * 8 : 0);
     static constexpr size_t smem_bytes() { return OFF_BASE + (SHARED ? (size_t)WARPS * (D2 / 2) * 8 : 0); }
@@ -85,13 +98,16 @@ struct MmaDecodeCfg {
     // of consecutive heads in different banks
     static constexpr int MO_LD = D1 * D2 + 8;
     static_assert(MA % 16 == 0, "h1*d1 must be a multiple of 16");
-    static_assert(D2 % 16 == 0, "d2 must be a multiple of 16");
+    static_assert(D2 % 16 == 0 || (KPA8 && D2 == 8), "d2 must be a multiple of 16 (or 8 with d1 = 8)");
     static_assert(D1 == 1 || D1 == 2 || D1 == 4 || D1 == 8 || D1 == 16, "d1 must be 1..16, a power of 2");
-    static_assert(D1 == 1 || (H1 >= 2 && 32 % H1 == 0), "h1 must divide 32 when d1 > 1");
+    static_assert(D1 == 1 || KPA8 || (H1 >= 2 && 32 % H1 == 0), "h1 must divide 32 when 1 < d1 < 8");
+    static_assert(!KPA8 || H1 % 2 == 0, "d1 = 8: h1 even (two heads per 16-row tile)");
     static_assert((size_t)SLICES * H * MO_LD * 4 + (size_t)SLICES * H * 8 + (size_t)H * DH * 4 + H * 8 <=
                       (size_t)STAGES * STAGE_BYTES,
                   "slice merge and merged partial must fit in the ring");
     static_assert(WARPS <= 31, "too many consumer warps");
+    static_assert(STAGES <= 12, "stage release counters");
+    static_assert(PRODUCER_WARP || WARPS <= 16, "sixteen warps at most without a producer warp");
     static_assert(smem_bytes() <= 227 * 1024, "shared memory");
     static_assert(!ORDER3 || (D1 == 1 && H2 == 1 && !SHARED && DB == 8 && DC == 8),
                   "third-order mode: TPA split, d_b = d_c = 8 (one c pair per fragment lane)");
@@ -106,13 +122,21 @@ using MmaKpaH4x4D8x16R2Shared = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2, true>;
 // TPA, h = 32, d_h = 64, R_K = R_V = 1 (the FlashTPA decoding benchmark's shape).
 using MmaTpaH32D64R1 = MmaDecodeCfg<32, 1, 64, 1, 1, 1, 8, 2, 2>;
 // KPA h = 4x8, d_h = 8x16, R_K = R_V = 4.
-using MmaKpaH4x8D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 8, 1, 2, 2>;
+using MmaKpaH4x8D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 8, 2, 1, 2>;
 // KPA h = 4x8, d_h = 8x16, R_K = R_V = 2.
-using MmaKpaH4x8D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 8, 1, 4, 2>;
+using MmaKpaH4x8D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 8, 2, 2, 2>;
 // KPA h = 4x4, d_h = 8x16, R_K = R_V = 2.
-using MmaKpaH4x4D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2>;
+using MmaKpaH4x4D8x16R2 = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 4, 1, 2>;
 // Third-order TPA, h = 16, d_h = 8 x 8, R_K = R_V = 2.
 using MmaTpa3H16D8x8R2 = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2, false, 8>;
+// The head splits of "Kronecker Product Attention" section 3.2 (d1 = d2 = 8, R_K = R_V = 2):
+// h = 4x4, 2x8, 8x2 (the 353M models) and 4x5, 2x10, 10x2 (the 773M models).
+using MmaKpaH4x4D8x8R2 = MmaDecodeCfg<32, 8, 8, 2, 2, 4, 4, 1, 2>;
+using MmaKpaH2x8D8x8R2 = MmaDecodeCfg<16, 8, 8, 2, 2, 8, 2, 2, 2>;
+using MmaKpaH8x2D8x8R2 = MmaDecodeCfg<64, 8, 8, 2, 2, 2, 8, 1, 2>;
+using MmaKpaH4x5D8x8R2 = MmaDecodeCfg<32, 8, 8, 2, 2, 5, 3, 2, 2>;
+using MmaKpaH2x10D8x8R2 = MmaDecodeCfg<16, 8, 8, 2, 2, 10, 1, 4, 2>;
+using MmaKpaH10x2D8x8R2 = MmaDecodeCfg<80, 8, 8, 2, 2, 2, 8, 1, 2>;
 
 #define KPA_MMA_VARIANTS(X)        \
     X(0, MmaTpaH16D64R2)           \
@@ -122,7 +146,13 @@ using MmaTpa3H16D8x8R2 = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2, false, 8>;
     X(4, MmaTpaH32D64R1)           \
     X(5, MmaTpaH16D64R2Shared)     \
     X(6, MmaKpaH4x4D8x16R2Shared)  \
-    X(7, MmaTpa3H16D8x8R2)
+    X(7, MmaTpa3H16D8x8R2)         \
+    X(8, MmaKpaH4x4D8x8R2)         \
+    X(9, MmaKpaH2x8D8x8R2)         \
+    X(10, MmaKpaH8x2D8x8R2)        \
+    X(11, MmaKpaH4x5D8x8R2)        \
+    X(12, MmaKpaH2x10D8x8R2)       \
+    X(13, MmaKpaH10x2D8x8R2)
 
 // Index of the variant that covers these dims, or -1.
 inline int mma_decode_variant(const Dims &d) {

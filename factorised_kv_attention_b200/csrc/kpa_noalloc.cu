@@ -59,8 +59,10 @@ extern "C" kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, c
                                          const void *vcache, int32_t capacity,
                                          const int32_t *seq_len, int32_t max_len, float sm_scale,
                                          float *out, kpa_stream stream) {
-    size_t need = 0;
-    kpa_status s = kpa_decode_workspace_size(cfg, batch, max_len, 0, &need);
+    if (batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
+    // the workspace of this (dense-query) decode, and where its counters sit in it
+    size_t need = 0, off = 0, count_bytes = 0;
+    kpa_status s = kpa::decode_dense_plan(cfg, batch, max_len, &need, &off, &count_bytes);
     if (s != KPA_OK) return s;
     if (need > (size_t)KPA_DECODE_NOALLOC_MAX_BYTES) return KPA_ERR_WORKSPACE;
     void *scratch = nullptr;
@@ -68,9 +70,6 @@ extern "C" kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, c
     if (s != KPA_OK) return s;
     // the decode's per-sequence counters must start at zero; an earlier call that
     // stopped on a device error may have left them set
-    size_t off = 0, count_bytes = 0;
-    s = kpa::decode_counter_region(cfg, batch, max_len, &off, &count_bytes);
-    if (s != KPA_OK) return s;
     if (batch > 0 && count_bytes > 0) {
         cudaError_t e = cudaMemsetAsync(static_cast<char *>(scratch) + off, 0, count_bytes,
                                         (cudaStream_t)stream);

@@ -303,7 +303,8 @@ kpa_status kpa_decode_noalloc(const kpa_config *cfg, int32_t batch, const void *
  * and reports KPA_ERR_TIMEOUT; with skip_tile >= 0 the CTA of split
  * `skip_split` of sequence 0 never issues the copy of its tile `skip_tile`, so
  * its consumers' wait runs out.  (-1, -1, 1000000000) restores the defaults.
- * Process-wide; not for concurrent use with real work. */
+ * The setting belongs to the calling host thread: it changes that thread's later
+ * calls only. */
 kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split, uint64_t wait_limit_ns);
 
 /* Testing and measurement: choose the decode kernel.  0 (the default) runs every
@@ -315,8 +316,16 @@ kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split, uint
  * R_Q R_K <= 32, R_K and R_V <= 4, bf16) with the factored score of Proposition 2.2
  * (the FlashTPA form: head-shared dots B^Q_r . B^K_r' per token, then a rank mix per
  * head) on CUDA cores, its splits merged by the combine pass; other calls are
- * unaffected.  Process-wide; returns KPA_ERR_INVALID_ARG for other values. */
+ * unaffected.  The setting belongs to the calling host thread (other threads keep
+ * their own, 0 unless they set it); returns KPA_ERR_INVALID_ARG for other values. */
 kpa_status kpa_test_set_decode_engine(int32_t engine);
+
+/* Testing only: y[i] = 2^x[i] for i < n (device arrays, float32) through the
+ * prefill's FMA-pipe exponential (Cody-Waite reduction to [-1/2, 1/2] and a fitted
+ * degree-4 polynomial, kpa_f32x2.cuh; inputs below -126 are taken as -126), so a
+ * test can compare it with CUDA's exp2f and with float64 over its whole domain.
+ * KPA_ERR_INVALID_ARG for n < 0 or null arrays; asynchronous on `stream`. */
+kpa_status kpa_test_exp2_poly(const float *x, float *y, int64_t n, kpa_stream stream);
 
 /* Wait for `stream`, then return in *code the per-device error word
  * (KPA_OK, KPA_ERR_TIMEOUT or KPA_ERR_DEVICE_CHECK) of the current device and

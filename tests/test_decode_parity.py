@@ -313,3 +313,25 @@ def test_decode_step_reads_the_appends_query_factors():
     vn = to_f64(natural(vc.cpu(), w.batch, w.capacity, s.e_v))
     want = oracle.decode(s, q_rot[:, 0], kn, vn, L.numpy(), keys_rotated=True, sm_scale=scale)
     assert_bf16_close(out.cpu().numpy(), want, "decode step from the append's query factors")
+
+
+@pytest.mark.parametrize("name", sorted(__import__("workloads").KPA_SECTION32))
+def test_section32_head_splits(name):
+    """The six head splits of the KPA paper's section 3.2 (d1 = d2 = 8, R = 2; h = 4x4,
+    2x8, 8x2, 4x5, 2x10, 10x2) run on the tensor cores, and match the oracle end to end
+    (RoPE on the reconstruction) and at stage level, on ragged lengths over several
+    tiles and splits, with a plain and a peaked softmax."""
+    from workloads import KPA_SECTION32
+    lib = kpa()
+    w = KPA_SECTION32[name].replace(batch=3, capacity=1200, length=0, ragged=(1, 1200), seed=61)
+    inp = decode_inputs(w)
+    cfg = lib.make_config(w.shape, w.dtype)
+    max_len = int(inp["seq_len"].max())
+    assert lib.kpa_decode_kernel_kind(cfg, w.batch, max_len) == "mma_sync"
+    got, kc, vc = _run(w, inp)
+    assert_bf16_close(got, oracle_decode_unrotated(w, inp), f"e2e {name}")
+    want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"])
+    assert_bf16_close(got, want, f"stage {name}")
+    scale = 64.0 / np.sqrt(w.shape.dh)
+    got, _, _ = _run(w, inp, sm_scale=float(scale))
+    assert_bf16_close(got, oracle_decode_unrotated(w, inp, sm_scale=scale), f"peaked {name}")

@@ -182,3 +182,80 @@ def test_prefill_from_query_factors(n_tok, starts):
         want = oracle.decode(s, q_rot[b, t][None], kn[b][None], vn[b][None], [L], keys_rotated=True,
                              sm_scale=scale)
         assert_bf16_close(got[b, t], want[0], f"prefill from query factors, row ({b},{t})")
+
+
+def _gpu_chain(lib, w, inp):
+    """The append+prefill path as the library runs it: kpa_append of the chunk (q_out),
+    kpa_prefill from q_out, then the decode step (kpa_append of token n_tok with its
+    query factors left in the workspace, kpa_decode_qf over n_tok + 1 slots)."""
+    s = w.shape
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, w.batch, w.capacity, "bf16")
+    start = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(lib.kpa_append_workspace_size(cfg, w.batch, w.n_tok), dtype=torch.uint8, device="cuda")
+    q_out = torch.empty(w.batch, w.n_tok, s.h, s.dh, dtype=torch.bfloat16, device="cuda")
+    W = inp["W"].cuda()
+    lib.kpa_append(cfg, w.batch, w.n_tok, inp["x"].cuda(), W, start, w.capacity, kc, vc, q_out, ws)
+    scale = 1.0 / np.sqrt(s.dh)
+    out = torch.full((w.batch, w.n_tok, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    lib.kpa_prefill(cfg, w.batch, w.n_tok, q_out, start, kc, vc, w.capacity, scale, out)
+    ws1 = torch.zeros(max(lib.kpa_append_workspace_size(cfg, w.batch, 1), 256), dtype=torch.uint8, device="cuda")
+    pos = torch.full((w.batch,), w.n_tok, dtype=torch.int32, device="cuda")
+    lib.kpa_append(cfg, w.batch, 1, inp["x_step"].cuda(), W, pos, w.capacity, kc, vc, None, ws1)
+    seq = torch.full((w.batch,), w.n_tok + 1, dtype=torch.int32, device="cuda")
+    wsd = torch.zeros(max(lib.kpa_decode_workspace_size(cfg, w.batch, w.n_tok + 1), 256), dtype=torch.uint8,
+                      device="cuda")
+    step = torch.full((w.batch, s.h, s.dh), float("nan"), dtype=torch.float32, device="cuda")
+    lib.kpa_decode_qf(cfg, w.batch, ws1.view(torch.float32), w.batch, 1, None, kc, vc, w.capacity, seq,
+                      w.n_tok + 1, scale, step, wsd)
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == 0
+    return out.cpu().numpy(), step.cpu().numpy(), scale
+
+
+def _oracle_records(w, inp):
+    """oracle.append of the chunk and of the decode step's token: the query rotated by
+    the oracle on its reconstruction, and the unrotated key and value records of slots
+    0 .. n_tok (the oracle rotates each key reconstruction itself when it attends)."""
+    s = w.shape
+    start = np.zeros(w.batch, dtype=np.int64)
+    q_rot, _, v_rec, k_rec = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start)
+    q1, _, v1, k1 = oracle.append(s, to_f64(inp["x_step"]), to_f64(inp["W"]), start + w.n_tok)
+    return q_rot, np.concatenate([k_rec, k1], axis=1), np.concatenate([v_rec, v1], axis=1), q1[:, 0]
+
+
+def test_append_prefill_decode_chain_against_the_plain_definition_every_row():
+    """The append+prefill configuration's shape at 2 x 512 tokens, end to end: every
+    prefill row and the decode step against oracle.append then oracle.prefill /
+    oracle.decode on the unrotated key records (keys_rotated=False: the oracle applies
+    RoPE to each reconstructed key at its slot)."""
+    lib = kpa()
+    w = APPEND_PREFILL.replace(batch=2, n_tok=512, capacity=576, seed=11)
+    inp = append_inputs(w)
+    got, step, scale = _gpu_chain(lib, w, inp)
+    q_rot, kf, vf, q1 = _oracle_records(w, inp)
+    want = oracle.prefill(w.shape, q_rot, kf, vf, [0] * w.batch, keys_rotated=False, sm_scale=scale)
+    assert_bf16_close(got, want, "prefill, every row, against the plain definition")
+    want1 = oracle.decode(w.shape, q1, kf, vf, [w.n_tok + 1] * w.batch, keys_rotated=False, sm_scale=scale)
+    assert_bf16_close(step, want1, "decode step against the plain definition")
+
+
+def test_append_prefill_decode_chain_full_config_against_the_plain_definition():
+    """Configuration 5 at full size, end to end: 64 sampled prefill rows (and the first
+    and last rows of two sequences) and the decode step of all 8 sequences against
+    oracle.append then the oracle's attention on the unrotated key records."""
+    lib = kpa()
+    w = APPEND_PREFILL
+    s = w.shape
+    inp = append_inputs(w)
+    got, step, scale = _gpu_chain(lib, w, inp)
+    q_rot, kf, vf, q1 = _oracle_records(w, inp)
+    rng = np.random.default_rng(12)
+    rows = sorted({(int(b), int(t)) for b, t in zip(rng.integers(0, w.batch, 64), rng.integers(0, w.n_tok, 64))})
+    rows += [(0, 0), (0, w.n_tok - 1), (w.batch - 1, 0), (w.batch - 1, w.n_tok - 1)]
+    for b, t in rows:
+        want = oracle.attend(s, q_rot[b, t][None, None], kf[b][None], vf[b][None], [[t + 1]],
+                             keys_rotated=False, sm_scale=scale)
+        assert_bf16_close(got[b, t], want[0, 0], f"prefill row ({b},{t}) against the plain definition")
+    want1 = oracle.decode(s, q1, kf, vf, [w.n_tok + 1] * w.batch, keys_rotated=False, sm_scale=scale)
+    assert_bf16_close(step, want1, "decode step at 2048 against the plain definition")

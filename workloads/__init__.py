@@ -175,9 +175,23 @@ TPA3_DECODE = DecodeWorkload(
     batch=8, capacity=4096, dtype="bf16", factor_std=float(2.0 ** (1.0 / 6.0)), q_std=1.0 / 8.0,
     seed=0, length=4096)
 
+# The head splits that "Kronecker Product Attention" evaluates in section 3.2 (its tables
+# 1 and 2): d1 = d2 = 8 (d_h = 64), R_K = R_V = 2, h = h1 x h2 with h = 16 (353M models)
+# or 20 (773M models).  The pages give no decode workload for them; these use the TPA
+# decode's batch, length and spreads.
+KPA_SECTION32_SPLITS = {"4x4": (4, 4), "2x8": (2, 8), "8x2": (8, 2), "4x5": (4, 5), "2x10": (2, 10),
+                        "10x2": (10, 2)}
+KPA_SECTION32 = {
+    f"kpa_h{name}_d8x8": DecodeWorkload(
+        name=f"KPA decode, split h={h1}x{h2}, d_h=8x8 (B=8, R=2+2, L=4096, bf16)",
+        shape=Shape(h1=h1, h2=h2, d1=8, d2=8, r_k=2, r_v=2, rope_base=10000.0),
+        batch=8, capacity=4096, dtype="bf16", factor_std=1.0 / np.sqrt(2.0), q_std=1.0 / 8.0, seed=0,
+        length=4096)
+    for name, (h1, h2) in KPA_SECTION32_SPLITS.items()}
+
 DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
                   "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE, "tpa_shared": TPA_SHARED_DECODE,
-                  "tpa_order3": TPA3_DECODE}
+                  "tpa_order3": TPA3_DECODE, **KPA_SECTION32}
 
 
 # --- draws ---------------------------------------------------------------------
@@ -258,3 +272,19 @@ def append_inputs(w: AppendWorkload) -> dict:
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact float64 copy of a float32 / bfloat16 tensor (for the oracle)."""
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def device_decode_factors(w: DecodeWorkload, device, seed: int):
+    """Factor records [B][capacity][E_K], [B][capacity][E_V] and the query [B][h][d_h]
+    drawn on the device (torch's generator, seeded) for throughput sweeps whose sizes
+    make host draws slow: every slot below the capacity holds a record ~ N(0, std^2),
+    the query ~ N(0, q_std^2), rounded to the workload's dtype.  No parity test uses
+    these draws; the oracle takes its inputs from decode_inputs."""
+    s = w.shape
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    kf = (torch.randn(w.batch, w.capacity, s.e_k, generator=g, device=device) * w.factor_std).to(dt)
+    vf = (torch.randn(w.batch, w.capacity, s.e_v, generator=g, device=device) * w.factor_std).to(dt)
+    q = (torch.randn(w.batch, s.h, s.dh, generator=g, device=device) * w.q_std).to(dt)
+    return kf, vf, q
