@@ -159,9 +159,16 @@ def test_split_invariance_and_determinism(name):
         outs[tps] = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"],
                                tokens_per_split=tps).cpu().numpy()
     ref = outs[0]
+    # Plans differ only in summation order, except that the d1 = 8 decode rounds each
+    # P' = p A^V once to fp16 (relative 2^-11) against a running maximum that depends on
+    # the plan.  Those roundings are independent per term, so two plans then agree to
+    # about 2^-12 of the output's norm (times a small factor from the terms' spread):
+    # 1e-3 relative.  Every other path keeps an exact bf16 hi + lo pair: 1e-5.
+    fp16_values = w.shape.d1 == 8 and not w.shape.shared_b and w.shape.order != 3
+    rel_tol = 1e-3 if fp16_values else 1e-5
     for tps, o in outs.items():
         max_abs, rel = errors(o, ref)
-        assert max_abs <= 2e-5 and rel <= 1e-5, f"split {tps}: {max_abs} {rel}"
+        assert max_abs <= 2e-5 and rel <= rel_tol, f"split {tps}: {max_abs} {rel}"
     again = run_decode(lib, w, cfg, kc, vc, inp["q"], inp["seq_len"], inp["q_pos"]).cpu().numpy()
     assert np.array_equal(again, ref), "rerun with the same split is not bitwise equal"
 
