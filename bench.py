@@ -42,7 +42,9 @@ KERNEL_SOURCES = ["factorised_kv_attention_b200/csrc/kpa_decode_mma.cu",
                   "factorised_kv_attention_b200/csrc/kpa_mma_decode.cuh",
                   "factorised_kv_attention_b200/csrc/kpa_decode_fma.cu",
                   "factorised_kv_attention_b200/csrc/kpa_internal.cuh",
-                  "factorised_kv_attention_b200/csrc/kpa_decode_merge.cuh"]
+                  "factorised_kv_attention_b200/csrc/kpa_decode_merge.cuh",
+                  "factorised_kv_attention_b200/csrc/kpa_f32x2.cuh",
+                  "factorised_kv_attention_b200/csrc/kpa_sm100.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 
 

@@ -240,11 +240,17 @@ cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void
 
 // ---------------------------------------------------------------------------
 // Split combine: out = (1/R_V) * sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
-// One block per (head, sequence): the split statistics are staged in shared
-// memory with all loads in flight, then each thread sums its features over the
-// splits with independent, unrolled loads.
+// One block per (head, sequence, chunk of up to 32 features): the split statistics
+// are staged in shared memory with all loads in flight; then the block's threads
+// take (feature, split phase) pairs, sum their features over every eighth split with
+// independent, unrolled loads, and the phases are added through shared memory.
+// Launched as a programmatic dependent of the decode kernel: it becomes resident
+// while the decode's last CTAs still run and waits for them before reading.
+namespace {
+
 constexpr int kCombineThreads = 256;
 constexpr int kCombineMaxSplits = 4096;
+constexpr int kCombineFeatures = 32;
 
 __global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, int tps,
@@ -254,13 +260,19 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
     __shared__ float w[kCombineMaxSplits];
     __shared__ float red[kCombineThreads / 32];
     __shared__ float s_den;
-    const int head = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int fch = d.dh < kCombineFeatures ? d.dh : kCombineFeatures;    // features per block
+    const int n_chunks = (d.dh + fch - 1) / fch;
+    const int head = blockIdx.x / n_chunks, f0 = (blockIdx.x % n_chunks) * fch;
+    const int b = blockIdx.y, tid = threadIdx.x;
+    asm volatile("griddepcontrol.wait;" ::: "memory");        // the decode's partials are complete
+    asm volatile("griddepcontrol.launch_dependents;");
     int L = seq_len[b];
     L = L < 0 ? 0 : (L > max_len ? max_len : L);
     const int ns = min(n_split, (L + tps - 1) / tps);
-    float *dst = out + ((size_t)b * d.h + head) * d.dh;
+    float *dst = out + ((size_t)b * d.h + head) * d.dh + f0;
+    const int nf = min(fch, d.dh - f0);
     if (ns == 0 || ns > kCombineMaxSplits) {
-        for (int f = tid; f < d.dh; f += kCombineThreads) dst[f] = 0.f;
+        for (int f = tid; f < nf; f += kCombineThreads) dst[f] = 0.f;
         return;
     }
     const float2 *ml = reinterpret_cast<const float2 *>(part_ml) + (size_t)b * n_split * d.h + head;
@@ -277,7 +289,7 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
     for (int k = 1; k < kCombineThreads / 32; ++k) M = fmaxf(M, red[k]);
     float den = 0.f;
     for (int i = tid; i < ns; i += kCombineThreads) {
-        const float wi = exp2f(w[i] - M);
+        const float wi = w[i] == -INFINITY ? 0.f : exp2f(w[i] - M);
         w[i] = wi;
         den += wi * ml[(size_t)i * d.h].y;
     }
@@ -291,46 +303,47 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
         s_den = t;
     }
     __syncthreads();
-    if (d.dh > kCombineThreads) {                          // wide heads: one feature per pass
-        const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh;
-        for (int ff = tid; ff < d.dh; ff += kCombineThreads) {
-            float t = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < ns; ++i) t += w[i] * po[(size_t)i * d.h * d.dh + ff];
-            dst[ff] = s_den > 0.f ? out_scale * t / s_den : 0.f;
-        }
-        return;
-    }
-    // features x split phases: threads that share a feature take every P-th split
-    const int P = kCombineThreads / d.dh;
-    const int f = tid % d.dh, phase = tid / d.dh;
+    // (feature, phase) pairs: the phases of one feature take every P-th split
+    const int P = kCombineThreads / fch;
+    const int f = tid % fch, phase = tid / fch;
     float num = 0.f;
-    if (phase < P) {
-        const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh + f;
-#pragma unroll 8
+    if (phase < P && f < nf) {
+        const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh + f0 + f;
+#pragma unroll 4
         for (int i = phase; i < ns; i += P) num += w[i] * po[(size_t)i * d.h * d.dh];
     }
     __syncthreads();
-    float *acc = w;                                        // reuse: [P][dh] partial sums
-    if (phase < P) acc[phase * d.dh + f] = num;
+    float *acc = w;                                        // reuse: [P][fch] partial sums
+    if (phase < P) acc[phase * fch + f] = num;
     __syncthreads();
-    for (int ff = tid; ff < d.dh; ff += kCombineThreads) {
+    for (int ff = tid; ff < nf; ff += kCombineThreads) {
         float t = 0.f;
-        for (int ph = 0; ph < P; ++ph) t += acc[ph * d.dh + ff];
+        for (int ph = 0; ph < P; ++ph) t += acc[ph * fch + ff];
         dst[ff] = s_den > 0.f ? out_scale * t / s_den : 0.f;
     }
 }
+
+}  // namespace
 
 cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_len,
                                   int max_len, const DecodePlan &plan, const float *part_o,
                                   const float *part_ml, float out_scale, float *out,
                                   cudaStream_t st) {
     if (plan.n_split > kCombineMaxSplits) return cudaErrorInvalidValue;
-    dim3 grid((unsigned)d.h, (unsigned)batch);
-    decode_combine_kernel<<<grid, kCombineThreads, 0, st>>>(d, seq_len, max_len,
-                                                            plan.tokens_per_split, plan.n_split,
-                                                            part_o, part_ml, out_scale, out);
-    return cudaGetLastError();
+    const int fch = d.dh < kCombineFeatures ? d.dh : kCombineFeatures;
+    const long long blocks = (long long)d.h * ((d.dh + fch - 1) / fch);
+    if (blocks > 0x7fffffffLL || batch > 65535) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)blocks, (unsigned)batch);
+    lc.blockDim = dim3(kCombineThreads);
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, decode_combine_kernel, d, seq_len, max_len, plan.tokens_per_split, plan.n_split,
+                              part_o, part_ml, out_scale, out);
 }
 
 }  // namespace kpa

@@ -25,6 +25,8 @@
 // returns.
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "kpa_decode_merge.cuh"
 #include "kpa_f32x2.cuh"
 #include "kpa_internal.cuh"
@@ -554,170 +556,179 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         for (int ch = 0; ch < CHUNKS; ++ch) {
             const int tok0 = tok_base + ch * 16;
             if (tok0 >= n_valid) break;
-            const bool tail = tok0 + 16 > n_valid;
-            const unsigned char *kg0 = kt + (size_t)(tok0 >> 3) * EK * 16;
-            // ---- scores of head 2 mt + hi1, tokens (gi, 2c) and (gi, 2c + 1)
-            float2 sc[MT][2];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) sc[mt][0] = sc[mt][1] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < RK; ++r) {
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi) {
-                    const unsigned char *grp = kg0 + (size_t)gi * EK * 16;
-                    uint32_t bk[KQ][2];
-                    const int e_b = A_K + r * H2 * D2 + i2 * D2;
-                    if constexpr (K8) {
-                        ldsm_x1_t(smem_u32(grp + (size_t)(e_b + (lane & 7)) * 16), bk[0][0]);
-                    } else if constexpr (KS % 2 == 0) {
-#pragma unroll
-                        for (int kp = 0; kp < KS / 2; ++kp)
-                            ldsm_x4_t(smem_u32(grp + (size_t)(e_b + kp * 32 + lane) * 16), bk[2 * kp][0],
-                                      bk[2 * kp][1], bk[2 * kp + 1][0], bk[2 * kp + 1][1]);
-                    } else {
-#pragma unroll
-                        for (int ks = 0; ks < KS; ++ks)
-                            ldsm_x2_t(smem_u32(grp + (size_t)(e_b + ks * 16 + (lane & 15)) * 16), bk[ks][0],
-                                      bk[ks][1]);
-                    }
-                    uint32_t ak[MT][2];
-                    a_frags<MT, D1>(smem_u32(grp + (size_t)r * MA * 16) + a_off, ak);
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                        if constexpr (K8) {
-                            mma16808(acc, qa_hi[mt][0][0], qa_hi[mt][0][1], bk[0][0]);
-                            mma16808(acc, qa_lo[mt][0][0], qa_lo[mt][0][1], bk[0][0]);
-                        } else {
-#pragma unroll
-                            for (int ks = 0; ks < KS; ++ks) {
-                                mma16816(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
-                                mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
-                            }
-                        }
-                        sc[mt][gi] = ffma2(make_float2(acc[0], acc[1]), unpack_bf16x2(ak[mt][0]), sc[mt][gi]);
-                        sc[mt][gi] = ffma2(make_float2(acc[2], acc[3]), unpack_bf16x2(ak[mt][1]), sc[mt][gi]);
-                    }
-                }
-            }
-            // ---- the sum over j1: lanes that differ in g & 3
-#pragma unroll
-            for (int off = 4; off <= 8; off <<= 1)
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
+            // a chunk that ends past the tile's valid tokens (the ragged end of a split)
+            // masks its scores and factors; full chunks carry none of that code
+            auto chunk = [&](auto tail_c) {
+                constexpr bool TAIL = decltype(tail_c)::value;
+                const unsigned char *kg0 = kt + (size_t)(tok0 >> 3) * EK * 16;
+                // ---- scores of head 2 mt + hi1, tokens (gi, 2c) and (gi, 2c + 1)
+                float2 sc[MT][2];
+    #pragma unroll
+                for (int mt = 0; mt < MT; ++mt) sc[mt][0] = sc[mt][1] = make_float2(0.f, 0.f);
+    #pragma unroll
+                for (int r = 0; r < RK; ++r) {
+    #pragma unroll
                     for (int gi = 0; gi < 2; ++gi) {
-                        sc[mt][gi].x += __shfl_xor_sync(0xffffffffu, sc[mt][gi].x, off);
-                        sc[mt][gi].y += __shfl_xor_sync(0xffffffffu, sc[mt][gi].y, off);
-                    }
-            if (tail) {
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi) {
-                    const int tk = tok0 + gi * 8 + 2 * c;
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        if (tk >= n_valid) sc[mt][gi].x = -INFINITY;
-                        if (tk + 1 >= n_valid) sc[mt][gi].y = -INFINITY;
-                    }
-                }
-            }
-            // ---- online softmax of this lane's head over the chunk's 16 tokens
-            bool grow = false;
-            float alpha[MT];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                float mx = fmaxf(fmaxf(sc[mt][0].x, sc[mt][0].y), fmaxf(sc[mt][1].x, sc[mt][1].y));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                alpha[mt] = 1.f;
-                if (mx > m_k[mt]) {                     // finite: the chunk has a valid token
-                    alpha[mt] = ex2_approx(m_k[mt] - mx);
-                    m_k[mt] = mx;
-                    grow = true;
-                }
-                const float m_new = m_k[mt];
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi) {
-                    sc[mt][gi].x = ex2_approx(sc[mt][gi].x - m_new);
-                    sc[mt][gi].y = ex2_approx(sc[mt][gi].y - m_new);
-                }
-                l_k[mt] = l_k[mt] * alpha[mt] + ((sc[mt][0].x + sc[mt][0].y) + (sc[mt][1].x + sc[mt][1].y));
-            }
-            if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) o[mt][nt][v] *= alpha[mt];
-            }
-            // ---- values: P'[(i1, j1), token] = p * A^V_r in fp16 (A operand: rows g, g + 8,
-            // tokens 2c, 2c + 1 of group 0 then of group 1)
-            const unsigned char *g0p = vt + (size_t)(tok0 >> 3) * EV * 16;
-            const unsigned char *g1p = g0p + (size_t)EV * 16;
-#pragma unroll
-            for (int r = 0; r < RV; ++r) {
-                uint32_t av[2][MT][2];
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi) {
-                    a_frags<MT, D1>(smem_u32((gi ? g1p : g0p) + (size_t)r * MA * 16) + a_off, av[gi]);
-                }
-                uint32_t pa[MT][4];
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-                    for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-                        for (int hr = 0; hr < 2; ++hr) {
-                            float2 x = fmul2(sc[mt][gi], unpack_bf16x2(av[gi][mt][hr]));
-                            if (tail) {   // garbage factors of masked tokens stay out (their weight is 0)
-                                const int tk = tok0 + gi * 8 + 2 * c;
-                                if (tk >= n_valid) x.x = 0.f;
-                                if (tk + 1 >= n_valid) x.y = 0.f;
-                            }
-                            pa[mt][2 * gi + hr] = pack_h2(x.x, x.y);
+                        const unsigned char *grp = kg0 + (size_t)gi * EK * 16;
+                        uint32_t bk[KQ][2];
+                        const int e_b = A_K + r * H2 * D2 + i2 * D2;
+                        if constexpr (K8) {
+                            ldsm_x1_t(smem_u32(grp + (size_t)(e_b + (lane & 7)) * 16), bk[0][0]);
+                        } else if constexpr (KS % 2 == 0) {
+    #pragma unroll
+                            for (int kp = 0; kp < KS / 2; ++kp)
+                                ldsm_x4_t(smem_u32(grp + (size_t)(e_b + kp * 32 + lane) * 16), bk[2 * kp][0],
+                                          bk[2 * kp][1], bk[2 * kp + 1][0], bk[2 * kp + 1][1]);
+                        } else {
+    #pragma unroll
+                            for (int ks = 0; ks < KS; ++ks)
+                                ldsm_x2_t(smem_u32(grp + (size_t)(e_b + ks * 16 + (lane & 15)) * 16), bk[ks][0],
+                                          bk[ks][1]);
                         }
-                }
-                const int e_b = A_V + r * H2 * D2 + i2 * D2;
-                const int mat = lane >> 3, mr = lane & 7;
-                if constexpr (K8) {
-                    // one n-tile: matrices (group 0, group 1) of the 8 features, lanes 0..15
-                    uint32_t b00, b01;
-                    ldsm_x2(smem_u32(((mat & 1) ? g1p : g0p) + (size_t)(e_b + mr) * 16), b00, b01);
-                    b00 = bf16x2_to_h2(b00);
-                    b01 = bf16x2_to_h2(b01);
-                    if (tail) {
-                        const int tk = tok0 + 2 * c;
-                        b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
-                        b01 = mask_pair(b01, tk + 8 < n_valid, tk + 9 < n_valid);
+                        uint32_t ak[MT][2];
+                        a_frags<MT, D1>(smem_u32(grp + (size_t)r * MA * 16) + a_off, ak);
+    #pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                            if constexpr (K8) {
+                                mma16808(acc, qa_hi[mt][0][0], qa_hi[mt][0][1], bk[0][0]);
+                                mma16808(acc, qa_lo[mt][0][0], qa_lo[mt][0][1], bk[0][0]);
+                            } else {
+    #pragma unroll
+                                for (int ks = 0; ks < KS; ++ks) {
+                                    mma16816(acc, qa_hi[mt][ks], bk[ks][0], bk[ks][1]);
+                                    mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
+                                }
+                            }
+                            sc[mt][gi] = ffma2(make_float2(acc[0], acc[1]), unpack_bf16x2(ak[mt][0]), sc[mt][gi]);
+                            sc[mt][gi] = ffma2(make_float2(acc[2], acc[3]), unpack_bf16x2(ak[mt][1]), sc[mt][gi]);
+                        }
                     }
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) mma16816h(o[mt][0], pa[mt], b00, b01);
                 }
-#pragma unroll
-                for (int np = 0; np < NT / 2; ++np) {
-                    const unsigned char *gp = (mat & 1) ? g1p : g0p;
-                    uint32_t b00, b01, b10, b11;
-                    ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mr) * 16), b00, b01, b10,
-                            b11);
-                    b00 = bf16x2_to_h2(b00);
-                    b01 = bf16x2_to_h2(b01);
-                    b10 = bf16x2_to_h2(b10);
-                    b11 = bf16x2_to_h2(b11);
-                    if (tail) {
-                        const int tk = tok0 + 2 * c;
-                        b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
-                        b10 = mask_pair(b10, tk < n_valid, tk + 1 < n_valid);
-                        b01 = mask_pair(b01, tk + 8 < n_valid, tk + 9 < n_valid);
-                        b11 = mask_pair(b11, tk + 8 < n_valid, tk + 9 < n_valid);
+                // ---- the sum over j1: lanes that differ in g & 3
+    #pragma unroll
+                for (int off = 4; off <= 8; off <<= 1)
+    #pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+    #pragma unroll
+                        for (int gi = 0; gi < 2; ++gi) {
+                            sc[mt][gi].x += __shfl_xor_sync(0xffffffffu, sc[mt][gi].x, off);
+                            sc[mt][gi].y += __shfl_xor_sync(0xffffffffu, sc[mt][gi].y, off);
+                        }
+                if constexpr (TAIL) {
+    #pragma unroll
+                    for (int gi = 0; gi < 2; ++gi) {
+                        const int tk = tok0 + gi * 8 + 2 * c;
+    #pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            if (tk >= n_valid) sc[mt][gi].x = -INFINITY;
+                            if (tk + 1 >= n_valid) sc[mt][gi].y = -INFINITY;
+                        }
                     }
-#pragma unroll
+                }
+                // ---- online softmax of this lane's head over the chunk's 16 tokens
+                bool grow = false;
+                float alpha[MT];
+    #pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    float mx = fmaxf(fmaxf(sc[mt][0].x, sc[mt][0].y), fmaxf(sc[mt][1].x, sc[mt][1].y));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    alpha[mt] = 1.f;
+                    if (mx > m_k[mt]) {                     // finite: the chunk has a valid token
+                        alpha[mt] = ex2_approx(m_k[mt] - mx);
+                        m_k[mt] = mx;
+                        grow = true;
+                    }
+                    const float m_new = m_k[mt];
+    #pragma unroll
+                    for (int gi = 0; gi < 2; ++gi) {
+                        sc[mt][gi].x = ex2_approx(sc[mt][gi].x - m_new);
+                        sc[mt][gi].y = ex2_approx(sc[mt][gi].y - m_new);
+                    }
+                    l_k[mt] = l_k[mt] * alpha[mt] + ((sc[mt][0].x + sc[mt][0].y) + (sc[mt][1].x + sc[mt][1].y));
+                }
+                if (__any_sync(0xffffffffu, grow)) {
+    #pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+    #pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+    #pragma unroll
+                            for (int v = 0; v < 4; ++v) o[mt][nt][v] *= alpha[mt];
+                }
+                // ---- values: P'[(i1, j1), token] = p * A^V_r in fp16 (A operand: rows g, g + 8,
+                // tokens 2c, 2c + 1 of group 0 then of group 1)
+                const unsigned char *g0p = vt + (size_t)(tok0 >> 3) * EV * 16;
+                const unsigned char *g1p = g0p + (size_t)EV * 16;
+    #pragma unroll
+                for (int r = 0; r < RV; ++r) {
+                    uint32_t av[2][MT][2];
+    #pragma unroll
+                    for (int gi = 0; gi < 2; ++gi) {
+                        a_frags<MT, D1>(smem_u32((gi ? g1p : g0p) + (size_t)r * MA * 16) + a_off, av[gi]);
+                    }
+                    uint32_t pa[MT][4];
+    #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
-                        mma16816h(o[mt][2 * np], pa[mt], b00, b01);
-                        mma16816h(o[mt][2 * np + 1], pa[mt], b10, b11);
+    #pragma unroll
+                        for (int gi = 0; gi < 2; ++gi)
+    #pragma unroll
+                            for (int hr = 0; hr < 2; ++hr) {
+                                float2 x = fmul2(sc[mt][gi], unpack_bf16x2(av[gi][mt][hr]));
+                                if constexpr (TAIL) {   // garbage factors of masked tokens stay out (their weight is 0)
+                                    const int tk = tok0 + gi * 8 + 2 * c;
+                                    if (tk >= n_valid) x.x = 0.f;
+                                    if (tk + 1 >= n_valid) x.y = 0.f;
+                                }
+                                pa[mt][2 * gi + hr] = pack_h2(x.x, x.y);
+                            }
+                    }
+                    const int e_b = A_V + r * H2 * D2 + i2 * D2;
+                    const int mat = lane >> 3, mr = lane & 7;
+                    if constexpr (K8) {
+                        // one n-tile: matrices (group 0, group 1) of the 8 features, lanes 0..15
+                        uint32_t b00, b01;
+                        ldsm_x2(smem_u32(((mat & 1) ? g1p : g0p) + (size_t)(e_b + mr) * 16), b00, b01);
+                        b00 = bf16x2_to_h2(b00);
+                        b01 = bf16x2_to_h2(b01);
+                        if constexpr (TAIL) {
+                            const int tk = tok0 + 2 * c;
+                            b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
+                            b01 = mask_pair(b01, tk + 8 < n_valid, tk + 9 < n_valid);
+                        }
+    #pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) mma16816h(o[mt][0], pa[mt], b00, b01);
+                    }
+    #pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const unsigned char *gp = (mat & 1) ? g1p : g0p;
+                        uint32_t b00, b01, b10, b11;
+                        ldsm_x4(smem_u32(gp + (size_t)(e_b + (2 * np + (mat >> 1)) * 8 + mr) * 16), b00, b01, b10,
+                                b11);
+                        b00 = bf16x2_to_h2(b00);
+                        b01 = bf16x2_to_h2(b01);
+                        b10 = bf16x2_to_h2(b10);
+                        b11 = bf16x2_to_h2(b11);
+                        if constexpr (TAIL) {
+                            const int tk = tok0 + 2 * c;
+                            b00 = mask_pair(b00, tk < n_valid, tk + 1 < n_valid);
+                            b10 = mask_pair(b10, tk < n_valid, tk + 1 < n_valid);
+                            b01 = mask_pair(b01, tk + 8 < n_valid, tk + 9 < n_valid);
+                            b11 = mask_pair(b11, tk + 8 < n_valid, tk + 9 < n_valid);
+                        }
+    #pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            mma16816h(o[mt][2 * np], pa[mt], b00, b01);
+                            mma16816h(o[mt][2 * np + 1], pa[mt], b10, b11);
+                        }
                     }
                 }
-            }
+        
+            };
+            if (tok0 + 16 > n_valid)
+                chunk(std::true_type{});
+            else
+                chunk(std::false_type{});
         }
         __syncwarp();
         if (lane == 0) {

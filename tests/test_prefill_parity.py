@@ -213,22 +213,37 @@ def _gpu_chain(lib, w, inp):
     return out.cpu().numpy(), step.cpu().numpy(), scale
 
 
+def _bf16(a):
+    """Round to bf16 (nearest even) and back to float64."""
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.float32).to(
+        torch.bfloat16).to(torch.float64).numpy()
+
+
 def _oracle_records(w, inp):
     """oracle.append of the chunk and of the decode step's token: the query rotated by
     the oracle on its reconstruction, and the unrotated key and value records of slots
-    0 .. n_tok (the oracle rotates each key reconstruction itself when it attends)."""
+    0 .. n_tok (the oracle rotates each key reconstruction itself when it attends).
+
+    The configuration stores bf16 factors, so the end-to-end oracle rounds to bf16 at
+    the two storage points, the cache records and the chunk's q_out (the survey's
+    reading of the rounding points); the decode step's query is assembled from fp32
+    factors and is not rounded.  The library rounds a key record after rotating its B,
+    the oracle before (it rotates the reconstruction): one bf16 rounding apart, which
+    the oracle alone puts at 4e-4 relative on this configuration."""
     s = w.shape
     start = np.zeros(w.batch, dtype=np.int64)
     q_rot, _, v_rec, k_rec = oracle.append(s, to_f64(inp["x"]), to_f64(inp["W"]), start)
     q1, _, v1, k1 = oracle.append(s, to_f64(inp["x_step"]), to_f64(inp["W"]), start + w.n_tok)
-    return q_rot, np.concatenate([k_rec, k1], axis=1), np.concatenate([v_rec, v1], axis=1), q1[:, 0]
+    kf = _bf16(np.concatenate([k_rec, k1], axis=1))
+    vf = _bf16(np.concatenate([v_rec, v1], axis=1))
+    return _bf16(q_rot), kf, vf, q1[:, 0]
 
 
 def test_append_prefill_decode_chain_against_the_plain_definition_every_row():
     """The append+prefill configuration's shape at 2 x 512 tokens, end to end: every
     prefill row and the decode step against oracle.append then oracle.prefill /
     oracle.decode on the unrotated key records (keys_rotated=False: the oracle applies
-    RoPE to each reconstructed key at its slot)."""
+    RoPE to each reconstructed key at its slot), bf16 at the storage points."""
     lib = kpa()
     w = APPEND_PREFILL.replace(batch=2, n_tok=512, capacity=576, seed=11)
     inp = append_inputs(w)
