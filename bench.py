@@ -787,14 +787,15 @@ def run_sweep(a):
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=stream):
                 step()
-            for _ in range(a.warmup):
-                graph.replay()
-            stream.synchronize()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps + 1)]
-            ev[0].record(stream)
-            for i in range(a.steps):
-                graph.replay()
-                ev[i + 1].record(stream)
+            with torch.cuda.stream(stream):          # replays run on the stream the events time
+                for _ in range(a.warmup):
+                    graph.replay()
+                stream.synchronize()
+                ev[0].record(stream)
+                for i in range(a.steps):
+                    graph.replay()
+                    ev[i + 1].record(stream)
             ev[-1].synchronize()
             per = np.array([ev[i].elapsed_time(ev[i + 1]) for i in range(a.steps)]) / layers * 1e3   # us per call
             code = kpa.kpa_read_device_error(stream)

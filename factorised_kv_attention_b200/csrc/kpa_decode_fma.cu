@@ -240,17 +240,18 @@ cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void
 
 // ---------------------------------------------------------------------------
 // Split combine: out = (1/R_V) * sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
-// One block per (head, sequence, chunk of up to 32 features): the split statistics
+// One block per (head, sequence, chunk of up to 16 features): the split statistics
 // are staged in shared memory with all loads in flight; then the block's threads
-// take (feature, split phase) pairs, sum their features over every eighth split with
-// independent, unrolled loads, and the phases are added through shared memory.
+// take (feature, split phase) pairs, sum their features over every 32nd split with
+// independent, unrolled loads (a few per thread, all in flight), and the phases are
+// added through shared memory.
 // Launched as a programmatic dependent of the decode kernel: it becomes resident
 // while the decode's last CTAs still run and waits for them before reading.
 namespace {
 
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 512;
 constexpr int kCombineMaxSplits = 4096;
-constexpr int kCombineFeatures = 32;
+constexpr int kCombineFeatures = 16;
 
 __global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, int tps,
@@ -309,7 +310,7 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
     float num = 0.f;
     if (phase < P && f < nf) {
         const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh + f0 + f;
-#pragma unroll 4
+#pragma unroll 8
         for (int i = phase; i < ns; i += P) num += w[i] * po[(size_t)i * d.h * d.dh];
     }
     __syncthreads();

@@ -552,7 +552,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         const int n_valid = min(TT, t1 - t0 - t * TT);
         const int tok_base = slice * CHUNKS * 16;
 
-#pragma unroll 1
+#pragma unroll
         for (int ch = 0; ch < CHUNKS; ++ch) {
             const int tok0 = tok_base + ch * 16;
             if (tok0 >= n_valid) break;
