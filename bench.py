@@ -70,6 +70,10 @@ def _args(argv=None):
     ap.add_argument("--batch", type=int, default=0, help="override: batch (profiling)")
     ap.add_argument("--tokens-per-split", type=int, default=0,
                     help="override the library's split of each sequence (profiling; multiple of 64)")
+    ap.add_argument("--split-sequence", action="store_true",
+                    help="one sequence split across the ranks: each rank holds a contiguous range of its tokens, "
+                         "decodes it with kpa_decode_lse, and the parts are all-gathered and merged "
+                         "(strong scaling)")
     ap.add_argument("--sweep", choices=["flashtpa"], default=None,
                     help="flashtpa: the FlashTPA decoding shape over sequence lengths 2^12..2^19 and batch "
                          "1, 2, 4, 8, 16 (one JSON line per point, then none of the other lines)")
@@ -118,6 +122,29 @@ def sum_over_ranks(x: float, world: int, device) -> float:
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def split_range(length: int, world: int, rank: int):
+    """The contiguous token range [lo, hi) of a sequence that rank `rank` of `world` holds:
+    equal ranges of whole 8-slot groups, the last rank taking the remainder."""
+    per = (length + world - 1) // world
+    per = (per + 7) // 8 * 8
+    lo = min(length, rank * per)
+    return lo, min(length, lo + per)
+
+
+def gather_parts(out, lse, world):
+    """Every rank's partial decode (out [B][h][d_h], lse [B][h]) gathered in rank order:
+    ([world][B][h][d_h], [world][B][h]).  The one exchange of a split sequence."""
+    import torch
+    if world == 1:
+        return out[None], lse[None]
+    import torch.distributed as dist
+    outs = [torch.empty_like(out) for _ in range(world)]
+    lses = [torch.empty_like(lse) for _ in range(world)]
+    dist.all_gather(outs, out.contiguous())
+    dist.all_gather(lses, lse.contiguous())
+    return torch.stack(outs), torch.stack(lses)
 
 
 def _kernel_hash():
@@ -735,6 +762,117 @@ def run_append_prefill(a):
     return 0
 
 
+def run_split(a):
+    """One sequence split across the ranks (strong scaling): rank r holds the tokens
+    split_range(L, world, r) of every layer's cache in slots 0 .. (kpa_append_factors_pos
+    rotates them at their global positions), decodes them with the query's global
+    position (kpa_decode_lse), and per layer the ranks' (out, lse) are all-gathered over
+    NCCL and merged on every rank (kpa_merge_lse).  Timed per step with CUDA events, the
+    max over ranks; the value counts each sequence's tokens once."""
+    import torch
+    import torch.distributed as dist
+    import factorised_kv_attention_b200 as kpa
+    from workloads import decode_inputs
+
+    rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    w = _workload(a.workload, a)
+    s = w.shape
+    first = decode_inputs(w.replace(seed=rank_seed(0)))      # every rank draws the same sequences
+    lens = first["seq_len"].numpy()
+    L = int(lens.max())
+    lo, hi = split_range(L, world, rank)
+    n = hi - lo
+    cap = max(8, (n + 7) // 8 * 8)
+    elt = 2 if w.dtype == "bf16" else 4
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    layer_bytes = int(lens.sum()) * (s.e_k + s.e_v) * elt
+    local_bytes = int(np.clip(lens - lo, 0, n).sum()) * (s.e_k + s.e_v) * elt
+    layers = a.layers or max(2, int(np.ceil(4 * l2 / max(local_bytes, 1))))
+    cfg = kpa.make_config(s, w.dtype)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    zero = torch.zeros(w.batch, dtype=torch.int32, device=dev)
+    off = torch.full((w.batch,), lo, dtype=torch.int32, device=dev)
+    seq_local = torch.from_numpy(np.clip(lens - lo, 0, n).astype(np.int32)).to(dev)
+    q_pos = first["q_pos"].to(dev)
+    max_local = int(seq_local.max().item())
+    kcs, vcs, qs = [], [], []
+    for layer in range(layers):
+        inp = first if layer == 0 else decode_inputs(w.replace(seed=rank_seed(0, layer)))
+        kc = torch.zeros(w.batch * cap * s.e_k, dtype=tdt, device=dev)
+        vc = torch.zeros(w.batch * cap * s.e_v, dtype=tdt, device=dev)
+        if n > 0:
+            kpa.kpa_append_factors_pos(cfg, w.batch, n, inp["kf"][:, lo:hi].contiguous().to(dev),
+                                       inp["vf"][:, lo:hi].contiguous().to(dev), zero, off, cap, kc, vc)
+        kcs.append(kc)
+        vcs.append(vc)
+        qs.append(inp["q"].to(dev))
+        del inp
+    ws = torch.zeros(max(kpa.kpa_decode_workspace_size(cfg, w.batch, max_local), 256), dtype=torch.uint8,
+                     device=dev)
+    out_l = torch.empty(w.batch, s.h, s.dh, dtype=torch.float32, device=dev)
+    lse_l = torch.empty(w.batch, s.h, dtype=torch.float32, device=dev)
+    outs = [torch.empty(w.batch, s.h, s.dh, dtype=torch.float32, device=dev) for _ in range(layers)]
+    sm_scale = 1.0 / float(np.sqrt(s.dh))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for layer in range(layers):
+            kpa.kpa_decode_lse(cfg, w.batch, qs[layer], q_pos, kcs[layer], vcs[layer], cap, seq_local, max_local,
+                               sm_scale, out_l, lse_l, ws, stream=stream)
+            po, pl = gather_parts(out_l, lse_l, world)
+            kpa.kpa_merge_lse(po, pl, outs[layer], stream=stream)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps + 1)]
+    ev[0].record(stream)
+    for i in range(a.steps):
+        step()
+        ev[i + 1].record(stream)
+    ev[-1].synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    per = np.array([ev[i].elapsed_time(ev[i + 1]) for i in range(a.steps)])
+    ms_step = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dev) / a.steps
+    code = kpa.kpa_read_device_error(stream)
+    if code != 0:
+        raise RuntimeError(f"device error word {code}")
+    t_layer = ms_step * 1e-3 / layers
+    peak, peak_kind = _hbm_peak()
+    n_split, _, _ = kpa.kpa_decode_plan(cfg, w.batch, max(max_local, 1))
+    line = {"metric": METRIC, "value": int(lens.sum()) * layers / (ms_step * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded, shapes of the pages' workloads)",
+            "config": dict(_config_json(w, layers, lens, world),
+                           parallelism=f"sequence split across {world} rank(s): contiguous token ranges, one "
+                                       "all-gather of (out, lse) per layer, log-sum-exp merge",
+                           tokens_per_rank=n, splits_per_sequence_per_rank=n_split),
+            "roofline": {"bound": "hbm", "achieved": layer_bytes / t_layer / 1e9, "peak": peak * world, "unit": "GB/s",
+                         "frac": layer_bytes / t_layer / 1e9 / (peak * world), "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs x {world} GPU(s)",
+                         "kernel": "kpa_decode_lse + all-gather + kpa_merge_lse, per layer",
+                         "algorithmic_bytes_per_launch": layer_bytes, "launch_us": t_layer * 1e6},
+            "ms_per_step_percentiles": {"median": float(np.median(per)), "p10": float(np.percentile(per, 10)),
+                                        "p90": float(np.percentile(per, 90))},
+            "gpu_launches": a.steps * layers * 3}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(a):
     """The FlashTPA decoding benchmark grid ("Tensor Product Attention Is All You Need"
     explainer, decoding-speed figures: sequence 2^12 .. 2^19, batch 1 .. 16) on the
@@ -822,6 +960,8 @@ def main(argv=None):
         return run_reference(a)
     if a.sweep:
         return run_sweep(a)
+    if a.split_sequence:
+        return run_split(a)
     if a.workload == "append_prefill":
         return run_append_prefill(a)
     return run_kpa(a)

@@ -81,6 +81,10 @@ _SIGS = {
     "kpa_test_set_decode_engine": ([_i32], ctypes.c_int),
     "kpa_decode_kernel_kind": ([_cfgp, _i32, _i32, _i32, _i32p], ctypes.c_int),
     "kpa_test_exp2_poly": ([_vp, _vp, ctypes.c_int64, _vp], ctypes.c_int),
+    "kpa_append_factors_pos": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
+    "kpa_decode_lse": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp],
+                       ctypes.c_int),
+    "kpa_merge_lse": ([_i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -253,6 +257,32 @@ def kpa_test_set_decode_hooks(skip_tile=-1, skip_split=-1, wait_limit_ns=1_000_0
 
 def kpa_test_set_decode_engine(engine=0):
     _check(_lib.kpa_test_set_decode_engine(engine), "kpa_test_set_decode_engine")
+
+
+def kpa_append_factors_pos(cfg, batch, n_tok, k_factors, v_factors, start_pos, pos_offset, capacity, kcache,
+                           vcache, stream=None):
+    """kpa_append_factors with the keys of slot start_pos[b] + t rotated at position
+    start_pos[b] + t + pos_offset[b] (a cache holding a range of a longer sequence)."""
+    _check(_lib.kpa_append_factors_pos(ctypes.byref(cfg), batch, n_tok, _addr(k_factors), _addr(v_factors),
+                                       _addr(start_pos), _addr(pos_offset), capacity, _addr(kcache), _addr(vcache),
+                                       _stream(stream)), "kpa_append_factors_pos")
+
+
+def kpa_decode_lse(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len, sm_scale, out, lse,
+                   workspace, ws_bytes=None, stream=None):
+    """kpa_decode that also writes each head's log-sum-exp of its scores into lse [batch][h]."""
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(_lib.kpa_decode_lse(ctypes.byref(cfg), batch, _addr(q), _addr(q_pos), _addr(kcache), _addr(vcache),
+                               capacity, _addr(seq_len), max_len, sm_scale, _addr(out), _addr(lse),
+                               _addr(workspace), ws_bytes, _stream(stream)), "kpa_decode_lse")
+
+
+def kpa_merge_lse(outs, lses, out, lse=None, stream=None):
+    """Log-sum-exp merge of normalised partial decodes: outs [n_parts][batch][h][d_h],
+    lses [n_parts][batch][h] -> out [batch][h][d_h] (and the merged lse when given)."""
+    n_parts, batch, heads, d_h = outs.shape
+    _check(_lib.kpa_merge_lse(batch, heads, d_h, n_parts, _addr(outs), _addr(lses), _addr(out), _addr(lse),
+                              _stream(stream)), "kpa_merge_lse")
 
 
 def kpa_test_exp2_poly(x, y, stream=None):

@@ -144,8 +144,9 @@ int cluster_capacity(int variant, int size) {
 // Split plan.  Auto splits aim at one wave of CTAs: ceil(sms * ctas_per_sm / batch)
 // pieces per sequence, each a multiple of 16 slots.
 // factored_rq > 0: the plan of the factored-score decode from query factors of that rank
+// no_fuse: the splits always end in the combine kernel (the call wants its log-sum-exp).
 kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int tps_req, int sms,
-                       DecodePlan *p, int factored_rq = 0) {
+                       DecodePlan *p, int factored_rq = 0, bool no_fuse = false) {
     if (tps_req < 0 || (tps_req > 0 && tps_req % 64 != 0)) return KPA_ERR_INVALID_ARG;
     p->variant = dt == KPA_BF16 && factored_rq == 0 ? mma_decode_variant(d) : -1;
     if (d.shared && p->variant < 0) return KPA_ERR_UNSUPPORTED;   // shared B: tensor-core variants only
@@ -232,8 +233,9 @@ kpa_status plan_decode(const Dims &d, kpa_dtype dt, int batch, int max_len, int 
     // copies one tile for nothing).  In several waves the later CTAs' latency overlaps the
     // running ones, and the copies of empty splits would only add DRAM traffic.
     p->spec = (int64_t)batch * p->n_split <= (int64_t)target;
-    p->fused = p->cluster ||
-               (p->variant >= 0 && (size_t)p->n_split * d.h * d.dh * sizeof(float) <= 256 * 1024);
+    if (no_fuse) p->cluster = 0;
+    p->fused = !no_fuse && (p->cluster ||
+                            (p->variant >= 0 && (size_t)p->n_split * d.h * d.dh * sizeof(float) <= 256 * 1024));
     const size_t o_bytes = (size_t)batch * p->n_split * d.h * d.dh * sizeof(float);
     const size_t ml_bytes = (size_t)batch * p->n_split * d.h * 2 * sizeof(float);
     p->part_o_off = 0;
@@ -293,28 +295,54 @@ kpa_status kpa_cache_bytes_per_token(const kpa_config *cfg, size_t *k_bytes, siz
     return KPA_OK;
 }
 
-kpa_status kpa_append_factors(const kpa_config *cfg, int32_t batch, int32_t n_tok,
-                              const void *k_factors, const void *v_factors,
-                              const int32_t *start_pos, int32_t capacity, void *kcache,
-                              void *vcache, kpa_stream stream) {
+}  // extern "C"
+
+namespace kpa {
+namespace {
+
+kpa_status append_factors_impl(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *k_factors,
+                               const void *v_factors, const int32_t *start_pos, const int32_t *pos_offset,
+                               int32_t capacity, void *kcache, void *vcache, kpa_stream stream) {
     kpa_status s = check_cfg(cfg, false, false);
     if (s != KPA_OK) return s;
     if (batch < 0 || n_tok < 0) return KPA_ERR_INVALID_ARG;
     if (capacity <= 0 || capacity % KPA_TOKEN_GROUP != 0) return KPA_ERR_INVALID_ARG;
+    // a shared B is rotated in the decode at the slot's own position
+    if (pos_offset && cfg->shared_b) return KPA_ERR_UNSUPPORTED;
     if (batch == 0 || n_tok == 0) return KPA_OK;
     if (!k_factors || !v_factors || !start_pos || !kcache || !vcache) return KPA_ERR_INVALID_ARG;
     if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(k_factors) || !aligned16(v_factors) ||
-        (reinterpret_cast<uintptr_t>(start_pos) & 3))
+        (reinterpret_cast<uintptr_t>(start_pos) & 3) || (reinterpret_cast<uintptr_t>(pos_offset) & 3))
         return KPA_ERR_INVALID_ARG;
     if ((int64_t)n_tok / KPA_TOKEN_GROUP + 2 > INT32_MAX || batch > 65535) return KPA_ERR_UNSUPPORTED;
     int *err = nullptr;
     s = device_state(&err, nullptr);
     if (s != KPA_OK) return s;
     const Dims d = dims_of(cfg);
-    cudaError_t e = launch_append_factors(d, cfg->dtype, batch, n_tok, k_factors, v_factors,
-                                          start_pos, capacity, kcache, vcache, rope_table(cfg),
-                                          err, (cudaStream_t)stream);
+    cudaError_t e = launch_append_factors(d, cfg->dtype, batch, n_tok, k_factors, v_factors, start_pos, pos_offset,
+                                          capacity, kcache, vcache, rope_table(cfg), err, (cudaStream_t)stream);
     return e == cudaSuccess ? KPA_OK : cuda_fail(e);
+}
+
+}  // namespace
+}  // namespace kpa
+
+extern "C" {
+
+kpa_status kpa_append_factors(const kpa_config *cfg, int32_t batch, int32_t n_tok,
+                              const void *k_factors, const void *v_factors,
+                              const int32_t *start_pos, int32_t capacity, void *kcache,
+                              void *vcache, kpa_stream stream) {
+    return append_factors_impl(cfg, batch, n_tok, k_factors, v_factors, start_pos, nullptr, capacity, kcache,
+                               vcache, stream);
+}
+
+kpa_status kpa_append_factors_pos(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *k_factors,
+                                  const void *v_factors, const int32_t *start_pos, const int32_t *pos_offset,
+                                  int32_t capacity, void *kcache, void *vcache, kpa_stream stream) {
+    if (!pos_offset && batch > 0 && n_tok > 0) return KPA_ERR_INVALID_ARG;
+    return append_factors_impl(cfg, batch, n_tok, k_factors, v_factors, start_pos, pos_offset, capacity, kcache,
+                               vcache, stream);
 }
 
 kpa_status kpa_decode_workspace_size(const kpa_config *cfg, int32_t batch, int32_t max_len,
@@ -384,7 +412,8 @@ namespace {
 kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, const float *qf, int32_t qf_stride,
                        int32_t qf_seq_stride, const int32_t *q_pos, const void *kcache, const void *vcache,
                        int32_t capacity, const int32_t *seq_len, int32_t max_len, float sm_scale,
-                       int32_t tokens_per_split, float *out, void *workspace, size_t ws_bytes, kpa_stream stream) {
+                       int32_t tokens_per_split, float *out, void *workspace, size_t ws_bytes, kpa_stream stream,
+                       float *lse = nullptr) {
     kpa_status s = check_cfg(cfg, false, false);
     if (s != KPA_OK) return s;
     if (batch < 0 || max_len < 0) return KPA_ERR_INVALID_ARG;
@@ -397,14 +426,15 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     if ((!q && !qf) || !kcache || !vcache || !seq_len || !out) return KPA_ERR_INVALID_ARG;
     if ((q && !aligned16(q)) || (qf && (reinterpret_cast<uintptr_t>(qf) & 3)) || !aligned16(kcache) ||
         !aligned16(vcache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seq_len) & 3) ||
-        (reinterpret_cast<uintptr_t>(q_pos) & 3))
+        (reinterpret_cast<uintptr_t>(q_pos) & 3) || (reinterpret_cast<uintptr_t>(lse) & 3))
         return KPA_ERR_INVALID_ARG;
     int *err = nullptr, sms = 0;
     s = device_state(&err, &sms);
     if (s != KPA_OK) return s;
     const Dims d = dims_of(cfg);
+    if (lse && d.shared) return KPA_ERR_UNSUPPORTED;              // (its keys rotate at the slot)
     DecodePlan p;
-    s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p);
+    s = plan_decode(d, cfg->dtype, batch, max_len, tokens_per_split, sms, &p, 0, lse != nullptr);
     if (s != KPA_OK) return s;
     // query factors: the factored score on request (TPA shapes), else the tensor-core
     // kernel, which assembles the query (never a third-order cache)
@@ -476,7 +506,9 @@ kpa_status decode_impl(const kpa_config *cfg, int32_t batch, const void *q, cons
     }
     if (e != cudaSuccess) return cuda_fail(e);
     if (max_len > 0 && p.fused) return KPA_OK;
-    e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml, out_scale, out, st);
+    // the partials' statistics are base 2 (the score scale carries log2 e): ln = log2 * ln 2
+    e = launch_decode_combine(d, batch, seq_len, max_len, p, part_o, part_ml, out_scale, out, st, lse,
+                              0.6931471805599453f);
     return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 
@@ -508,6 +540,28 @@ kpa_status kpa_decode(const kpa_config *cfg, int32_t batch, const void *q, const
                       void *workspace, size_t ws_bytes, kpa_stream stream) {
     return kpa_decode_split(cfg, batch, q, q_pos, kcache, vcache, capacity, seq_len, max_len,
                             sm_scale, 0, out, workspace, ws_bytes, stream);
+}
+
+kpa_status kpa_decode_lse(const kpa_config *cfg, int32_t batch, const void *q, const int32_t *q_pos,
+                          const void *kcache, const void *vcache, int32_t capacity, const int32_t *seq_len,
+                          int32_t max_len, float sm_scale, float *out, float *lse, void *workspace, size_t ws_bytes,
+                          kpa_stream stream) {
+    if (!lse && batch > 0 && cfg) return KPA_ERR_INVALID_ARG;
+    return decode_impl(cfg, batch, q, nullptr, 0, 0, q_pos, kcache, vcache, capacity, seq_len, max_len, sm_scale, 0,
+                       out, workspace, ws_bytes, stream, lse);
+}
+
+kpa_status kpa_merge_lse(int32_t batch, int32_t heads, int32_t d_h, int32_t n_parts, const float *outs,
+                         const float *lses, float *out, float *lse, kpa_stream stream) {
+    if (batch < 0 || heads < 0 || d_h < 0 || n_parts < 0) return KPA_ERR_INVALID_ARG;
+    if ((int64_t)batch * heads == 0 || d_h == 0) return KPA_OK;
+    if (n_parts == 0 || !outs || !lses || !out) return KPA_ERR_INVALID_ARG;
+    if (d_h > 1024 || heads > 65535 || batch > 65535 || n_parts > 4096) return KPA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(outs) & 3) || (reinterpret_cast<uintptr_t>(lses) & 3) ||
+        (reinterpret_cast<uintptr_t>(out) & 3) || (reinterpret_cast<uintptr_t>(lse) & 3))
+        return KPA_ERR_INVALID_ARG;
+    cudaError_t e = launch_merge_lse(batch, heads, d_h, n_parts, outs, lses, out, lse, (cudaStream_t)stream);
+    return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 
 kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,

@@ -39,8 +39,8 @@ template <> struct Pack8<float> {
 template <typename T>
 __global__ void __launch_bounds__(256)
 append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__restrict__ vf,
-                      const int32_t *__restrict__ start_pos, int cap, T *__restrict__ kc,
-                      T *__restrict__ vc, RopeTable rope, int *err) {
+                      const int32_t *__restrict__ start_pos, const int32_t *__restrict__ pos_offset, int cap,
+                      T *__restrict__ kc, T *__restrict__ vc, RopeTable rope, int *err) {
     __shared__ float2 cs[kGroup][kMaxHalfD2];   // (cos, sin) per token of the group, per m
 
     const int b = blockIdx.y;
@@ -70,10 +70,13 @@ append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__re
     const int rot_end = d.order == 3 ? a_size + R * d.d1 : E;
     const bool rot_k = is_k && !d.shared;         // a shared B is stored unrotated
     if (rot_k) {
+        // the position of slot s is s, or s + pos_offset[b] for a cache that holds a range of
+        // a longer sequence
+        const int64_t off = pos_offset ? (int64_t)pos_offset[b] : 0;
         for (int i = threadIdx.x; i < kGroup * half; i += blockDim.x) {
             const int k = i / half, m = i % half;
             float c, s;
-            rope_cs((double)(g * kGroup + k), rope.theta[m], c, s);
+            rope_cs((double)(g * kGroup + k + off), rope.theta[m], c, s);
             cs[k][m] = make_float2(c, s);
         }
         __syncthreads();
@@ -120,17 +123,17 @@ append_factors_kernel(Dims d, int n_tok, const T *__restrict__ kf, const T *__re
 
 cudaError_t launch_append_factors(const Dims &d, kpa_dtype dt, int batch, int n_tok,
                                   const void *kf, const void *vf, const int32_t *start_pos,
-                                  int cap, void *kc, void *vc, const RopeTable &rope, int *err,
-                                  cudaStream_t st) {
+                                  const int32_t *pos_offset, int cap, void *kc, void *vc, const RopeTable &rope,
+                                  int *err, cudaStream_t st) {
     // a run of n_tok slots touches at most n_tok/8 + 2 groups
     dim3 grid((unsigned)(n_tok / kGroup + 2), (unsigned)batch, 2);
     if (dt == KPA_BF16)
         append_factors_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            d, n_tok, (const __nv_bfloat16 *)kf, (const __nv_bfloat16 *)vf, start_pos, cap,
+            d, n_tok, (const __nv_bfloat16 *)kf, (const __nv_bfloat16 *)vf, start_pos, pos_offset, cap,
             (__nv_bfloat16 *)kc, (__nv_bfloat16 *)vc, rope, err);
     else
         append_factors_kernel<float><<<grid, 256, 0, st>>>(d, n_tok, (const float *)kf,
-                                                           (const float *)vf, start_pos, cap,
+                                                           (const float *)vf, start_pos, pos_offset, cap,
                                                            (float *)kc, (float *)vc, rope, err);
     return cudaGetLastError();
 }

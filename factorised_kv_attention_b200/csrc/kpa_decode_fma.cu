@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, int tps,
                       int n_split, const float *__restrict__ part_o,
                       const float *__restrict__ part_ml, float out_scale,
-                      float *__restrict__ out) {
+                      float *__restrict__ out, float *__restrict__ lse, float lse_scale) {
     __shared__ float w[kCombineMaxSplits];
     __shared__ float red[kCombineThreads / 32];
     __shared__ float s_den;
@@ -274,6 +274,7 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
     const int nf = min(fch, d.dh - f0);
     if (ns == 0 || ns > kCombineMaxSplits) {
         for (int f = tid; f < nf; f += kCombineThreads) dst[f] = 0.f;
+        if (lse && f0 == 0 && tid == 0) lse[(size_t)b * d.h + head] = -INFINITY;   // no scores
         return;
     }
     const float2 *ml = reinterpret_cast<const float2 *>(part_ml) + (size_t)b * n_split * d.h + head;
@@ -302,6 +303,7 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
         float t = 0.f;
         for (int k = 0; k < kCombineThreads / 32; ++k) t += red[k];
         s_den = t;
+        if (lse && f0 == 0) lse[(size_t)b * d.h + head] = t > 0.f ? (M + log2f(t)) * lse_scale : -INFINITY;
     }
     __syncthreads();
     // (feature, phase) pairs: the phases of one feature take every P-th split
@@ -329,7 +331,7 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
 cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_len,
                                   int max_len, const DecodePlan &plan, const float *part_o,
                                   const float *part_ml, float out_scale, float *out,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, float *lse, float lse_scale) {
     if (plan.n_split > kCombineMaxSplits) return cudaErrorInvalidValue;
     const int fch = d.dh < kCombineFeatures ? d.dh : kCombineFeatures;
     const long long blocks = (long long)d.h * ((d.dh + fch - 1) / fch);
@@ -344,7 +346,55 @@ cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_l
     lc.attrs = attr;
     lc.numAttrs = 1;
     return cudaLaunchKernelEx(&lc, decode_combine_kernel, d, seq_len, max_len, plan.tokens_per_split, plan.n_split,
-                              part_o, part_ml, out_scale, out);
+                              part_o, part_ml, out_scale, out, lse, lse_scale);
+}
+
+namespace {
+
+// One block per (head, sequence), one thread per feature: the parts' weights
+// exp(lse_p - LSE) are formed once per block in shared memory.
+constexpr int kMergeMaxParts = 4096;
+
+__global__ void __launch_bounds__(1024)
+merge_lse_kernel(int heads, int d_h, int n_parts, const float *__restrict__ outs, const float *__restrict__ lses,
+                 float *__restrict__ out, float *__restrict__ lse_out) {
+    __shared__ float w[kMergeMaxParts];
+    __shared__ float s_max, s_den;
+    const int head = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const size_t bh = (size_t)b * heads + head, per_part = (size_t)gridDim.y * heads;
+    if (tid == 0) {
+        float M = -INFINITY;
+        for (int p = 0; p < n_parts; ++p) M = fmaxf(M, lses[p * per_part + bh]);
+        float den = 0.f;
+        for (int p = 0; p < n_parts; ++p) {
+            const float l = lses[p * per_part + bh];
+            const float wp = l == -INFINITY ? 0.f : expf(l - M);
+            w[p] = wp;
+            den += wp;
+        }
+        s_max = M;
+        s_den = den;
+        if (lse_out) lse_out[bh] = den > 0.f ? M + logf(den) : -INFINITY;
+    }
+    __syncthreads();
+    const float inv = s_den > 0.f ? 1.f / s_den : 0.f;
+    for (int f = tid; f < d_h; f += blockDim.x) {
+        float acc = 0.f;
+        for (int p = 0; p < n_parts; ++p)
+            if (w[p] != 0.f) acc = fmaf(w[p], outs[(p * per_part + bh) * d_h + f], acc);
+        out[bh * d_h + f] = acc * inv;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_merge_lse(int batch, int heads, int d_h, int n_parts, const float *outs, const float *lses,
+                             float *out, float *lse_out, cudaStream_t st) {
+    if (n_parts > kMergeMaxParts || d_h > 1024) return cudaErrorInvalidValue;
+    const int threads = d_h < 32 ? 32 : (d_h + 31) / 32 * 32;
+    merge_lse_kernel<<<dim3((unsigned)heads, (unsigned)batch), threads, 0, st>>>(heads, d_h, n_parts, outs, lses, out,
+                                                                                 lse_out);
+    return cudaGetLastError();
 }
 
 }  // namespace kpa

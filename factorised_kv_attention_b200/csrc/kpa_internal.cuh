@@ -104,10 +104,12 @@ inline cudaError_t ensure_dynamic_smem(size_t bytes) {
 void record_cuda_error(cudaError_t e);
 
 // ---- host-side launchers (one per kernel file) ------------------------------
+// pos_offset (nullable, device [batch]): the keys of slot s are rotated at position
+// s + pos_offset[b] instead of s
 cudaError_t launch_append_factors(const Dims &d, kpa_dtype dt, int batch, int n_tok,
                                   const void *kf, const void *vf, const int32_t *start_pos,
-                                  int cap, void *kc, void *vc, const RopeTable &rope, int *err,
-                                  cudaStream_t st);
+                                  const int32_t *pos_offset, int cap, void *kc, void *vc, const RopeTable &rope,
+                                  int *err, cudaStream_t st);
 
 struct DecodePlan {
     int variant;         // tensor-core kernel variant, or -1 for the CUDA-core kernel
@@ -134,10 +136,17 @@ cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void
                               const DecodePlan &plan, float *part_o, float *part_ml,
                               const RopeTable &rope, int *err, cudaStream_t st, int sms);
 
+// lse (nullable, [batch][h]): also the natural-log log-sum-exp of each head's scores,
+// (M + log2 L) * lse_scale with the partials' base-2 statistics (lse_scale = ln 2)
 cudaError_t launch_decode_combine(const Dims &d, int batch, const int32_t *seq_len,
                                   int max_len, const DecodePlan &plan, const float *part_o,
                                   const float *part_ml, float out_scale, float *out,
-                                  cudaStream_t st);
+                                  cudaStream_t st, float *lse = nullptr, float lse_scale = 0.f);
+
+// out[b][h] = sum_p exp(lse_p - LSE) out_p[b][h] over n_parts normalised partial outputs,
+// LSE = ln sum_p exp(lse_p); lse_out (nullable) receives LSE
+cudaError_t launch_merge_lse(int batch, int heads, int d_h, int n_parts, const float *outs, const float *lses,
+                             float *out, float *lse_out, cudaStream_t st);
 
 size_t decode_fma_smem_bytes(const Dims &d, kpa_dtype dt, int tile);
 

@@ -187,6 +187,45 @@ kpa_status kpa_decode(const kpa_config *cfg, int32_t batch, const void *q, const
                       const int32_t *seq_len, int32_t max_len, float sm_scale, float *out,
                       void *workspace, size_t ws_bytes, kpa_stream stream);
 
+/* One long sequence split across GPUs (or any set of caches that each hold a
+ * contiguous range of its tokens): each part decodes its range with the query's
+ * global position and also reports, per head, the log-sum-exp of its scores; an
+ * exchange of (out, lse) between the parts and kpa_merge_lse give the decode of the
+ * whole range.  This is the split-KV merge of the pages' decoding kernel ("Tensor
+ * Product Attention Is All You Need" explainer, "FlashTPA Decoding": the cache is
+ * processed in blocks with an online log-sum-exp) carried across devices.
+ *
+ * kpa_append_factors_pos: kpa_append_factors whose token t of sequence b goes to
+ * slot start_pos[b] + t but is rotated at position start_pos[b] + t + pos_offset[b]
+ * (pos_offset: device [batch] int32, required), so a cache that holds positions
+ * p0 .. p0 + n - 1 of a sequence can keep them in slots 0 .. n - 1.  Other rules as
+ * kpa_append_factors; KPA_ERR_UNSUPPORTED for a shared-B cache (its keys are rotated
+ * in the decode at the slot's position). */
+kpa_status kpa_append_factors_pos(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *k_factors,
+                                  const void *v_factors, const int32_t *start_pos, const int32_t *pos_offset,
+                                  int32_t capacity, void *kcache, void *vcache, kpa_stream stream);
+
+/* kpa_decode that also writes lse [batch][h] float32 (required): the natural
+ * logarithm of sum_s exp(sm_scale q . k_s) over the sequence's slots (the softmax
+ * normaliser, with the key reconstruction's 1/R_K; -inf for an empty sequence).  Its
+ * splits always end in the combine kernel (two launches).  The workspace is sized by
+ * kpa_decode_workspace_size.  KPA_ERR_UNSUPPORTED for a shared-B cache; other rules
+ * as kpa_decode. */
+kpa_status kpa_decode_lse(const kpa_config *cfg, int32_t batch, const void *q, const int32_t *q_pos,
+                          const void *kcache, const void *vcache, int32_t capacity, const int32_t *seq_len,
+                          int32_t max_len, float sm_scale, float *out, float *lse, void *workspace, size_t ws_bytes,
+                          kpa_stream stream);
+
+/* Merge n_parts normalised partial decodes of the same queries (the log-sum-exp
+ * merge): out[b][h] = sum_p exp(lse_p - LSE) out_p[b][h] with LSE = ln sum_p exp(lse_p); a part with lse = -inf (no tokens) adds
+ * nothing, and a head with no tokens in any part gets zeros and LSE = -inf.
+ *   outs [n_parts][batch][heads][d_h] float32, lses [n_parts][batch][heads] float32
+ *   out  [batch][heads][d_h] float32, lse (nullable) [batch][heads]: LSE
+ * All device pointers (4-byte aligned); d_h <= 1024, n_parts <= 4096.  Asynchronous
+ * on `stream`. */
+kpa_status kpa_merge_lse(int32_t batch, int32_t heads, int32_t d_h, int32_t n_parts, const float *outs,
+                         const float *lses, float *out, float *lse, kpa_stream stream);
+
 /* kpa_decode with an explicit split of each sequence into pieces of
  * tokens_per_split slots (a positive multiple of 64, or 0 for the library's
  * choice).  The workspace must be sized with the same tokens_per_split. */

@@ -65,7 +65,7 @@ def _bind(path: str):
     lib.oracle_rotate_record.argtypes = [c_int] * 5 + [c_double, c_double, _dp]
     lib.oracle_project.argtypes = [c_int, c_int, c_int, _dp, _dp, _dp]
     lib.oracle_attend.argtypes = ([c_int] * 6 + [c_double] + [c_int, c_int, _dp, _i64p, _dp, _dp,
-                                   c_int, _i32p, c_int, c_double, _dp, c_int, _i32p])
+                                   c_int, _i32p, c_int, c_double, _dp, c_int, _i32p, _dp])
     lib.oracle_attend.restype = c_int
     lib.oracle_cache_numbers_per_token.argtypes = [c_int] * 6
     lib.oracle_cache_numbers_per_token.restype = ctypes.c_int64
@@ -197,12 +197,13 @@ def compression(h1, h2, d1, d2, r_k, r_v) -> float:
 
 # ------------------------------------------------------------ attention core
 def attend(shape, q, kf, vf, n_keys, *, q_pos=None, keys_rotated=False, sm_scale=None,
-           heads=None) -> np.ndarray:
+           heads=None, return_lse=False):
     """Softmax attention over factor-cache slots (see ``oracle_attend`` in C).
 
     q  [B][n_q][h][dh]; kf, vf [B][cap][E]; n_keys [B][n_q]; q_pos [B][n_q] or None.
     ``heads``: optional iterable of flat ``b*h + head`` indices; other heads come
-    back as NaN.
+    back as NaN.  With ``return_lse`` also the softmax normaliser of each row,
+    ln sum_s exp(score_s), as [B][n_q][h] (-inf with no visible slot).
     """
     s = shape
     h, dh = s.h1 * s.h2, s.d1 * s.d2
@@ -219,25 +220,30 @@ def attend(shape, q, kf, vf, n_keys, *, q_pos=None, keys_rotated=False, sm_scale
         sm_scale = 1.0 / np.sqrt(dh)
     out = np.full((B, n_q, h, dh), np.nan)
     hl = None if heads is None else np.ascontiguousarray(np.asarray(list(heads), dtype=np.int32))
+    lse = np.full((B, n_q, h), np.nan) if return_lse else None
     rc = _load().oracle_attend(
         s.h1, s.h2, s.d1, s.d2, s.r_k, s.r_v, float(s.rope_base), B, n_q, _ptr(q),
         None if qp is None else _ptr(qp, _i64p), _ptr(kf), _ptr(vf), cap, _ptr(nk, _i32p),
         1 if keys_rotated else 0, float(sm_scale), _ptr(out),
-        0 if hl is None else int(hl.size), None if hl is None else _ptr(hl, _i32p))
+        0 if hl is None else int(hl.size), None if hl is None else _ptr(hl, _i32p),
+        None if lse is None else _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_attend rejected its arguments")
-    return out
+    return (out, lse) if return_lse else out
 
 
 def decode(shape, q, kf, vf, seq_len, *, q_pos=None, keys_rotated=False, sm_scale=None,
-           heads=None) -> np.ndarray:
-    """One query row per sequence: q [B][h][dh] -> out [B][h][dh]."""
+           heads=None, return_lse=False):
+    """One query row per sequence: q [B][h][dh] -> out [B][h][dh] (and with
+    ``return_lse`` the softmax normaliser [B][h], see ``attend``)."""
     q = _f64(q)
     B = q.shape[0]
-    out = attend(shape, q[:, None], kf, vf, np.asarray(seq_len).reshape(B, 1),
+    res = attend(shape, q[:, None], kf, vf, np.asarray(seq_len).reshape(B, 1),
                  q_pos=None if q_pos is None else np.asarray(q_pos).reshape(B, 1),
-                 keys_rotated=keys_rotated, sm_scale=sm_scale, heads=heads)
-    return out[:, 0]
+                 keys_rotated=keys_rotated, sm_scale=sm_scale, heads=heads, return_lse=return_lse)
+    if return_lse:
+        return res[0][:, 0], res[1][:, 0]
+    return res[:, 0]
 
 
 def decode_shared_b(shape, q, kf, va, seq_len, *, q_pos=None, sm_scale=None, heads=None) -> np.ndarray:

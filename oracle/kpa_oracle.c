@@ -165,6 +165,8 @@ void oracle_project(int n_tok, int d_model, int n_out, const double *x,
  *  out      [batch][n_q][h][dh]
  *  heads    optional list of n_heads flat (b*h + head) indices to compute;
  *           NULL computes all.  Rows of skipped heads are left untouched.
+ *  lse      optional [batch][n_q][h]: the softmax normaliser of each row,
+ *           ln sum_s exp(score_s) (-inf with no visible slot); NULL skips it.
  *
  * For each (b, head, t): k_s = row `head` of (1/R_K) sum_r A^K_r(s) (x) B^K_r(s)
  * rotated by R_KPA(s); q rotated by R_KPA(q_pos); score_s = sm_scale * q.k_s;
@@ -176,7 +178,7 @@ int oracle_attend(int h1, int h2, int d1, int d2, int r_k, int r_v, double rope_
                   int batch, int n_q, const double *q, const int64_t *q_pos,
                   const double *kf, const double *vf, int cap, const int32_t *n_keys,
                   int keys_rotated, double sm_scale, double *out,
-                  int n_heads, const int32_t *heads)
+                  int n_heads, const int32_t *heads, double *lse)
 {
     const int h = h1 * h2, dh = d1 * d2;
     const int ek = r_k * (h1 * d1 + h2 * d2), ev = r_v * (h1 * d1 + h2 * d2);
@@ -228,12 +230,17 @@ int oracle_attend(int h1, int h2, int d1, int d2, int r_k, int r_v, double rope_
         for (int t = 0; t < n_q; ++t) {
             const int nk = n_keys[(size_t)b * n_q + t] < cap ? n_keys[(size_t)b * n_q + t] : cap;
             double *row = scores + (size_t)t * max_keys;
-            if (nk <= 0) continue;
+            double *lrow = lse ? lse + ((size_t)b * n_q + t) * h + head : NULL;
+            if (nk <= 0) {
+                if (lrow) *lrow = -INFINITY;
+                continue;
+            }
             double mx = row[0];
             for (int s = 1; s < nk; ++s) if (row[s] > mx) mx = row[s];
             double sum = 0.0;
             for (int s = 0; s < nk; ++s) { row[s] = exp(row[s] - mx); sum += row[s]; }
             for (int s = 0; s < nk; ++s) row[s] /= sum;
+            if (lrow) *lrow = mx + log(sum);
         }
         /* pass 2: out[t] = sum_s p[t][s] v_s */
         for (int t = 0; t < n_q; ++t) {

@@ -198,9 +198,10 @@ def check_relative_position(seed=7):
 
 
 # --------------------------------------------------- softmax attention (SDPA)
-def _reference_attention(s: Shape, q, q_pos, kf, vf, n_keys, sm_scale):
+def _reference_attention(s: Shape, q, q_pos, kf, vf, n_keys, sm_scale, return_lse=False):
     """numpy.kron reconstruction, numpy.kron rotation matrices and torch's
-    scaled_dot_product_attention (float64, CPU) with a boolean visibility mask."""
+    scaled_dot_product_attention (float64, CPU) with a boolean visibility mask.  With
+    return_lse also torch.logsumexp of the masked scores Q K^T * sm_scale."""
     B, n_q = q.shape[0], q.shape[1]
     cap = kf.shape[1]
     h, dh = s.h, s.dh
@@ -224,7 +225,11 @@ def _reference_attention(s: Shape, q, q_pos, kf, vf, n_keys, sm_scale):
         torch.from_numpy(Q).permute(0, 2, 1, 3), torch.from_numpy(K).permute(0, 2, 1, 3),
         torch.from_numpy(V).permute(0, 2, 1, 3), attn_mask=torch.from_numpy(mask)[:, None],
         scale=sm_scale).permute(0, 2, 1, 3).numpy()
-    return out
+    if not return_lse:
+        return out
+    scores = np.einsum("bqhd,bkhd->bqhk", Q, K) * sm_scale
+    scores = np.where(mask[:, :, None, :], scores, -np.inf)
+    return out, torch.logsumexp(torch.from_numpy(scores), dim=-1).numpy()
 
 
 def check_attention_matches_sdpa(seed=8):
@@ -239,6 +244,26 @@ def check_attention_matches_sdpa(seed=8):
         got = oracle.attend(s, q, kf, vf, n_keys, q_pos=q_pos, sm_scale=scale)
         want = _reference_attention(s, q, q_pos, kf, vf, n_keys, scale)
         _close(got, want, 1e-11, f"attention vs SDPA {s}")
+
+
+def check_attention_lse(seed=18):
+    """The softmax normaliser ln sum_s exp(score_s) of each row against torch.logsumexp
+    of the reference scores; one visible slot gives that slot's score; none gives -inf."""
+    rng = np.random.default_rng(seed)
+    for s in [SHAPES[0], SHAPES[3], Shape(h1=2, h2=2, d1=4, d2=4, r_k=2, r_v=1)]:
+        B, n_q, cap = 2, 3, 9
+        q = rng.standard_normal((B, n_q, s.h, s.dh))
+        kf = rng.standard_normal((B, cap, s.e_k)); vf = rng.standard_normal((B, cap, s.e_v))
+        q_pos = rng.integers(0, 600000, size=(B, n_q))
+        n_keys = rng.integers(1, cap + 1, size=(B, n_q)).astype(np.int32)
+        n_keys[0, 0] = 1
+        scale = 0.7 / math.sqrt(s.dh)
+        got_o, got_l = oracle.attend(s, q, kf, vf, n_keys, q_pos=q_pos, sm_scale=scale, return_lse=True)
+        want_o, want_l = _reference_attention(s, q, q_pos, kf, vf, n_keys, scale, return_lse=True)
+        _close(got_o, want_o, 1e-11, f"attention (with lse) vs SDPA {s}")
+        _close(got_l, want_l, 1e-11, f"lse vs logsumexp {s}")
+    _, l0 = oracle.attend(s, q, kf, vf, np.zeros((B, n_q), np.int32), q_pos=q_pos, return_lse=True)
+    assert np.all(np.isneginf(l0)), "no visible slot: -inf"
 
 
 def check_attention_closed_forms(seed=9):
@@ -438,7 +463,7 @@ ALL_CHECKS = [
     check_kron_is_numpy_kron, check_reconstruct_is_kron_sum, check_tpa_split_is_outer_product,
     check_prop22_factored_score, check_rope_golden_frequencies, check_rope_tpa_is_textbook,
     check_rope_kpa_is_identity_kron_rotation, check_thm24_rotating_b_equals_rotating_reconstruction,
-    check_relative_position, check_attention_matches_sdpa, check_attention_closed_forms,
+    check_relative_position, check_attention_matches_sdpa, check_attention_lse, check_attention_closed_forms,
     check_prefill_rows_are_decodes, check_projection_is_matmul, check_append_scores_follow_eq9,
     check_cache_sizes_golden, check_shared_b_attention, check_order3_attention,
 ]

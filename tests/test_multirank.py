@@ -3,7 +3,10 @@ them, check the pieces that decide the reported numbers.
 
   - each rank draws its own batch (replicas shard the batch; no data exchange);
   - device times combine as the maximum over ranks, work as the sum over ranks;
-  - the reference arm runs on rank 0 only: other ranks exit 0 without work or output.
+  - the reference arm runs on rank 0 only: other ranks exit 0 without work or output;
+  - a sequence split across the ranks: the ranges cover it exactly, and each rank's
+    partial decode (the oracle's, over its range, with the normaliser) gathered over
+    the process group and merged by the log-sum-exp rule is the whole sequence's decode.
 """
 import contextlib
 import io
@@ -44,6 +47,32 @@ def _worker(rank, world, port, results):
         gathered = [None] * world
         dist.all_gather_object(gathered, lens)
         out["lens"] = gathered
+        # one sequence split across the ranks: keys stored rotated at their global positions
+        import numpy as np
+        import torch
+
+        import oracle
+        from workloads import KPA_LONG, to_f64
+        ws = KPA_LONG.replace(capacity=304, length=300, seed=9)
+        si = decode_inputs(ws)
+        s = ws.shape
+        kf, vf, q = to_f64(si["kf"]), to_f64(si["vf"]), to_f64(si["q"])
+        kr = np.stack([[oracle.rotate_record(s.h1, s.h2, s.d1, s.d2, s.r_k, s.rope_base, t, kf[b, t])
+                        for t in range(ws.capacity)] for b in range(ws.batch)])
+        lo, hi = bench.split_range(300, world, rank)
+        q_rot = np.stack([[oracle.rope_kpa(s.d1, s.d2, s.rope_base, 300, q[b, h]) for h in range(s.h)]
+                          for b in range(ws.batch)])
+        o_p, l_p = oracle.decode(s, q_rot, kr[:, lo:hi], vf[:, lo:hi], [hi - lo] * ws.batch, keys_rotated=True,
+                                 return_lse=True)
+        outs, lses = bench.gather_parts(torch.from_numpy(o_p), torch.from_numpy(l_p), world)
+        outs, lses = outs.numpy(), lses.numpy()
+        M = lses.max(axis=0)
+        wgt = np.exp(lses - M)
+        merged = (wgt[..., None] * outs).sum(axis=0) / wgt.sum(axis=0)[..., None]
+        whole = oracle.decode(s, q, kf, vf, si["seq_len"].numpy(), q_pos=si["q_pos"].numpy())
+        out["split_err"] = float(np.max(np.abs(merged - whole)))
+        out["ranges"] = [bench.split_range(L, W, r) for L in (0, 1, 9, 300, 524288, 4101) for W in (1, 2, 3, 8)
+                         for r in range(W)]
         buf = io.StringIO()
         with contextlib.redirect_stdout(buf):
             rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "1"]) if rank != 0 else 0
@@ -77,3 +106,13 @@ def test_two_gloo_ranks():
     assert lens == got[1]["lens"]
     assert lens[0] != lens[1], "replicas must draw different batches"
     assert got[1]["ref_rc"] == 0 and got[1]["ref_out"] == "", "reference arm runs on rank 0 only"
+    for rank in range(world):
+        assert got[rank]["split_err"] <= 1e-12, f"split-sequence merge: {got[rank]['split_err']}"
+    # the ranges of a split cover [0, L) with contiguous, ordered, group-aligned pieces
+    it = iter(got[0]["ranges"])
+    for L in (0, 1, 9, 300, 524288, 4101):
+        for W in (1, 2, 3, 8):
+            ranges = [next(it) for _ in range(W)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == L
+            for (a0, a1), (b0, b1) in zip(ranges[:-1], ranges[1:]):
+                assert a1 == b0 and a0 <= a1 and (a1 % 8 == 0 or a1 == L)

@@ -33,6 +33,7 @@ MUTATIONS = [
      "return (int64_t)(r_k + r_v) * ((int64_t)h1 + (int64_t)h2 * d2);"),
     ("value row from the key factors", "oracle_kron_sum_row(h1, h2, d1, d2, r_v, vf + ((size_t)b * cap + s) * ev,",
      "oracle_kron_sum_row(h1, h2, d1, d2, r_v, kf + ((size_t)b * cap + s) * ev,"),
+    ("normaliser without the maximum", "if (lrow) *lrow = mx + log(sum);", "if (lrow) *lrow = log(sum);"),
 ]
 
 
