@@ -330,9 +330,66 @@ def _cpu_baseline(w, inp, seconds, steps=None, q_factors=None, call_seconds=2.5,
     return base, times
 
 
+def _cpu_baseline_prefill(w, inp, seconds, steps=None, call_seconds=2.5):
+    """The float64 oracle on the append+prefill workload: a call takes the first n
+    prompt tokens of one sequence through oracle.append (projection, the rank-major
+    split, RoPE on the B factors and on the assembled query) and oracle.prefill (each
+    row over the block's slots up to its own).  n is the largest of 2048, 1024, ... 64
+    whose time, scaled from a 64-token call by the prefill's n^2, fits call_seconds.
+    Calls run over the sequences in turn until `seconds` pass (or `steps` calls)."""
+    import oracle
+    from workloads import to_f64
+    oracle.build()
+    s = w.shape
+    x, W = to_f64(inp["x"]), to_f64(inp["W"])
+    scale = 1.0 / float(np.sqrt(s.dh))
+
+    def call(b, n):
+        t0 = time.perf_counter()
+        q_rot, k_rot, v_rec, _ = oracle.append(s, x[b:b + 1, :n], W, [0])
+        oracle.prefill(s, q_rot, k_rot, v_rec, [0], keys_rotated=True, sm_scale=scale)
+        return time.perf_counter() - t0
+
+    t64 = max(call(0, 64), 1e-6)
+    n = 64
+    while n < w.n_tok and t64 * (2 * n / 64) ** 2 <= call_seconds:
+        n *= 2
+    n = min(n, w.n_tok)
+    done, t_total, times, b = 0, 0.0, [], 0
+    while (steps is None and t_total < seconds) or (steps is not None and len(times) < steps):
+        dt = call(b, n)
+        times.append(dt)
+        t_total += dt
+        done += n
+        b = (b + 1) % w.batch
+    return {"value": done / t_total, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{len(times)} calls of the first {n} prompt tokens of one sequence (of {w.n_tok}): float64 "
+                      f"projection, RoPE and causal prefill over the block, OpenMP over heads, {t_total:.1f} s",
+            "cpu_model": _cpu_model()}, times
+
+
 def run_reference(a):
     rank, world, _ = _dist()
     if rank != 0:
+        return 0
+    if a.workload == "append_prefill":
+        from workloads import APPEND_PREFILL, append_inputs
+        w = APPEND_PREFILL
+        inp = append_inputs(w)
+        per_call = min(2.5, 120.0 / max(a.steps + a.warmup, 1))
+        _cpu_baseline_prefill(w, inp, 0, steps=a.warmup, call_seconds=per_call)
+        base, times = _cpu_baseline_prefill(w, inp, 0, steps=a.steps, call_seconds=per_call)
+        line = {"impl": "reference", "metric": "append + causal prefill + decode step, tokens/s (2048-token chunks); "
+                                              "TFLOP/s vs B200 bf16 peak",
+                "value": base["value"], "unit": "tokens/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+                "ms_per_step": 1e3 * float(np.sum(times)) / max(len(times), 1), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_tok, "d_model": w.shape.d_model,
+                           "sample": "one call per step: a block of prompt tokens of one sequence"},
+                "cpu_baseline": base,
+                "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
         return 0
     from workloads import decode_inputs
     w = _workload(a.workload, a)
@@ -754,6 +811,8 @@ def run_append_prefill(a):
                     "d2h_bytes_per_step": int(out_host.numel() * 4 + out1_host.numel() * 4),
                     "ms_per_step": ms_e2e},
             "clocks": clocks, "gpu_launches": a.steps * launches_per_step}
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"], _ = _cpu_baseline_prefill(w, inp, a.cpu_seconds)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
