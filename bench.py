@@ -77,6 +77,12 @@ def _args(argv=None):
     ap.add_argument("--sweep", choices=["flashtpa"], default=None,
                     help="flashtpa: the FlashTPA decoding shape over sequence lengths 2^12..2^19 and batch "
                          "1, 2, 4, 8, 16 (one JSON line per point, then none of the other lines)")
+    ap.add_argument("--prefill-split", default="kpa_h4x4_d8x16_r2",
+                    choices=["kpa_h4x4_d8x16_r2", "tpa_h16_d1x128_r2", "kpa_h4x4_d8x16_r4"],
+                    help="append_prefill: the Kronecker split of its h=16, d_h=128 (the tcgen05 prefill takes the "
+                         "first, the mma.sync prefill the others)")
+    ap.add_argument("--prefill-engine", type=int, default=0, choices=(0, 1),
+                    help="1: the mma.sync prefill on every split (measurement)")
     ap.add_argument("--settle-seconds", type=float, default=1.0,
                     help="untimed load before timing while clocks are sampled (0 for profiling)")
     a = ap.parse_args(argv)
@@ -373,8 +379,8 @@ def run_reference(a):
     if rank != 0:
         return 0
     if a.workload == "append_prefill":
-        from workloads import APPEND_PREFILL, append_inputs
-        w = APPEND_PREFILL
+        from workloads import APPEND_PREFILL_SPLITS, append_inputs
+        w = APPEND_PREFILL_SPLITS[a.prefill_split]
         inp = append_inputs(w)
         per_call = min(2.5, 120.0 / max(a.steps + a.warmup, 1))
         _cpu_baseline_prefill(w, inp, 0, steps=a.warmup, call_seconds=per_call)
@@ -676,7 +682,7 @@ def run_append_prefill(a):
     import torch
     import torch.distributed as dist
     import factorised_kv_attention_b200 as kpa
-    from workloads import APPEND_PREFILL, append_inputs
+    from workloads import APPEND_PREFILL_SPLITS, append_inputs
 
     rank, world, local = _dist()
     torch.cuda.set_device(local)
@@ -684,10 +690,12 @@ def run_append_prefill(a):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    w = APPEND_PREFILL
+    w = APPEND_PREFILL_SPLITS[a.prefill_split]
     s = w.shape
     inp = append_inputs(w.replace(seed=rank_seed(rank)))
     cfg = kpa.make_config(s, "bf16")
+    kpa.kpa_test_set_prefill_engine(a.prefill_engine)
+    prefill_kernel = kpa.kpa_prefill_kernel_kind(cfg)
     x, W, x1 = inp["x"].to(dev), inp["W"].to(dev), inp["x_step"].to(dev)
     kc = torch.zeros(w.batch * w.capacity * s.e_k, dtype=torch.bfloat16, device=dev)
     vc = torch.zeros(w.batch * w.capacity * s.e_v, dtype=torch.bfloat16, device=dev)
@@ -719,12 +727,22 @@ def run_append_prefill(a):
     def prefill():
         kpa.kpa_prefill(cfg, w.batch, w.n_tok, q, start, kc, vc, w.capacity, scale, out, stream=stream)
 
+    # the decode step reads the one-token append's query factors where a tensor-core decode
+    # variant takes this split (kpa_decode_qf), else the append's dense rotated query
+    step_qf = kpa.kpa_decode_kernel_kind(cfg, w.batch, w.n_tok + 1) == "mma_sync"
+    q1 = torch.empty(w.batch, 1, s.h, s.dh, dtype=torch.bfloat16, device=dev)
+
     def decode_step():
         # one-token append (matrix-vector projection, RoPE, cache write; query factors into
         # its workspace), then decode straight from those query factors
-        kpa.kpa_append(cfg, w.batch, 1, x1, W, pos1, w.capacity, kc, vc, None, ws1, stream=stream)
-        kpa.kpa_decode_qf(cfg, w.batch, qf1, w.batch, 1, None, kc, vc, w.capacity, len1, w.n_tok + 1, scale, out1,
-                          wsd, stream=stream)
+        if step_qf:
+            kpa.kpa_append(cfg, w.batch, 1, x1, W, pos1, w.capacity, kc, vc, None, ws1, stream=stream)
+            kpa.kpa_decode_qf(cfg, w.batch, qf1, w.batch, 1, None, kc, vc, w.capacity, len1, w.n_tok + 1, scale,
+                              out1, wsd, stream=stream)
+        else:
+            kpa.kpa_append(cfg, w.batch, 1, x1, W, pos1, w.capacity, kc, vc, q1, ws1, stream=stream)
+            kpa.kpa_decode(cfg, w.batch, q1, None, kc, vc, w.capacity, len1, w.n_tok + 1, scale, out1, wsd,
+                           stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(a.warmup):
@@ -798,7 +816,7 @@ def run_append_prefill(a):
             "roofline": {"bound": "tensor", "achieved": pre_tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": pre_tf / peak, "traffic": None,
                          "peak_source": f"{kind} bf16_tflops (burst; fp16 dense rate is the same)",
-                         "kernel": "kpa_prefill", "algorithmic_flop_per_launch": pre_flop,
+                         "kernel": f"kpa_prefill ({prefill_kernel})", "algorithmic_flop_per_launch": pre_flop,
                          "launch_us": t_pre * 1e6},
             "append": {"achieved_tflops": app_tf, "frac": app_tf / peak, "launch_us": t_app * 1e6,
                        "algorithmic_flop_per_launch": proj_flop},

@@ -80,6 +80,8 @@ _SIGS = {
     "kpa_test_set_decode_hooks": ([_i32, _i32, ctypes.c_uint64], ctypes.c_int),
     "kpa_test_set_decode_engine": ([_i32], ctypes.c_int),
     "kpa_decode_kernel_kind": ([_cfgp, _i32, _i32, _i32, _i32p], ctypes.c_int),
+    "kpa_prefill_kernel_kind": ([_cfgp, _i32p], ctypes.c_int),
+    "kpa_test_set_prefill_engine": ([_i32], ctypes.c_int),
     "kpa_test_exp2_poly": ([_vp, _vp, ctypes.c_int64, _vp], ctypes.c_int),
     "kpa_append_factors_pos": ([_cfgp, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp], ctypes.c_int),
     "kpa_decode_lse": ([_cfgp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp],
@@ -172,6 +174,16 @@ def kpa_decode_kernel_kind(cfg, batch, max_len, tokens_per_split=0):
     return DECODE_KERNEL_NAMES[k.value]
 
 
+PREFILL_KERNEL_NAMES = {1: "mma_sync", 2: "tcgen05"}
+
+
+def kpa_prefill_kernel_kind(cfg):
+    """Name of the kernel kpa_prefill runs for this config on the calling thread."""
+    k = ctypes.c_int32()
+    _check(_lib.kpa_prefill_kernel_kind(ctypes.byref(cfg), ctypes.byref(k)), "kpa_prefill_kernel_kind")
+    return PREFILL_KERNEL_NAMES[k.value]
+
+
 def kpa_decode_qf(cfg, batch, q_factors, qf_stride, qf_seq_stride, q_pos, kcache, vcache, capacity, seq_len,
                   max_len, sm_scale, out, workspace, ws_bytes=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
@@ -257,6 +269,10 @@ def kpa_test_set_decode_hooks(skip_tile=-1, skip_split=-1, wait_limit_ns=1_000_0
 
 def kpa_test_set_decode_engine(engine=0):
     _check(_lib.kpa_test_set_decode_engine(engine), "kpa_test_set_decode_engine")
+
+
+def kpa_test_set_prefill_engine(engine=0):
+    _check(_lib.kpa_test_set_prefill_engine(engine), "kpa_test_set_prefill_engine")
 
 
 def kpa_append_factors_pos(cfg, batch, n_tok, k_factors, v_factors, start_pos, pos_offset, capacity, kcache,

@@ -10,6 +10,7 @@
 #include "kpa_decode_factored.cuh"
 #include "kpa_internal.cuh"
 #include "kpa_mma_decode.cuh"
+#include "kpa_prefill_mma.cuh"
 
 namespace kpa {
 
@@ -119,6 +120,7 @@ thread_local DecodeTestHooks t_hooks = {-1, -1, 1000000000ull};
 // score for decodes from query factors on TPA shapes (testing and measurement: both are
 // slower than the defaults on the shapes measured so far).
 thread_local int t_decode_engine = 0;
+thread_local int t_prefill_engine = 0;
 
 DecodeTestHooks current_hooks() { return t_hooks; }
 
@@ -573,6 +575,26 @@ kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int3
     return KPA_OK;
 }
 
+// Which prefill kernel takes these dims on the calling thread: the tcgen05 kernel
+// where it is instantiated (unless the thread chose the mma.sync kernel), else the
+// mma.sync kernel where it fits, else -1.
+static int prefill_kind(const Dims &d) {
+    if (d.order == 3) return -1;
+    if (prefill_supported(d) && t_prefill_engine == 0) return KPA_PREFILL_KERNEL_TCGEN05;
+    return prefill_mma_supported(d) ? KPA_PREFILL_KERNEL_MMA_SYNC : -1;
+}
+
+kpa_status kpa_prefill_kernel_kind(const kpa_config *cfg, int32_t *kind) {
+    kpa_status s = check_cfg(cfg, false, false);
+    if (s != KPA_OK) return s;
+    if (!kind) return KPA_ERR_INVALID_ARG;
+    if (cfg->dtype != KPA_BF16) return KPA_ERR_UNSUPPORTED;
+    const int k = prefill_kind(dims_of(cfg));
+    if (k < 0) return KPA_ERR_UNSUPPORTED;
+    *kind = k;
+    return KPA_OK;
+}
+
 // The prefill with a dense bf16 query (q) or with query factors (qf.ptr).
 static kpa_status prefill_impl(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *q,
                                const PrefillQf &qf, const int32_t *start_pos, const void *kcache,
@@ -586,7 +608,8 @@ static kpa_status prefill_impl(const kpa_config *cfg, int32_t batch, int32_t n_t
     if (qf.ptr && (qf.stride <= 0 || qf.seq_stride < 0 || qf.tok_stride < 0)) return KPA_ERR_INVALID_ARG;
     if (cfg->dtype != KPA_BF16 || cfg->order == 3) return KPA_ERR_UNSUPPORTED;
     const Dims d = dims_of(cfg);
-    if (!prefill_supported(d)) return KPA_ERR_UNSUPPORTED;
+    const int kind = prefill_kind(d);
+    if (kind < 0) return KPA_ERR_UNSUPPORTED;
     if (qf.ptr && cfg->r_q > kPrefillQfMaxRq) return KPA_ERR_UNSUPPORTED;
     if (batch == 0 || n_tok == 0) return KPA_OK;
     if (batch > 65535 || d.h > 65535 || (int64_t)batch * n_tok > INT32_MAX / 2) return KPA_ERR_UNSUPPORTED;
@@ -598,9 +621,13 @@ static kpa_status prefill_impl(const kpa_config *cfg, int32_t batch, int32_t n_t
     s = device_state(&err, nullptr);
     if (s != KPA_OK) return s;
     const float qscale = (float)((double)sm_scale / (double)d.rk * 1.4426950408889634);
-    cudaError_t e = launch_prefill(d, batch, n_tok, q, qf, start_pos, kcache, vcache, capacity, qscale,
-                                   (float)(1.0 / (double)d.rv), out, rope_table(cfg), err,
-                                   current_hooks().wait_limit_ns, (cudaStream_t)stream);
+    const float out_scale = (float)(1.0 / (double)d.rv);
+    cudaError_t e = kind == KPA_PREFILL_KERNEL_TCGEN05
+                        ? launch_prefill(d, batch, n_tok, q, qf, start_pos, kcache, vcache, capacity, qscale,
+                                         out_scale, out, rope_table(cfg), err, current_hooks().wait_limit_ns,
+                                         (cudaStream_t)stream)
+                        : launch_prefill_mma(d, batch, n_tok, q, qf, start_pos, kcache, vcache, capacity, qscale,
+                                             out_scale, out, rope_table(cfg), err, (cudaStream_t)stream);
     return e == cudaSuccess ? KPA_OK : cuda_fail(e);
 }
 
@@ -684,6 +711,12 @@ kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split,
     t_hooks.skip_tile = skip_tile;
     t_hooks.skip_split = skip_split;
     t_hooks.wait_limit_ns = wait_limit_ns;
+    return KPA_OK;
+}
+
+kpa_status kpa_test_set_prefill_engine(int32_t engine) {
+    if (engine < 0 || engine > 1) return KPA_ERR_INVALID_ARG;
+    t_prefill_engine = engine;
     return KPA_OK;
 }
 

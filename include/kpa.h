@@ -261,18 +261,34 @@ kpa_status kpa_decode_qf(const kpa_config *cfg, int32_t batch, const float *q_fa
 /* Causal chunked attention in factor space (prefill).  Row t of sequence b is
  * the query at position start_pos[b] + t and sees slots 0 .. start_pos[b] + t
  * (its own key included), which must already be in the cache (kpa_append or
- * kpa_append_factors).  K/V tiles are rebuilt from the factors on chip only.
+ * kpa_append_factors).  K/V tiles are rebuilt from the factors on chip only
+ * ("Kronecker Product Attention", section 2.2, eq 4; Proposition 2.2), with fp16
+ * products and fp32 accumulation.
  *   q    [batch][n_tok][h][d_h]  config dtype, already rotated
  *   out  [batch][n_tok][h][d_h]  float32
  *   start_pos [batch] int32; a row whose last slot is outside the cache is
  *   skipped (zeros) and sets KPA_ERR_DEVICE_CHECK.
- *   workspace at least kpa_prefill_workspace_size bytes (may be 0). */
+ *   workspace at least kpa_prefill_workspace_size bytes (may be 0).
+ * Takes bf16 caches of order 2 with d_h <= 128 whose per-head factor slices fit the
+ * kernel's staging (R_K (d1 + d2) + R_V (d1 + d2) up to about 600 elements);
+ * KPA_ERR_UNSUPPORTED otherwise.  kpa_prefill_kernel_kind says which kernel runs. */
 kpa_status kpa_prefill_workspace_size(const kpa_config *cfg, int32_t batch, int32_t n_tok,
                                       size_t *bytes);
 kpa_status kpa_prefill(const kpa_config *cfg, int32_t batch, int32_t n_tok, const void *q,
                        const int32_t *start_pos, const void *kcache, const void *vcache,
                        int32_t capacity, float sm_scale, float *out, void *workspace,
                        size_t ws_bytes, kpa_stream stream);
+
+/* Which kernel kpa_prefill and kpa_prefill_qf run for this config on the calling
+ * thread:
+ *   KPA_PREFILL_KERNEL_TCGEN05    d1 = 8, d2 = 16, R_K = R_V = 2 (S, P and O in tensor
+ *                                 memory; two 128-row query halves per CTA)
+ *   KPA_PREFILL_KERNEL_MMA_SYNC   every other split it takes (128 query rows per CTA on
+ *                                 mma.sync m16n8k16), or every split after
+ *                                 kpa_test_set_prefill_engine(1)
+ * KPA_ERR_UNSUPPORTED where neither applies (fp32, third order, d_h > 128). */
+enum { KPA_PREFILL_KERNEL_MMA_SYNC = 1, KPA_PREFILL_KERNEL_TCGEN05 = 2 };
+kpa_status kpa_prefill_kernel_kind(const kpa_config *cfg, int32_t *kind);
 
 /* kpa_prefill with the queries given as factors ("Kronecker Product Attention", eq 2
  * for Q): the kernel forms each query row (1/R_Q) sum_r A^Q_r (x) B^Q_r in fp32 and
@@ -358,6 +374,13 @@ kpa_status kpa_test_set_decode_hooks(int32_t skip_tile, int32_t skip_split, uint
  * unaffected.  The setting belongs to the calling host thread (other threads keep
  * their own, 0 unless they set it); returns KPA_ERR_INVALID_ARG for other values. */
 kpa_status kpa_test_set_decode_engine(int32_t engine);
+
+/* Testing and measurement: choose the prefill kernel.  0 (the default) runs the
+ * tcgen05 kernel where it is instantiated and the mma.sync kernel elsewhere; 1 runs
+ * the mma.sync kernel for every split it takes, so the two can be compared on the
+ * same shape.  Belongs to the calling host thread; KPA_ERR_INVALID_ARG for other
+ * values. */
+kpa_status kpa_test_set_prefill_engine(int32_t engine);
 
 /* Testing only: y[i] = 2^x[i] for i < n (device arrays, float32) through the
  * prefill's FMA-pipe exponential (Cody-Waite reduction to [-1/2, 1/2] and a fitted

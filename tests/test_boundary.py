@@ -84,13 +84,43 @@ def test_shared_b_needs_equal_ranks():
     assert e.value.status == kpa.KPA_ERR_INVALID_ARG
 
 
-def test_shared_b_prefill_shape_limit():
-    """The prefill kernel covers d1 = 8, d2 = 16, R = 2 whether B is shared or not; a
-    shared-B TPA shape is outside it (checked before any device call)."""
-    s = Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2, r_q=6, d_model=2048, shared_b=1)
-    cfg = kpa.make_config(s, "bf16")
+def test_prefill_kernel_kinds():
+    """The tcgen05 prefill takes d1 = 8, d2 = 16, R = 2 (B shared or not); the mma.sync
+    prefill every other order-2 bf16 split with d_h <= 128 whose factor slices fit its
+    staging, and the tcgen05 split too after kpa_test_set_prefill_engine(1).  d_h > 128,
+    oversized slices and fp32 are refused before any device call."""
+    def kind(**kw):
+        return kpa.kpa_prefill_kernel_kind(kpa.make_config(Shape(**kw), "bf16"))
+
+    c5 = dict(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2)
+    assert kind(**c5) == "tcgen05"
+    assert kind(**c5, shared_b=1) == "tcgen05"
+    for split in (dict(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2), dict(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2,
+                                                                    shared_b=1),
+                  dict(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4), dict(h1=2, h2=8, d1=8, d2=8, r_k=2, r_v=2),
+                  dict(h1=3, h2=2, d1=4, d2=6, r_k=2, r_v=2), dict(h1=8, h2=1, d1=1, d2=128, r_k=3, r_v=2)):
+        assert kind(**split) == "mma_sync", split
+    try:
+        kpa.kpa_test_set_prefill_engine(1)
+        assert kind(**c5) == "mma_sync"
+    finally:
+        kpa.kpa_test_set_prefill_engine(0)
+    assert kind(**c5) == "tcgen05"
     with pytest.raises(kpa.KpaError) as e:
-        kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)
+        kpa.kpa_test_set_prefill_engine(2)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+    for bad in (dict(h1=4, h2=4, d1=16, d2=16, r_k=2, r_v=2),          # d_h = 256
+                dict(h1=1, h2=1, d1=1, d2=128, r_k=8, r_v=8)):         # 2 x 1032-element slices
+        cfg = kpa.make_config(Shape(**bad), "bf16")
+        with pytest.raises(kpa.KpaError) as e:
+            kpa.kpa_prefill_kernel_kind(cfg)
+        assert e.value.status == kpa.KPA_ERR_UNSUPPORTED, bad
+        with pytest.raises(kpa.KpaError) as e:
+            kpa.kpa_prefill(cfg, 1, 16, A, A, A, A, 64, 0.1, A, stream=0)
+        assert e.value.status == kpa.KPA_ERR_UNSUPPORTED, bad
+    cfg = kpa.make_config(Shape(**c5), "f32")
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_prefill_kernel_kind(cfg)
     assert e.value.status == kpa.KPA_ERR_UNSUPPORTED
 
 

@@ -146,6 +146,19 @@ APPEND_PREFILL = AppendWorkload(
     shape=Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, rope_base=10000.0),
     batch=8, n_tok=2048, capacity=2112, seed=0)
 
+# The append+prefill configuration on other splits of the same h = 16 heads and
+# d_h = 128 features: the TPA split of "Kronecker Product Attention", section 2.2
+# (h1 = h, d1 = 1), and the KPA split at rank 4.  Same chunk, batch, d_model and R_Q.
+APPEND_PREFILL_SPLITS = {
+    "kpa_h4x4_d8x16_r2": APPEND_PREFILL,
+    "tpa_h16_d1x128_r2": APPEND_PREFILL.replace(
+        name="TPA append+prefill (B=8, n=2048, d_model=2048, h=16x1, d_h=1x128, R_Q=6, R=2+2)",
+        shape=dataclasses.replace(APPEND_PREFILL.shape, h1=16, h2=1, d1=1, d2=128)),
+    "kpa_h4x4_d8x16_r4": APPEND_PREFILL.replace(
+        name="KPA append+prefill (B=8, n=2048, d_model=2048, h=4x4, d_h=8x16, R_Q=6, R=4+4)",
+        shape=dataclasses.replace(APPEND_PREFILL.shape, r_k=4, r_v=4)),
+}
+
 # The decoding benchmark shape of the FlashTPA figures ("Tensor Product Attention Is
 # All You Need" explainer, decoding-speed benchmarks): d_model 2048, h = 32, d_h = 64,
 # R_Q = 16, R_K = R_V = 1, sequences 2^12 .. 2^19, batch 1 .. 16.  Here batch 1 at 2^19
