@@ -67,7 +67,7 @@ def _args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override: fixed length (profiling)")
-    ap.add_argument("--batch", type=int, default=0, help="override: batch (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override: batch (profiling; append_prefill too)")
     ap.add_argument("--tokens-per-split", type=int, default=0,
                     help="override the library's split of each sequence (profiling; multiple of 64)")
     ap.add_argument("--split-sequence", action="store_true",
@@ -691,6 +691,8 @@ def run_append_prefill(a):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     w = APPEND_PREFILL_SPLITS[a.prefill_split]
+    if a.batch:
+        w = w.replace(batch=a.batch)
     s = w.shape
     inp = append_inputs(w.replace(seed=rank_seed(rank)))
     cfg = kpa.make_config(s, "bf16")

@@ -129,7 +129,7 @@ constexpr int kMaxClusterSplits = 16;
 // How many clusters of `size` CTAs of a tensor-core variant can be resident at once
 // on this device (cached per device).
 int cluster_capacity(int variant, int size) {
-    constexpr int kMaxVariants = 16;
+    constexpr int kMaxVariants = 24;
     static std::atomic<int> known[kMaxDevices][kMaxVariants][kMaxClusterSplits + 1];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || variant < 0 ||

@@ -137,6 +137,10 @@ using MmaKpaH8x2D8x8R2 = MmaDecodeCfg<64, 8, 8, 2, 2, 2, 8, 1, 2>;
 using MmaKpaH4x5D8x8R2 = MmaDecodeCfg<32, 8, 8, 2, 2, 5, 3, 2, 2>;
 using MmaKpaH2x10D8x8R2 = MmaDecodeCfg<16, 8, 8, 2, 2, 10, 1, 4, 2>;
 using MmaKpaH10x2D8x8R2 = MmaDecodeCfg<80, 8, 8, 2, 2, 2, 8, 1, 2>;
+// The append+prefill configuration's h = 16, d_h = 128 in two more splits: TPA (h1 = 16,
+// d1 = 1; 1152-byte records, so 64 tokens per stage) and KPA h = 4x4, d_h = 8x16 at rank 4.
+using MmaTpaH16D128R2 = MmaDecodeCfg<16, 1, 128, 2, 2, 1, 4, 1, 2>;
+using MmaKpaH4x4D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 4, 4, 1, 2>;
 
 #define KPA_MMA_VARIANTS(X)        \
     X(0, MmaTpaH16D64R2)           \
@@ -152,7 +156,9 @@ using MmaKpaH10x2D8x8R2 = MmaDecodeCfg<80, 8, 8, 2, 2, 2, 8, 1, 2>;
     X(10, MmaKpaH8x2D8x8R2)        \
     X(11, MmaKpaH4x5D8x8R2)        \
     X(12, MmaKpaH2x10D8x8R2)       \
-    X(13, MmaKpaH10x2D8x8R2)
+    X(13, MmaKpaH10x2D8x8R2)       \
+    X(14, MmaTpaH16D128R2)         \
+    X(15, MmaKpaH4x4D8x16R4)
 
 // Index of the variant that covers these dims, or -1.
 inline int mma_decode_variant(const Dims &d) {

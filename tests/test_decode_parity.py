@@ -268,8 +268,10 @@ def _qf_case(shape, batch, cap, seed):
 
 @pytest.mark.parametrize("shape", [
     Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2, r_q=6, d_model=2048, rope_base=10000.0),
-    Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2, r_q=4, d_model=1024, rope_base=10000.0)],
-    ids=["kpa_h4x4", "tpa_h16"])
+    Shape(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2, r_q=4, d_model=1024, rope_base=10000.0),
+    Shape(h1=16, h2=1, d1=1, d2=128, r_k=2, r_v=2, r_q=6, d_model=2048, rope_base=10000.0),
+    Shape(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4, r_q=6, d_model=2048, rope_base=10000.0)],
+    ids=["kpa_h4x4", "tpa_h16", "tpa_h16_d128", "kpa_h4x4_r4"])
 def test_decode_from_query_factors(shape):
     """kpa_decode_qf: the query as factor records (record layout), rotated in the kernel at
     q_pos, against the oracle with the float64 assembly (1/R_Q) sum_r A^Q_r (x) B^Q_r."""
@@ -333,6 +335,37 @@ def test_section32_head_splits(name):
     from workloads import KPA_SECTION32
     lib = kpa()
     w = KPA_SECTION32[name].replace(batch=3, capacity=1200, length=0, ragged=(1, 1200), seed=61)
+    inp = decode_inputs(w)
+    cfg = lib.make_config(w.shape, w.dtype)
+    max_len = int(inp["seq_len"].max())
+    assert lib.kpa_decode_kernel_kind(cfg, w.batch, max_len) == "mma_sync"
+    got, kc, vc = _run(w, inp)
+    assert_bf16_close(got, oracle_decode_unrotated(w, inp), f"e2e {name}")
+    want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"])
+    assert_bf16_close(got, want, f"stage {name}")
+    scale = 64.0 / np.sqrt(w.shape.dh)
+    got, kc, vc = _run(w, inp, sm_scale=float(scale))
+    want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"],
+                                    sm_scale=scale)
+    assert_bf16_close(got, want, f"peaked {name}")
+
+
+# The append+prefill configuration's h = 16, d_h = 128 in its TPA split and at rank 4:
+# the tensor-core decode variants that take those splits' decode steps.
+SPLIT_DECODES = {
+    "tpa_h16_d1x128_r2": Shape(h1=16, h2=1, d1=1, d2=128, r_k=2, r_v=2),
+    "kpa_h4x4_d8x16_r4": Shape(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SPLIT_DECODES))
+def test_more_split_decodes(name):
+    """The TPA split of h = 16, d_h = 128 (1152-byte records, 64 tokens a stage) and the
+    KPA split at rank 4 run on the tensor cores and match the oracle end to end, at stage
+    level, and with a peaked softmax (scale x 64) at stage level, on ragged lengths."""
+    lib = kpa()
+    w = KPA_MEDIUM.replace(shape=SPLIT_DECODES[name], batch=3, capacity=1200, length=0, ragged=(1, 1200),
+                           factor_std=1.0 / np.sqrt(2.0), seed=62)
     inp = decode_inputs(w)
     cfg = lib.make_config(w.shape, w.dtype)
     max_len = int(inp["seq_len"].max())
