@@ -202,9 +202,23 @@ KPA_SECTION32 = {
         length=4096)
     for name, (h1, h2) in KPA_SECTION32_SPLITS.items()}
 
+# The append+prefill configuration's h = 16, d_h = 128 in its TPA split and at rank 4,
+# as decode workloads with the TPA decode's batch, length and spreads.
+SPLIT_DECODES = {
+    "tpa_h16_d1x128": DecodeWorkload(
+        name="TPA decode, h=16x1, d_h=1x128 (B=8, R=2+2, L=4096, bf16)",
+        shape=Shape(h1=16, h2=1, d1=1, d2=128, r_k=2, r_v=2, rope_base=10000.0),
+        batch=8, capacity=4096, dtype="bf16", factor_std=1.0 / np.sqrt(2.0), q_std=1.0 / 8.0, seed=0,
+        length=4096),
+    "kpa_h4x4_d8x16_r4": DecodeWorkload(
+        name="KPA decode, h=4x4, d_h=8x16 (B=8, R=4+4, L=4096, bf16)",
+        shape=Shape(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4, rope_base=10000.0),
+        batch=8, capacity=4096, dtype="bf16", factor_std=0.5, q_std=1.0 / 8.0, seed=0, length=4096),
+}
+
 DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
                   "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE, "tpa_shared": TPA_SHARED_DECODE,
-                  "tpa_order3": TPA3_DECODE, **KPA_SECTION32}
+                  "tpa_order3": TPA3_DECODE, **KPA_SECTION32, **SPLIT_DECODES}
 
 
 # --- draws ---------------------------------------------------------------------
