@@ -693,7 +693,7 @@ def run_append_prefill(a):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     w = APPEND_PREFILL_SPLITS[a.prefill_split]
     if a.batch:
-        w = w.replace(batch=a.batch)
+        w = w.replace(batch=a.batch, name=w.name + f" [batch overridden to {a.batch}]")
     s = w.shape
     inp = append_inputs(w.replace(seed=rank_seed(rank)))
     cfg = kpa.make_config(s, "bf16")
