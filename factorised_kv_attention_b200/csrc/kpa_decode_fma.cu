@@ -240,11 +240,13 @@ cudaError_t launch_decode_fma(const Dims &d, kpa_dtype dt, int batch, const void
 
 // ---------------------------------------------------------------------------
 // Split combine: out = (1/R_V) * sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
-// One block per (head, sequence, chunk of up to 16 features): the split statistics
-// are staged in shared memory with all loads in flight; then the block's threads
-// take (feature, split phase) pairs, sum their features over every 32nd split with
-// independent, unrolled loads (a few per thread, all in flight), and the phases are
-// added through shared memory.
+// One block per (head, sequence, chunk of up to 16 features).  The block's threads
+// take (feature, split phase) pairs; right after the wait on the decode, each thread
+// requests its partial outputs (every 32nd split, up to kCombinePre of them into
+// registers) and the first threads the splits' (m, l), all in one round trip to L2.
+// The maximum, the weights and their sum are then formed in shared memory, each
+// thread weighs the outputs it already holds, and the phases are added through shared
+// memory.
 // Launched as a programmatic dependent of the decode kernel: it becomes resident
 // while the decode's last CTAs still run and waits for them before reading.
 namespace {
@@ -252,6 +254,7 @@ namespace {
 constexpr int kCombineThreads = 512;
 constexpr int kCombineMaxSplits = 4096;
 constexpr int kCombineFeatures = 16;
+constexpr int kCombinePre = 8;           // partial outputs per thread requested up front
 
 __global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, int tps,
@@ -260,11 +263,11 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
                       float *__restrict__ out, float *__restrict__ lse, float lse_scale) {
     __shared__ float w[kCombineMaxSplits];
     __shared__ float red[kCombineThreads / 32];
-    __shared__ float s_den;
+    __shared__ float s_max, s_den;
     const int fch = d.dh < kCombineFeatures ? d.dh : kCombineFeatures;    // features per block
     const int n_chunks = (d.dh + fch - 1) / fch;
     const int head = blockIdx.x / n_chunks, f0 = (blockIdx.x % n_chunks) * fch;
-    const int b = blockIdx.y, tid = threadIdx.x;
+    const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     asm volatile("griddepcontrol.wait;" ::: "memory");        // the decode's partials are complete
     asm volatile("griddepcontrol.launch_dependents;");
     int L = seq_len[b];
@@ -277,27 +280,50 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
         if (lse && f0 == 0 && tid == 0) lse[(size_t)b * d.h + head] = -INFINITY;   // no scores
         return;
     }
+    // (feature, phase) pairs: the phases of one feature take every P-th split
+    const int P = kCombineThreads / fch;
+    const int f = tid % fch, phase = tid / fch;
+    const bool worker = phase < P && f < nf;
+    const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh + f0 + f;
+    const size_t po_stride = (size_t)d.h * d.dh;
+    float pre[kCombinePre];
+#pragma unroll
+    for (int k = 0; k < kCombinePre; ++k) {
+        const int i = phase + k * P;
+        pre[k] = worker && i < ns ? __ldcg(po + (size_t)i * po_stride) : 0.f;
+    }
     const float2 *ml = reinterpret_cast<const float2 *>(part_ml) + (size_t)b * n_split * d.h + head;
     float M = -INFINITY;
-    for (int i = tid; i < ns; i += kCombineThreads) {
-        const float m = ml[(size_t)i * d.h].x;
-        w[i] = m;
-        M = fmaxf(M, m);
+    float2 mine[kCombineMaxSplits / kCombineThreads];
+#pragma unroll
+    for (int k = 0; k < kCombineMaxSplits / kCombineThreads; ++k) {
+        const int i = tid + k * kCombineThreads;
+        mine[k] = i < ns ? __ldcg(ml + (size_t)i * d.h) : make_float2(-INFINITY, 0.f);
+        M = fmaxf(M, mine[k].x);
     }
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if ((tid & 31) == 0) red[tid >> 5] = M;
+    if (lane == 0) red[wid] = M;
     __syncthreads();
-    M = red[0];
-    for (int k = 1; k < kCombineThreads / 32; ++k) M = fmaxf(M, red[k]);
+    if (tid == 0) {
+        float t = red[0];
+        for (int k = 1; k < kCombineThreads / 32; ++k) t = fmaxf(t, red[k]);
+        s_max = t;
+    }
+    __syncthreads();
+    M = s_max;
     float den = 0.f;
-    for (int i = tid; i < ns; i += kCombineThreads) {
-        const float wi = w[i] == -INFINITY ? 0.f : exp2f(w[i] - M);
-        w[i] = wi;
-        den += wi * ml[(size_t)i * d.h].y;
+#pragma unroll
+    for (int k = 0; k < kCombineMaxSplits / kCombineThreads; ++k) {
+        const int i = tid + k * kCombineThreads;
+        if (i < ns) {
+            const float wi = mine[k].x == -INFINITY ? 0.f : exp2f(mine[k].x - M);
+            w[i] = wi;
+            den += wi * mine[k].y;
+        }
     }
     for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-    __syncthreads();
-    if ((tid & 31) == 0) red[tid >> 5] = den;
+    __syncthreads();                                       // red reused; w complete
+    if (lane == 0) red[wid] = den;
     __syncthreads();
     if (tid == 0) {
         float t = 0.f;
@@ -305,17 +331,17 @@ decode_combine_kernel(Dims d, const int32_t *__restrict__ seq_len, int max_len, 
         s_den = t;
         if (lse && f0 == 0) lse[(size_t)b * d.h + head] = t > 0.f ? (M + log2f(t)) * lse_scale : -INFINITY;
     }
-    __syncthreads();
-    // (feature, phase) pairs: the phases of one feature take every P-th split
-    const int P = kCombineThreads / fch;
-    const int f = tid % fch, phase = tid / fch;
     float num = 0.f;
-    if (phase < P && f < nf) {
-        const float *po = part_o + ((size_t)b * n_split * d.h + head) * d.dh + f0 + f;
-#pragma unroll 8
-        for (int i = phase; i < ns; i += P) num += w[i] * po[(size_t)i * d.h * d.dh];
+    if (worker) {
+#pragma unroll
+        for (int k = 0; k < kCombinePre; ++k) {
+            const int i = phase + k * P;
+            if (i < ns) num += w[i] * pre[k];
+        }
+#pragma unroll 4
+        for (int i = phase + kCombinePre * P; i < ns; i += P) num += w[i] * __ldcg(po + (size_t)i * po_stride);
     }
-    __syncthreads();
+    __syncthreads();                                       // s_den set; every w read
     float *acc = w;                                        // reuse: [P][fch] partial sums
     if (phase < P) acc[phase * fch + f] = num;
     __syncthreads();
