@@ -12,7 +12,7 @@
 // share every rebuilt K/V tile and take turns on the tensor pipe:
 //   - a producer warp streams the head's factor slices of each key tile into shared
 //     memory with TMA, two tiles ahead (and loads the Q tile once);
-//   - four rebuild warps form the K tile (token rows) and the V^T tile (feature rows)
+//   - eight rebuild warps form the K tile (token rows) and the V^T tile (feature rows)
 //     in the 128-byte-swizzled K-major layouts tcgen05.mma reads, from ldmatrix.trans
 //     fragments of the factors through stmatrix / stmatrix.trans; K runs one tile
 //     ahead of V, K is double-buffered;
