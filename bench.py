@@ -56,7 +56,7 @@ def _args(argv=None):
     ap.add_argument("--impl", choices=["kpa", "reference"], default="kpa")
     ap.add_argument("--workload", default="kpa_long",
                     help="tpa_decode | tpa_shared | tpa_order3 | kpa_medium | kpa_long | tiny_kpa | flashtpa | "
-                         "tpa_h16_d1x128 | kpa_h4x4_d8x16_r4 | kpa_h{4x4,2x8,8x2,4x5,2x10,10x2}_d8x8 | "
+                         "tpa_h61 | tpa_h16_d1x128 | kpa_h4x4_d8x16_r4 | kpa_h{4x4,2x8,8x2,4x5,2x10,10x2}_d8x8 | "
                          "append_prefill")
     ap.add_argument("--layers", type=int, default=0,
                     help="0 = enough layer caches to exceed 4 x L2 (at least 2)")

@@ -198,13 +198,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     constexpr int MA = C::MA, D1 = C::D1, D2 = C::D2, RK = C::RK, RV = C::RV, H2 = C::H2;
     constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
-    constexpr int MT = MA / 16, KS = D2 / 16, NT = D2 / 8;
+    // MR record rows (the cache's h1 d1; MA pads them to whole 16-row tiles), HR the
+    // cache's heads: the query, the partials and the outputs have HR heads
+    constexpr int MR = C::MR, HR1 = C::HR1, HR = C::HR, HS = C::HS;
+    constexpr int MT = MA / 16, MTW = MT / HS, KS = D2 / 16, NT = D2 / 8;
     constexpr int EK = C::EK, EV = C::EV;
     constexpr int WARPS = C::WARPS, SLICES = C::SLICES, CHUNKS = C::CHUNKS, STAGES = C::STAGES;
     constexpr int TT = C::TT;
     constexpr int KBYTES = TT * EK * 2, STAGE_BYTES = C::STAGE_BYTES;
     constexpr int RED_LD = C::RED_LD;               // floats per token row of the j1 scratch
-    constexpr int A_K = RK * MA, A_V = RV * MA;     // start of B in a key / value record
+    constexpr int A_K = RK * MR, A_V = RV * MR;     // start of B in a key / value record
     // third order: query pair i = (head, m, jc) -> its first feature (head, 2m, jc); the
     // records' b and c factors start at A_K (A_V) and A_K + RK DB (A_V + RV DB)
     auto o3_pair_feature = [](int i) {
@@ -277,18 +280,18 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const bool rotate = a.q_pos != nullptr;
     int L = a.seq_len[b];
     const double qpos = rotate ? (double)a.q_pos[b] : 0.0;
-    constexpr int QPT = (H * DH / 2 + WARPS * 32 - 1) / (WARPS * 32);   // query pairs per thread
+    constexpr int QPT = (HR * DH / 2 + WARPS * 32 - 1) / (WARPS * 32);  // query pairs per thread
     __nv_bfloat162 qv[QPT];
     if (warp < WARPS && !a.qf) {
-        const __nv_bfloat162 *qb = reinterpret_cast<const __nv_bfloat162 *>(a.q + (size_t)b * H * DH);
+        const __nv_bfloat162 *qb = reinterpret_cast<const __nv_bfloat162 *>(a.q + (size_t)b * HR * DH);
 #pragma unroll
         for (int k = 0; k < QPT; ++k) {
             const int i = tid + k * WARPS * 32;
-            if (i < H * DH / 2) {
+            if (i < HR * DH / 2) {
                 if constexpr (C::ORDER3) {
                     // third order: the RoPE pair of (head, m, c index) is features (2m DC + jc, + DC)
                     const int e0 = o3_pair_feature(i);
-                    qv[k] = __halves2bfloat162(a.q[(size_t)b * H * DH + e0], a.q[(size_t)b * H * DH + e0 + C::DC]);
+                    qv[k] = __halves2bfloat162(a.q[(size_t)b * HR * DH + e0], a.q[(size_t)b * HR * DH + e0 + C::DC]);
                 } else {
                     qv[k] = qb[i];
                 }
@@ -298,7 +301,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     // query factors: the sequence's E_Q values (at most QF_PT per consumer thread) are
     // requested here, in the same round trip as the other inputs
     constexpr int QF_PT = C::QF_MAX / (WARPS * 32);
-    const int eq = a.qf ? a.rq * (H1 * D1 + H2 * D2) : 0;
+    const int eq = a.qf ? a.rq * (HR1 * D1 + H2 * D2) : 0;
     float qfv[QF_PT];
     if (warp < WARPS && a.qf) {
         const float *qfb = a.qf + (size_t)b * a.qf_seq_stride;
@@ -314,7 +317,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     }
     if (t0 >= L && !a.cluster) {                           // empty split (a cluster member stays)
         if (a.fused && L == 0 && split == 0)                // an empty sequence gets zeros
-            for (int i = tid; i < H * DH; i += C::THREADS) a.out[(size_t)b * H * DH + i] = 0.f;
+            for (int i = tid; i < HR * DH; i += C::THREADS) a.out[(size_t)b * HR * DH + i] = 0.f;
         if (tid == 0 && spec && !mbar_wait(full0, 0, hooks.wait_limit_ns))
             raise_error(a.err, kErrTimeout);               // its speculative copy lands first
         return;
@@ -391,7 +394,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         // shared-memory rows (E_Q <= H * Q_LD, checked by the host), the outputs are kept in
         // registers until every thread has read its factors, then written over them.
         // One thread per 8 features of a (head, j1) row.
-        constexpr int CH = D2 / 8, ITEMS = H * D1 * CH;
+        constexpr int CH = D2 / 8, ITEMS = HR * D1 * CH;
         constexpr int IPT = (ITEMS + WARPS * 32 - 1) / (WARPS * 32);
         static_assert(C::QF_MAX <= H * C::Q_LD, "query factors staged in the query rows");
 #pragma unroll
@@ -400,7 +403,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             if (e < eq) qs[e] = qfv[k];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-        const int qa_b = a.rq * H1 * D1;                  // first B^Q element of the record
+        const int qa_b = a.rq * HR1 * D1;                 // first B^Q element of the record
         const float rs = a.qscale / (float)a.rq;
         float acc[IPT][8];
 #pragma unroll
@@ -412,7 +415,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 const int head = it / (D1 * CH), rem = it % (D1 * CH), j1 = rem / CH, j2 = (rem % CH) * 8;
                 const int i1 = head / H2, i2h = head % H2;
                 for (int r = 0; r < a.rq; ++r) {
-                    const float av = qs[(r * H1 + i1) * D1 + j1];
+                    const float av = qs[(r * HR1 + i1) * D1 + j1];
                     const float4 *bq = reinterpret_cast<const float4 *>(qs + qa_b + (r * H2 + i2h) * D2 + j2);
                     const float4 b0 = bq[0], b1 = bq[1];
                     acc[k][0] += av * b0.x;
@@ -449,7 +452,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
 #pragma unroll
     for (int k = 0; k < QPT; ++k) {
         const int i = tid + k * WARPS * 32;
-        if (i < H * DH / 2 && !a.qf) {
+        if (i < HR * DH / 2 && !a.qf) {
             const float2 x = __bfloat1622float2(qv[k]);
             float2 y = x;
             if constexpr (C::ORDER3) {
@@ -484,10 +487,12 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             st[i] = make_float2(cth, sth);
         }
     }
+    if constexpr (HR < H)                                  // padded heads: zero query rows
+        for (int i = tid; i < (H - HR) * C::Q_LD; i += WARPS * 32) qs[(size_t)HR * C::Q_LD + i] = 0.f;
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
 
     // ------------------------------------------------------------ consumers
-    const int i2 = warp % H2, slice = warp / H2;
+    const int i2 = warp % H2, hs = (warp / H2) % HS, slice = warp / (H2 * HS);
     const int g = lane >> 2, c = lane & 3;
     float *mo = reinterpret_cast<float *>(smem);                   // [SLICES][H][DH] (after the loop)
     constexpr int MO_LD = C::MO_LD;
@@ -586,7 +591,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                                           bk[ks][1]);
                         }
                         uint32_t ak[MT][2];
-                        a_frags<MT, D1>(smem_u32(grp + (size_t)r * MA * 16) + a_off, ak);
+                        a_frags<MT, D1>(smem_u32(grp + (size_t)r * MR * 16) + a_off, ak);
     #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -665,7 +670,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                     uint32_t av[2][MT][2];
     #pragma unroll
                     for (int gi = 0; gi < 2; ++gi) {
-                        a_frags<MT, D1>(smem_u32((gi ? g1p : g0p) + (size_t)r * MA * 16) + a_off, av[gi]);
+                        a_frags<MT, D1>(smem_u32((gi ? g1p : g0p) + (size_t)r * MR * 16) + a_off, av[gi]);
                     }
                     uint32_t pa[MT][4];
     #pragma unroll
@@ -792,14 +797,14 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     float *abuf = pbuf + H1 * 16;                            // [H1] rescale factors
 
     // query fragments (A operand, row = (i1, j1), k = j2), hi and lo parts
-    uint32_t qa_hi[MT][KS][4], qa_lo[MT][KS][4];
+    uint32_t qa_hi[MTW][KS][4], qa_lo[MTW][KS][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-                const int row = mt * 16 + g + ((v & 1) ? 8 : 0);
+                const int row = (hs * MTW + mt) * 16 + g + ((v & 1) ? 8 : 0);
                 const int j2 = ks * 16 + 2 * c + ((v & 2) ? 8 : 0);
                 const int i1 = row / D1, j1 = row % D1;
                 const float *src = qs + (i1 * H2 + i2) * C::Q_LD + j1 * D2 + j2;
@@ -817,15 +822,15 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const float2 *step_s = reinterpret_cast<const float2 *>(smem + C::OFF_STEP);
     float2 *base_s = reinterpret_cast<float2 *>(smem + C::OFF_BASE) + (size_t)warp * (D2 / 2);
 
-    float o[MT][NT][4];
+    float o[MTW][NT][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
     // softmax state: per owned row (D1 == 1: rows are heads) or per lane head (D1 > 1)
-    float m_row[MT][2], l_row[MT][2];
+    float m_row[MTW][2], l_row[MTW][2];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
+    for (int mt = 0; mt < MTW; ++mt) {
         m_row[mt][0] = m_row[mt][1] = -INFINITY;
         l_row[mt][0] = l_row[mt][1] = 0.f;
     }
@@ -874,9 +879,9 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         }
             }
             // ---- scores: sc[mt][gi][v] = sum_r A^K_r * (Q_i2 B~^K_r), rows (i1,j1), tokens 2c, 2c+1
-            float2 sc[MT][2][2];
+            float2 sc[MTW][2][2];
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
+            for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
                 for (int gi = 0; gi < 2; ++gi) sc[mt][gi][0] = sc[mt][gi][1] = make_float2(0.f, 0.f);
 #pragma unroll
@@ -918,7 +923,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         }
                     }
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
+                    for (int mt = 0; mt < MTW; ++mt) {
                         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int ks = 0; ks < KS; ++ks) {
@@ -937,9 +942,9 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                                 (tk + 1 < n_valid && !(isfinite(acc[1]) && isfinite(acc[3]))))
                                 raise_error(a.err, kErrDeviceCheck);
                         }
-                        const int row0 = mt * 16 + g;
-                        const float2 a0 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MA + row0) * 16 + 4 * c));
-                        const float2 a1 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MA + row0 + 8) * 16 + 4 * c));
+                        const int row0 = (hs * MTW + mt) * 16 + g;
+                        const float2 a0 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MR + row0) * 16 + 4 * c));
+                        const float2 a1 = unpack_bf16x2(lds_u32(grp + (size_t)(r * MR + row0 + 8) * 16 + 4 * c));
                         sc[mt][gi][0] = ffma2(make_float2(acc[0], acc[1]), a0, sc[mt][gi][0]);
                         sc[mt][gi][1] = ffma2(make_float2(acc[2], acc[3]), a1, sc[mt][gi][1]);
                     }
@@ -950,7 +955,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             if constexpr (D1 == 1) {
                 // rows are heads: row g of m-tile mt is head mt*16+g, row g+8 head mt*16+g+8
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
+                for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
                         if (tail) {
@@ -985,10 +990,10 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             } else {
                 // sum over j1 once per (head, token): partials through the warp's scratch
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
+                for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
                     for (int gi = 0; gi < 2; ++gi) {
-                        const int tk = gi * 8 + 2 * c, row = mt * 16 + g;
+                        const int tk = gi * 8 + 2 * c, row = (hs * MTW + mt) * 16 + g;
                         red[tk * RED_LD + row] = sc[mt][gi][0].x;
                         red[(tk + 1) * RED_LD + row] = sc[mt][gi][0].y;
                         red[tk * RED_LD + row + 8] = sc[mt][gi][1].x;
@@ -1032,10 +1037,10 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 if (lane < H1) abuf[lane] = alpha;
                 __syncwarp();
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
+                for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
-                        const int i1 = (mt * 16 + g + 8 * hr) / D1;
+                        const int i1 = ((hs * MTW + mt) * 16 + g + 8 * hr) / D1;
                         const float al = abuf[i1];
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
@@ -1053,14 +1058,14 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
             const unsigned char *g1p = g0p + (size_t)EV * 16;
 #pragma unroll
             for (int r = 0; r < RV; ++r) {
-                uint32_t pa_hi[MT][4], pa_lo[MT][4];
+                uint32_t pa_hi[MTW][4], pa_lo[MTW][4];
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const int row0 = mt * 16 + g;
-                    const uint32_t w00 = lds_u32(g0p + (size_t)(r * MA + row0) * 16 + 4 * c);
-                    const uint32_t w10 = lds_u32(g0p + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
-                    const uint32_t w01 = lds_u32(g1p + (size_t)(r * MA + row0) * 16 + 4 * c);
-                    const uint32_t w11 = lds_u32(g1p + (size_t)(r * MA + row0 + 8) * 16 + 4 * c);
+                for (int mt = 0; mt < MTW; ++mt) {
+                    const int row0 = (hs * MTW + mt) * 16 + g;
+                    const uint32_t w00 = lds_u32(g0p + (size_t)(r * MR + row0) * 16 + 4 * c);
+                    const uint32_t w10 = lds_u32(g0p + (size_t)(r * MR + row0 + 8) * 16 + 4 * c);
+                    const uint32_t w01 = lds_u32(g1p + (size_t)(r * MR + row0) * 16 + 4 * c);
+                    const uint32_t w11 = lds_u32(g1p + (size_t)(r * MR + row0 + 8) * 16 + 4 * c);
                     float2 x0 = fmul2(sc[mt][0][0], unpack_bf16x2(w00));
                     float2 x1 = fmul2(sc[mt][0][1], unpack_bf16x2(w10));
                     float2 x2 = fmul2(sc[mt][1][0], unpack_bf16x2(w01));
@@ -1122,7 +1127,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         b11 = mask_pair(b11, tk + 8 < n_valid, tk + 9 < n_valid);
                     }
 #pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
+                    for (int mt = 0; mt < MTW; ++mt) {
                         if constexpr (C::ORDER3) {
                             mma16816h(o[mt][2 * np], pa_hi[mt], b00, b01);
                             mma16816h(o[mt][2 * np], pa_lo[mt], b00, b01);
@@ -1148,7 +1153,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         // the values' fp16 features b (x) c: an overflow makes the partial non-finite
         bool fin = true;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+        for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -1159,7 +1164,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     // l: complete sums per head
     if constexpr (D1 == 1) {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
+        for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
                 float l = l_row[mt][hr];
@@ -1177,10 +1182,10 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     const bool ok = !(aborted || flags[0]);
     if (!ok && !a.cluster) return;
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int mt = 0; mt < MTW; ++mt)
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
-            const int row = mt * 16 + g + 8 * hr;
+            const int row = (hs * MTW + mt) * 16 + g + 8 * hr;
             const int i1 = row / D1, j1 = row % D1;
             const int head = i1 * H2 + i2;
             float *dst = mo + ((size_t)slice * H + head) * MO_LD + j1 * D2;
@@ -1204,12 +1209,12 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     }
     }  // KPA8
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
-    float *po = a.part_o + ((size_t)(b * a.n_split + split) * H) * DH;
-    float *pml = a.part_ml + ((size_t)(b * a.n_split + split) * H) * 2;
+    float *po = a.part_o + ((size_t)(b * a.n_split + split) * HR) * DH;
+    float *pml = a.part_ml + ((size_t)(b * a.n_split + split) * HR) * 2;
     // One float4 column of the merged partial per thread.  Each thread forms the
     // log-sum-exp weights 2^(m_slice - M) of its own head from the slice statistics,
     // so the merge needs no further barrier.
-    constexpr int N4 = H * DH / 4;
+    constexpr int N4 = HR * DH / 4;                  // the cache's heads (padded ones dropped)
     static_assert(DH % 4 == 0 && (MO_LD % 4) == 0 && ((size_t)SLICES * H * (MO_LD + 2)) % 4 == 0,
                   "float4 columns of the slice-merge buffer and of the merged partial");
     for (int c4 = tid; c4 < N4; c4 += WARPS * 32) {
@@ -1241,8 +1246,8 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         if (a.cluster) {
             *reinterpret_cast<float4 *>(cp + c4 * 4) = acc;
             if (col == 0) {
-                cp[H * DH + head] = M;
-                cp[H * DH + H + head] = l;
+                cp[HR * DH + head] = M;
+                cp[HR * DH + HR + head] = l;
             }
         } else {
             reinterpret_cast<float4 *>(po)[c4] = acc;
@@ -1264,7 +1269,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     }
     asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32));
     if (!flags[1]) return;
-    merge_split_partials<H, DH>(a.part_o, a.part_ml, a.n_split, n_b, b, a.out_scale, a.out, tid, WARPS * 32);
+    merge_split_partials<HR, DH>(a.part_o, a.part_ml, a.n_split, n_b, b, a.out_scale, a.out, tid, WARPS * 32);
     if (tid == 0) a.counters[b] = 0;                 // ready for the next call
     return;
     }  // global merge
@@ -1277,22 +1282,22 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     cl.sync();
     if (warp < WARPS) {
         const int n_cl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
-        const int per = (H * DH + n_cl - 1) / n_cl;
-        const int lo = rank * per, hi = min(H * DH, lo + per);
+        const int per = (HR * DH + n_cl - 1) / n_cl;
+        const int lo = rank * per, hi = min(HR * DH, lo + per);
         float *cpl = reinterpret_cast<float *>(smem) + SLICES * H * C::MO_LD + SLICES * H * 2;
         for (int idx = lo + tid; idx < hi; idx += WARPS * 32) {
             const int head = idx / DH;
             float M = -INFINITY;
-            for (int r = 0; r < n_cl; ++r) M = fmaxf(M, cl.map_shared_rank(cpl, r)[H * DH + head]);
+            for (int r = 0; r < n_cl; ++r) M = fmaxf(M, cl.map_shared_rank(cpl, r)[HR * DH + head]);
             float num = 0.f, den = 0.f;
             for (int r = 0; r < n_cl; ++r) {
                 const float *rp = cl.map_shared_rank(cpl, r);
-                const float m = rp[H * DH + head];
+                const float m = rp[HR * DH + head];
                 const float w = m == -INFINITY ? 0.f : exp2f(m - M);
                 num += w * rp[idx];
-                den += w * rp[H * DH + H + head];
+                den += w * rp[HR * DH + HR + head];
             }
-            a.out[(size_t)b * H * DH + idx] = den > 0.f ? a.out_scale * num / den : 0.f;
+            a.out[(size_t)b * HR * DH + idx] = den > 0.f ? a.out_scale * num / den : 0.f;
         }
     }
     cl.sync();                                       // peers read this CTA's shared memory

@@ -49,22 +49,29 @@ struct DecodeArgs {
 //   DB      > 0: a third-order TPA cache (h = MA heads, d1 = 1, d2 = d_h = DB * DC):
 //           records [a | b | c] with b in R^DB, c in R^DC, and the keys' features
 //           b (x) c formed in registers as fp16 for both products.
+//   HS      warps that split the CTA's 16-row head tiles between them (d1 = 1, h2 = 1):
+//           warps = HS * SLICES, each with MA / 16 / HS tiles of its token slice.
+//   MR      > 0: the records' A parts have MR = h1 d1 rows, padded to MA (a multiple of
+//           16) in the tiles (d1 = 1, h2 = 1): the padded query rows are zero, their
+//           outputs are never written, and the partials and outputs keep MR heads.
 template <int MA_, int D1_, int D2_, int RK_, int RV_, int H2_, int SLICES_, int CHUNKS_, int STAGES_,
-          bool SHARED_ = false, int DB_ = 0>
+          bool SHARED_ = false, int DB_ = 0, int HS_ = 1, int MR_ = 0>
 struct MmaDecodeCfg {
     static constexpr int MA = MA_, D1 = D1_, D2 = D2_, RK = RK_, RV = RV_, H2 = H2_;
+    static constexpr int HS = HS_, MR = MR_ > 0 ? MR_ : MA_;
     static constexpr int SLICES = SLICES_, CHUNKS = CHUNKS_, STAGES = STAGES_;
     static constexpr bool SHARED = SHARED_;
     static constexpr bool ORDER3 = DB_ > 0;
     static constexpr int DB = ORDER3 ? DB_ : 1, DC = ORDER3 ? D2_ / DB : D2_;
     static constexpr int H1 = MA / D1, H = H1 * H2, DH = D1 * D2;
-    static constexpr int EK = ORDER3 ? RK * (MA + DB + DC) : RK * (MA + H2 * D2);
-    static constexpr int EV = ORDER3 ? RV * (MA + DB + DC) : SHARED ? RV * MA : RV * (MA + H2 * D2);
+    static constexpr int HR1 = MR / D1, HR = HR1 * H2;           // the cache's heads (H: padded)
+    static constexpr int EK = ORDER3 ? RK * (MA + DB + DC) : RK * (MR + H2 * D2);
+    static constexpr int EV = ORDER3 ? RV * (MA + DB + DC) : SHARED ? RV * MR : RV * (MR + H2 * D2);
     // d1 = 8 (no shared B, second order): the rows of each 16-row query tile pair up
     // two j1 of one head per lane, so the sum over j1 and the softmax stay in registers,
     // and the value product runs once in fp16 (P' = p A^V and B^V rounded to fp16)
     static constexpr bool KPA8 = D1 == 8 && !SHARED && !ORDER3;
-    static constexpr int WARPS = H2 * SLICES;
+    static constexpr int WARPS = H2 * SLICES * HS;
     // A warp of its own streams the tiles, or (KPA8) the last consumer warp to release a
     // stage issues its next tile: sixteen consumer warps then keep 128 registers each
     // (a seventeenth warp would put five warps, at most 96 registers each, on one SM
@@ -97,7 +104,11 @@ struct MmaDecodeCfg {
     // row stride (floats) of the slice-merge buffer: 8 floats of padding put the rows
     // of consecutive heads in different banks
     static constexpr int MO_LD = D1 * D2 + 8;
-    static_assert(MA % 16 == 0, "h1*d1 must be a multiple of 16");
+    static_assert(MA % 16 == 0, "h1*d1 (padded) must be a multiple of 16");
+    static_assert(MR <= MA && MR > MA - 16, "MR pads to MA within one 16-row tile");
+    static_assert((MR == MA && HS == 1) || (D1 == 1 && H2 == 1 && !SHARED && !ORDER3),
+                  "padded rows and split head tiles: second-order TPA splits without a shared B");
+    static_assert((MA / 16) % HS == 0, "head tiles split evenly between the warps");
     static_assert(D2 % 16 == 0 || (KPA8 && D2 == 8), "d2 must be a multiple of 16 (or 8 with d1 = 8)");
     static_assert(D1 == 1 || D1 == 2 || D1 == 4 || D1 == 8 || D1 == 16, "d1 must be 1..16, a power of 2");
     static_assert(D1 == 1 || KPA8 || (H1 >= 2 && 32 % H1 == 0), "h1 must divide 32 when 1 < d1 < 8");
@@ -141,6 +152,10 @@ using MmaKpaH10x2D8x8R2 = MmaDecodeCfg<80, 8, 8, 2, 2, 2, 8, 1, 2>;
 // d1 = 1; 1152-byte records, so 64 tokens per stage) and KPA h = 4x4, d_h = 8x16 at rank 4.
 using MmaTpaH16D128R2 = MmaDecodeCfg<16, 1, 128, 2, 2, 1, 4, 1, 2>;
 using MmaKpaH4x4D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 4, 4, 1, 2>;
+// TPA h = 61, d_h = 64, R = 2: the TPA explainer's 773M model.  61 heads pad to 4 tiles
+// of 16 rows, one per warp of a token slice (HS = 4, two slices: 8 consumer warps);
+// 1000-byte records, 64 tokens a stage.
+using MmaTpaH61D64R2 = MmaDecodeCfg<64, 1, 64, 2, 2, 1, 2, 2, 2, false, 0, 4, 61>;
 
 #define KPA_MMA_VARIANTS(X)        \
     X(0, MmaTpaH16D64R2)           \
@@ -158,14 +173,15 @@ using MmaKpaH4x4D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 4, 4, 1, 2>;
     X(12, MmaKpaH2x10D8x8R2)       \
     X(13, MmaKpaH10x2D8x8R2)       \
     X(14, MmaTpaH16D128R2)         \
-    X(15, MmaKpaH4x4D8x16R4)
+    X(15, MmaKpaH4x4D8x16R4)       \
+    X(16, MmaTpaH61D64R2)
 
 // Index of the variant that covers these dims, or -1.
 inline int mma_decode_variant(const Dims &d) {
 #define KPA_MMA_MATCH(IDX, CFG)                                                                    \
     if (d.rk == CFG::RK && d.rv == CFG::RV &&                                                      \
         (CFG::ORDER3 ? (d.order == 3 && d.h1 == CFG::MA && d.h2 == 1 && d.d1 == CFG::DB && d.d2 == CFG::DC) \
-                     : (d.order != 3 && d.h1 * d.d1 == CFG::MA && d.d1 == CFG::D1 && d.d2 == CFG::D2 &&  \
+                     : (d.order != 3 && d.h1 * d.d1 == CFG::MR && d.d1 == CFG::D1 && d.d2 == CFG::D2 &&  \
                         d.h2 == CFG::H2 && (d.shared != 0) == CFG::SHARED)))                       \
         return IDX;
     KPA_MMA_VARIANTS(KPA_MMA_MATCH)

@@ -26,6 +26,8 @@ SMALL = {
     "kpa_long_base": KPA_LONG.replace(capacity=4104, length=4101, seed=3),
     "tiny_kpa_scaled": TINY_KPA.replace(factor_std=1.0 / np.sqrt(2.0), seed=4),
     "flashtpa": FLASHTPA_DECODE.replace(batch=3, capacity=1536, length=0, ragged=(1, 1536), seed=6),
+    "tpa_h61": __import__("workloads").TPA_H61_DECODE.replace(batch=3, capacity=1024, length=0, ragged=(1, 1024),
+                                                             seed=7),
     "kpa_odd": KPA_MEDIUM.replace(shape=KPA_MEDIUM.shape.__class__(h1=3, h2=2, d1=2, d2=6, r_k=3,
                                                                    r_v=1, rope_base=10000.0),
                                   batch=2, capacity=200, ragged=(1, 200), seed=5),
@@ -379,3 +381,24 @@ def test_more_split_decodes(name):
     want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"],
                                     sm_scale=scale)
     assert_bf16_close(got, want, f"peaked {name}")
+
+
+def test_tpa_h61_on_the_tensor_cores():
+    """The TPA explainer's 773M model, h = 61, d_h = 64, R = 2 (500 numbers per token):
+    61 heads padded to four 16-row tiles split over four warps of a token slice; the
+    padded query rows are zero and the 61 heads' outputs match the oracle end to end,
+    at stage level and with a peaked softmax, on ragged lengths over several tiles."""
+    from workloads import TPA_H61_DECODE
+    lib = kpa()
+    w = TPA_H61_DECODE.replace(batch=3, capacity=1200, length=0, ragged=(1, 1200), seed=63)
+    inp = decode_inputs(w)
+    cfg = lib.make_config(w.shape, w.dtype)
+    assert lib.kpa_decode_kernel_kind(cfg, w.batch, int(inp["seq_len"].max())) == "mma_sync"
+    got, kc, vc = _run(w, inp)
+    assert_bf16_close(got, oracle_decode_unrotated(w, inp), "e2e tpa h=61")
+    want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"])
+    assert_bf16_close(got, want, "stage tpa h=61")
+    scale = 64.0 / np.sqrt(w.shape.dh)
+    got, kc, vc = _run(w, inp, sm_scale=float(scale))
+    want = oracle_decode_from_cache(w, kc.cpu(), vc.cpu(), inp["q"], inp["seq_len"], inp["q_pos"], sm_scale=scale)
+    assert_bf16_close(got, want, "peaked tpa h=61")

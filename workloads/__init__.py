@@ -216,7 +216,16 @@ SPLIT_DECODES = {
         batch=8, capacity=4096, dtype="bf16", factor_std=0.5, q_std=1.0 / 8.0, seed=0, length=4096),
 }
 
-DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
+# The TPA explainer's 773M-parameter TPA model: h = 61 heads, d_h = 64, R_K = R_V = 2,
+# 500 numbers per token ("KV Cache Efficiency at the Evaluated Configurations"); the
+# TPA decode's batch, length and spreads.
+TPA_H61_DECODE = DecodeWorkload(
+    name="TPA decode, 773M model's h=61x1, d_h=1x64 (B=8, R=2+2, L=4096, bf16)",
+    shape=Shape(h1=61, h2=1, d1=1, d2=64, r_k=2, r_v=2, rope_base=10000.0),
+    batch=8, capacity=4096, dtype="bf16", factor_std=1.0 / np.sqrt(2.0), q_std=1.0 / 8.0, seed=0,
+    length=4096)
+
+DECODE_CONFIGS = {"tiny_kpa": TINY_KPA, "tpa_h61": TPA_H61_DECODE, "tpa_decode": TPA_DECODE, "kpa_medium": KPA_MEDIUM,
                   "kpa_long": KPA_LONG, "flashtpa": FLASHTPA_DECODE, "tpa_shared": TPA_SHARED_DECODE,
                   "tpa_order3": TPA3_DECODE, **KPA_SECTION32, **SPLIT_DECODES}
 
