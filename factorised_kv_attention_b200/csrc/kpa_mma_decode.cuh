@@ -130,8 +130,10 @@ using MmaTpaH16D64R2 = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2>;
 using MmaTpaH16D64R2Shared = MmaDecodeCfg<16, 1, 64, 2, 2, 1, 8, 1, 2, true>;
 // KPA h = 4x4, d_h = 8x16, R = 2 with one B shared by keys and values.
 using MmaKpaH4x4D8x16R2Shared = MmaDecodeCfg<32, 8, 16, 2, 2, 4, 2, 2, 2, true>;
-// TPA, h = 32, d_h = 64, R_K = R_V = 1 (the FlashTPA decoding benchmark's shape).
-using MmaTpaH32D64R1 = MmaDecodeCfg<32, 1, 64, 1, 1, 1, 8, 2, 2>;
+// TPA, h = 32, d_h = 64, R_K = R_V = 1 (the FlashTPA decoding benchmark's shape): the
+// two head tiles split over two warps of each of four token slices (one warp holding
+// both spilled).
+using MmaTpaH32D64R1 = MmaDecodeCfg<32, 1, 64, 1, 1, 1, 4, 4, 2, false, 0, 2>;
 // KPA h = 4x8, d_h = 8x16, R_K = R_V = 4.
 using MmaKpaH4x8D8x16R4 = MmaDecodeCfg<32, 8, 16, 4, 4, 8, 2, 1, 2>;
 // KPA h = 4x8, d_h = 8x16, R_K = R_V = 2.
