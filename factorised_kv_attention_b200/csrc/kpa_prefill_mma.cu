@@ -17,7 +17,8 @@
 //     and adds P V (P rounded to fp16) into its fp32 output tile.
 // The scores carry sm_scale / R_K log2(e) folded into Q before it is rounded to fp16;
 // the output is scaled by 1 / R_V.  Rows whose position is outside the cache are
-// written as zeros and raise the device-check error.
+// written as zeros and raise the device-check error; so does an output made non-finite
+// by a value outside the fp16 range.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -436,18 +437,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_mma_kernel(const PrefillM
     const int row0 = wrow0 + (lane >> 2), row1 = row0 + 8;
     const bool ok0 = row0 < a.n_tok && pos0 < a.cap, ok1 = row1 < a.n_tok && pos1 < a.cap;
     const float f0 = l0 > 0.f ? a.out_scale / l0 : 0.f, f1 = l1 > 0.f ? a.out_scale / l1 : 0.f;
+    bool finite = true;
 #pragma unroll
     for (int nt = 0; nt < DH / 8; ++nt) {
         const int f = nt * 8 + 2 * (lane & 3);
         if (f < a.dh) {
-            if (row0 < a.n_tok)
-                *reinterpret_cast<float2 *>(out_b + ((size_t)row0 * h + head) * a.dh + f) =
-                    ok0 ? make_float2(o[nt][0] * f0, o[nt][1] * f0) : make_float2(0.f, 0.f);
-            if (row1 < a.n_tok)
-                *reinterpret_cast<float2 *>(out_b + ((size_t)row1 * h + head) * a.dh + f) =
-                    ok1 ? make_float2(o[nt][2] * f1, o[nt][3] * f1) : make_float2(0.f, 0.f);
+            const float2 y0 = ok0 ? make_float2(o[nt][0] * f0, o[nt][1] * f0) : make_float2(0.f, 0.f);
+            const float2 y1 = ok1 ? make_float2(o[nt][2] * f1, o[nt][3] * f1) : make_float2(0.f, 0.f);
+            if (row0 < a.n_tok) {
+                *reinterpret_cast<float2 *>(out_b + ((size_t)row0 * h + head) * a.dh + f) = y0;
+                finite = finite && isfinite(y0.x) && isfinite(y0.y);
+            }
+            if (row1 < a.n_tok) {
+                *reinterpret_cast<float2 *>(out_b + ((size_t)row1 * h + head) * a.dh + f) = y1;
+                finite = finite && isfinite(y1.x) && isfinite(y1.y);
+            }
         }
     }
+    // a value outside the fp16 range (a rebuilt K or V element, or P) makes rows non-finite
+    if (__any_sync(0xffffffffu, !finite) && lane == 0) raise_error(a.err, kErrDeviceCheck);
 }
 
 struct SliceDims {

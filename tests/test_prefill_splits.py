@@ -221,3 +221,28 @@ def test_append_prefill_split_against_the_plain_definition(name):
     want = oracle.prefill(s, _bf16(q_rot), _bf16(k_rec), _bf16(v_rec), [0] * w.batch, keys_rotated=False,
                           sm_scale=scale)
     assert_bf16_close(out.cpu().numpy(), want, f"append + prefill {name} against the plain definition")
+
+
+@pytest.mark.parametrize("name", ["tpa_h8_d1x64_r2", "c5"])
+def test_prefill_fp16_overflow_is_reported(name):
+    """A cached factor whose rebuilt keys leave the fp16 range (an fp16 operand of the
+    products) in a visible slot makes rows non-finite, which both prefill kernels
+    report as KPA_ERR_DEVICE_CHECK."""
+    lib = kpa()
+    s = C5_SPLIT if name == "c5" else SPLITS[name]
+    starts, n_tok, cap = [0, 0], 130, 256
+    batch = len(starts)
+    w = KPA_MEDIUM.replace(shape=s, batch=batch, capacity=cap, ragged=(), length=cap,
+                           factor_std=1.0 / np.sqrt(2.0), seed=56)
+    inp = decode_inputs(w)
+    inp["kf"][1, 20, s.r_k * s.h1 * s.d1 + 3] = 1.0e6      # a B^K element of a visible slot
+    cfg = lib.make_config(s, "bf16")
+    kc, vc = planes(s, batch, cap, "bf16")
+    zero = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    lib.kpa_append_factors(cfg, batch, cap, inp["kf"].cuda(), inp["vf"].cuda(), zero, cap, kc, vc)
+    assert lib.kpa_prefill_kernel_kind(cfg) == ("tcgen05" if name == "c5" else "mma_sync")
+    lib.kpa_read_device_error()                              # clear
+    q = _query(s, batch, n_tok, seed=13)
+    _prefill(lib, cfg, batch, n_tok, q, torch.tensor(starts, dtype=torch.int32), kc, vc, cap, 1.0 / np.sqrt(s.dh))
+    torch.cuda.synchronize()
+    assert lib.kpa_read_device_error() == lib.KPA_ERR_DEVICE_CHECK
