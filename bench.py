@@ -79,9 +79,10 @@ def _args(argv=None):
                     help="flashtpa: the FlashTPA decoding shape over sequence lengths 2^12..2^19 and batch "
                          "1, 2, 4, 8, 16 (one JSON line per point, then none of the other lines)")
     ap.add_argument("--prefill-split", default="kpa_h4x4_d8x16_r2",
-                    choices=["kpa_h4x4_d8x16_r2", "tpa_h16_d1x128_r2", "kpa_h4x4_d8x16_r4"],
-                    help="append_prefill: the Kronecker split of its h=16, d_h=128 (the tcgen05 prefill takes the "
-                         "first, the mma.sync prefill the others)")
+                    choices=["kpa_h4x4_d8x16_r2", "tpa_h16_d1x128_r2", "kpa_h4x4_d8x16_r4", "kpa353m_h4x4_d8x8_r2"],
+                    help="append_prefill: the Kronecker split of its h=16, d_h=128, or the KPA paper's 353M split "
+                         "(d_model 1024, d_h=8x8); the tcgen05 prefill takes the d1=8, R=2 splits, the mma.sync "
+                         "prefill the others")
     ap.add_argument("--prefill-engine", type=int, default=0, choices=(0, 1),
                     help="1: the mma.sync prefill on every split (measurement)")
     ap.add_argument("--settle-seconds", type=float, default=1.0,

@@ -86,12 +86,13 @@ template <int D1_, int D2_, int RK_, int RV_>
 struct PrefillCfg {
     static constexpr int D1 = D1_, D2 = D2_, RK = RK_, RV = RV_;
     static constexpr int DH = D1 * D2;
-    static_assert(D1 == 8 && D2 == 16, "the fragment mapping covers d1 = 8, d2 = 16");
-    static_assert(RK == 2 && RV == 2, "one ldmatrix.x4 covers the B rows of two ranks");
+    static_assert(D1 == 8 && (D2 == 16 || D2 == 8), "the fragment mapping covers d1 = 8, d2 = 16 or 8");
+    static_assert(RK == 2 && RV == 2, "one ldmatrix covers the B rows of two ranks");
+    static constexpr int HB = D2 / 8;                          // 8-element boxes of a B row
     static constexpr uint32_t Q_HALF = HQ * DH * 2;
     static constexpr uint32_t KV_TILE = TK * DH * 2;
-    static constexpr uint32_t K_ST = 3 * RK * kBox;          // A_r (1 box) and B_r (2 boxes) per rank
-    static constexpr uint32_t V_ST = 3 * RV * kBox;
+    static constexpr uint32_t K_ST = (1 + HB) * RK * kBox;   // A_r (1 box) and B_r (HB boxes) per rank
+    static constexpr uint32_t V_ST = (1 + HB) * RV * kBox;
     static constexpr size_t OFF_Q = 0;                         // two halves
     static constexpr size_t OFF_K = OFF_Q + 2 * Q_HALF;        // two buffers
     static constexpr size_t OFF_V = OFF_K + 2 * KV_TILE;       // one buffer
@@ -129,6 +130,11 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t (&r)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
+}
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -324,8 +330,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 for (int r = 0; r < R; ++r) {
                     tma_load_2d(smem_u32(st + r * kBox), map, (r * a.h1 * D1 + i1 * D1) * kGroup, grp, full);
 #pragma unroll
-                    for (int hb = 0; hb < 2; ++hb)
-                        tma_load_2d(smem_u32(st + (R + 2 * r + hb) * kBox), bmap,
+                    for (int hb = 0; hb < C::HB; ++hb)
+                        tma_load_2d(smem_u32(st + (R + C::HB * r + hb) * kBox), bmap,
                                     (b0 + (r * a.h2 + i2) * C::D2 + hb * 8) * kGroup, grp, full);
                 }
                 issued[is_v ? 1 : 0][s] = t;
@@ -434,50 +440,67 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                         av[r][j1] = __uint_as_float(
                             (uint32_t)(*reinterpret_cast<const uint16_t *>(st + r * kBox + g * 128 + j1 * 16 + tok * 2))
                             << 16);
-                // B_r[tok][hb*8 + 2c .. +1] for (r, hb) = block 0..3
-                uint32_t bw[4];
-                ldsm_x4_t(smem_u32(st + (2 + blk) * kBox + g * 128 + brow * 16), bw);
-                float2 bf[4];
+                // B_r[tok][hb*8 + 2c .. +1] for (r, hb) = block r * HB + hb
+                constexpr int HB = C::HB, NBLK = 2 * HB;
+                float2 bf[NBLK];
+                if constexpr (HB == 2) {
+                    uint32_t bw[4];
+                    ldsm_x4_t(smem_u32(st + (2 + blk) * kBox + g * 128 + brow * 16), bw);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) bf[i] = unpack_bf16x2(bw[i]);
+                    for (int i = 0; i < 4; ++i) bf[i] = unpack_bf16x2(bw[i]);
+                } else {
+                    uint32_t bw[2];                          // lanes 0..15 address the two blocks
+                    ldsm_x2_t(smem_u32(st + (2 + (blk & 1)) * kBox + g * 128 + brow * 16), bw);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) bf[i] = unpack_bf16x2(bw[i]);
+                }
                 if (SHARED && !is_v) {
-                    // shared B is cached unrotated: rotate this lane's pairs m = c and 4 + c of its
-                    // token at the token's slot ("Kronecker Product Attention", Thm 2.4)
+                    // shared B is cached unrotated: rotate this lane's pairs m = c (and 4 + c when
+                    // d2 = 16) of its token at the token's slot ("Kronecker Product Attention", Thm 2.4)
                     const double pos = (double)(t * TK + g * kGroup + tok);
-                    float c0, s0, c1, s1;
+                    float c0, s0, c1 = 1.f, s1 = 0.f;
                     rope_cs_fast(pos, a.theta[lane & 3], c0, s0);
-                    rope_cs_fast(pos, a.theta[4 + (lane & 3)], c1, s1);
+                    if constexpr (HB == 2) rope_cs_fast(pos, a.theta[4 + (lane & 3)], c1, s1);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float cc = (i & 1) ? c1 : c0, ss = (i & 1) ? s1 : s0;
+                    for (int i = 0; i < NBLK; ++i) {
+                        const float cc = (i % HB) ? c1 : c0, ss = (i % HB) ? s1 : s0;
                         bf[i] = make_float2(bf[i].x * cc - bf[i].y * ss, bf[i].x * ss + bf[i].y * cc);
                     }
                 }
-                uint32_t w[8][2];
+                uint32_t w[8][HB];
 #pragma unroll
                 for (int j1 = 0; j1 < 8; ++j1)
 #pragma unroll
-                    for (int hb = 0; hb < 2; ++hb) {
+                    for (int hb = 0; hb < HB; ++hb) {
                         float2 acc = fmul2(make_float2(av[0][j1], av[0][j1]), bf[hb]);
-                        acc = ffma2(make_float2(av[1][j1], av[1][j1]), bf[2 + hb], acc);
+                        acc = ffma2(make_float2(av[1][j1], av[1][j1]), bf[HB + hb], acc);
                         w[j1][hb] = pack_half2(acc.x, acc.y);
                     }
                 if (edge && t * TK + g * kGroup + tok > max_slot) {
 #pragma unroll
-                    for (int j1 = 0; j1 < 8; ++j1) w[j1][0] = w[j1][1] = 0u;
-                }
-                // this lane addresses row brow of block blk of each x4 store: (j1 = 2i + blk/2, hb = blk%2)
+                    for (int j1 = 0; j1 < 8; ++j1)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int f0 = (2 * i + (blk >> 1)) * 16 + (blk & 1) * 8;     // first feature of the block
+                        for (int hb = 0; hb < HB; ++hb) w[j1][hb] = 0u;
+                }
+                // this lane addresses row brow of block blk of each x4 store: d2 = 16, (j1 = 2i +
+                // blk/2, hb = blk%2); d2 = 8, j1 = 4i + blk
+#pragma unroll
+                for (int i = 0; i < 8 / (4 / HB); ++i) {
+                    const int f0 = HB == 2 ? (2 * i + (blk >> 1)) * 16 + (blk & 1) * 8 : (4 * i + blk) * 8;
+                    uint32_t w0, w1, w2, w3;
+                    if constexpr (HB == 2) {
+                        w0 = w[2 * i][0], w1 = w[2 * i][HB - 1], w2 = w[2 * i + 1][0], w3 = w[2 * i + 1][HB - 1];
+                    } else {
+                        w0 = w[4 * i][0], w1 = w[4 * i + 1][0], w2 = w[4 * i + 2][0], w3 = w[4 * i + 3][0];
+                    }
                     if (!is_v) {
                         const int row = g * kGroup + brow;                          // token row
                         const uint32_t ad = dst + (f0 >> 6) * (TK * 128) + sw128_chunk(row, (f0 & 63) >> 3);
-                        stsm_x4(ad, w[2 * i][0], w[2 * i][1], w[2 * i + 1][0], w[2 * i + 1][1]);
+                        stsm_x4(ad, w0, w1, w2, w3);
                     } else {
                         const int row = f0 + brow;                                  // feature row
                         const uint32_t ad = dst + (g >> 3) * (DH * 128) + sw128_chunk(row, g & 7);
-                        stsm_x4_t(ad, w[2 * i][0], w[2 * i][1], w[2 * i + 1][0], w[2 * i + 1][1]);
+                        stsm_x4_t(ad, w0, w1, w2, w3);
                     }
                 }
             }
@@ -695,6 +718,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 }
 
 using PrefillKpaH4x4D8x16R2 = PrefillCfg<8, 16, 2, 2>;
+using PrefillKpaD8x8R2 = PrefillCfg<8, 8, 2, 2>;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -739,16 +763,16 @@ bool make_factor_map(CUtensorMap *map, const void *plane, uint64_t groups, uint6
 }  // namespace
 
 bool prefill_supported(const Dims &d) {
-    return d.d1 == PrefillKpaH4x4D8x16R2::D1 && d.d2 == PrefillKpaH4x4D8x16R2::D2 &&
-           d.rk == PrefillKpaH4x4D8x16R2::RK && d.rv == PrefillKpaH4x4D8x16R2::RV;
+    return d.d1 == 8 && (d.d2 == 16 || d.d2 == 8) && d.rk == 2 && d.rv == 2;
 }
 
-cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const PrefillQf &qf,
-                           const int32_t *start_pos, const void *kc, const void *vc, int cap, float qscale,
-                           float out_scale, float *out, const RopeTable &rope, int *err,
-                           unsigned long long wait_limit_ns, cudaStream_t st) {
-    using C = PrefillKpaH4x4D8x16R2;
-    if (!prefill_supported(d)) return cudaErrorInvalidValue;
+namespace {
+
+template <class C>
+cudaError_t launch_prefill_cfg(const Dims &d, int batch, int n_tok, const void *q, const PrefillQf &qf,
+                               const int32_t *start_pos, const void *kc, const void *vc, int cap, float qscale,
+                               float out_scale, float *out, const RopeTable &rope, int *err,
+                               unsigned long long wait_limit_ns, cudaStream_t st) {
     PrefillArgs a;
     a.batch = batch;
     a.n_tok = n_tok;
@@ -791,6 +815,20 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     else
         prefill_kernel<C, false, false><<<grid, kThreads, C::SMEM, st>>>(tmq, tmk, tmv, a);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, const PrefillQf &qf,
+                           const int32_t *start_pos, const void *kc, const void *vc, int cap, float qscale,
+                           float out_scale, float *out, const RopeTable &rope, int *err,
+                           unsigned long long wait_limit_ns, cudaStream_t st) {
+    if (!prefill_supported(d)) return cudaErrorInvalidValue;
+    if (d.d2 == 8)
+        return launch_prefill_cfg<PrefillKpaD8x8R2>(d, batch, n_tok, q, qf, start_pos, kc, vc, cap, qscale,
+                                                     out_scale, out, rope, err, wait_limit_ns, st);
+    return launch_prefill_cfg<PrefillKpaH4x4D8x16R2>(d, batch, n_tok, q, qf, start_pos, kc, vc, cap, qscale,
+                                                      out_scale, out, rope, err, wait_limit_ns, st);
 }
 
 }  // namespace kpa

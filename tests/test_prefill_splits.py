@@ -1,8 +1,8 @@
-"""kpa_prefill on the Kronecker splits that the tcgen05 prefill is not instantiated
-for, which run on the mma.sync prefill: the TPA split (h1 = h, d1 = 1), R = 4, the
-KPA paper's section 3.2 head/feature splits, uneven ranks, d2 not a multiple of 4,
-d1 > d2, a shared B, and queries given as factors, each against the float64 oracle;
-and the mma.sync prefill on the tcgen05 kernel's own split (GPU)."""
+"""kpa_prefill on Kronecker splits other than the append+prefill configuration's: the
+TPA split (h1 = h, d1 = 1), R = 4, uneven ranks, d2 not a multiple of 4, d1 > d2, a
+shared B and queries given as factors run on the mma.sync prefill; the KPA paper's
+section 3.2 splits (d1 = d2 = 8, R = 2) run on the tcgen05 prefill.  Each against the
+float64 oracle, and both kernels on the splits the tcgen05 one takes (GPU)."""
 import dataclasses
 
 import numpy as np
@@ -20,12 +20,18 @@ SPLITS = {
     "tpa_h8_d1x128_rk3_rv2": Shape(h1=8, h2=1, d1=1, d2=128, r_k=3, r_v=2),
     "kpa_h4x4_d8x16_r4": Shape(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4),
     "kpa_h2x8_d8x8_r2": Shape(h1=2, h2=8, d1=8, d2=8, r_k=2, r_v=2),
+    "kpa_h10x2_d8x8_r2": Shape(h1=10, h2=2, d1=8, d2=8, r_k=2, r_v=2),
     "kpa_h4x4_d8x16_rk3_rv1": Shape(h1=4, h2=4, d1=8, d2=16, r_k=3, r_v=1),
     "kpa_h3x2_d4x6_r2": Shape(h1=3, h2=2, d1=4, d2=6, r_k=2, r_v=2),
     "kpa_h4x2_d16x4_r2": Shape(h1=4, h2=2, d1=16, d2=4, r_k=2, r_v=2),
 }
 # the tcgen05 kernel's split
 C5_SPLIT = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2)
+
+
+def _kind(s):
+    """The prefill kernel a split runs on by default."""
+    return "tcgen05" if s.d1 == 8 and s.d2 in (8, 16) and s.r_k == 2 and s.r_v == 2 else "mma_sync"
 
 
 def _cache(lib, s, batch, cap, seed, factor_std=1.0 / np.sqrt(2.0)):
@@ -72,7 +78,7 @@ def test_prefill_split_against_oracle(name, starts, n_tok):
     batch = len(starts)
     cap = max(512, (max(starts) + n_tok + 7) // 8 * 8)
     cfg, kc, vc = _cache(lib, s, batch, cap, seed=51)
-    assert lib.kpa_prefill_kernel_kind(cfg) == "mma_sync"
+    assert lib.kpa_prefill_kernel_kind(cfg) == _kind(s)
     q = _query(s, batch, n_tok, seed=8)
     start = torch.tensor(starts, dtype=torch.int32)
     scale = 1.0 / np.sqrt(s.dh)
@@ -118,11 +124,11 @@ def test_prefill_split_shared_b():
     assert_bf16_close(out.cpu().numpy(), _oracle(s, q, kc, vc, batch, cap, starts, scale), "shared-B TPA prefill")
 
 
-def test_prefill_mma_kernel_on_the_tcgen05_split():
-    """The tcgen05 kernel's split, on both kernels (kpa_test_set_prefill_engine): each
+@pytest.mark.parametrize("s", [C5_SPLIT, SPLITS["kpa_h2x8_d8x8_r2"]], ids=["d8x16", "d8x8"])
+def test_prefill_mma_kernel_on_the_tcgen05_split(s):
+    """The tcgen05 kernel's splits, on both kernels (kpa_test_set_prefill_engine): each
     against the oracle, so the two prefill kernels are checked on one shape."""
     lib = kpa()
-    s = C5_SPLIT
     starts, n_tok, cap = [0, 77], 400, 512
     batch = len(starts)
     cfg, kc, vc = _cache(lib, s, batch, cap, seed=54)

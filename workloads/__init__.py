@@ -157,6 +157,11 @@ APPEND_PREFILL_SPLITS = {
     "kpa_h4x4_d8x16_r4": APPEND_PREFILL.replace(
         name="KPA append+prefill (B=8, n=2048, d_model=2048, h=4x4, d_h=8x16, R_Q=6, R=4+4)",
         shape=dataclasses.replace(APPEND_PREFILL.shape, r_k=4, r_v=4)),
+    # the KPA paper's 353M models (section 3.2): d_model 1024, h = 16 as 4x4, d_h = 64 as
+    # 8x8, R = 2; the same chunk, batch and R_Q
+    "kpa353m_h4x4_d8x8_r2": APPEND_PREFILL.replace(
+        name="KPA append+prefill, 353M model split (B=8, n=2048, d_model=1024, h=4x4, d_h=8x8, R_Q=6, R=2+2)",
+        shape=dataclasses.replace(APPEND_PREFILL.shape, d2=8, d_model=1024)),
 }
 
 # The decoding benchmark shape of the FlashTPA figures ("Tensor Product Attention Is
