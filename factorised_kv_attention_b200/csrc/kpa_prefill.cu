@@ -87,8 +87,11 @@ struct PrefillCfg {
     static constexpr int D1 = D1_, D2 = D2_, RK = RK_, RV = RV_;
     static constexpr int DH = D1 * D2;
     static_assert(D1 == 8 && (D2 == 16 || D2 == 8), "the fragment mapping covers d1 = 8, d2 = 16 or 8");
-    static_assert(RK == 2 && RV == 2, "one ldmatrix covers the B rows of two ranks");
+    static_assert(RK == RV && (RK == 2 || (RK == 4 && D2 == 16)), "ranks: 2, or 4 with d2 = 16");
     static constexpr int HB = D2 / 8;                          // 8-element boxes of a B row
+    // factor stages: two at R = 2; one at R = 4, where two stages of four ranks' slices
+    // would not fit beside the Q, K and V tiles
+    static constexpr int FST = RK == 2 ? 2 : 1;
     static constexpr uint32_t Q_HALF = HQ * DH * 2;
     static constexpr uint32_t KV_TILE = TK * DH * 2;
     static constexpr uint32_t K_ST = (1 + HB) * RK * kBox;   // A_r (1 box) and B_r (HB boxes) per rank
@@ -96,11 +99,12 @@ struct PrefillCfg {
     static constexpr size_t OFF_Q = 0;                         // two halves
     static constexpr size_t OFF_K = OFF_Q + 2 * Q_HALF;        // two buffers
     static constexpr size_t OFF_V = OFF_K + 2 * KV_TILE;       // one buffer
-    static constexpr size_t OFF_KST = OFF_V + KV_TILE;         // two stages
-    static constexpr size_t OFF_VST = OFF_KST + 2 * K_ST;      // two stages
-    static constexpr size_t OFF_BAR = OFF_VST + 2 * V_ST;
+    static constexpr size_t OFF_KST = OFF_V + KV_TILE;         // FST stages
+    static constexpr size_t OFF_VST = OFF_KST + FST * K_ST;    // FST stages
+    static constexpr size_t OFF_BAR = OFF_VST + FST * V_ST;
     static constexpr int NBAR = 24;
     static constexpr size_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 // mbarrier slots
@@ -315,11 +319,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const int grp0 = (int)((int64_t)b * a.cap / kGroup);
             const int ea = RK * a.h1 * D1;     // first B element of a key record
             const int va = RV * a.h1 * D1;
-            int issued[2][2] = {{-1, -1}, {-1, -1}};
+            int issued[2][2] = {{-1, -1}, {-1, -1}};          // [plane][stage < FST]
             // the head's factor slices of tile t: A_r[i1] (one box) and B_r[i2] (two boxes) per rank
             auto issue_factors = [&](int t, bool is_v) -> bool {
-                const int s = t & 1, grp = grp0 + t * (TK / kGroup);
-                if (t >= 2 && !wait((is_v ? B_VST_EMPTY : B_KST_EMPTY) + s, ((t >> 1) - 1) & 1)) return false;
+                constexpr int FST = C::FST;
+                const int s = t % FST, grp = grp0 + t * (TK / kGroup);
+                if (t >= FST && !wait((is_v ? B_VST_EMPTY : B_KST_EMPTY) + s, ((t / FST) - 1) & 1)) return false;
                 const uint32_t full = bar((is_v ? B_VST_FULL : B_KST_FULL) + s);
                 mbar_expect_tx(full, is_v ? C::V_ST : C::K_ST);
                 unsigned char *st = smem + (is_v ? C::OFF_VST + s * C::V_ST : C::OFF_KST + s * C::K_ST);
@@ -360,9 +365,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 #pragma unroll
             for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-                for (int s = 0; s < 2; ++s)
+                for (int s = 0; s < C::FST; ++s)
                     if (issued[pl][s] >= 0)
-                        (void)mbar_wait(bar((pl ? B_VST_FULL : B_KST_FULL) + s), (issued[pl][s] >> 1) & 1, limit);
+                        (void)mbar_wait(bar((pl ? B_VST_FULL : B_KST_FULL) + s), (issued[pl][s] / C::FST) & 1, limit);
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issue
@@ -425,32 +430,37 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         const int blk = lane >> 3, brow = lane & 7;   // ldmatrix / stmatrix row this lane addresses
         // Rebuild one plane of tile t: K (token rows, stmatrix) or V^T (feature rows, stmatrix.trans).
         auto rebuild = [&](int t, bool is_v) {
-            const unsigned char *st = smem + (is_v ? C::OFF_VST + (t & 1) * C::V_ST : C::OFF_KST + (t & 1) * C::K_ST);
+            const int fs = t % C::FST;                                    // factor stage
+            const unsigned char *st = smem + (is_v ? C::OFF_VST + fs * C::V_ST : C::OFF_KST + fs * C::K_ST);
             const uint32_t dst = smem_u32(smem + (is_v ? C::OFF_V : C::OFF_K + (t & 1) * C::KV_TILE));
             const bool edge = t * TK + TK - 1 > max_slot;
 #pragma unroll 1
             for (int gi = 0; gi < TK / kGroup / kRebuildWarps; ++gi) {
                 const int g = rw + gi * kRebuildWarps;      // group of the tile, 0..15
-                // A_r[tok][j1], r = 0, 1: one 16-byte row per j1 holds the group's 8 tokens
-                float av[2][8];
+                // A_r[tok][j1], r < R: one 16-byte row per j1 holds the group's 8 tokens
+                constexpr int R = RK;
+                float av[R][8];
 #pragma unroll
-                for (int r = 0; r < 2; ++r)
+                for (int r = 0; r < R; ++r)
 #pragma unroll
                     for (int j1 = 0; j1 < 8; ++j1)
                         av[r][j1] = __uint_as_float(
                             (uint32_t)(*reinterpret_cast<const uint16_t *>(st + r * kBox + g * 128 + j1 * 16 + tok * 2))
                             << 16);
                 // B_r[tok][hb*8 + 2c .. +1] for (r, hb) = block r * HB + hb
-                constexpr int HB = C::HB, NBLK = 2 * HB;
+                constexpr int HB = C::HB, NBLK = R * HB;
                 float2 bf[NBLK];
                 if constexpr (HB == 2) {
-                    uint32_t bw[4];
-                    ldsm_x4_t(smem_u32(st + (2 + blk) * kBox + g * 128 + brow * 16), bw);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) bf[i] = unpack_bf16x2(bw[i]);
+                    for (int q4 = 0; q4 < NBLK / 4; ++q4) {          // four blocks (two ranks) per load
+                        uint32_t bw[4];
+                        ldsm_x4_t(smem_u32(st + (R + 4 * q4 + blk) * kBox + g * 128 + brow * 16), bw);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) bf[4 * q4 + i] = unpack_bf16x2(bw[i]);
+                    }
                 } else {
                     uint32_t bw[2];                          // lanes 0..15 address the two blocks
-                    ldsm_x2_t(smem_u32(st + (2 + (blk & 1)) * kBox + g * 128 + brow * 16), bw);
+                    ldsm_x2_t(smem_u32(st + (R + (blk & 1)) * kBox + g * 128 + brow * 16), bw);
 #pragma unroll
                     for (int i = 0; i < 2; ++i) bf[i] = unpack_bf16x2(bw[i]);
                 }
@@ -473,7 +483,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 #pragma unroll
                     for (int hb = 0; hb < HB; ++hb) {
                         float2 acc = fmul2(make_float2(av[0][j1], av[0][j1]), bf[hb]);
-                        acc = ffma2(make_float2(av[1][j1], av[1][j1]), bf[HB + hb], acc);
+#pragma unroll
+                        for (int r = 1; r < R; ++r)
+                            acc = ffma2(make_float2(av[r][j1], av[r][j1]), bf[r * HB + hb], acc);
                         w[j1][hb] = pack_half2(acc.x, acc.y);
                     }
                 if (edge && t * TK + g * kGroup + tok > max_slot) {
@@ -506,8 +518,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
         };
         auto step = [&](int t, bool is_v) -> bool {
-            const int s = t & 1;
-            bool ok = wait((is_v ? B_VST_FULL : B_KST_FULL) + s, (t >> 1) & 1);
+            const int s = t & 1, fs = t % C::FST;           // K buffer, factor stage
+            bool ok = wait((is_v ? B_VST_FULL : B_KST_FULL) + fs, (t / C::FST) & 1);
             if (ok && !is_v && t >= 2) ok = wait(B_K_EMPTY + s, ((t >> 1) - 1) & 1);
             if (ok && is_v && t >= 1) ok = wait(B_V_EMPTY, (t - 1) & 1);
             if (!__all_sync(0xffffffffu, ok)) return false;
@@ -516,7 +528,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(is_v ? B_V_FULL : B_K_FULL + s));
-                mbar_arrive(bar((is_v ? B_VST_EMPTY : B_KST_EMPTY) + s));
+                mbar_arrive(bar((is_v ? B_VST_EMPTY : B_KST_EMPTY) + fs));
             }
             return true;
         };
@@ -719,6 +731,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 
 using PrefillKpaH4x4D8x16R2 = PrefillCfg<8, 16, 2, 2>;
 using PrefillKpaD8x8R2 = PrefillCfg<8, 8, 2, 2>;
+using PrefillKpaD8x16R4 = PrefillCfg<8, 16, 4, 4>;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -763,7 +776,7 @@ bool make_factor_map(CUtensorMap *map, const void *plane, uint64_t groups, uint6
 }  // namespace
 
 bool prefill_supported(const Dims &d) {
-    return d.d1 == 8 && (d.d2 == 16 || d.d2 == 8) && d.rk == 2 && d.rv == 2;
+    return d.d1 == 8 && d.rk == d.rv && ((d.d2 == 16 && (d.rk == 2 || d.rk == 4)) || (d.d2 == 8 && d.rk == 2));
 }
 
 namespace {
@@ -827,6 +840,9 @@ cudaError_t launch_prefill(const Dims &d, int batch, int n_tok, const void *q, c
     if (d.d2 == 8)
         return launch_prefill_cfg<PrefillKpaD8x8R2>(d, batch, n_tok, q, qf, start_pos, kc, vc, cap, qscale,
                                                      out_scale, out, rope, err, wait_limit_ns, st);
+    if (d.rk == 4)
+        return launch_prefill_cfg<PrefillKpaD8x16R4>(d, batch, n_tok, q, qf, start_pos, kc, vc, cap, qscale,
+                                                      out_scale, out, rope, err, wait_limit_ns, st);
     return launch_prefill_cfg<PrefillKpaH4x4D8x16R2>(d, batch, n_tok, q, qf, start_pos, kc, vc, cap, qscale,
                                                       out_scale, out, rope, err, wait_limit_ns, st);
 }

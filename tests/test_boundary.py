@@ -85,10 +85,10 @@ def test_shared_b_needs_equal_ranks():
 
 
 def test_prefill_kernel_kinds():
-    """The tcgen05 prefill takes d1 = 8, d2 = 16 or 8, R = 2 (B shared or not); the mma.sync
-    prefill every other order-2 bf16 split with d_h <= 128 whose factor slices fit its
-    staging, and the tcgen05 split too after kpa_test_set_prefill_engine(1).  d_h > 128,
-    oversized slices and fp32 are refused before any device call."""
+    """The tcgen05 prefill takes d1 = 8 with d2 = 16 (R = 2 or 4) or d2 = 8 (R = 2), B shared or
+    not; the mma.sync prefill every other order-2 bf16 split with d_h <= 128 whose factor
+    slices fit its staging, and the tcgen05 splits too after kpa_test_set_prefill_engine(1).
+    d_h > 128, oversized slices and fp32 are refused before any device call."""
     def kind(**kw):
         return kpa.kpa_prefill_kernel_kind(kpa.make_config(Shape(**kw), "bf16"))
 
@@ -97,9 +97,10 @@ def test_prefill_kernel_kinds():
     assert kind(**c5, shared_b=1) == "tcgen05"
     for h1, h2 in ((4, 4), (2, 8), (8, 2), (4, 5), (2, 10), (10, 2)):    # section 3.2's splits
         assert kind(h1=h1, h2=h2, d1=8, d2=8, r_k=2, r_v=2) == "tcgen05", (h1, h2)
+    assert kind(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4) == "tcgen05"                  # rank 4
     for split in (dict(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2), dict(h1=16, h2=1, d1=1, d2=64, r_k=2, r_v=2,
                                                                     shared_b=1),
-                  dict(h1=4, h2=4, d1=8, d2=16, r_k=4, r_v=4), dict(h1=2, h2=8, d1=8, d2=8, r_k=4, r_v=4),
+                  dict(h1=4, h2=4, d1=8, d2=16, r_k=3, r_v=1), dict(h1=2, h2=8, d1=8, d2=8, r_k=4, r_v=4),
                   dict(h1=3, h2=2, d1=4, d2=6, r_k=2, r_v=2), dict(h1=8, h2=1, d1=1, d2=128, r_k=3, r_v=2)):
         assert kind(**split) == "mma_sync", split
     try:

@@ -1,7 +1,7 @@
 """kpa_prefill on Kronecker splits other than the append+prefill configuration's: the
 TPA split (h1 = h, d1 = 1), R = 4, uneven ranks, d2 not a multiple of 4, d1 > d2, a
-shared B and queries given as factors run on the mma.sync prefill; the KPA paper's
-section 3.2 splits (d1 = d2 = 8, R = 2) run on the tcgen05 prefill.  Each against the
+shared B and queries given as factors run on the mma.sync prefill; d1 = 8 with R = 4
+and the KPA paper's section 3.2 splits (d1 = d2 = 8, R = 2) run on the tcgen05 prefill.  Each against the
 float64 oracle, and both kernels on the splits the tcgen05 one takes (GPU)."""
 import dataclasses
 
@@ -31,7 +31,9 @@ C5_SPLIT = Shape(h1=4, h2=4, d1=8, d2=16, r_k=2, r_v=2)
 
 def _kind(s):
     """The prefill kernel a split runs on by default."""
-    return "tcgen05" if s.d1 == 8 and s.d2 in (8, 16) and s.r_k == 2 and s.r_v == 2 else "mma_sync"
+    if s.d1 == 8 and s.r_k == s.r_v and ((s.d2 == 16 and s.r_k in (2, 4)) or (s.d2 == 8 and s.r_k == 2)):
+        return "tcgen05"
+    return "mma_sync"
 
 
 def _cache(lib, s, batch, cap, seed, factor_std=1.0 / np.sqrt(2.0)):
@@ -124,7 +126,8 @@ def test_prefill_split_shared_b():
     assert_bf16_close(out.cpu().numpy(), _oracle(s, q, kc, vc, batch, cap, starts, scale), "shared-B TPA prefill")
 
 
-@pytest.mark.parametrize("s", [C5_SPLIT, SPLITS["kpa_h2x8_d8x8_r2"]], ids=["d8x16", "d8x8"])
+@pytest.mark.parametrize("s", [C5_SPLIT, SPLITS["kpa_h2x8_d8x8_r2"], SPLITS["kpa_h4x4_d8x16_r4"]],
+                         ids=["d8x16", "d8x8", "d8x16_r4"])
 def test_prefill_mma_kernel_on_the_tcgen05_split(s):
     """The tcgen05 kernel's splits, on both kernels (kpa_test_set_prefill_engine): each
     against the oracle, so the two prefill kernels are checked on one shape."""
