@@ -557,21 +557,26 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
         const int n_valid = min(TT, t1 - t0 - t * TT);
         const int tok_base = slice * CHUNKS * 16;
 
-#pragma unroll
-        for (int ch = 0; ch < CHUNKS; ++ch) {
-            const int tok0 = tok_base + ch * 16;
-            if (tok0 >= n_valid) break;
-            // a chunk that ends past the tile's valid tokens (the ragged end of a split)
-            // masks its scores and factors; full chunks carry none of that code
-            auto chunk = [&](auto tail_c) {
+            // NC chunks of 16 tokens from tok0 on, with one softmax update: the score
+            // products of the NC chunks are independent, so a warp has NC of them in
+            // flight.  A chunk that ends past the tile's valid tokens (the ragged end of
+            // a split, NC = 1) masks its scores and factors; full chunks carry none of
+            // that code
+            auto chunk = [&](auto tail_c, auto nc_c, const int tok0) {
                 constexpr bool TAIL = decltype(tail_c)::value;
-                const unsigned char *kg0 = kt + (size_t)(tok0 >> 3) * EK * 16;
-                // ---- scores of head 2 mt + hi1, tokens (gi, 2c) and (gi, 2c + 1)
-                float2 sc[MT][2];
+                constexpr int NC = decltype(nc_c)::value;
+                static_assert(!TAIL || NC == 1, "a ragged chunk runs alone");
+                // ---- scores of head 2 mt + hi1, tokens (gi, 2c) and (gi, 2c + 1) of chunk cc
+                float2 sc[NC][MT][2];
     #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) sc[mt][0] = sc[mt][1] = make_float2(0.f, 0.f);
+                for (int cc = 0; cc < NC; ++cc)
+    #pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) sc[cc][mt][0] = sc[cc][mt][1] = make_float2(0.f, 0.f);
+    #pragma unroll
+                for (int cc = 0; cc < NC; ++cc)
     #pragma unroll
                 for (int r = 0; r < RK; ++r) {
+                    const unsigned char *kg0 = kt + (size_t)((tok0 + cc * 16) >> 3) * EK * 16;
     #pragma unroll
                     for (int gi = 0; gi < 2; ++gi) {
                         const unsigned char *grp = kg0 + (size_t)gi * EK * 16;
@@ -605,8 +610,10 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                                     mma16816(acc, qa_lo[mt][ks], bk[ks][0], bk[ks][1]);
                                 }
                             }
-                            sc[mt][gi] = ffma2(make_float2(acc[0], acc[1]), unpack_bf16x2(ak[mt][0]), sc[mt][gi]);
-                            sc[mt][gi] = ffma2(make_float2(acc[2], acc[3]), unpack_bf16x2(ak[mt][1]), sc[mt][gi]);
+                            sc[cc][mt][gi] =
+                                ffma2(make_float2(acc[0], acc[1]), unpack_bf16x2(ak[mt][0]), sc[cc][mt][gi]);
+                            sc[cc][mt][gi] =
+                                ffma2(make_float2(acc[2], acc[3]), unpack_bf16x2(ak[mt][1]), sc[cc][mt][gi]);
                         }
                     }
                 }
@@ -614,11 +621,13 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
     #pragma unroll
                 for (int off = 4; off <= 8; off <<= 1)
     #pragma unroll
+                    for (int cc = 0; cc < NC; ++cc)
+    #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
     #pragma unroll
                         for (int gi = 0; gi < 2; ++gi) {
-                            sc[mt][gi].x += __shfl_xor_sync(0xffffffffu, sc[mt][gi].x, off);
-                            sc[mt][gi].y += __shfl_xor_sync(0xffffffffu, sc[mt][gi].y, off);
+                            sc[cc][mt][gi].x += __shfl_xor_sync(0xffffffffu, sc[cc][mt][gi].x, off);
+                            sc[cc][mt][gi].y += __shfl_xor_sync(0xffffffffu, sc[cc][mt][gi].y, off);
                         }
                 if constexpr (TAIL) {
     #pragma unroll
@@ -626,17 +635,21 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         const int tk = tok0 + gi * 8 + 2 * c;
     #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
-                            if (tk >= n_valid) sc[mt][gi].x = -INFINITY;
-                            if (tk + 1 >= n_valid) sc[mt][gi].y = -INFINITY;
+                            if (tk >= n_valid) sc[0][mt][gi].x = -INFINITY;
+                            if (tk + 1 >= n_valid) sc[0][mt][gi].y = -INFINITY;
                         }
                     }
                 }
-                // ---- online softmax of this lane's head over the chunk's 16 tokens
+                // ---- online softmax of this lane's head over the NC chunks' tokens
                 bool grow = false;
                 float alpha[MT];
     #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    float mx = fmaxf(fmaxf(sc[mt][0].x, sc[mt][0].y), fmaxf(sc[mt][1].x, sc[mt][1].y));
+                    float mx = -INFINITY;
+    #pragma unroll
+                    for (int cc = 0; cc < NC; ++cc)
+                        mx = fmaxf(mx, fmaxf(fmaxf(sc[cc][mt][0].x, sc[cc][mt][0].y),
+                                             fmaxf(sc[cc][mt][1].x, sc[cc][mt][1].y)));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                     alpha[mt] = 1.f;
@@ -646,12 +659,17 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         grow = true;
                     }
                     const float m_new = m_k[mt];
+                    float lsum = 0.f;
     #pragma unroll
-                    for (int gi = 0; gi < 2; ++gi) {
-                        sc[mt][gi].x = ex2_approx(sc[mt][gi].x - m_new);
-                        sc[mt][gi].y = ex2_approx(sc[mt][gi].y - m_new);
+                    for (int cc = 0; cc < NC; ++cc) {
+    #pragma unroll
+                        for (int gi = 0; gi < 2; ++gi) {
+                            sc[cc][mt][gi].x = ex2_approx(sc[cc][mt][gi].x - m_new);
+                            sc[cc][mt][gi].y = ex2_approx(sc[cc][mt][gi].y - m_new);
+                        }
+                        lsum += (sc[cc][mt][0].x + sc[cc][mt][0].y) + (sc[cc][mt][1].x + sc[cc][mt][1].y);
                     }
-                    l_k[mt] = l_k[mt] * alpha[mt] + ((sc[mt][0].x + sc[mt][0].y) + (sc[mt][1].x + sc[mt][1].y));
+                    l_k[mt] = l_k[mt] * alpha[mt] + lsum;
                 }
                 if (__any_sync(0xffffffffu, grow)) {
     #pragma unroll
@@ -663,10 +681,12 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 }
                 // ---- values: P'[(i1, j1), token] = p * A^V_r in fp16 (A operand: rows g, g + 8,
                 // tokens 2c, 2c + 1 of group 0 then of group 1)
-                const unsigned char *g0p = vt + (size_t)(tok0 >> 3) * EV * 16;
-                const unsigned char *g1p = g0p + (size_t)EV * 16;
+    #pragma unroll
+                for (int cc = 0; cc < NC; ++cc)
     #pragma unroll
                 for (int r = 0; r < RV; ++r) {
+                    const unsigned char *g0p = vt + (size_t)((tok0 + cc * 16) >> 3) * EV * 16;
+                    const unsigned char *g1p = g0p + (size_t)EV * 16;
                     uint32_t av[2][MT][2];
     #pragma unroll
                     for (int gi = 0; gi < 2; ++gi) {
@@ -679,7 +699,7 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                         for (int gi = 0; gi < 2; ++gi)
     #pragma unroll
                             for (int hr = 0; hr < 2; ++hr) {
-                                float2 x = fmul2(sc[mt][gi], unpack_bf16x2(av[gi][mt][hr]));
+                                float2 x = fmul2(sc[cc][mt][gi], unpack_bf16x2(av[gi][mt][hr]));
                                 if constexpr (TAIL) {   // garbage factors of masked tokens stay out (their weight is 0)
                                     const int tk = tok0 + gi * 8 + 2 * c;
                                     if (tk >= n_valid) x.x = 0.f;
@@ -730,11 +750,19 @@ decode_mma_kernel(DecodeArgs a, RopeTable rope, DecodeTestHooks hooks) {
                 }
         
             };
-            if (tok0 + 16 > n_valid)
-                chunk(std::true_type{});
-            else
-                chunk(std::false_type{});
-        }
+            if (n_valid >= tok_base + CHUNKS * 16) {
+                chunk(std::false_type{}, std::integral_constant<int, CHUNKS>{}, tok_base);
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < CHUNKS; ++ch) {
+                    const int tok0 = tok_base + ch * 16;
+                    if (tok0 >= n_valid) break;
+                    if (tok0 + 16 > n_valid)
+                        chunk(std::true_type{}, std::integral_constant<int, 1>{}, tok0);
+                    else
+                        chunk(std::false_type{}, std::integral_constant<int, 1>{}, tok0);
+                }
+            }
         __syncwarp();
         if (lane == 0) {
             // the warp is done with stage s: the last of the WARPS releases issues tile
