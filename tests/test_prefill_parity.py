@@ -225,8 +225,8 @@ def _oracle_records(w, inp):
     0 .. n_tok (the oracle rotates each key reconstruction itself when it attends).
 
     The configuration stores bf16 factors, so the end-to-end oracle rounds to bf16 at
-    the two storage points, the cache records and the chunk's q_out (the survey's
-    reading of the rounding points); the decode step's query is assembled from fp32
+    the two storage points, the cache records and the chunk's q_out (the pages fix no
+    rounding points; these are where the library stores bf16); the decode step's query is assembled from fp32
     factors and is not rounded.  The library rounds a key record after rotating its B,
     the oracle before (it rotates the reconstruction): one bf16 rounding apart, which
     the oracle alone puts at 4e-4 relative on this configuration."""
