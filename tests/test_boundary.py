@@ -233,3 +233,76 @@ def test_package_refuses_to_load_without_the_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import factorised_kv_attention_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "ImportError" in r.stderr and "libkpa.so" in r.stderr
+
+
+PCFG = kpa.make_config(APPEND_PREFILL.shape, "bf16")
+
+
+def _prefill(**over):
+    args = dict(batch=2, n_tok=64, q=A, start_pos=A, kcache=A, vcache=A, capacity=128, sm_scale=0.1, out=A)
+    args.update(over)
+    kpa.kpa_prefill(PCFG, args["batch"], args["n_tok"], args["q"], args["start_pos"], args["kcache"],
+                    args["vcache"], args["capacity"], args["sm_scale"], args["out"], stream=0)
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(start_pos=None), dict(kcache=None), dict(vcache=None), dict(out=None),
+    dict(q=A + 2), dict(kcache=A + 8), dict(vcache=A + 4), dict(out=A + 4), dict(start_pos=A + 1),
+    dict(capacity=60), dict(capacity=0), dict(batch=-1), dict(n_tok=-1),
+    dict(sm_scale=float("nan")), dict(sm_scale=float("inf")),
+], ids=str)
+def test_prefill_rejects_before_launch(over):
+    with pytest.raises(kpa.KpaError) as e:
+        _prefill(**over)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def test_prefill_empty_is_a_no_op():
+    _prefill(batch=0, q=None, start_pos=None, kcache=None, vcache=None, out=None)
+    _prefill(n_tok=0, q=None, start_pos=None, kcache=None, vcache=None, out=None)
+
+
+@pytest.mark.parametrize("stride", [dict(qf_stride=0), dict(qf_seq_stride=-1), dict(qf_tok_stride=-1)], ids=str)
+def test_prefill_qf_rejects_bad_strides(stride):
+    s = dict(qf_stride=1, qf_seq_stride=4096, qf_tok_stride=2)
+    s.update(stride)
+    with pytest.raises(kpa.KpaError) as e:
+        kpa.kpa_prefill_qf(PCFG, 2, 64, A, s["qf_stride"], s["qf_seq_stride"], s["qf_tok_stride"], A, A, A, 128,
+                           0.1, A, stream=0)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def _append(**over):
+    args = dict(batch=2, n_tok=64, x=A, w=A, start_pos=A, capacity=128, kcache=A, vcache=A, q_out=None,
+                workspace=None, ws_bytes=0)
+    args.update(over)
+    kpa.kpa_append(PCFG, args["batch"], args["n_tok"], args["x"], args["w"], args["start_pos"], args["capacity"],
+                   args["kcache"], args["vcache"], args["q_out"], args["workspace"], args["ws_bytes"], stream=0)
+
+
+@pytest.mark.parametrize("over", [
+    dict(x=None), dict(w=None), dict(start_pos=None), dict(kcache=None), dict(vcache=None),
+    dict(x=A + 2), dict(w=A + 8), dict(kcache=A + 4), dict(start_pos=A + 2), dict(q_out=A + 4),
+    dict(capacity=12), dict(capacity=0), dict(batch=-1), dict(n_tok=-1),
+], ids=str)
+def test_append_rejects_before_launch(over):
+    with pytest.raises(kpa.KpaError) as e:
+        _append(**over)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+
+
+def test_append_workspace_checked_before_launch():
+    """q_out needs the workspace kpa_append_workspace_size gives (the query factors in fp32),
+    256-byte aligned; an empty call is a no-op."""
+    need = kpa.kpa_append_workspace_size(PCFG, 2, 64)
+    e_q = APPEND_PREFILL.shape.r_q * (APPEND_PREFILL.shape.h1 * APPEND_PREFILL.shape.d1 +
+                                      APPEND_PREFILL.shape.h2 * APPEND_PREFILL.shape.d2)
+    assert need >= 2 * 64 * e_q * 4 and need % 256 == 0
+    for over in (dict(q_out=A), dict(q_out=A, workspace=A, ws_bytes=need - 1), dict(workspace=A, ws_bytes=0)):
+        with pytest.raises(kpa.KpaError) as e:
+            _append(**over)
+        assert e.value.status == kpa.KPA_ERR_WORKSPACE, over
+    with pytest.raises(kpa.KpaError) as e:
+        _append(q_out=A, workspace=A + 16, ws_bytes=need)
+    assert e.value.status == kpa.KPA_ERR_INVALID_ARG
+    _append(batch=0, x=None, w=None, start_pos=None, kcache=None, vcache=None)
